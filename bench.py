@@ -1,0 +1,485 @@
+#!/usr/bin/env python
+"""Benchmark of the Mamba-2 SSD hot path on B200: chunked prefill tokens/s (the
+long-context workload: 1 x 65536 tokens, H=64, P=64, G=8, N=128, chunk 256, bf16)
+plus decode steps/s (256 sequences with 2 MiB FP32 states), each with its HBM
+roofline fraction, and the FP64 oracle timed on the host cores beside them.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+  torchrun --nproc-per-node N bench.py --gpus N ...   (one rank per GPU)
+
+One JSON line is printed by rank 0. Multi-GPU runs are replicas: every rank runs
+its own independent problem (different seed), there is no data-path collective,
+`value` is the tokens all ranks processed divided by the slowest rank's time, and
+scaling is weak.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from mamba_ssd_state_02_b200 import workloads as W  # noqa: E402
+
+METRIC = "SSD prefill tokens/s & decode steps/s on 1 B200; % of HBM/tensor roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PREFILL_CONFIG = 2
+DECODE_CONFIG = 4
+
+
+# ------------------------------------------------------------------------------ ranks
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def dist_setup(world: int, backend: str):
+    if world > 1 and not torch.distributed.is_initialized():
+        import datetime
+        torch.distributed.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def max_over_ranks(v: float, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (identity without a process group)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return float(v)
+    t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        if device is not None and device.type == "cuda":
+            torch.distributed.barrier(device_ids=[device.index])
+        else:
+            torch.distributed.barrier()
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Independent problem per rank: same recipe, different seed."""
+    return base + 7919 * rank
+
+
+# ------------------------------------------------------------------------------ peaks / bytes
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def path_bytes(w: W.Workload) -> int:
+    """Algorithmic bytes of one prefill call: each input read once, each output
+    written once (x, B, C, dt_raw, y, initial and final states, per-head params)."""
+    T, H, P, G, N = w.total_tokens, w.nheads, w.headdim, w.ngroups, w.dstate
+    e = 2 if w.dtype == torch.bfloat16 else 4
+    b = T * H * P * e * 2 + T * G * N * e * 2 + T * H * 4 + w.nseq * H * P * N * 4 + 3 * H * 4
+    if w.init != "zero":
+        b += w.nseq * H * P * N * 4
+    return b
+
+
+def path_flops(w: W.Workload) -> int:
+    """Tensor-core flops of the chunked method (2 per multiply-add), with the masked
+    causal half of each Q x Q block excluded. Per token-head: C.B^T shared by the
+    group's H/G heads Q*N/(H/G), intra-chunk M.X Q*P, chunk state 2*N*P, C.h 2*N*P."""
+    Q, H, P, G, N = w.chunk, w.nheads, w.headdim, w.ngroups, w.dstate
+    per = Q * N // (H // G) + Q * P + 4 * N * P
+    return w.total_tokens * H * per
+
+
+def kernel_bytes(name: str, w: W.Workload, nchunks: int) -> int:
+    """Algorithmic bytes one launch of each kernel must move for the prefill workload
+    (inputs read once, outputs written once, intermediates of the pipeline counted
+    where the kernel reads or writes them)."""
+    T, H, P, G, N, Q = w.total_tokens, w.nheads, w.headdim, w.ngroups, w.dstate, w.chunk
+    e = 2 if w.dtype == torch.bfloat16 else 4
+    x = T * H * P * e
+    bc = T * G * N * e
+    dtq = nchunks * H * Q * 4
+    st = nchunks * H * P * N * 4
+    fin = w.nseq * H * P * N * 4
+    return {
+        "ssd_chunk_table": nchunks * 16,
+        "ssd_chunk_cumsum": T * H * 4 + 2 * dtq,
+        "ssd_chunk_state": x + bc + 2 * dtq + st,
+        "ssd_state_passing": 2 * st + fin + nchunks * H * 4,
+        "ssd_chunk_scan": 2 * x + 2 * bc + 2 * dtq + st,
+    }.get(name, 0)
+
+
+def decode_step_bytes(nseq, H, P, G, N, e=2) -> int:
+    return 2 * nseq * H * P * N * 4 + 2 * nseq * H * P * e + 2 * nseq * G * N * e + nseq * H * 4
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "mamba_ssd_state_02_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(workload, {}).get(kernel)
+    if not e or e.get("source_hash") != source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 100 ms while running."""
+    FIELDS = ["timestamp", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device):
+        self.proc = None
+        self.file = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            self.sel = str(device.index)
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.sel, "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "20"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self, window=None):
+        """Summary of the samples taken inside `window` = (t0, t1) host wall-clock
+        seconds (all samples if None; the nearest later sample if none fall inside)."""
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.strip().split(", ") for r in self.file.read().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        import datetime
+        parsed = []
+        for r in rows:
+            if len(r) < len(self.FIELDS):
+                continue
+            try:
+                ts = datetime.datetime.strptime(r[0].strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                parsed.append((ts, float(r[1]), float(r[2]), r[5:9]))
+            except ValueError:
+                continue
+        sel = parsed
+        if window is not None:
+            sel = [p for p in parsed if window[0] <= p[0] <= window[1]]
+            if not sel:
+                later = [p for p in parsed if p[0] >= window[0]]
+                sel = later[:1]
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ts, a, b, rs in sel:
+            sm.append(a)
+            mx.append(b)
+            for k, v in zip(names, rs):
+                if v.strip().lower() == "active":
+                    reasons.add(k)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------ oracle baseline
+def oracle_sample(w: W.Workload, tokens: int, heads: int, seed_rank: int = 0):
+    """Time the FP64 oracle (as it stands) on the first `tokens` tokens of sequence 0
+    for `heads` heads; returns (tokens/s of the full workload's width, threads, desc)."""
+    from oracle import oracle as O
+    tok = W.make_tokens(w, 0, tokens)
+    par = W.make_params(w)
+    threads = max(1, len(os.sched_getaffinity(0)))
+    pairs = [(0, h) for h in range(heads)]
+    O.build()
+    t0 = time.perf_counter()
+    O.ssd_scan(tok["x"], tok["dt_raw"], par["dt_bias"], par["A"], tok["B"], tok["C"], par["D"],
+               pairs=pairs, nthreads=threads)
+    dt = time.perf_counter() - t0
+    tok_heads_per_s = tokens * heads / dt
+    return tok_heads_per_s / w.nheads, threads, dt
+
+
+# ------------------------------------------------------------------------------ our arm
+def bench_ours(args, rank, world, local_rank):
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist_setup(world, "nccl")
+    from mamba_ssd_state_02_b200 import build
+    if rank == 0:
+        build.build()
+    barrier(dev)
+    from mamba_ssd_state_02_b200 import ssd
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+
+    # ---- prefill (long-context workload)
+    w = W.config(PREFILL_CONFIG, seed=rank_seed(1000 + PREFILL_CONFIG, rank))
+    inp = W.make_all(w, device=dev)
+    L = w.seqlens[0]
+    r4 = lambda t: t.view(w.nseq, L, *t.shape[1:])
+    x, dtr, Bm, Cm = r4(inp["x"]), r4(inp["dt_raw"]), r4(inp["B"]), r4(inp["C"])
+    y = torch.empty_like(x)
+    fin = torch.empty(w.nseq, w.nheads, w.headdim, w.dstate, dtype=torch.float32, device=dev)
+    dims = ssd.make_dims(w.total_tokens, w.nheads, w.headdim, w.ngroups, w.dstate, ssd.SSD_DTYPE_BF16,
+                         batch=w.nseq, seqlen=L)
+    ws = torch.empty(ssd.workspace_size(dims, w.chunk), dtype=torch.uint8, device=dev)
+    variant = ssd.scan_variant(dims, w.chunk)
+
+    def step():
+        ssd.scan_fwd(x, dtr, inp["dt_bias"], inp["A"], Bm, Cm, inp["D"], init_state=inp["init_state"],
+                     chunk=w.chunk, y=y, final_state=fin, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    ssd.device_status()
+    launches_per_call = ssd.last_launch_count()
+    stream = torch.cuda.current_stream(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    ssd.profile_enable(True)
+    t_wall0 = time.time()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    barrier(dev)
+    ms_total = ev0.elapsed_time(ev1)
+    kprof = ssd.profile_read()
+    ssd.profile_enable(False)
+    time.sleep(0.1)
+    clk = clocks.stop((t_wall0, t_wall1))
+    ssd.device_status()
+    ms_step = max_over_ranks(ms_total / args.steps, dev)
+    value = world * w.total_tokens / (ms_step / 1e3)
+
+    # Dominant kernel roofline (per-launch device time from events inside the timed region).
+    nchunks = w.nseq * math.ceil(L / w.chunk)
+    dom = max((k for k in kprof if not k.startswith("_")), key=lambda k: kprof[k][1])
+    n_l, t_l = kprof[dom]
+    kb = kernel_bytes(dom, w, nchunks)
+    achieved = kb / (t_l / n_l / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": hbm,
+                "peak_source": peak_src, "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                "bytes_per_launch": kb, "ms_per_launch": round(t_l / n_l, 4),
+                "traffic": ncu_traffic(dom, w.name)}
+    pb = path_bytes(w)
+    pf = path_flops(w)
+    t_bw = pb / (hbm * 1e9)
+    t_tc = pf / (float(peaks["bf16_tflops"]) * 1e12)
+    path_roof = {"bytes": pb, "flops": pf, "roofline_ms": round(max(t_bw, t_tc) * 1e3, 4),
+                 "bound": "hbm" if t_bw >= t_tc else "tensor",
+                 "frac": round(max(t_bw, t_tc) * 1e3 / ms_step, 4),
+                 "frac_nominal_8tbs": round(pb / 8e12 * 1e3 / ms_step, 4)}
+    kernels = {k: {"launches": v[0], "ms_per_launch": round(v[1] / max(1, v[0]), 4)}
+               for k, v in kprof.items()}
+
+    # ---- end to end through the public call with host buffers
+    host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in inp.items()
+            if k in ("x", "dt_raw", "B", "C", "dt_bias", "A", "D", "init_state")}
+    y_h = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    f_h = torch.empty(fin.shape, dtype=fin.dtype).pin_memory()
+    dbuf = {k: (None if v is None else torch.empty_like(v, device=dev)) for k, v in host.items()}
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = y_h.numel() * y_h.element_size() + f_h.numel() * f_h.element_size()
+
+    def e2e_step():
+        for k, v in host.items():
+            if v is not None:
+                dbuf[k].copy_(v, non_blocking=True)
+        ssd.scan_fwd(r4(dbuf["x"]), r4(dbuf["dt_raw"]), dbuf["dt_bias"], dbuf["A"], r4(dbuf["B"]),
+                     r4(dbuf["C"]), dbuf["D"], init_state=dbuf["init_state"], chunk=w.chunk, y=y,
+                     final_state=fin, workspace=ws)
+        y_h.copy_(y, non_blocking=True)
+        f_h.copy_(fin, non_blocking=True)
+
+    e2e_steps = max(1, min(args.steps, 5))
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(dev)
+    ev0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1) / e2e_steps, dev)
+    e2e = {"value": world * w.total_tokens / (e2e_ms / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3),
+           "steps": e2e_steps}
+    del host, dbuf, inp, x, dtr, Bm, Cm, y, ws
+    torch.cuda.empty_cache()
+
+    # ---- decode (256 sequences, FP32 states from a 2048-token prefill)
+    decode = bench_decode(args, ssd, dev, rank, world, hbm, peak_src)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.nseq, "seq_len": L, "nheads": w.nheads,
+                   "headdim": w.headdim, "ngroups": w.ngroups, "dstate": w.dstate, "chunk": w.chunk,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (%.2f GB per step vs 126 MB L2), no flush" % (pb / 1e9),
+                   "variant": variant},
+        "roofline": roofline, "path_roofline": path_roof, "kernels": kernels,
+        "clocks": clk, "e2e": e2e, "gpu_launches": launches_per_call * args.steps,
+        "decode": decode,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, threads, secs = oracle_sample(w, 16384, w.nheads)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                "sample": f"all {w.nheads} heads of the first 16384 tokens "
+                                          f"({secs:.1f} s wall)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def bench_decode(args, ssd, dev, rank, world, hbm, peak_src):
+    w = W.config(DECODE_CONFIG, seed=rank_seed(1000 + DECODE_CONFIG, rank))
+    nseq, H, P, G, N, prefix = w.nseq, w.nheads, w.headdim, w.ngroups, w.dstate, w.seqlens[0]
+    steps_timed = max(args.steps, 64)
+    Ltot = prefix + w.decode_steps
+    par = W.make_params(w, device=dev)
+    b_idx = torch.arange(nseq, device=dev, dtype=torch.int64)
+    pre_rows = (b_idx[:, None] * Ltot + torch.arange(prefix, device=dev)[None, :]).reshape(-1)
+    pre = W.make_tokens(w, 0, 0, rows=pre_rows)
+    rs = lambda t: t.reshape(nseq, prefix, *t.shape[1:])
+    _, state = ssd.scan_fwd(rs(pre["x"]), rs(pre["dt_raw"]), par["dt_bias"], par["A"], rs(pre["B"]),
+                            rs(pre["C"]), par["D"], chunk=w.chunk)
+    del pre
+    torch.cuda.empty_cache()
+    nstep_inputs = min(w.decode_steps, steps_timed + args.warmup)
+    step_rows = (torch.arange(nstep_inputs, device=dev)[:, None] + prefix + b_idx[None, :] * Ltot).reshape(-1)
+    stp = W.make_tokens(w, 0, 0, rows=step_rows)
+    xs = stp["x"].view(-1, nseq, H, P)
+    dts = stp["dt_raw"].view(-1, nseq, H)
+    Bs = stp["B"].view(-1, nseq, G, N)
+    Cs = stp["C"].view(-1, nseq, G, N)
+    y = torch.empty(nseq, H, P, dtype=w.dtype, device=dev)
+    k = [0]
+
+    def step():
+        i = k[0] % nstep_inputs
+        ssd.state_update(state, xs[i], dts[i], par["dt_bias"], par["A"], Bs[i], Cs[i], par["D"], y=y)
+        k[0] += 1
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    ssd.device_status()
+    stream = torch.cuda.current_stream(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(steps_timed):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / steps_timed, dev)
+    sb = decode_step_bytes(nseq, H, P, G, N)
+    achieved = sb / (ms / 1e3) / 1e9
+    return {"workload": w.name, "steps_per_s": 1e3 / ms, "replicas": world,
+            "tokens_per_s": world * nseq * 1e3 / ms, "ms_per_step": round(ms, 4),
+            "steps_timed": steps_timed,
+            "roofline": {"bound": "hbm", "kernel": "ssd_state_update", "achieved": round(achieved, 1),
+                         "peak": hbm, "peak_source": peak_src, "unit": "GB/s",
+                         "frac": round(achieved / hbm, 4), "bytes_per_launch": sb,
+                         "traffic": ncu_traffic("ssd_state_update", w.name)}}
+
+
+# ------------------------------------------------------------------------------ reference arm
+def bench_reference(args, rank, world):
+    """The FP64 oracle on the host cores as the reference arm: same workload, metric
+    and unit; each step a bounded sample (all heads of the first 4096 tokens)."""
+    if rank != 0:
+        return
+    w = W.config(PREFILL_CONFIG)
+    tokens = 4096
+    for _ in range(args.warmup):
+        oracle_sample(w, tokens, w.nheads)
+    times, threads = [], 1
+    for _ in range(args.steps):
+        v, threads, secs = oracle_sample(w, tokens, w.nheads)
+        times.append(secs)
+    sec = statistics.mean(times)
+    value = tokens / sec
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(sec * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.nseq, "seq_len": w.seqlens[0], "nheads": w.nheads,
+                   "headdim": w.headdim, "ngroups": w.ngroups, "dstate": w.dstate, "chunk": w.chunk},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"per step: all {w.nheads} heads of the first {tokens} tokens"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    rank, world, local_rank = dist_env()
+    if args.impl == "reference":
+        bench_reference(args, rank, world)
+        return
+    try:
+        bench_ours(args, rank, world, local_rank)
+    finally:
+        if torch.distributed.is_available() and torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,176 @@
+/*
+ * libssd: the Mamba-2 SSD selective scan (chunked prefill) and its per-token decode
+ * step, for NVIDIA B200 (sm_100a).
+ *
+ * The operation. For every sequence and head h (group g = h / (H/G), heads share B
+ * and C within a group "like GQA": JAX Nemotron 3 Nano page, NemotronConfig
+ * `mamba_ngroups`), token by token:
+ *
+ *     dt_t   = softplus(dt_raw[t,h] + dt_bias[h])          RL-Kernel issue page, Figure 2
+ *     h_t    = exp(dt_t * A[h]) * h_{t-1} + dt_t * x_t B_t^T      (FP32 state, ibid. §1)
+ *     y_t[p] = sum_n C_t[n] * h_t[p][n] + D[h] * x_t[p]           (D skip: JAX page,
+ *                                                                  "Key Components")
+ *
+ * starting from the caller's initial state (or zero). Prefill evaluates this with
+ * the chunked SSD algorithm (JAX page, "Key Components" 1: "Chunked SSD algorithm
+ * keeps memory usage bounded"; RL-Kernel issue page, Figure 2: "SSD chunked scan"),
+ * decode with the per-token recurrent update (RL-Kernel issue page, §1 and §2:
+ * causal_conv1d_update + selective_state_update). The state is stored [P][N] with N
+ * contiguous (the transpose of B x^T).
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library never
+ *     frees or retains them. Layouts are row-major and contiguous:
+ *         x, y        [T, H, P]           (dtype: float32 or bf16)
+ *         B, C        [T, G, N]           (same dtype as x)
+ *         dt_raw      [T, H]              float32
+ *         dt_bias, A, D [H]               float32 (A must be <= 0 and finite)
+ *         states      [nseq, H, P, N]     float32
+ *     where T is the number of tokens in the call (dense: batch*seqlen).
+ *   - Work is enqueued on `stream` and the call returns without waiting for it.
+ *     Errors found on the host are returned at once; errors found by a kernel
+ *     (bad cu_seqlens, A > 0, a bounded wait that ran out) are latched in a device
+ *     error word that ssd_get_device_status() reads and clears.
+ *   - Fail closed: geometry outside the supported set returns SSD_ERR_UNSUPPORTED
+ *     and nothing is launched; there is no CPU or other fallback (RL-Kernel issue
+ *     page, §4.1 "fail closed on unsupported strict geometry" and §7).
+ *   - Functions are thread-safe; ssd_last_error() is per host thread.
+ */
+#ifndef SSD_H
+#define SSD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same handle type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* ssd_stream_t;
+
+typedef enum {
+    SSD_OK = 0,
+    SSD_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, negative size, inconsistent dims */
+    SSD_ERR_UNSUPPORTED = 2,   /* valid but outside the supported geometry (fail closed) */
+    SSD_ERR_CUDA = 3,          /* a CUDA runtime call failed (message in ssd_last_error) */
+    SSD_ERR_TIMEOUT = 4        /* a device-side bounded wait expired */
+} ssd_status;
+
+typedef enum {
+    SSD_DTYPE_F32 = 0,         /* x, B, C, y are float32 */
+    SSD_DTYPE_BF16 = 1         /* x, B, C, y are bf16; dt, A, D and states stay float32 */
+} ssd_dtype;
+
+/*
+ * Problem description.
+ *   Dense mode (cu_seqlens == NULL): nseq = batch sequences of seqlen tokens each,
+ *     T = batch * seqlen; token t of sequence b is packed row b*seqlen + t.
+ *   Packed varlen mode (cu_seqlens != NULL): nseq sequences, T = total_tokens, which
+ *     must equal cu_seqlens[nseq]; sequence s owns rows [cu_seqlens[s], cu_seqlens[s+1]).
+ *     batch and seqlen are ignored.
+ *   nheads H, headdim P, ngroups G (H % G == 0), dstate N.
+ *   workspace / workspace_bytes: optional device scratch of at least the size
+ *     ssd_scan_fwd_workspace_size() reports (256-byte aligned). When workspace is
+ *     NULL the call allocates and frees scratch itself with cudaMallocAsync /
+ *     cudaFreeAsync on `stream`. The decode step needs no workspace.
+ */
+typedef struct {
+    int64_t batch;
+    int64_t seqlen;
+    int32_t nseq;
+    int64_t total_tokens;
+    int32_t nheads;
+    int32_t headdim;
+    int32_t ngroups;
+    int32_t dstate;
+    ssd_dtype dtype;
+    void* workspace;
+    size_t workspace_bytes;
+} ssd_dims;
+
+/*
+ * Bytes of device scratch ssd_scan_fwd needs for `dims` and `chunk`, written to
+ * *bytes. Returns SSD_OK, or the status ssd_scan_fwd would return for these dims.
+ */
+ssd_status ssd_scan_fwd_workspace_size(const ssd_dims* dims, int chunk, size_t* bytes);
+
+/*
+ * Chunked SSD prefill (the operation above) over every sequence of the call.
+ *   x, dt_raw, dt_bias, A, B, C, D: inputs (layouts above).
+ *   init_state: [nseq,H,P,N] float32, or NULL for zero initial states.
+ *   cu_seqlens: [nseq+1] int32 device array, or NULL for dense mode. Chunks are
+ *     anchored at each sequence start and the state never crosses a sequence
+ *     boundary (RL-Kernel issue page, §7 "sequence-anchored chunks", §8 Q4
+ *     "cu_seqlens-aware chunking"); a sequence's last chunk may be partial.
+ *   y: [T,H,P] output, same dtype as x (bf16 rounded to nearest even).
+ *   final_state: [nseq,H,P,N] float32 output (the state after each sequence's last
+ *     token; the initial state for an empty sequence), or NULL.
+ *   chunk: 64, 128 or 256 tokens per chunk. The result does not depend on it
+ *     beyond rounding.
+ * Supported: P and N in {16, 32, 64, 128}; x/B/C/y 16-byte aligned; other arrays
+ * 4-byte aligned. x, B, C and y must not overlap each other or the states.
+ */
+ssd_status ssd_scan_fwd(const void* x, const float* dt_raw, const float* dt_bias, const float* A,
+                        const void* B, const void* C, const float* D, const float* init_state,
+                        const int32_t* cu_seqlens, void* y, float* final_state,
+                        const ssd_dims* dims, int chunk, ssd_stream_t stream);
+
+/*
+ * One decode step for nseq = dims->batch sequences (dims->seqlen must be 1; varlen
+ * fields are ignored): per sequence and head, dt = softplus(dt_raw + dt_bias),
+ * state <- exp(dt*A) * state + dt * x B^T in place, y = state . C + D * x.
+ *   state: [nseq,H,P,N] float32, read and overwritten.
+ *   x [nseq,H,P], B/C [nseq,G,N] (dims->dtype), dt_raw [nseq,H] float32.
+ *   y: [nseq,H,P] output, dims->dtype.
+ * Same support set as ssd_scan_fwd; no workspace.
+ */
+ssd_status ssd_state_update(float* state, const void* x, const float* dt_raw, const float* dt_bias,
+                            const float* A, const void* B, const void* C, const float* D, void* y,
+                            const ssd_dims* dims, ssd_stream_t stream);
+
+/*
+ * Waits for `stream`, then reads and clears the device error word: SSD_OK, or the
+ * first error a kernel latched since the last read (SSD_ERR_INVALID_ARG for bad
+ * cu_seqlens or A > 0, SSD_ERR_TIMEOUT for an expired bounded wait). SSD_ERR_CUDA
+ * if the wait itself failed.
+ */
+ssd_status ssd_get_device_status(ssd_stream_t stream);
+
+/* Message for the last non-OK status returned on this host thread ("" if none). */
+const char* ssd_last_error(void);
+
+/*
+ * Name of the kernel pipeline ssd_scan_fwd uses for these dims and chunk
+ * ("tc": tcgen05 tensor-core kernels; "simt": CUDA-core FP32 kernels), or "" when
+ * the dims are rejected.
+ */
+const char* ssd_scan_fwd_variant(const ssd_dims* dims, int chunk);
+
+/* Number of kernels the last successful call on this host thread enqueued. */
+int ssd_last_launch_count(void);
+
+/*
+ * Per-kernel timing (tracing). While enabled, every kernel the library enqueues is
+ * bracketed by a pair of CUDA events on its stream; ssd_profile_read() waits for
+ * the recorded events and reports, per kernel name, the launches and the summed
+ * device time since profiling was enabled (or last read). Enabling resets the
+ * totals. At most 65536 launches are kept between reads; later ones are counted
+ * in `dropped`. Device time only: the events add no host synchronisation.
+ */
+typedef struct {
+    const char* name;      /* kernel name (static string) */
+    int launches;
+    double total_ms;
+} ssd_kernel_time;
+
+void ssd_profile_enable(int on);
+/* Fills up to `max` entries, returns how many kernel names had launches, or -1 if
+ * waiting on an event failed. *dropped (nullable) receives the unrecorded count. */
+int ssd_profile_read(ssd_kernel_time* out, int max, int* dropped);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_H */

@@ -1,0 +1,449 @@
+// libssd C ABI: argument validation (fail closed), workspace planning and kernel
+// dispatch for the chunked SSD prefill and the decode step. All kernels of the
+// library live in this translation unit (the .cuh files), so they share the device
+// error word without relocatable device code.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "ssd.h"
+#include "ssd_common.cuh"
+#include "ssd_decode.cuh"
+#include "ssd_scan_simt.cuh"
+
+namespace ssd {
+namespace {
+
+thread_local std::string t_last_error;
+thread_local int t_launches = 0;
+
+ssd_status fail(ssd_status st, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    t_last_error = buf;
+    return st;
+}
+
+ssd_status cuda_fail(cudaError_t e, const char* what) {
+    return fail(SSD_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// ---------------------------------------------------------------------------------
+// Per-kernel event timing (ssd_profile_enable / ssd_profile_read).
+enum Stage { ST_TABLE, ST_CUMSUM, ST_CHUNK_STATE, ST_STATE_PASSING, ST_CHUNK_SCAN, ST_STATE_UPDATE,
+             ST_COUNT };
+const char* const kStageName[ST_COUNT] = {"ssd_chunk_table", "ssd_chunk_cumsum", "ssd_chunk_state",
+                                          "ssd_state_passing", "ssd_chunk_scan", "ssd_state_update"};
+constexpr size_t kMaxRecords = 65536;
+
+struct Profiler {
+    std::mutex mu;
+    bool on = false;
+    struct Rec { int stage; cudaEvent_t a, b; };
+    std::vector<Rec> recs;
+    std::vector<cudaEvent_t> pool;
+    int dropped = 0;
+    cudaEvent_t get() {
+        if (!pool.empty()) {
+            cudaEvent_t e = pool.back();
+            pool.pop_back();
+            return e;
+        }
+        cudaEvent_t e = nullptr;
+        if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+        return e;
+    }
+};
+Profiler g_prof;
+
+// Brackets one kernel launch with events when profiling is on.
+struct StageScope {
+    int stage;
+    cudaStream_t st;
+    cudaEvent_t a = nullptr;
+    StageScope(int s, cudaStream_t stream) : stage(s), st(stream) {
+        std::lock_guard<std::mutex> lk(g_prof.mu);
+        if (!g_prof.on) return;
+        if (g_prof.recs.size() >= kMaxRecords) {
+            ++g_prof.dropped;
+            return;
+        }
+        a = g_prof.get();
+        if (a) cudaEventRecord(a, st);
+    }
+    ~StageScope() {
+        if (!a) return;
+        std::lock_guard<std::mutex> lk(g_prof.mu);
+        cudaEvent_t b = g_prof.get();
+        if (!b) {
+            g_prof.pool.push_back(a);
+            return;
+        }
+        cudaEventRecord(b, st);
+        g_prof.recs.push_back({stage, a, b});
+    }
+};
+
+bool pow2_in(int v, int lo, int hi) { return v >= lo && v <= hi && (v & (v - 1)) == 0; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Validate dims/chunk and fill the plan (no pointers looked at here).
+ssd_status make_plan(const ssd_dims* d, int chunk, bool varlen, Plan* pl) {
+    if (!d) return fail(SSD_ERR_INVALID_ARG, "dims is NULL");
+    if (d->nheads <= 0 || d->headdim <= 0 || d->ngroups <= 0 || d->dstate <= 0)
+        return fail(SSD_ERR_INVALID_ARG, "nheads, headdim, ngroups and dstate must be positive");
+    if (d->nheads % d->ngroups != 0)
+        return fail(SSD_ERR_UNSUPPORTED, "nheads (%d) must be a multiple of ngroups (%d)", d->nheads,
+                    d->ngroups);
+    if (!pow2_in(d->headdim, 16, 128))
+        return fail(SSD_ERR_UNSUPPORTED, "headdim %d not in {16,32,64,128}", d->headdim);
+    if (!pow2_in(d->dstate, 16, 128))
+        return fail(SSD_ERR_UNSUPPORTED, "dstate %d not in {16,32,64,128}", d->dstate);
+    if (chunk != 64 && chunk != 128 && chunk != 256)
+        return fail(SSD_ERR_UNSUPPORTED, "chunk %d not in {64,128,256}", chunk);
+    if (d->dtype != SSD_DTYPE_F32 && d->dtype != SSD_DTYPE_BF16)
+        return fail(SSD_ERR_INVALID_ARG, "unknown dtype %d", (int)d->dtype);
+    Plan p;
+    p.H = d->nheads;
+    p.P = d->headdim;
+    p.G = d->ngroups;
+    p.N = d->dstate;
+    p.Q = chunk;
+    p.bf16 = d->dtype == SSD_DTYPE_BF16;
+    p.varlen = varlen;
+    if (varlen) {
+        if (d->nseq < 0 || d->total_tokens < 0)
+            return fail(SSD_ERR_INVALID_ARG, "nseq and total_tokens must be >= 0");
+        p.nseq = d->nseq;
+        p.T = d->total_tokens;
+        p.max_chunks = p.T / chunk + p.nseq;
+    } else {
+        if (d->batch < 0 || d->seqlen < 0) return fail(SSD_ERR_INVALID_ARG, "batch and seqlen must be >= 0");
+        if (d->batch > INT32_MAX) return fail(SSD_ERR_UNSUPPORTED, "batch too large");
+        p.nseq = (int32_t)d->batch;
+        p.seqlen = d->seqlen;
+        if (d->seqlen > 0 && d->batch > INT64_MAX / d->seqlen)
+            return fail(SSD_ERR_INVALID_ARG, "batch*seqlen overflows");
+        p.T = d->batch * d->seqlen;
+        p.max_chunks = d->batch * ((d->seqlen + chunk - 1) / chunk);
+    }
+    // Packed token rows and chunk indices are int32 on the device.
+    if (p.T >= INT32_MAX || p.max_chunks >= INT32_MAX / 2)
+        return fail(SSD_ERR_UNSUPPORTED, "more than 2^31-1 tokens in one call");
+    if (p.T * (int64_t)p.H * p.P >= (int64_t)1 << 40)
+        return fail(SSD_ERR_UNSUPPORTED, "x has more than 2^40 elements");
+    // Workspace carving (256-byte aligned pieces).
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off = align_up(off + bytes, 256);
+        return o;
+    };
+    const size_t mc = (size_t)p.max_chunks;
+    p.off_table = take(sizeof(ChunkEntry) * (mc > 0 ? mc : 1));
+    p.off_first = take(sizeof(int32_t) * ((size_t)p.nseq + 1));
+    p.off_count = take(sizeof(int32_t));
+    p.off_dt = take(sizeof(float) * mc * p.H * p.Q);
+    p.off_acum = take(sizeof(float) * mc * p.H * p.Q);
+    p.off_states = take(sizeof(float) * mc * p.H * p.P * p.N);
+    p.bytes = off;
+    *pl = p;
+    return SSD_OK;
+}
+
+// ---------------------------------------------------------------------------------
+// SIMT pipeline launch, templated on the geometry.
+template <typename T, int Q, int P, int N>
+ssd_status launch_simt(const Plan& pl, char* ws, const T* x, const float* dt_raw,
+                       const float* dt_bias, const float* A, const T* B, const T* C,
+                       const float* D, const float* init, const int32_t* cu, T* y, float* fin,
+                       cudaStream_t st) {
+    auto* table = reinterpret_cast<ChunkEntry*>(ws + pl.off_table);
+    auto* first = reinterpret_cast<int32_t*>(ws + pl.off_first);
+    auto* count = reinterpret_cast<int32_t*>(ws + pl.off_count);
+    auto* dtc = reinterpret_cast<float*>(ws + pl.off_dt);
+    auto* acum = reinterpret_cast<float*>(ws + pl.off_acum);
+    auto* states = reinterpret_cast<float*>(ws + pl.off_states);
+    const int H = pl.H, G = pl.G;
+    int n = 0;
+    {
+        StageScope sc(ST_TABLE, st);
+        k_chunk_table<<<1, kTableThreads, 0, st>>>(cu, pl.nseq, pl.T, pl.seqlen, Q, table, first, count);
+    }
+    ++n;
+    if (pl.max_chunks > 0) {
+        const unsigned mc = (unsigned)pl.max_chunks;
+        {
+            StageScope sc(ST_CUMSUM, st);
+            k_chunk_cumsum<Q><<<dim3(mc, (H + 31) / 32), 256, 0, st>>>(dt_raw, dt_bias, A, table,
+                                                                        count, H, dtc, acum);
+        }
+        {
+            StageScope sc(ST_CHUNK_STATE, st);
+            k_chunk_state_simt<T, Q, P, N><<<dim3(mc, H), 256, 0, st>>>(x, B, dtc, acum, table,
+                                                                         count, H, G, states);
+        }
+        n += 2;
+    }
+    if (pl.nseq > 0) {
+        StageScope sc(ST_STATE_PASSING, st);
+        k_state_passing<Q><<<dim3(pl.nseq, H, (P * N + 255) / 256), 256, 0, st>>>(
+            states, acum, table, first, init, fin, H, P * N);
+        ++n;
+    }
+    if (pl.max_chunks > 0) {
+        constexpr size_t smem = chunk_scan_simt_smem<Q, P, N>();
+        cudaError_t e = cudaFuncSetAttribute(k_chunk_scan_simt<T, Q, P, N>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(chunk_scan)");
+        StageScope sc(ST_CHUNK_SCAN, st);
+        k_chunk_scan_simt<T, Q, P, N><<<dim3((unsigned)pl.max_chunks, H, Q / 32), 256, smem, st>>>(
+            x, B, C, D, dtc, acum, states, table, count, H, G, y);
+        ++n;
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch (simt scan)");
+    t_launches = n;
+    return SSD_OK;
+}
+
+template <typename T, int Q>
+ssd_status dispatch_PN(const Plan& pl, char* ws, const void* x, const float* dt_raw,
+                       const float* dt_bias, const float* A, const void* B, const void* C,
+                       const float* D, const float* init, const int32_t* cu, void* y, float* fin,
+                       cudaStream_t st) {
+#define SSD_CASE(PP, NN)                                                                       \
+    if (pl.P == PP && pl.N == NN)                                                              \
+        return launch_simt<T, Q, PP, NN>(pl, ws, (const T*)x, dt_raw, dt_bias, A, (const T*)B, \
+                                         (const T*)C, D, init, cu, (T*)y, fin, st);
+#define SSD_CASES_N(PP) SSD_CASE(PP, 16) SSD_CASE(PP, 32) SSD_CASE(PP, 64) SSD_CASE(PP, 128)
+    SSD_CASES_N(16) SSD_CASES_N(32) SSD_CASES_N(64) SSD_CASES_N(128)
+#undef SSD_CASES_N
+#undef SSD_CASE
+    return fail(SSD_ERR_UNSUPPORTED, "headdim/dstate combination");
+}
+
+template <typename T>
+ssd_status dispatch_Q(const Plan& pl, char* ws, const void* x, const float* dt_raw,
+                      const float* dt_bias, const float* A, const void* B, const void* C,
+                      const float* D, const float* init, const int32_t* cu, void* y, float* fin,
+                      cudaStream_t st) {
+    switch (pl.Q) {
+        case 64: return dispatch_PN<T, 64>(pl, ws, x, dt_raw, dt_bias, A, B, C, D, init, cu, y, fin, st);
+        case 128: return dispatch_PN<T, 128>(pl, ws, x, dt_raw, dt_bias, A, B, C, D, init, cu, y, fin, st);
+        case 256: return dispatch_PN<T, 256>(pl, ws, x, dt_raw, dt_bias, A, B, C, D, init, cu, y, fin, st);
+    }
+    return fail(SSD_ERR_UNSUPPORTED, "chunk");
+}
+
+template <typename T, int P, int N>
+void launch_decode(float* state, const void* x, const float* dt_raw, const float* dt_bias,
+                   const float* A, const void* B, const void* C, const float* D, void* y,
+                   int64_t nseq, int H, int G, cudaStream_t st) {
+    StageScope sc(ST_STATE_UPDATE, st);
+    k_state_update<T, P, N><<<(unsigned)(nseq * H), kDecodeThreads, 0, st>>>(
+        state, (const T*)x, dt_raw, dt_bias, A, (const T*)B, (const T*)C, D, (T*)y, H, G);
+}
+
+template <typename T>
+ssd_status dispatch_decode(int P, int N, float* state, const void* x, const float* dt_raw,
+                           const float* dt_bias, const float* A, const void* B, const void* C,
+                           const float* D, void* y, int64_t nseq, int H, int G, cudaStream_t st) {
+#define SSD_CASE(PP, NN)                                                                \
+    if (P == PP && N == NN) {                                                           \
+        launch_decode<T, PP, NN>(state, x, dt_raw, dt_bias, A, B, C, D, y, nseq, H, G, st); \
+        return SSD_OK;                                                                  \
+    }
+#define SSD_CASES_N(PP) SSD_CASE(PP, 16) SSD_CASE(PP, 32) SSD_CASE(PP, 64) SSD_CASE(PP, 128)
+    SSD_CASES_N(16) SSD_CASES_N(32) SSD_CASES_N(64) SSD_CASES_N(128)
+#undef SSD_CASES_N
+#undef SSD_CASE
+    return fail(SSD_ERR_UNSUPPORTED, "headdim/dstate combination");
+}
+
+}  // namespace
+}  // namespace ssd
+
+using namespace ssd;
+
+extern "C" {
+
+ssd_status ssd_scan_fwd_workspace_size(const ssd_dims* dims, int chunk, size_t* bytes) {
+    if (!bytes) return fail(SSD_ERR_INVALID_ARG, "bytes is NULL");
+    // Covers both modes for the fields given: the dense reading (batch, seqlen) and
+    // the packed reading (nseq, total_tokens); the larger of the valid ones wins.
+    Plan dense, packed;
+    const ssd_status sd = make_plan(dims, chunk, false, &dense);
+    const ssd_status sp = make_plan(dims, chunk, true, &packed);
+    if (sd != SSD_OK && sp != SSD_OK) return sd;
+    size_t b = 0;
+    if (sd == SSD_OK) b = dense.bytes;
+    if (sp == SSD_OK && packed.bytes > b) b = packed.bytes;
+    t_last_error.clear();
+    *bytes = b;
+    return SSD_OK;
+}
+
+ssd_status ssd_scan_fwd(const void* x, const float* dt_raw, const float* dt_bias, const float* A,
+                        const void* B, const void* C, const float* D, const float* init_state,
+                        const int32_t* cu_seqlens, void* y, float* final_state,
+                        const ssd_dims* dims, int chunk, ssd_stream_t stream) {
+    Plan pl;
+    ssd_status s = make_plan(dims, chunk, cu_seqlens != nullptr, &pl);
+    if (s != SSD_OK) return s;
+    if (!dt_bias || !A || !D) return fail(SSD_ERR_INVALID_ARG, "dt_bias, A and D must be non-NULL");
+    if (pl.T > 0 && (!x || !dt_raw || !B || !C || !y))
+        return fail(SSD_ERR_INVALID_ARG, "x, dt_raw, B, C and y must be non-NULL");
+    if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(y, 16))
+        return fail(SSD_ERR_INVALID_ARG, "x, B, C and y must be 16-byte aligned");
+    if (!aligned(dt_raw, 4) || !aligned(dt_bias, 4) || !aligned(A, 4) || !aligned(D, 4) ||
+        !aligned(init_state, 16) || !aligned(final_state, 16) || !aligned(cu_seqlens, 4))
+        return fail(SSD_ERR_INVALID_ARG, "float/int arrays must be 4-byte aligned, states 16-byte");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (pl.nseq == 0) {
+        t_launches = 0;
+        t_last_error.clear();
+        return SSD_OK;
+    }
+    char* ws = static_cast<char*>(dims->workspace);
+    bool owned = false;
+    if (ws) {
+        if (dims->workspace_bytes < pl.bytes)
+            return fail(SSD_ERR_INVALID_ARG, "workspace_bytes %zu < required %zu", dims->workspace_bytes,
+                        pl.bytes);
+        if (!aligned(ws, 256)) return fail(SSD_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    } else {
+        cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&ws), pl.bytes, st);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(workspace)");
+        owned = true;
+    }
+    if (pl.bf16)
+        s = dispatch_Q<__nv_bfloat16>(pl, ws, x, dt_raw, dt_bias, A, B, C, D, init_state, cu_seqlens, y,
+                                      final_state, st);
+    else
+        s = dispatch_Q<float>(pl, ws, x, dt_raw, dt_bias, A, B, C, D, init_state, cu_seqlens, y,
+                              final_state, st);
+    if (owned) {
+        cudaError_t e = cudaFreeAsync(ws, st);
+        if (e != cudaSuccess && s == SSD_OK) return cuda_fail(e, "cudaFreeAsync(workspace)");
+    }
+    if (s == SSD_OK) t_last_error.clear();
+    return s;
+}
+
+ssd_status ssd_state_update(float* state, const void* x, const float* dt_raw, const float* dt_bias,
+                            const float* A, const void* B, const void* C, const float* D, void* y,
+                            const ssd_dims* dims, ssd_stream_t stream) {
+    if (!dims) return fail(SSD_ERR_INVALID_ARG, "dims is NULL");
+    Plan pl;
+    ssd_dims d = *dims;
+    if (d.seqlen != 1) return fail(SSD_ERR_INVALID_ARG, "decode takes seqlen == 1 (got %lld)",
+                                   (long long)d.seqlen);
+    ssd_status s = make_plan(&d, 64, false, &pl);
+    if (s != SSD_OK) return s;
+    if (pl.nseq == 0) {
+        t_launches = 0;
+        t_last_error.clear();
+        return SSD_OK;
+    }
+    if (!state || !x || !dt_raw || !dt_bias || !A || !B || !C || !D || !y)
+        return fail(SSD_ERR_INVALID_ARG, "all decode pointers must be non-NULL");
+    if (!aligned(state, 16) || !aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(y, 16))
+        return fail(SSD_ERR_INVALID_ARG, "state, x, B, C and y must be 16-byte aligned");
+    if (!aligned(dt_raw, 4) || !aligned(dt_bias, 4) || !aligned(A, 4) || !aligned(D, 4))
+        return fail(SSD_ERR_INVALID_ARG, "float arrays must be 4-byte aligned");
+    if ((int64_t)pl.nseq * pl.H >= INT32_MAX) return fail(SSD_ERR_UNSUPPORTED, "nseq*nheads too large");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (pl.bf16)
+        s = dispatch_decode<__nv_bfloat16>(pl.P, pl.N, state, x, dt_raw, dt_bias, A, B, C, D, y,
+                                           pl.nseq, pl.H, pl.G, st);
+    else
+        s = dispatch_decode<float>(pl.P, pl.N, state, x, dt_raw, dt_bias, A, B, C, D, y, pl.nseq,
+                                   pl.H, pl.G, st);
+    if (s != SSD_OK) return s;
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch (state update)");
+    t_launches = 1;
+    t_last_error.clear();
+    return SSD_OK;
+}
+
+ssd_status ssd_get_device_status(ssd_stream_t stream) {
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    int code = 0;
+    e = cudaMemcpyFromSymbol(&code, g_device_error, sizeof code);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyFromSymbol(error word)");
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyToSymbol(error word)");
+    if (code == 0) {
+        t_last_error.clear();
+        return SSD_OK;
+    }
+    if (code == SSD_ERR_TIMEOUT) return fail(SSD_ERR_TIMEOUT, "a device-side bounded wait expired");
+    return fail((ssd_status)code, "a kernel rejected its data (bad cu_seqlens, or A > 0 / not finite)");
+}
+
+const char* ssd_last_error(void) { return t_last_error.c_str(); }
+
+const char* ssd_scan_fwd_variant(const ssd_dims* dims, int chunk) {
+    Plan pl;
+    if (make_plan(dims, chunk, false, &pl) != SSD_OK) return "";
+    return "simt";
+}
+
+int ssd_last_launch_count(void) { return t_launches; }
+
+void ssd_profile_enable(int on) {
+    std::lock_guard<std::mutex> lk(g_prof.mu);
+    g_prof.on = on != 0;
+    if (g_prof.on) {
+        for (auto& r : g_prof.recs) {
+            g_prof.pool.push_back(r.a);
+            g_prof.pool.push_back(r.b);
+        }
+        g_prof.recs.clear();
+        g_prof.dropped = 0;
+    }
+}
+
+int ssd_profile_read(ssd_kernel_time* out, int max, int* dropped) {
+    std::lock_guard<std::mutex> lk(g_prof.mu);
+    double ms[ST_COUNT] = {0};
+    int cnt[ST_COUNT] = {0};
+    int rc = 0;
+    for (auto& r : g_prof.recs) {
+        float t = 0.f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess)
+            rc = -1;
+        ms[r.stage] += t;
+        cnt[r.stage] += 1;
+        g_prof.pool.push_back(r.a);
+        g_prof.pool.push_back(r.b);
+    }
+    g_prof.recs.clear();
+    if (dropped) *dropped = g_prof.dropped;
+    g_prof.dropped = 0;
+    if (rc) return fail(SSD_ERR_CUDA, "waiting on a profiling event failed"), -1;
+    int k = 0;
+    for (int i = 0; i < ST_COUNT; ++i)
+        if (cnt[i] > 0) {
+            if (out && k < max) out[k] = {kStageName[i], cnt[i], ms[i]};
+            ++k;
+        }
+    return k;
+}
+
+}  // extern "C"

@@ -1,0 +1,244 @@
+"""Python binding of libssd (argument marshalling only).
+
+Every step of the SSD path runs in the CUDA kernels of ``libssd.so``; this module
+checks shapes and dtypes, passes ``data_ptr()`` values and the current CUDA stream
+through the C ABI declared in ``include/ssd.h``, and turns non-OK statuses into
+exceptions. There is no fallback: if the library is missing, importing this
+module raises.
+
+Functions mirror the C entry points:
+  scan_fwd(x, dt_raw, dt_bias, A, B, C, D, init_state=None, cu_seqlens=None,
+           chunk=128, y=None, final_state=None, workspace=None)
+  state_update(state, x, dt_raw, dt_bias, A, B, C, D, y=None)
+  device_status(), scan_variant(...), workspace_size(...), last_launch_count()
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libssd.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m mamba_ssd_state_02_b200.build` "
+        "(nvcc, sm_100a). The SSD path has no fallback.")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_CUDA, SSD_ERR_TIMEOUT = range(5)
+SSD_DTYPE_F32, SSD_DTYPE_BF16 = 0, 1
+_STATUS = {1: "SSD_ERR_INVALID_ARG", 2: "SSD_ERR_UNSUPPORTED", 3: "SSD_ERR_CUDA", 4: "SSD_ERR_TIMEOUT"}
+
+
+class SSDDims(ctypes.Structure):
+    """Mirror of ``ssd_dims`` (include/ssd.h)."""
+    _fields_ = [
+        ("batch", ctypes.c_int64),
+        ("seqlen", ctypes.c_int64),
+        ("nseq", ctypes.c_int32),
+        ("total_tokens", ctypes.c_int64),
+        ("nheads", ctypes.c_int32),
+        ("headdim", ctypes.c_int32),
+        ("ngroups", ctypes.c_int32),
+        ("dstate", ctypes.c_int32),
+        ("dtype", ctypes.c_int32),
+        ("workspace", ctypes.c_void_p),
+        ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
+_p = ctypes.c_void_p
+_lib.ssd_scan_fwd_workspace_size.argtypes = [ctypes.POINTER(SSDDims), ctypes.c_int,
+                                             ctypes.POINTER(ctypes.c_size_t)]
+_lib.ssd_scan_fwd_workspace_size.restype = ctypes.c_int
+_lib.ssd_scan_fwd.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p,
+                              ctypes.POINTER(SSDDims), ctypes.c_int, _p]
+_lib.ssd_scan_fwd.restype = ctypes.c_int
+_lib.ssd_state_update.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, ctypes.POINTER(SSDDims), _p]
+_lib.ssd_state_update.restype = ctypes.c_int
+_lib.ssd_get_device_status.argtypes = [_p]
+_lib.ssd_get_device_status.restype = ctypes.c_int
+_lib.ssd_last_error.argtypes = []
+_lib.ssd_last_error.restype = ctypes.c_char_p
+_lib.ssd_scan_fwd_variant.argtypes = [ctypes.POINTER(SSDDims), ctypes.c_int]
+_lib.ssd_scan_fwd_variant.restype = ctypes.c_char_p
+_lib.ssd_last_launch_count.argtypes = []
+_lib.ssd_last_launch_count.restype = ctypes.c_int
+
+
+class SSDKernelTime(ctypes.Structure):
+    """Mirror of ``ssd_kernel_time``."""
+    _fields_ = [("name", ctypes.c_char_p), ("launches", ctypes.c_int), ("total_ms", ctypes.c_double)]
+
+
+_lib.ssd_profile_enable.argtypes = [ctypes.c_int]
+_lib.ssd_profile_enable.restype = None
+_lib.ssd_profile_read.argtypes = [ctypes.POINTER(SSDKernelTime), ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
+_lib.ssd_profile_read.restype = ctypes.c_int
+
+
+class SSDError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{_STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+def _check(status: int) -> None:
+    if status != SSD_OK:
+        raise SSDError(status, _lib.ssd_last_error().decode())
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SSD_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return SSD_DTYPE_F32
+    raise TypeError(f"x/B/C must be float32 or bfloat16, got {t.dtype}")
+
+
+def _need(t, name, shape, dtype, device):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda or t.device != device:
+        raise ValueError(f"{name} must be on {device}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def make_dims(T, H, P, G, N, dtype_code, batch=None, seqlen=None, nseq=None, workspace=None):
+    d = SSDDims()
+    if nseq is not None:          # packed varlen
+        d.batch, d.seqlen, d.nseq, d.total_tokens = 0, 0, int(nseq), int(T)
+    else:
+        d.batch, d.seqlen, d.nseq, d.total_tokens = int(batch), int(seqlen), 0, 0
+    d.nheads, d.headdim, d.ngroups, d.dstate, d.dtype = H, P, G, N, dtype_code
+    if workspace is not None:
+        d.workspace, d.workspace_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    return d
+
+
+def workspace_size(dims: SSDDims, chunk: int) -> int:
+    b = ctypes.c_size_t(0)
+    _check(_lib.ssd_scan_fwd_workspace_size(ctypes.byref(dims), int(chunk), ctypes.byref(b)))
+    return int(b.value)
+
+
+def scan_variant(dims: SSDDims, chunk: int) -> str:
+    return _lib.ssd_scan_fwd_variant(ctypes.byref(dims), int(chunk)).decode()
+
+
+def last_launch_count() -> int:
+    return int(_lib.ssd_last_launch_count())
+
+
+def profile_enable(on: bool = True) -> None:
+    """Start (and reset) or stop per-kernel CUDA-event timing inside the library."""
+    _lib.ssd_profile_enable(1 if on else 0)
+
+
+def profile_read() -> dict:
+    """{kernel name: (launches, total device ms)} since enable / the last read."""
+    buf = (SSDKernelTime * 32)()
+    dropped = ctypes.c_int(0)
+    n = _lib.ssd_profile_read(buf, 32, ctypes.byref(dropped))
+    if n < 0:
+        raise SSDError(SSD_ERR_CUDA, _lib.ssd_last_error().decode())
+    out = {buf[i].name.decode(): (int(buf[i].launches), float(buf[i].total_ms)) for i in range(min(n, 32))}
+    if dropped.value:
+        out["_dropped"] = (int(dropped.value), 0.0)
+    return out
+
+
+def device_status(device=None) -> None:
+    """Wait for the current stream and raise if a kernel latched an error."""
+    _check(_lib.ssd_get_device_status(_stream(device)))
+
+
+def scan_fwd(x, dt_raw, dt_bias, A, B, C, D, init_state=None, cu_seqlens=None, chunk=128,
+             y=None, final_state=None, workspace=None, batch=None):
+    """Chunked SSD prefill.
+
+    Dense: x [batch, L, H, P], dt_raw [batch, L, H], B/C [batch, L, G, N].
+    Packed varlen (cu_seqlens int32 [nseq+1] on the device): x [T, H, P],
+    dt_raw [T, H], B/C [T, G, N].
+    Returns (y, final_state); final_state [nseq, H, P, N] float32.
+    """
+    dev = x.device
+    varlen = cu_seqlens is not None
+    if varlen:
+        T, H, P = x.shape
+        nseq = cu_seqlens.numel() - 1
+        tok = (T,)
+    else:
+        if x.dim() != 4:
+            raise ValueError("dense x must be [batch, L, H, P]")
+        bsz, L, H, P = x.shape
+        nseq = bsz
+        tok = (bsz, L)
+    G, N = B.shape[-2], B.shape[-1]
+    dt = x.dtype
+    _need(x, "x", tok + (H, P), dt, dev)
+    _need(dt_raw, "dt_raw", tok + (H,), torch.float32, dev)
+    _need(B, "B", tok + (G, N), dt, dev)
+    _need(C, "C", tok + (G, N), dt, dev)
+    for name, v in (("dt_bias", dt_bias), ("A", A), ("D", D)):
+        _need(v, name, (H,), torch.float32, dev)
+    if init_state is not None:
+        _need(init_state, "init_state", (nseq, H, P, N), torch.float32, dev)
+    if varlen:
+        _need(cu_seqlens, "cu_seqlens", (nseq + 1,), torch.int32, dev)
+    if y is None:
+        y = torch.empty_like(x)
+    _need(y, "y", tok + (H, P), dt, dev)
+    if final_state is None:
+        final_state = torch.empty(nseq, H, P, N, dtype=torch.float32, device=dev)
+    _need(final_state, "final_state", (nseq, H, P, N), torch.float32, dev)
+    if varlen:
+        dims = make_dims(x.shape[0], H, P, G, N, _dtype_code(x), nseq=nseq, workspace=workspace)
+    else:
+        dims = make_dims(bsz * L, H, P, G, N, _dtype_code(x), batch=bsz, seqlen=L, workspace=workspace)
+    with torch.cuda.device(dev):
+        _check(_lib.ssd_scan_fwd(_ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C),
+                                 _ptr(D), _ptr(init_state), _ptr(cu_seqlens), _ptr(y),
+                                 _ptr(final_state), ctypes.byref(dims), int(chunk), _stream(dev)))
+    return y, final_state
+
+
+def state_update(state, x, dt_raw, dt_bias, A, B, C, D, y=None):
+    """One decode step in place on ``state`` [nseq,H,P,N] float32.
+    x [nseq,H,P], dt_raw [nseq,H], B/C [nseq,G,N]. Returns y [nseq,H,P]."""
+    dev = x.device
+    nseq, H, P = x.shape
+    G, N = B.shape[-2], B.shape[-1]
+    _need(state, "state", (nseq, H, P, N), torch.float32, dev)
+    _need(x, "x", (nseq, H, P), x.dtype, dev)
+    _need(dt_raw, "dt_raw", (nseq, H), torch.float32, dev)
+    _need(B, "B", (nseq, G, N), x.dtype, dev)
+    _need(C, "C", (nseq, G, N), x.dtype, dev)
+    for name, v in (("dt_bias", dt_bias), ("A", A), ("D", D)):
+        _need(v, name, (H,), torch.float32, dev)
+    if y is None:
+        y = torch.empty_like(x)
+    _need(y, "y", (nseq, H, P), x.dtype, dev)
+    dims = make_dims(nseq, H, P, G, N, _dtype_code(x), batch=nseq, seqlen=1)
+    with torch.cuda.device(dev):
+        _check(_lib.ssd_state_update(_ptr(state), _ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A),
+                                     _ptr(B), _ptr(C), _ptr(D), _ptr(y), ctypes.byref(dims),
+                                     _stream(dev)))
+    return y

@@ -1,0 +1,96 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point the
+header declares, and rejects unsupported geometry on the host (fail closed)
+before any CUDA work."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for f in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if f.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", f)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(ssd_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("ssd_scan_fwd", "ssd_state_update", "ssd_scan_fwd_workspace_size",
+              "ssd_get_device_status", "ssd_last_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(ssd):
+    lib = ctypes.CDLL(ssd.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def _dims(ssd, **kw):
+    base = dict(T=256, H=8, P=64, G=2, N=128, dtype_code=ssd.SSD_DTYPE_BF16, batch=1, seqlen=256)
+    base.update(kw)
+    return ssd.make_dims(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(H=6, G=4), "UNSUPPORTED"),        # H % G != 0
+    (dict(P=48), "UNSUPPORTED"),
+    (dict(P=256), "UNSUPPORTED"),
+    (dict(N=8), "UNSUPPORTED"),
+    (dict(N=96), "UNSUPPORTED"),
+    (dict(H=0), "INVALID_ARG"),
+    (dict(batch=-1), "INVALID_ARG"),
+])
+def test_bad_geometry_fails_closed(ssd, kw, status):
+    d = _dims(ssd, **kw)
+    if "batch" not in kw:         # the size query also accepts the packed reading of dims
+        with pytest.raises(ssd.SSDError, match=status):
+            ssd.workspace_size(d, 128)
+    rc = ssd._lib.ssd_scan_fwd(None, None, None, None, None, None, None, None, None, None, None,
+                               ctypes.byref(d), 128, None)
+    assert rc == getattr(ssd, "SSD_ERR_" + status)
+    assert ssd._lib.ssd_last_error().decode()
+    if "batch" not in kw:
+        assert ssd.scan_variant(d, 128) == ""
+
+
+@pytest.mark.parametrize("chunk", [0, 32, 100, 512])
+def test_bad_chunk_fails_closed(ssd, chunk):
+    with pytest.raises(ssd.SSDError, match="UNSUPPORTED"):
+        ssd.workspace_size(_dims(ssd), chunk)
+
+
+def test_null_and_misaligned_pointers_rejected_on_host(ssd):
+    d = _dims(ssd)
+    p = 1 << 20                       # never dereferenced: validation stops first
+    rc = ssd._lib.ssd_scan_fwd(p, p, p, p, p, p, p, None, None, None, None, ctypes.byref(d), 128, None)
+    assert rc == ssd.SSD_ERR_INVALID_ARG          # y is NULL
+    rc = ssd._lib.ssd_scan_fwd(p + 2, p, p, p, p, p, p, None, None, p, None, ctypes.byref(d), 128, None)
+    assert rc == ssd.SSD_ERR_INVALID_ARG          # x misaligned
+    d1 = _dims(ssd, seqlen=2)
+    rc = ssd._lib.ssd_state_update(p, p, p, p, p, p, p, p, p, ctypes.byref(d1), None)
+    assert rc == ssd.SSD_ERR_INVALID_ARG          # decode needs seqlen == 1
+    too_small = _dims(ssd)
+    too_small.workspace, too_small.workspace_bytes = p, 16
+    rc = ssd._lib.ssd_scan_fwd(p, p, p, p, p, p, p, None, None, p, None, ctypes.byref(too_small), 128, None)
+    assert rc == ssd.SSD_ERR_INVALID_ARG          # workspace too small
+
+
+def test_workspace_size_grows_with_tokens(ssd):
+    a = ssd.workspace_size(_dims(ssd, T=256, seqlen=256), 128)
+    b = ssd.workspace_size(_dims(ssd, T=4096, seqlen=4096), 128)
+    assert 0 < a < b
+    packed = ssd.make_dims(1000, 8, 64, 2, 128, ssd.SSD_DTYPE_BF16, nseq=7)
+    assert ssd.workspace_size(packed, 64) > 0
+
+
+def test_variant_names(ssd):
+    assert ssd.scan_variant(_dims(ssd), 128) in ("tc", "simt")
+    assert ssd.scan_variant(_dims(ssd, dtype_code=ssd.SSD_DTYPE_F32, P=16, N=16, H=4, G=1), 64) == "simt"
