@@ -102,7 +102,7 @@ def path_flops(w: W.Workload) -> int:
     return w.total_tokens * H * per
 
 
-def kernel_bytes(name: str, w: W.Workload, nchunks: int) -> int:
+def kernel_bytes(name: str, w: W.Workload, nchunks: int, variant: str = "simt", nsegs: int = 0) -> int:
     """Algorithmic bytes one launch of each kernel must move for the prefill workload
     (inputs read once, outputs written once, intermediates of the pipeline counted
     where the kernel reads or writes them)."""
@@ -113,6 +113,15 @@ def kernel_bytes(name: str, w: W.Workload, nchunks: int) -> int:
     dtq = nchunks * H * Q * 4
     st = nchunks * H * P * N * 4
     fin = w.nseq * H * P * N * 4
+    if variant == "tc":
+        sst = nsegs * H * P * N * 4           # segment states (fp32)
+        dtr = T * H * 4
+        return {
+            "ssd_chunk_table": nsegs * 16,
+            "ssd_chunk_state": x + bc + dtr + sst + nsegs * H * 4,
+            "ssd_state_passing": 2 * sst + fin + nsegs * H * 4,
+            "ssd_chunk_scan": 2 * x + 2 * bc + dtr + sst,
+        }.get(name, 0)
     return {
         "ssd_chunk_table": nchunks * 16,
         "ssd_chunk_cumsum": T * H * 4 + 2 * dtq,
@@ -262,6 +271,7 @@ def bench_ours(args, rank, world, local_rank):
                          batch=w.nseq, seqlen=L)
     ws = torch.empty(ssd.workspace_size(dims, w.chunk), dtype=torch.uint8, device=dev)
     variant = ssd.scan_variant(dims, w.chunk)
+    seg_tokens = ssd.segment_tokens(dims, w.chunk)
 
     def step():
         ssd.scan_fwd(x, dtr, inp["dt_bias"], inp["A"], Bm, Cm, inp["D"], init_state=inp["init_state"],
@@ -298,9 +308,10 @@ def bench_ours(args, rank, world, local_rank):
 
     # Dominant kernel roofline (per-launch device time from events inside the timed region).
     nchunks = w.nseq * math.ceil(L / w.chunk)
+    nsegs = w.nseq * math.ceil(L / seg_tokens) if seg_tokens else 0
     dom = max((k for k in kprof if not k.startswith("_")), key=lambda k: kprof[k][1])
     n_l, t_l = kprof[dom]
-    kb = kernel_bytes(dom, w, nchunks)
+    kb = kernel_bytes(dom, w, nchunks, variant, nsegs)
     achieved = kb / (t_l / n_l / 1e3) / 1e9
     roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": hbm,
                 "peak_source": peak_src, "unit": "GB/s", "frac": round(achieved / hbm, 4),
@@ -314,8 +325,12 @@ def bench_ours(args, rank, world, local_rank):
                  "bound": "hbm" if t_bw >= t_tc else "tensor",
                  "frac": round(max(t_bw, t_tc) * 1e3 / ms_step, 4),
                  "frac_nominal_8tbs": round(pb / 8e12 * 1e3 / ms_step, 4)}
-    kernels = {k: {"launches": v[0], "ms_per_launch": round(v[1] / max(1, v[0]), 4)}
-               for k, v in kprof.items()}
+    kernels = {}
+    for k, v in kprof.items():
+        kms = v[1] / max(1, v[0])
+        kbk = kernel_bytes(k, w, nchunks, variant, nsegs)
+        kernels[k] = {"launches": v[0], "ms_per_launch": round(kms, 4),
+                      "gbs": round(kbk / (kms / 1e3) / 1e9, 1) if kms > 0 and kbk else None}
 
     # ---- end to end through the public call with host buffers
     host = {k: (None if v is None else v.cpu().pin_memory()) for k, v in inp.items()
@@ -363,7 +378,7 @@ def bench_ours(args, rank, world, local_rank):
                    "headdim": w.headdim, "ngroups": w.ngroups, "dstate": w.dstate, "chunk": w.chunk,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "inputs larger than L2 (%.2f GB per step vs 126 MB L2), no flush" % (pb / 1e9),
-                   "variant": variant},
+                   "variant": variant, "segment_tokens": seg_tokens},
         "roofline": roofline, "path_roofline": path_roof, "kernels": kernels,
         "clocks": clk, "e2e": e2e, "gpu_launches": launches_per_call * args.steps,
         "decode": decode,
@@ -460,6 +475,41 @@ def bench_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def ncu_case(args):
+    """Small fixed workloads for ncu captures (no timing, no JSON): `decode` runs
+    W + K decode steps of 256 sequences on a random 512 MiB FP32 state; `prefill`
+    runs W + K prefill calls of the long-context workload."""
+    from mamba_ssd_state_02_b200 import build
+    build.build()
+    from mamba_ssd_state_02_b200 import ssd
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    if args.ncu_case == "decode":
+        w = W.config(DECODE_CONFIG)
+        nseq, H, P, G, N = w.nseq, w.nheads, w.headdim, w.ngroups, w.dstate
+        par = W.make_params(w, device=dev)
+        state = (W.normal(w.seed, W.STREAM["init_state"], nseq * H * P * N, 0, dev) * 0.1).float()
+        state = state.view(nseq, H, P, N)
+        rows = torch.arange(nseq, device=dev, dtype=torch.int64)
+        tok = W.make_tokens(w, 0, 0, rows=rows)
+        y = torch.empty(nseq, H, P, dtype=w.dtype, device=dev)
+        for _ in range(args.warmup + args.steps):
+            ssd.state_update(state, tok["x"], tok["dt_raw"], par["dt_bias"], par["A"], tok["B"], tok["C"],
+                             par["D"], y=y)
+    else:
+        w = W.config(PREFILL_CONFIG)
+        inp = W.make_all(w, device=dev)
+        L = w.seqlens[0]
+        r4 = lambda t: t.view(w.nseq, L, *t.shape[1:])
+        y = torch.empty_like(r4(inp["x"]))
+        for _ in range(args.warmup + args.steps):
+            ssd.scan_fwd(r4(inp["x"]), r4(inp["dt_raw"]), inp["dt_bias"], inp["A"], r4(inp["B"]),
+                         r4(inp["C"]), inp["D"], chunk=w.chunk, y=y)
+    ssd.device_status()
+    torch.cuda.synchronize(dev)
+    print(f"ncu case {args.ncu_case}: {args.warmup + args.steps} calls ok", flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -467,7 +517,12 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ncu-case", choices=["decode", "prefill"], default=None,
+                    help="run a small fixed workload for an ncu capture instead of the benchmark")
     args = ap.parse_args(argv)
+    if args.ncu_case:
+        ncu_case(args)
+        return
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     rank, world, local_rank = dist_env()

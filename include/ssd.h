@@ -147,6 +147,13 @@ const char* ssd_last_error(void);
  */
 const char* ssd_scan_fwd_variant(const ssd_dims* dims, int chunk);
 
+/*
+ * Tokens per segment of the tensor-core pipeline for these dims (the unit whose
+ * state is materialised between its kernels), or 0 for the CUDA-core pipeline or
+ * rejected dims.
+ */
+int ssd_scan_fwd_segment_tokens(const ssd_dims* dims, int chunk);
+
 /* Number of kernels the last successful call on this host thread enqueued. */
 int ssd_last_launch_count(void);
 
@@ -165,6 +172,16 @@ typedef struct {
 } ssd_kernel_time;
 
 void ssd_profile_enable(int on);
+
+/*
+ * Diagnostic for the tensor-core path's shared-memory operand formats: multiplies two
+ * 128x128 row-major bf16 device matrices X1, X2 four ways on the tcgen05 tensor cores
+ * (each with a different pairing of TMA-written / thread-written and K-major /
+ * MN-major operands) and writes out[4][128][128] float32:
+ *   out[0] = X1 X2^T, out[1] = out[3] = X1 X2[:, :64], out[2] = X1^T X2[:, :64]
+ * (columns >= 64 of out[1..3] are zero). Enqueued on `stream`; no workspace.
+ */
+ssd_status ssd_selftest_umma(const void* X1, const void* X2, float* out, ssd_stream_t stream);
 /* Fills up to `max` entries, returns how many kernel names had launches, or -1 if
  * waiting on an event failed. *dropped (nullable) receives the unrecorded count. */
 int ssd_profile_read(ssd_kernel_time* out, int max, int* dropped);

@@ -63,6 +63,11 @@ struct Plan {
     // workspace byte offsets
     size_t off_table = 0, off_first = 0, off_count = 0, off_dt = 0, off_acum = 0, off_states = 0;
     size_t bytes = 0;
+    // tensor-core pipeline (tc): segment length (tokens), segment slots, state slots
+    bool tc = false;
+    int Ls = 0;
+    int64_t max_segs = 0;
+    size_t off_seg_acum = 0;
 };
 
 }  // namespace ssd

@@ -11,10 +11,16 @@
 #include <string>
 #include <vector>
 
+#include <cudaTypedefs.h>
+
+#include <cstdlib>
+
 #include "ssd.h"
 #include "ssd_common.cuh"
 #include "ssd_decode.cuh"
 #include "ssd_scan_simt.cuh"
+#include "ssd_scan_tc.cuh"
+#include "ssd_tc_selftest.cuh"
 
 namespace ssd {
 namespace {
@@ -92,6 +98,37 @@ struct StageScope {
     }
 };
 
+// ---------------------------------------------------------------------------------
+// TMA descriptors (driver entry point, resolved once).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }();
+    return fn;
+}
+
+// 3-D bf16 tensor map: dims {d0 (contiguous), d1, d2}, byte strides s1, s2, box
+// {64, 1, 128} (or {64, 128, 1} for 2-D data), 128-byte swizzle, zero fill.
+bool make_map3(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+               uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {s1, s2};
+    cuuint32_t box[3] = {b0, b1, b2};
+    cuuint32_t es[3] = {1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 bool pow2_in(int v, int lo, int hi) { return v >= lo && v <= hi && (v & (v - 1)) == 0; }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -143,6 +180,28 @@ ssd_status make_plan(const ssd_dims* d, int chunk, bool varlen, Plan* pl) {
         return fail(SSD_ERR_UNSUPPORTED, "more than 2^31-1 tokens in one call");
     if (p.T * (int64_t)p.H * p.P >= (int64_t)1 << 40)
         return fail(SSD_ERR_UNSUPPORTED, "x has more than 2^40 elements");
+    // Tensor-core pipeline: bf16, headdim 64, dstate 128, heads per group a multiple of 4.
+    p.tc = p.bf16 && p.P == tc::kP && p.N == tc::kN && (p.H / p.G) % tc::kHeads == 0;
+    auto segs_for = [&](int64_t Ls) -> int64_t {
+        return varlen ? p.T / Ls + p.nseq : (int64_t)p.nseq * ((p.seqlen + Ls - 1) / Ls);
+    };
+    if (p.tc) {
+        // Segment length: the longest of 2048/1024/512/256 tokens that still gives at least
+        // two work units (segment x 4 heads) per SM of a 148-SM B200.
+        int Ls = 256;
+        for (int cand : {2048, 1024, 512}) {
+            if (segs_for(cand) * (p.H / tc::kHeads) >= 2 * 148) {
+                Ls = cand;
+                break;
+            }
+        }
+        if (const char* e = getenv("SSD_SEGMENT_TOKENS")) {
+            const int v = atoi(e);
+            if (v >= tc::kTile && v % tc::kTile == 0 && v <= (1 << 20)) Ls = v;
+        }
+        p.Ls = Ls;
+        p.max_segs = segs_for(Ls);
+    }
     // Workspace carving (256-byte aligned pieces).
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -150,13 +209,22 @@ ssd_status make_plan(const ssd_dims* d, int chunk, bool varlen, Plan* pl) {
         off = align_up(off + bytes, 256);
         return o;
     };
-    const size_t mc = (size_t)p.max_chunks;
-    p.off_table = take(sizeof(ChunkEntry) * (mc > 0 ? mc : 1));
-    p.off_first = take(sizeof(int32_t) * ((size_t)p.nseq + 1));
-    p.off_count = take(sizeof(int32_t));
-    p.off_dt = take(sizeof(float) * mc * p.H * p.Q);
-    p.off_acum = take(sizeof(float) * mc * p.H * p.Q);
-    p.off_states = take(sizeof(float) * mc * p.H * p.P * p.N);
+    if (p.tc) {
+        const size_t ms = (size_t)p.max_segs;
+        p.off_table = take(sizeof(ChunkEntry) * (ms > 0 ? ms : 1));
+        p.off_first = take(sizeof(int32_t) * ((size_t)p.nseq + 1));
+        p.off_count = take(sizeof(int32_t));
+        p.off_states = take(sizeof(float) * ms * p.H * p.P * p.N);
+        p.off_seg_acum = take(sizeof(float) * ms * p.H);
+    } else {
+        const size_t mc = (size_t)p.max_chunks;
+        p.off_table = take(sizeof(ChunkEntry) * (mc > 0 ? mc : 1));
+        p.off_first = take(sizeof(int32_t) * ((size_t)p.nseq + 1));
+        p.off_count = take(sizeof(int32_t));
+        p.off_dt = take(sizeof(float) * mc * p.H * p.Q);
+        p.off_acum = take(sizeof(float) * mc * p.H * p.Q);
+        p.off_states = take(sizeof(float) * mc * p.H * p.P * p.N);
+    }
     p.bytes = off;
     *pl = p;
     return SSD_OK;
@@ -214,6 +282,66 @@ ssd_status launch_simt(const Plan& pl, char* ws, const T* x, const float* dt_raw
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch (simt scan)");
+    t_launches = n;
+    return SSD_OK;
+}
+
+// ---------------------------------------------------------------------------------
+// Tensor-core pipeline launch (bf16, P = 64, N = 128).
+ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_raw, const float* dt_bias,
+                     const float* A, const void* B, const void* C, const float* D, const float* init,
+                     const int32_t* cu, void* y, float* fin, cudaStream_t st) {
+    auto* table = reinterpret_cast<ChunkEntry*>(ws + pl.off_table);
+    auto* first = reinterpret_cast<int32_t*>(ws + pl.off_first);
+    auto* count = reinterpret_cast<int32_t*>(ws + pl.off_count);
+    auto* seg_state = reinterpret_cast<float*>(ws + pl.off_states);
+    auto* seg_acum = reinterpret_cast<float*>(ws + pl.off_seg_acum);
+    const int H = pl.H, G = pl.G;
+    int n = 0;
+    {
+        StageScope sc(ST_TABLE, st);
+        k_chunk_table<<<1, kTableThreads, 0, st>>>(cu, pl.nseq, pl.T, pl.seqlen, pl.Ls, table, first, count);
+    }
+    ++n;
+    if (pl.max_segs > 0 && pl.T > 0) {
+        CUtensorMap mx, mb, mc;
+        const uint64_t T = (uint64_t)pl.T;
+        if (!make_map3(&mx, x, tc::kP, H, T, (uint64_t)tc::kP * 2, (uint64_t)H * tc::kP * 2, 64, 1, tc::kTile) ||
+            !make_map3(&mb, B, tc::kN, G, T, (uint64_t)tc::kN * 2, (uint64_t)G * tc::kN * 2, 64, 1, tc::kTile) ||
+            !make_map3(&mc, C, tc::kN, G, T, (uint64_t)tc::kN * 2, (uint64_t)G * tc::kN * 2, 64, 1, tc::kTile))
+            return fail(SSD_ERR_CUDA, "cuTensorMapEncodeTiled failed (x/B/C tensor maps)");
+        cudaError_t e = cudaFuncSetAttribute(tc::k_tc_segment_state, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             tc::kSmemA);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(tc::k_tc_chunk_scan, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::kSmemB);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(tc kernels)");
+        const dim3 grid((unsigned)pl.max_segs, H / tc::kHeads);
+        {
+            StageScope sc(ST_CHUNK_STATE, st);
+            tc::k_tc_segment_state<<<grid, 128, tc::kSmemA, st>>>(mx, mb, dt_raw, dt_bias, A, table, count, H, G,
+                                                                  seg_state, seg_acum);
+        }
+        ++n;
+        {
+            StageScope sc(ST_STATE_PASSING, st);
+            tc::k_tc_segment_passing<<<dim3(pl.nseq, H, (tc::kP * tc::kN) / 256), 256, 0, st>>>(
+                seg_state, seg_acum, first, init, fin, H);
+        }
+        ++n;
+        {
+            StageScope sc(ST_CHUNK_SCAN, st);
+            tc::k_tc_chunk_scan<<<grid, 128, tc::kSmemB, st>>>(mx, mb, mc, dt_raw, dt_bias, A, D, table, count, H,
+                                                               G, seg_state, (__nv_bfloat16*)y);
+        }
+        ++n;
+    } else {
+        StageScope sc(ST_STATE_PASSING, st);
+        tc::k_tc_segment_passing<<<dim3(pl.nseq, H, (tc::kP * tc::kN) / 256), 256, 0, st>>>(
+            seg_state, seg_acum, first, init, fin, H);
+        ++n;
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch (tc scan)");
     t_launches = n;
     return SSD_OK;
 }
@@ -328,7 +456,9 @@ ssd_status ssd_scan_fwd(const void* x, const float* dt_raw, const float* dt_bias
         if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(workspace)");
         owned = true;
     }
-    if (pl.bf16)
+    if (pl.tc)
+        s = launch_tc(pl, ws, x, dt_raw, dt_bias, A, B, C, D, init_state, cu_seqlens, y, final_state, st);
+    else if (pl.bf16)
         s = dispatch_Q<__nv_bfloat16>(pl, ws, x, dt_raw, dt_bias, A, B, C, D, init_state, cu_seqlens, y,
                                       final_state, st);
     else
@@ -401,10 +531,36 @@ const char* ssd_last_error(void) { return t_last_error.c_str(); }
 const char* ssd_scan_fwd_variant(const ssd_dims* dims, int chunk) {
     Plan pl;
     if (make_plan(dims, chunk, false, &pl) != SSD_OK) return "";
-    return "simt";
+    return pl.tc ? "tc" : "simt";
 }
 
 int ssd_last_launch_count(void) { return t_launches; }
+
+int ssd_scan_fwd_segment_tokens(const ssd_dims* dims, int chunk) {
+    Plan pl;
+    if (make_plan(dims, chunk, dims && dims->batch == 0 && dims->nseq > 0, &pl) != SSD_OK) return 0;
+    return pl.tc ? pl.Ls : 0;
+}
+
+ssd_status ssd_selftest_umma(const void* X1, const void* X2, float* out, ssd_stream_t stream) {
+    if (!X1 || !X2 || !out) return fail(SSD_ERR_INVALID_ARG, "selftest pointers must be non-NULL");
+    if (!aligned(X1, 16) || !aligned(X2, 16) || !aligned(out, 16))
+        return fail(SSD_ERR_INVALID_ARG, "selftest pointers must be 16-byte aligned");
+    CUtensorMap m1, m2;
+    if (!make_map3(&m1, X1, 128, 128, 1, 256, 256 * 128, 64, 128, 1) ||
+        !make_map3(&m2, X2, 128, 128, 1, 256, 256 * 128, 64, 128, 1))
+        return fail(SSD_ERR_CUDA, "cuTensorMapEncodeTiled failed (selftest)");
+    cudaError_t e = cudaFuncSetAttribute(tc::k_umma_selftest, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         tc::kSelftestSmem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(selftest)");
+    tc::k_umma_selftest<<<1, 128, tc::kSelftestSmem, reinterpret_cast<cudaStream_t>(stream)>>>(
+        m1, m2, (const __nv_bfloat16*)X1, (const __nv_bfloat16*)X2, out);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch (selftest)");
+    t_launches = 1;
+    t_last_error.clear();
+    return SSD_OK;
+}
 
 void ssd_profile_enable(int on) {
     std::lock_guard<std::mutex> lk(g_prof.mu);

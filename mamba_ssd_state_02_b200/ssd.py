@@ -66,6 +66,8 @@ _lib.ssd_last_error.argtypes = []
 _lib.ssd_last_error.restype = ctypes.c_char_p
 _lib.ssd_scan_fwd_variant.argtypes = [ctypes.POINTER(SSDDims), ctypes.c_int]
 _lib.ssd_scan_fwd_variant.restype = ctypes.c_char_p
+_lib.ssd_scan_fwd_segment_tokens.argtypes = [ctypes.POINTER(SSDDims), ctypes.c_int]
+_lib.ssd_scan_fwd_segment_tokens.restype = ctypes.c_int
 _lib.ssd_last_launch_count.argtypes = []
 _lib.ssd_last_launch_count.restype = ctypes.c_int
 
@@ -75,6 +77,8 @@ class SSDKernelTime(ctypes.Structure):
     _fields_ = [("name", ctypes.c_char_p), ("launches", ctypes.c_int), ("total_ms", ctypes.c_double)]
 
 
+_lib.ssd_selftest_umma.argtypes = [_p, _p, _p, _p]
+_lib.ssd_selftest_umma.restype = ctypes.c_int
 _lib.ssd_profile_enable.argtypes = [ctypes.c_int]
 _lib.ssd_profile_enable.restype = None
 _lib.ssd_profile_read.argtypes = [ctypes.POINTER(SSDKernelTime), ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
@@ -143,6 +147,10 @@ def scan_variant(dims: SSDDims, chunk: int) -> str:
     return _lib.ssd_scan_fwd_variant(ctypes.byref(dims), int(chunk)).decode()
 
 
+def segment_tokens(dims: SSDDims, chunk: int) -> int:
+    return int(_lib.ssd_scan_fwd_segment_tokens(ctypes.byref(dims), int(chunk)))
+
+
 def last_launch_count() -> int:
     return int(_lib.ssd_last_launch_count())
 
@@ -162,6 +170,18 @@ def profile_read() -> dict:
     out = {buf[i].name.decode(): (int(buf[i].launches), float(buf[i].total_ms)) for i in range(min(n, 32))}
     if dropped.value:
         out["_dropped"] = (int(dropped.value), 0.0)
+    return out
+
+
+def selftest_umma(X1: torch.Tensor, X2: torch.Tensor) -> torch.Tensor:
+    """Run the tensor-core operand-format diagnostic on two [128,128] bf16 matrices;
+    returns out [4,128,128] float32 (see ssd_selftest_umma in include/ssd.h)."""
+    dev = X1.device
+    for name, t in (("X1", X1), ("X2", X2)):
+        _need(t, name, (128, 128), torch.bfloat16, dev)
+    out = torch.empty(4, 128, 128, dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _check(_lib.ssd_selftest_umma(_ptr(X1), _ptr(X2), _ptr(out), _stream(dev)))
     return out
 
 
