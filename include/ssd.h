@@ -174,12 +174,13 @@ typedef struct {
 void ssd_profile_enable(int on);
 
 /*
- * Diagnostic for the tensor-core path's shared-memory operand formats: multiplies two
- * 128x128 row-major bf16 device matrices X1, X2 four ways on the tcgen05 tensor cores
- * (each with a different pairing of TMA-written / thread-written and K-major /
- * MN-major operands) and writes out[4][128][128] float32:
- *   out[0] = X1 X2^T, out[1] = out[3] = X1 X2[:, :64], out[2] = X1^T X2[:, :64]
- * (columns >= 64 of out[1..3] are zero). Enqueued on `stream`; no workspace.
+ * Diagnostic for the tensor-core path's operand formats: multiplies two 128x128
+ * row-major bf16 device matrices X1, X2 five ways on the tcgen05 tensor cores (each
+ * with a different pairing of TMA-written / thread-written, K-major / MN-major shared
+ * memory operands, or an A operand held in tensor memory) and writes
+ * out[5][128][128] float32:
+ *   out[0] = X1 X2^T, out[1] = out[3] = out[4] = X1 X2[:, :64], out[2] = X1^T X2[:, :64]
+ * (columns >= 64 of out[1..4] are zero). Enqueued on `stream`; no workspace.
  */
 ssd_status ssd_selftest_umma(const void* X1, const void* X2, float* out, ssd_stream_t stream);
 /* Fills up to `max` entries, returns how many kernel names had launches, or -1 if

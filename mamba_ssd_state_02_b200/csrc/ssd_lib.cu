@@ -330,7 +330,8 @@ ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_ra
         ++n;
         {
             StageScope sc(ST_CHUNK_SCAN, st);
-            tc::k_tc_chunk_scan<<<grid, 128, tc::kSmemB, st>>>(mx, mb, mc, dt_raw, dt_bias, A, D, table, count, H,
+            const dim3 gridB((unsigned)pl.max_segs, H / tc::kHeadsB);
+            tc::k_tc_chunk_scan<<<gridB, tc::kThreadsB, tc::kSmemB, st>>>(mx, mb, mc, dt_raw, dt_bias, A, D, table, count, H,
                                                                G, seg_state, (__nv_bfloat16*)y);
         }
         ++n;

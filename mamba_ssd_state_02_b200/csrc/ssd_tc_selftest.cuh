@@ -6,7 +6,8 @@
 //   r1[t][p] = sum_k X1[t][k] X2[k][p]   A: thread K-major, B: TMA MN-major  (N=64)
 //   r2[m][p] = sum_k X1[k][m] X2[k][p]   A: TMA MN-major,   B: thread MN-major
 //   r3[t][p] = sum_k X1[t][k] X2[k][p]   A: TMA K-major,    B: thread MN-major
-// out is [4][128][128] fp32; columns >= 64 of r1..r3 are written as zero.
+//   r4[t][p] = sum_k X1[t][k] X2[k][p]   A: thread-written TMEM, B: TMA MN-major
+// out is [5][128][128] fp32; columns >= 64 of r1..r4 are written as zero.
 #pragma once
 
 #include "ssd_tc_ptx.cuh"
@@ -66,7 +67,19 @@ k_umma_selftest(const __grid_constant__ CUtensorMap map1, const __grid_constant_
             st_shared_v4(smem_u32(twb) + swz(r, c), v.x, v.y, v.z, v.w);
         }
     }
+    // A operand of r4 in TMEM: row r (lane r) = X1[r][:], bf16 pairs per column 320..383.
+    {
+        const int r = tid;
+        const uint32_t* src = reinterpret_cast<const uint32_t*>(X1 + r * 128);
+        for (int q = 0; q < 2; ++q) {
+            uint32_t v[32];
+            for (int j = 0; j < 32; ++j) v[j] = src[q * 32 + j];
+            tmem_st32(tmem_addr(tbase, warp * 32, 320 + q * 32), v);
+        }
+        tmem_wait_st();
+    }
     fence_proxy_async_smem();
+    tc_fence_before();
     bool ok = __syncthreads_and(mbar_wait(&bar_tma, 0));
 
     if (tid == 0 && ok) {
@@ -83,6 +96,9 @@ k_umma_selftest(const __grid_constant__ CUtensorMap map1, const __grid_constant_
         for (int k = 0; k < 8; ++k)
             umma_bf16(tbase + 256, desc_kmajor(a1, 128, k), desc_mnmajor(tb, k, 16384), idesc_bf16(128, 64, 0, 1),
                       k > 0);
+        for (int k = 0; k < 8; ++k)
+            umma_bf16_ts(tbase + 384, tbase + 320 + 8 * k, desc_mnmajor(a2, k, 16384), idesc_bf16(128, 64, 0, 1),
+                         k > 0);
         umma_commit(&bar_mma);
     }
     __syncwarp();
@@ -97,9 +113,10 @@ k_umma_selftest(const __grid_constant__ CUtensorMap map1, const __grid_constant_
         tmem_wait_ld();
         for (int j = 0; j < 32; ++j) out[(0 * 128 + row) * 128 + q * 32 + j] = ok ? __uint_as_float(r[j]) : 0.f;
     }
-    for (int m = 1; m < 4; ++m) {
+    for (int m = 1; m < 5; ++m) {
+        const uint32_t col = m < 4 ? 128 + (m - 1) * 64 : 384;
         for (int q = 0; q < 2; ++q) {
-            tmem_ld32(lane_base + 128 + (m - 1) * 64 + q * 32, r);
+            tmem_ld32(lane_base + col + q * 32, r);
             tmem_wait_ld();
             for (int j = 0; j < 32; ++j)
                 out[(m * 128 + row) * 128 + q * 32 + j] = ok ? __uint_as_float(r[j]) : 0.f;

@@ -175,11 +175,11 @@ def profile_read() -> dict:
 
 def selftest_umma(X1: torch.Tensor, X2: torch.Tensor) -> torch.Tensor:
     """Run the tensor-core operand-format diagnostic on two [128,128] bf16 matrices;
-    returns out [4,128,128] float32 (see ssd_selftest_umma in include/ssd.h)."""
+    returns out [5,128,128] float32 (see ssd_selftest_umma in include/ssd.h)."""
     dev = X1.device
     for name, t in (("X1", X1), ("X2", X2)):
         _need(t, name, (128, 128), torch.bfloat16, dev)
-    out = torch.empty(4, 128, 128, dtype=torch.float32, device=dev)
+    out = torch.empty(5, 128, 128, dtype=torch.float32, device=dev)
     with torch.cuda.device(dev):
         _check(_lib.ssd_selftest_umma(_ptr(X1), _ptr(X2), _ptr(out), _stream(dev)))
     return out

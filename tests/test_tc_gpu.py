@@ -22,7 +22,7 @@ def test_umma_operand_formats(ssd, cuda_dev):
     torch.cuda.synchronize()
     ssd.device_status()
     a, b = X1.double(), X2.double()
-    ref = [a @ b.T, a @ b[:, :64], a.T @ b[:, :64], a @ b[:, :64]]
+    ref = [a @ b.T, a @ b[:, :64], a.T @ b[:, :64], a @ b[:, :64], a @ b[:, :64]]
     got = out.cpu().double()
     for i, r in enumerate(ref):
         cols = r.shape[1]
