@@ -315,10 +315,10 @@ ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_ra
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(tc::k_tc_chunk_scan, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::kSmemB);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(tc kernels)");
-        const dim3 grid((unsigned)pl.max_segs, H / tc::kHeads);
         {
             StageScope sc(ST_CHUNK_STATE, st);
-            tc::k_tc_segment_state<<<grid, 128, tc::kSmemA, st>>>(mx, mb, dt_raw, dt_bias, A, table, count, H, G,
+            tc::k_tc_segment_state<<<(unsigned)(pl.max_segs * (H / tc::kHeads)), tc::kThreadsTc, tc::kSmemA,
+                                     st>>>(mx, mb, dt_raw, dt_bias, A, table, count, H, G,
                                                                   seg_state, seg_acum);
         }
         ++n;
@@ -330,8 +330,7 @@ ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_ra
         ++n;
         {
             StageScope sc(ST_CHUNK_SCAN, st);
-            const dim3 gridB((unsigned)pl.max_segs, H / tc::kHeadsB);
-            tc::k_tc_chunk_scan<<<gridB, tc::kThreadsB, tc::kSmemB, st>>>(mx, mb, mc, dt_raw, dt_bias, A, D, table, count, H,
+            tc::k_tc_chunk_scan<<<(unsigned)(pl.max_segs * (H / tc::kHeadsB)), tc::kThreadsTc, tc::kSmemB, st>>>(mx, mb, mc, dt_raw, dt_bias, A, D, table, count, H,
                                                                G, seg_state, (__nv_bfloat16*)y);
         }
         ++n;

@@ -78,131 +78,215 @@ __device__ __forceinline__ void tile_cumsum(const float* __restrict__ dt_raw, co
 }
 
 // ---------------------------------------------------------------------------------
-// Pass A: zero-start segment states S_seg (fp32, layout [seg][H][N][P]) and the
-// segment's total sum of dt*A (seg_acum[seg][H]).
-constexpr int kSmemA = 128 * 1024 + 1024;
+// Shared by both passes.
+constexpr int kRoleWarps = 2;                    // warp 0: TMA producer, warp 1: UMMA issuer
+constexpr int kComputeWarps = 16;                // four compute warpgroups (cw = 0..3)
+constexpr int kThreadsTc = 32 * (kRoleWarps + kComputeWarps);
 
-__global__ void __launch_bounds__(128, 1)
+__device__ __forceinline__ void compute_bar() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
+
+// Wait with a shared abort flag: once any wait has timed out, every later wait
+// returns at once, so all roles run to the end without blocking each other.
+__device__ __forceinline__ void wait_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort_flag) return;
+        if (clock64() - t0 > kWaitBudgetCycles) {
+            latch_error(SSD_ERR_TIMEOUT);
+            *abort_flag = 1;
+            return;
+        }
+    }
+}
+
+// Inclusive scan of `a` over the 128 rows of one compute warpgroup (rows r = 32*q +
+// lane); `part` holds the four per-warp totals of that warpgroup. Two compute_bar()s.
+__device__ __forceinline__ float wg_scan(float a, int q, int lane, float* part) {
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float v = __shfl_up_sync(0xffffffffu, a, off);
+        if (lane >= off) a += v;
+    }
+    if (lane == 31) part[q] = a;
+    compute_bar();
+    float pre = 0.f;
+    for (int w = 0; w < q; ++w) pre += part[w];
+    return a + pre;
+}
+
+// ---------------------------------------------------------------------------------
+// Pass A: zero-start segment states S_seg (fp32, layout [seg][H][N][P]) and the
+// segment's total sum of dt*A (seg_acum[seg][H]). One CTA per (segment, 4 heads);
+// compute warpgroup cw owns head cw for the decay weights and column quarter cw of
+// every w*X row. Tiles run from the segment end backwards so the decay to the end is
+// a running sum. Shared memory: two B stages, a four-slot X ring (one per head), two
+// w*X hi/lo buffer pairs. TMEM: S_seg of the 4 heads (64 columns each).
+constexpr int kSmemA = 192 * 1024 + 1024;
+
+__global__ void __launch_bounds__(kThreadsTc, 1)
 k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
                    const float* __restrict__ dt_raw, const float* __restrict__ dt_bias,
                    const float* __restrict__ A, const ChunkEntry* __restrict__ segs,
                    const int32_t* __restrict__ nsegs, int H, int G, float* __restrict__ seg_state,
                    float* __restrict__ seg_acum) {
-    const int sg = blockIdx.x;
+    const int nq = H / kHeads;
+    const int sg = blockIdx.x / nq;
     if (sg >= *nsegs) return;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sB = sm;                       // [2][128 s][64 n]
-    uint8_t* sX = sm + 32768;               // [4][128 s][64 p]
-    uint8_t* sHi = sm + 98304;              // [128 s][64 p]
-    uint8_t* sLo = sm + 114688;             // [128 s][64 p]
-    __shared__ float acs2[kHeads][kTile], dts[kHeads][kTile], wsum[4][kHeads];
-    __shared__ uint64_t bar_load, bar_mma;
+    uint8_t* sB = sm;                       // stage st at st*32768: [2][128 s][64 n]
+    uint8_t* sX = sm + 65536;               // slot hh at hh*16384: [128 s][64 p]
+    uint8_t* sWx = sm + 131072;             // buffer b at b*32768: hi [128 s][64 p], lo at +16384
+    __shared__ float wts[kHeads][kTile];
+    __shared__ float part[kHeads][4], tile_tot[kHeads];
+    __shared__ uint64_t full_b[2], empty_b[2], full_x[kHeads], empty_x[kHeads], ops_ready[2], mma_done[2];
     __shared__ uint32_t tmem_slot;
+    __shared__ int abort_flag;
 
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int h0 = blockIdx.y * kHeads, g = h0 / (H / G);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int h0 = (blockIdx.x % nq) * kHeads, g = h0 / (H / G);
     const ChunkEntry seg = segs[sg];
     const int ntiles = (seg.len + kTile - 1) / kTile;
 
     if (tid == 0) {
-        mbar_init(&bar_load, 1);
-        mbar_init(&bar_mma, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&full_b[i], 1);
+            mbar_init(&empty_b[i], 1);
+            mbar_init(&ops_ready[i], kComputeWarps);
+            mbar_init(&mma_done[i], 1);
+        }
+        for (int i = 0; i < kHeads; ++i) {
+            mbar_init(&full_x[i], 1);
+            mbar_init(&empty_x[i], kComputeWarps);
+        }
+        abort_flag = 0;
         fence_barrier_init();
         prefetch_tmap(&map_x);
         prefetch_tmap(&map_b);
     }
-    if (warp == 0) {
+    if (warp == 1) {
         tmem_alloc(&tmem_slot, 256);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tS = tmem_slot;            // S_seg for head hh at columns [64*hh, 64*hh + 64)
+    const uint32_t tS = tmem_slot;          // head hh at columns [64 hh, 64 hh + 64)
+    volatile int* abort_p = &abort_flag;
 
-    float suffix[kHeads] = {0.f, 0.f, 0.f, 0.f};   // log2-scaled sum of dt*A over later tiles
-    uint32_t ph_load = 0, ph_mma = 0;
-    bool ok = true, first_mma = true;
-    for (int it = ntiles - 1; it >= 0 && ok; --it) {
-        const int64_t t0 = seg.start + (int64_t)it * kTile;
-        const int tl = min(kTile, seg.len - it * kTile);
-        if (tid == 0) {
-            mbar_arrive_expect_tx(&bar_load, 32768 + kHeads * 16384);
-            tma_load_3d(sB, &map_b, &bar_load, 0, g, (int)t0);
-            tma_load_3d(sB + 16384, &map_b, &bar_load, 64, g, (int)t0);
-            for (int hh = 0; hh < kHeads; ++hh) tma_load_3d(sX + hh * 16384, &map_x, &bar_load, 0, h0 + hh, (int)t0);
-        }
-        tile_cumsum(dt_raw, dt_bias, A, H, h0, t0, tl, acs2, dts, wsum);
-        ok = __syncthreads_and(mbar_wait(&bar_load, ph_load));
-        ph_load ^= 1;
-        const int s = tid;
-        for (int hh = 0; hh < kHeads && ok; ++hh) {
-            // w_s = exp(sum of dt*A after s up to the segment end) * dt_s
-            const float w = exp2f(suffix[hh] + acs2[hh][kTile - 1] - acs2[hh][s]) * dts[hh][s];
-            const uint32_t xrow = smem_u32(sX + hh * 16384);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const uint4 v = ld_shared_v4(xrow + swz(s, c));
-                const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-                uint32_t hi[4], lo[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float2 f = bf16x2_to_f2(in[q]);
-                    const float p0 = f.x * w, p1 = f.y * w;
-                    const __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
-                    const float2 hf = __bfloat1622float2(hb);
-                    hi[q] = *reinterpret_cast<const uint32_t*>(&hb);
-                    lo[q] = pack_bf16(p0 - hf.x, p1 - hf.y);
+    if (warp == 0) {
+        if (lane == 0) {
+            for (int k = 0; k < ntiles; ++k) {            // k-th tile processed = tile ntiles-1-k
+                const int t0 = seg.start + (ntiles - 1 - k) * kTile, st = k & 1;
+                if (k >= 2) wait_abort(&empty_b[st], ((k - 2) >> 1) & 1, abort_p);
+                mbar_arrive_expect_tx(&full_b[st], 32768);
+                tma_load_3d(sB + st * 32768, &map_b, &full_b[st], 0, g, t0);
+                tma_load_3d(sB + st * 32768 + 16384, &map_b, &full_b[st], 64, g, t0);
+                for (int hh = 0; hh < kHeads; ++hh) {
+                    if (k >= 1) wait_abort(&empty_x[hh], (k - 1) & 1, abort_p);
+                    mbar_arrive_expect_tx(&full_x[hh], 16384);
+                    tma_load_3d(sX + hh * 16384, &map_x, &full_x[hh], 0, h0 + hh, t0);
                 }
-                st_shared_v4(smem_u32(sHi) + swz(s, c), hi[0], hi[1], hi[2], hi[3]);
-                st_shared_v4(smem_u32(sLo) + swz(s, c), lo[0], lo[1], lo[2], lo[3]);
             }
-            fence_proxy_async_smem();
-            __syncthreads();
-            if (tid == 0) {
-                tc_fence_after();
-                const uint32_t idesc = idesc_bf16(128, 64, 1, 1);
-                const uint32_t aB = smem_u32(sB), aHi = smem_u32(sHi), aLo = smem_u32(sLo);
-                const uint32_t d = tS + hh * 64;
-                for (int k = 0; k < 8; ++k)
-                    umma_bf16(d, desc_mnmajor(aB, k, 16384), desc_mnmajor(aHi, k, 16384), idesc,
-                              !(first_mma && k == 0));
-                for (int k = 0; k < 8; ++k)
-                    umma_bf16(d, desc_mnmajor(aB, k, 16384), desc_mnmajor(aLo, k, 16384), idesc, true);
-                umma_commit(&bar_mma);
-            }
-            __syncwarp();
-            ok = __syncthreads_and(mbar_wait(&bar_mma, ph_mma));
-            ph_mma ^= 1;
         }
-        first_mma = false;
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(128, 64, 1, 1);
+            for (int k = 0; k < ntiles; ++k) {
+                const int st = k & 1;
+                wait_abort(&full_b[st], (k >> 1) & 1, abort_p);
+                const uint32_t aB = smem_u32(sB + st * 32768);
+                for (int hh = 0; hh < kHeads; ++hh) {
+                    const int j = k * kHeads + hh, b = j & 1;
+                    wait_abort(&ops_ready[b], (j >> 1) & 1, abort_p);
+                    tc_fence_after();
+                    const uint32_t aHi = smem_u32(sWx + b * 32768), aLo = aHi + 16384;
+                    const uint32_t d = tS + hh * 64;
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_bf16(d, desc_mnmajor(aB, kk, 16384), desc_mnmajor(aHi, kk, 16384), idesc,
+                                  !(k == 0 && kk == 0));
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_bf16(d, desc_mnmajor(aB, kk, 16384), desc_mnmajor(aLo, kk, 16384), idesc, true);
+                    umma_commit(&mma_done[b]);
+                    if (hh == kHeads - 1) umma_commit(&empty_b[st]);
+                }
+            }
+        }
+    } else {
+        const int cw = (warp - kRoleWarps) >> 2, q = warp & 3, r = q * 32 + lane;
+        float suffix = 0.f;                 // log2-scaled sum of dt*A of head cw after this tile
+        for (int k = 0; k < ntiles; ++k) {
+            const int it = ntiles - 1 - k;
+            const int64_t t0 = seg.start + (int64_t)it * kTile;
+            const int tl = min(kTile, seg.len - it * kTile);
+            // decay-to-segment-end weights of head cw: w_s = exp(sum_{r>s} dt_r A) dt_s
+            {
+                const float Ah = A[h0 + cw];
+                if (r == 0 && k == 0 && (!(Ah <= 0.f) || isinf(Ah))) latch_error(SSD_ERR_INVALID_ARG);
+                const float dtv = r < tl ? softplus_f32(dt_raw[(t0 + r) * H + h0 + cw] + dt_bias[h0 + cw]) : 0.f;
+                compute_bar();              // previous tile's weights no longer read
+                const float incl = wg_scan(dtv * Ah, q, lane, part[cw]) * kLog2e;
+                if (r == kTile - 1) tile_tot[cw] = incl;
+                compute_bar();
+                const float tot = tile_tot[cw];
+                wts[cw][r] = exp2f(suffix + tot - incl) * dtv;
+                suffix += tot;
+                compute_bar();
+            }
+            for (int hh = 0; hh < kHeads; ++hh) {
+                const int j = k * kHeads + hh, b = j & 1;
+                if (j >= 2) wait_abort(&mma_done[b], ((j - 2) >> 1) & 1, abort_p);
+                wait_abort(&full_x[hh], k & 1, abort_p);
+                const float w = wts[hh][r];
+                const uint32_t xrow = smem_u32(sX + hh * 16384);
+                const uint32_t hi = smem_u32(sWx + b * 32768), lo = hi + 16384;
 #pragma unroll
-        for (int hh = 0; hh < kHeads; ++hh) suffix[hh] += acs2[hh][kTile - 1];
-        __syncthreads();
-    }
-
-    // Write S_seg: thread = TMEM lane = state row n; 64 fp32 columns p per head.
-    tc_fence_after();
-    const int n = tid;
-    for (int hh = 0; hh < kHeads; ++hh) {
-        float* dst = seg_state + (((int64_t)sg * H + h0 + hh) * kN + n) * kP;
-        for (int q = 0; q < 2; ++q) {
-            uint32_t r[32];
-            tmem_ld32(tmem_addr(tS, warp * 32, hh * 64 + q * 32), r);
+                for (int c = 2 * cw; c < 2 * cw + 2; ++c) {
+                    const uint4 v = ld_shared_v4(xrow + swz(r, c));
+                    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+                    uint32_t oh[4], ol[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = bf16x2_to_f2(in[e]);
+                        const float p0 = f.x * w, p1 = f.y * w;
+                        const __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
+                        const float2 hf = __bfloat1622float2(hb);
+                        oh[e] = *reinterpret_cast<const uint32_t*>(&hb);
+                        ol[e] = pack_bf16(p0 - hf.x, p1 - hf.y);
+                    }
+                    st_shared_v4(hi + swz(r, c), oh[0], oh[1], oh[2], oh[3]);
+                    st_shared_v4(lo + swz(r, c), ol[0], ol[1], ol[2], ol[3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&empty_x[hh]);
+                    mbar_arrive(&ops_ready[b]);
+                }
+            }
+        }
+        // Wait for the last UMMAs, then write S_seg of head cw: thread = state row n.
+        const int jl = ntiles * kHeads - 1;
+        wait_abort(&mma_done[jl & 1], (jl >> 1) & 1, abort_p);
+        if (ntiles * kHeads >= 2) wait_abort(&mma_done[(jl - 1) & 1], ((jl - 1) >> 1) & 1, abort_p);
+        tc_fence_after();
+        float* dst = seg_state + (((int64_t)sg * H + h0 + cw) * kN + r) * kP;
+        for (int half = 0; half < 2; ++half) {
+            uint32_t v[32];
+            tmem_ld32(tS + ((uint32_t)(q * 32) << 16) + cw * 64 + half * 32, v);
             tmem_wait_ld();
-            float4* d4 = reinterpret_cast<float4*>(dst + q * 32);
+            float4* d4 = reinterpret_cast<float4*>(dst + half * 32);
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                d4[j] = ok ? make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                         __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]))
-                           : make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int e = 0; e < 8; ++e)
+                d4[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                                    __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
         }
-        if (tid == 0) seg_acum[(int64_t)sg * H + h0 + hh] = ntiles > 0 ? suffix[hh] / kLog2e : 0.f;
+        if (r == 0) seg_acum[(int64_t)sg * H + h0 + cw] = suffix / kLog2e;
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tS, 256);
+    if (warp == 1) tmem_dealloc(tS, 256);
 }
 
 // ---------------------------------------------------------------------------------
@@ -242,61 +326,43 @@ k_tc_segment_passing(float* __restrict__ seg_state, const float* __restrict__ se
 }
 
 // ---------------------------------------------------------------------------------
-// Pass B: outputs y for one (segment, 4 heads), chunk by chunk.
+// Pass B: outputs y for one (segment, 2 heads), chunk by chunk.
 //
-// One CTA per (segment, 2 heads). Warp roles (320 threads): warp 0 issues the TMA
-// loads, warp 1 issues the UMMAs, warps 2..9 form two compute warpgroups (cw = 0, 1)
-// that split every row's columns in halves. Compute thread (cw, r) owns TMEM lane r = 32*(warp%4) + lane and holds
-// the FP32 running state h[head][n = r][p in its half] in registers.
-// Shared memory: two C/B stages (tile i+1 loads while tile i computes), a two-slot
-// ring of X tiles (one per head), and one w*X and one bf16 h operand tile.
-// TMEM: C B^T (128 cols), two M buffers (A operands, bf16 pairs, 64 cols each), and
-// the Y, Z, S accumulators (64 cols each). Per head the compute warps build M for
-// head hh while the UMMAs of head hh-1 run, then drain head hh-1 (y rows, state
-// update) and write the h / w*X operands of head hh.
-constexpr int kThreadsB = 320;
-constexpr int kHeadsB = 2;          // heads per pass-B CTA
+// Warp 0 issues the TMA loads, warp 1 the UMMAs; the four compute warpgroups
+// (cw = 0..3) split every row's 64 columns in quarters (and the 128 source columns
+// of M in 32-wide blocks). Compute thread (cw, r) owns TMEM lane r = 32*(warp%4) +
+// lane and holds the FP32 running state h[head][n = r][p in its quarter].
+// Shared memory: two C/B stages (tile i+1 loads while tile i computes), a two-slot X
+// ring (one per head), one w*X and one bf16 h operand tile. TMEM: C B^T (128 cols),
+// two M buffers (A operands, bf16 pairs, 64 cols each), Y, Z, S (64 cols each). Per
+// head the compute warps build M for head hh while the UMMAs of head hh-1 run, then
+// drain head hh-1 (y rows, state update) and write the operands of head hh.
+constexpr int kHeadsB = 2;
 constexpr int kSmemB = 192 * 1024 + 1024;
 
-__device__ __forceinline__ void compute_bar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
-
-// Wait with a shared abort flag: once any wait has timed out, every later wait
-// returns at once, so all roles run to the end without blocking each other.
-__device__ __forceinline__ void wait_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-    if (mbar_try_wait(bar, parity)) return;
-    const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
-        if (*abort_flag) return;
-        if (clock64() - t0 > kWaitBudgetCycles) {
-            latch_error(SSD_ERR_TIMEOUT);
-            *abort_flag = 1;
-            return;
-        }
-    }
-}
-
-__global__ void __launch_bounds__(kThreadsB, 1)
+__global__ void __launch_bounds__(kThreadsTc, 1)
 k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
                 const __grid_constant__ CUtensorMap map_c, const float* __restrict__ dt_raw,
                 const float* __restrict__ dt_bias, const float* __restrict__ A, const float* __restrict__ D,
                 const ChunkEntry* __restrict__ segs, const int32_t* __restrict__ nsegs, int H, int G,
                 const float* __restrict__ hin, __nv_bfloat16* __restrict__ y) {
-    const int sg = blockIdx.x;
+    const int nhp = H / kHeadsB;
+    const int sg = blockIdx.x / nhp;
     if (sg >= *nsegs) return;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sCB = sm;                      // stage st: C at st*65536 ([2][128 t][64 n]), B at +32768
-    uint8_t* sX = sm + 131072;              // slot j: [128 s][64 p] at j*16384
+    uint8_t* sX = sm + 131072;              // slot hh: [128 s][64 p] at hh*16384
     uint8_t* sW = sm + 163840;              // [128 s][64 p]  w * X
     uint8_t* sH = sm + 180224;              // [128 n][64 p]  bf16 h_in
     __shared__ float ac2[kHeadsB][kTile], dts[kHeadsB][kTile], uw[kHeadsB][kTile], ww[kHeadsB][kTile];
-    __shared__ float wpart[2][4];
+    __shared__ float part[4][4];
     __shared__ uint64_t full_cb[2], empty_cb[2], full_x[2], empty_x[2], cb_done, ops_ready, mma_done;
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int h0 = blockIdx.y * kHeadsB, g = h0 / (H / G);
+    const int h0 = (blockIdx.x % nhp) * kHeadsB, g = h0 / (H / G);
     const ChunkEntry seg = segs[sg];
     const int ntiles = (seg.len + kTile - 1) / kTile;
 
@@ -305,10 +371,10 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             mbar_init(&full_cb[i], 1);
             mbar_init(&empty_cb[i], 1);
             mbar_init(&full_x[i], 1);
-            mbar_init(&empty_x[i], 8);
+            mbar_init(&empty_x[i], kComputeWarps);
         }
         mbar_init(&cb_done, 1);
-        mbar_init(&ops_ready, 8);
+        mbar_init(&ops_ready, kComputeWarps);
         mbar_init(&mma_done, 1);
         abort_flag = 0;
         fence_barrier_init();
@@ -340,10 +406,9 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 tma_load_3d(cbuf + 32768, &map_b, &full_cb[st], 0, g, t0);
                 tma_load_3d(cbuf + 49152, &map_b, &full_cb[st], 64, g, t0);
                 for (int hh = 0; hh < kHeadsB; ++hh) {
-                    const int j = it * kHeadsB + hh, slot = j & 1;
-                    if (j >= 2) wait_abort(&empty_x[slot], ((j - 2) >> 1) & 1, abort_p);
-                    mbar_arrive_expect_tx(&full_x[slot], 16384);
-                    tma_load_3d(sX + slot * 16384, &map_x, &full_x[slot], 0, h0 + hh, t0);
+                    if (it >= 1) wait_abort(&empty_x[hh], (it - 1) & 1, abort_p);
+                    mbar_arrive_expect_tx(&full_x[hh], 16384);
+                    tma_load_3d(sX + hh * 16384, &map_x, &full_x[hh], 0, h0 + hh, t0);
                 }
             }
         }
@@ -365,7 +430,7 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                     const int j = it * kHeadsB + hh;
                     wait_abort(&ops_ready, j & 1, abort_p);
                     tc_fence_after();
-                    const uint32_t aX = smem_u32(sX + (hh & 1) * 16384), tMh = tM + (hh & 1) * 64;
+                    const uint32_t aX = smem_u32(sX + hh * 16384), tMh = tM + hh * 64;
                     for (int k = 0; k < 8; ++k) umma_bf16_ts(tY, tMh + 8 * k, desc_mnmajor(aX, k, 16384), id_km, k > 0);
                     for (int k = 0; k < 8; ++k)
                         umma_bf16(tZ, desc_kmajor(aC, 128, k), desc_mnmajor(aH, k, 16384), id_km, k > 0);
@@ -378,17 +443,17 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
         }
     } else {
         // ------------------------------------------------------------ compute warpgroups
-        const int q = warp & 3;                 // TMEM lane quarter of this warp
-        const int r = q * 32 + lane;            // row: token t, source s or state row n
-        const int cw = (warp - 2) >> 2;         // column half
+        const int q = warp & 3;                     // TMEM lane quarter of this warp
+        const int r = q * 32 + lane;                // row: token t, source s or state row n
+        const int cw = (warp - kRoleWarps) >> 2;    // column quarter / source block
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-        float h[kHeadsB][32];                    // h[head][n = r][p = 32*cw + j]
+        float h[kHeadsB][16];                       // h[head][n = r][p = 16*cw + j]
 #pragma unroll
         for (int hh = 0; hh < kHeadsB; ++hh) {
             const float4* src =
-                reinterpret_cast<const float4*>(hin + (((int64_t)sg * H + h0 + hh) * kN + r) * kP + 32 * cw);
+                reinterpret_cast<const float4*>(hin + (((int64_t)sg * H + h0 + hh) * kN + r) * kP + 16 * cw);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
+            for (int j = 0; j < 4; ++j) {
                 const float4 v = src[j];
                 h[hh][4 * j] = v.x;
                 h[hh][4 * j + 1] = v.y;
@@ -397,20 +462,21 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             }
         }
 
-        // Epilogue of head e: y rows (this thread's token r, its 32 columns) and the
-        // state update h <- exp(Acum_end) h + S (this thread's state row r).
+        // Head e done: y rows (token r, this quarter's 16 columns) and the state
+        // update h <- exp(Acum_end) h + S (state row r).
         auto drain = [&](int e, int64_t t0, int tl) {
             const float et = exp2f(ac2[e][r]);
             const float Dh = D[h0 + e];
-            const uint32_t xrow = smem_u32(sX + (e & 1) * 16384);
-            uint32_t ry[32], rz[32];
-            tmem_ld32(tY + lane_off + 32 * cw, ry);
-            tmem_ld32(tZ + lane_off + 32 * cw, rz);
+            const uint32_t xrow = smem_u32(sX + e * 16384);
+            uint32_t ry[16], rz[16], rs[16];
+            tmem_ld16(tY + lane_off + 16 * cw, ry);
+            tmem_ld16(tZ + lane_off + 16 * cw, rz);
+            tmem_ld16(tS + lane_off + 16 * cw, rs);
             tmem_wait_ld();
-            uint32_t o[16];
+            uint32_t o[8];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const uint4 xv = ld_shared_v4(xrow + swz(r, 4 * cw + c));
+            for (int c = 0; c < 2; ++c) {
+                const uint4 xv = ld_shared_v4(xrow + swz(r, 2 * cw + c));
                 const uint32_t xin[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
                 for (int jj = 0; jj < 4; ++jj) {
@@ -422,44 +488,35 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 }
             }
             if (r < tl) {
-                uint4* dst = reinterpret_cast<uint4*>(y + ((t0 + r) * H + h0 + e) * kP + 32 * cw);
-#pragma unroll
-                for (int c = 0; c < 4; ++c) dst[c] = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+                uint4* dst = reinterpret_cast<uint4*>(y + ((t0 + r) * H + h0 + e) * kP + 16 * cw);
+                dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+                dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
             }
-            uint32_t rs[32];
-            tmem_ld32(tS + lane_off + 32 * cw, rs);
-            tmem_wait_ld();
             const float decay = exp2f(ac2[e][kTile - 1]);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) h[e][j] = fmaf(decay, h[e][j], __uint_as_float(rs[j]));
+            for (int j = 0; j < 16; ++j) h[e][j] = fmaf(decay, h[e][j], __uint_as_float(rs[j]));
         };
 
         for (int it = 0; it < ntiles; ++it) {
             const int64_t t0 = seg.start + (int64_t)it * kTile;
             const int tl = min(kTile, seg.len - it * kTile);
-            // -------- dt, log2-scaled cumulative dt*A, and the decay weights of this tile
-            compute_bar();
+            // -------- dt and log2-scaled cumulative dt*A (head cw for cw < 2) and weights
             {
-                const int hh = cw;
+                const int hh = cw & 1;
                 const float Ah = A[h0 + hh];
-                if (r == 0 && it == 0 && (!(Ah <= 0.f) || isinf(Ah))) latch_error(SSD_ERR_INVALID_ARG);
+                if (cw == 0 && r == 0 && it == 0 && (!(Ah <= 0.f) || isinf(Ah))) latch_error(SSD_ERR_INVALID_ARG);
                 const float dtv = r < tl ? softplus_f32(dt_raw[(t0 + r) * H + h0 + hh] + dt_bias[h0 + hh]) : 0.f;
-                float a = dtv * Ah;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const float v = __shfl_up_sync(0xffffffffu, a, off);
-                    if (lane >= off) a += v;
+                compute_bar();              // previous tile's arrays no longer read
+                const float av = wg_scan(dtv * Ah, q, lane, part[cw]) * kLog2e;
+                if (cw < kHeadsB) {
+                    ac2[hh][r] = av;
+                    dts[hh][r] = dtv;
                 }
-                if (lane == 31) wpart[cw][q] = a;
                 compute_bar();
-                float pre = 0.f;
-                for (int w = 0; w < q; ++w) pre += wpart[cw][w];
-                const float av = (a + pre) * kLog2e;
-                ac2[hh][r] = av;
-                dts[hh][r] = dtv;
-                compute_bar();
-                uw[hh][r] = exp2f(ac2[hh][(r | 31)] - av) * dtv;
-                ww[hh][r] = exp2f(ac2[hh][kTile - 1] - av) * dtv;
+                if (cw < kHeadsB) {
+                    uw[hh][r] = exp2f(ac2[hh][(r | 31)] - av) * dtv;
+                    ww[hh][r] = exp2f(ac2[hh][kTile - 1] - av) * dtv;
+                }
                 compute_bar();
             }
             wait_abort(&cb_done, it & 1, abort_p);
@@ -468,43 +525,38 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
 #pragma unroll
             for (int hh = 0; hh < kHeadsB; ++hh) {
                 const int j = it * kHeadsB + hh;
-                // -------- (c) M[t][s] for head hh, t = r, s in [64 cw, 64 cw + 64) -> TMEM
+                // -------- (c) M[t][s] for head hh, t = r, s in source block cw -> TMEM
                 {
                     const float* ac = ac2[hh];
                     const float at = ac[r];
-                    const int bt = r >> 5;
+                    const int bt = q;               // block of t = r >> 5
+                    uint32_t pk[16];
+                    if (cw > bt) {
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        const int sb = 2 * cw + half;              // 32-wide source block
-                        uint32_t pk[16];
-                        if (sb > bt) {
+                        for (int k = 0; k < 16; ++k) pk[k] = 0u;
+                    } else {
+                        uint32_t rc[32];
+                        tmem_ld32(tCB + lane_off + 32 * cw, rc);
+                        tmem_wait_ld();
+                        if (cw < bt) {
+                            const float v = exp2f(at - ac[32 * cw + 31]);
 #pragma unroll
-                            for (int k = 0; k < 16; ++k) pk[k] = 0u;
+                            for (int k = 0; k < 16; ++k) {
+                                const int s0 = 32 * cw + 2 * k;
+                                pk[k] = pack_bf16(__uint_as_float(rc[2 * k]) * v * uw[hh][s0],
+                                                  __uint_as_float(rc[2 * k + 1]) * v * uw[hh][s0 + 1]);
+                            }
                         } else {
-                            uint32_t rc[32];
-                            tmem_ld32(tCB + lane_off + 32 * sb, rc);
-                            tmem_wait_ld();
-                            if (sb < bt) {
-                                const float v = exp2f(at - ac[32 * sb + 31]);
 #pragma unroll
-                                for (int k = 0; k < 16; ++k) {
-                                    const int s0 = 32 * sb + 2 * k;
-                                    pk[k] = pack_bf16(__uint_as_float(rc[2 * k]) * v * uw[hh][s0],
-                                                      __uint_as_float(rc[2 * k + 1]) * v * uw[hh][s0 + 1]);
-                                }
-                            } else {
-#pragma unroll
-                                for (int k = 0; k < 16; ++k) {
-                                    const int s0 = 32 * sb + 2 * k;
-                                    const float m0 = s0 <= r ? __uint_as_float(rc[2 * k]) * exp2f(at - ac[s0]) * dts[hh][s0] : 0.f;
-                                    const float m1 = s0 + 1 <= r ? __uint_as_float(rc[2 * k + 1]) * exp2f(at - ac[s0 + 1]) * dts[hh][s0 + 1] : 0.f;
-                                    pk[k] = pack_bf16(m0, m1);
-                                }
+                            for (int k = 0; k < 16; ++k) {
+                                const int s0 = 32 * cw + 2 * k;
+                                const float m0 = s0 <= r ? __uint_as_float(rc[2 * k]) * exp2f(at - ac[s0]) * dts[hh][s0] : 0.f;
+                                const float m1 = s0 + 1 <= r ? __uint_as_float(rc[2 * k + 1]) * exp2f(at - ac[s0 + 1]) * dts[hh][s0 + 1] : 0.f;
+                                pk[k] = pack_bf16(m0, m1);
                             }
                         }
-                        // 16 packed columns at tM[hh&1] + 16*sb
-                        tmem_st16(tM + (hh & 1) * 64 + lane_off + 16 * sb, pk);
                     }
+                    tmem_st16(tM + hh * 64 + lane_off + 16 * cw, pk);
                     tmem_wait_st();
                 }
                 // -------- drain head hh-1 (its UMMAs overlapped the M build above)
@@ -513,23 +565,23 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                     tc_fence_after();
                     drain(hh - 1, t0, tl);
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&empty_x[(hh - 1) & 1]);
+                    if (lane == 0) mbar_arrive(&empty_x[hh - 1]);
                 }
                 // -------- (a) bf16 h_in of head hh, (b) w * X of head hh
                 {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
+                    for (int c = 0; c < 2; ++c) {
                         uint32_t pk[4];
 #pragma unroll
                         for (int jj = 0; jj < 4; ++jj) pk[jj] = pack_bf16(h[hh][8 * c + 2 * jj], h[hh][8 * c + 2 * jj + 1]);
-                        st_shared_v4(smem_u32(sH) + swz(r, 4 * cw + c), pk[0], pk[1], pk[2], pk[3]);
+                        st_shared_v4(smem_u32(sH) + swz(r, 2 * cw + c), pk[0], pk[1], pk[2], pk[3]);
                     }
-                    wait_abort(&full_x[hh & 1], (j >> 1) & 1, abort_p);
+                    wait_abort(&full_x[hh], it & 1, abort_p);
                     const float w = ww[hh][r];
-                    const uint32_t xrow = smem_u32(sX + (hh & 1) * 16384);
+                    const uint32_t xrow = smem_u32(sX + hh * 16384);
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const uint4 v = ld_shared_v4(xrow + swz(r, 4 * cw + c));
+                    for (int c = 0; c < 2; ++c) {
+                        const uint4 v = ld_shared_v4(xrow + swz(r, 2 * cw + c));
                         const uint32_t in[4] = {v.x, v.y, v.z, v.w};
                         uint32_t o[4];
 #pragma unroll
@@ -537,7 +589,7 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                             const float2 f = bf16x2_to_f2(in[jj]);
                             o[jj] = pack_bf16(f.x * w, f.y * w);
                         }
-                        st_shared_v4(smem_u32(sW) + swz(r, 4 * cw + c), o[0], o[1], o[2], o[3]);
+                        st_shared_v4(smem_u32(sW) + swz(r, 2 * cw + c), o[0], o[1], o[2], o[3]);
                     }
                 }
                 fence_proxy_async_smem();
@@ -549,7 +601,7 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             tc_fence_after();
             drain(kHeadsB - 1, t0, tl);
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty_x[(kHeadsB - 1) & 1]);
+            if (lane == 0) mbar_arrive(&empty_x[kHeadsB - 1]);
         }
     }
     tc_fence_before();
