@@ -191,26 +191,31 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            const uint32_t idesc = idesc_bf16(128, 64, 1, 1);
-            for (int k = 0; k < ntiles; ++k) {
-                const int st = k & 1;
-                wait_abort(&full_b[st], (k >> 1) & 1, abort_p);
-                const uint32_t aB = smem_u32(sB + st * 32768);
-                for (int hh = 0; hh < kHeads; ++hh) {
-                    const int j = k * kHeads + hh, b = j & 1;
-                    wait_abort(&ops_ready[b], (j >> 1) & 1, abort_p);
-                    tc_fence_after();
-                    const uint32_t aHi = smem_u32(sWx + b * 32768), aLo = aHi + 16384;
-                    const uint32_t d = tS + hh * 64;
+        // UMMA issuer: the whole warp runs the loop (warp-uniform descriptors), one
+        // elected lane issues.
+        const uint32_t idesc = idesc_bf16(128, 64, 1, 1);
+        const uint64_t dWx0 = smem_desc(smem_u32(sWx), 16384, 1024);
+        for (int k = 0; k < ntiles; ++k) {
+            const int st = k & 1;
+            wait_abort(&full_b[st], (k >> 1) & 1, abort_p);
+            const uint64_t dB = smem_desc(smem_u32(sB + st * 32768), 16384, 1024);
+            for (int hh = 0; hh < kHeads; ++hh) {
+                const int j = k * kHeads + hh, b = j & 1;
+                wait_abort(&ops_ready[b], (j >> 1) & 1, abort_p);
+                tc_fence_after();
+                const uint64_t dHi = desc_add(dWx0, b * 32768), dLo = desc_add(dHi, 16384);
+                const uint32_t d = tS + hh * 64;
+                if (elect_one()) {
+#pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        umma_bf16(d, desc_mnmajor(aB, kk, 16384), desc_mnmajor(aHi, kk, 16384), idesc,
-                                  !(k == 0 && kk == 0));
+                        umma_bf16(d, desc_add(dB, kk * kMnStep), desc_add(dHi, kk * kMnStep), idesc, !(k == 0 && kk == 0));
+#pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        umma_bf16(d, desc_mnmajor(aB, kk, 16384), desc_mnmajor(aLo, kk, 16384), idesc, true);
+                        umma_bf16(d, desc_add(dB, kk * kMnStep), desc_add(dLo, kk * kMnStep), idesc, true);
                     umma_commit(&mma_done[b]);
                     if (hh == kHeads - 1) umma_commit(&empty_b[st]);
                 }
+                __syncwarp();
             }
         }
     } else {
@@ -230,7 +235,7 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
                 if (r == kTile - 1) tile_tot[cw] = incl;
                 compute_bar();
                 const float tot = tile_tot[cw];
-                wts[cw][r] = exp2f(suffix + tot - incl) * dtv;
+                wts[cw][r] = fast_exp2(suffix + tot - incl) * dtv;
                 suffix += tot;
                 compute_bar();
             }
@@ -414,31 +419,44 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ UMMA issuer
-        if (lane == 0) {
-            const uint32_t id_cb = idesc_bf16(128, 128, 0, 0);
-            const uint32_t id_km = idesc_bf16(128, 64, 0, 1), id_mm = idesc_bf16(128, 64, 1, 1);
-            const uint32_t aW = smem_u32(sW), aH = smem_u32(sH);
-            for (int it = 0; it < ntiles; ++it) {
-                const int st = it & 1;
-                wait_abort(&full_cb[st], (it >> 1) & 1, abort_p);
-                tc_fence_after();
-                const uint32_t aC = smem_u32(sCB + st * 65536), aB = aC + 32768;
+        // The whole warp runs the loop (warp-uniform descriptors), one elected lane issues.
+        const uint32_t id_cb = idesc_bf16(128, 128, 0, 0);
+        const uint32_t id_km = idesc_bf16(128, 64, 0, 1), id_mm = idesc_bf16(128, 64, 1, 1);
+        const uint64_t dW = smem_desc(smem_u32(sW), 16384, 1024), dH = smem_desc(smem_u32(sH), 16384, 1024);
+        const uint64_t dX0 = smem_desc(smem_u32(sX), 16384, 1024);
+        for (int it = 0; it < ntiles; ++it) {
+            const int st = it & 1;
+            wait_abort(&full_cb[st], (it >> 1) & 1, abort_p);
+            tc_fence_after();
+            const uint32_t aC = smem_u32(sCB + st * 65536);
+            const uint64_t dCk = smem_desc(aC, 16, 1024), dBk = smem_desc(aC + 32768, 16, 1024);
+            const uint64_t dBm = smem_desc(aC + 32768, 16384, 1024);
+            if (elect_one()) {
+#pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    umma_bf16(tCB, desc_kmajor(aC, 128, k), desc_kmajor(aB, 128, k), id_cb, k > 0);
+                    umma_bf16(tCB, desc_add(dCk, kmajor_step(128, k)), desc_add(dBk, kmajor_step(128, k)), id_cb, k > 0);
                 umma_commit(&cb_done);
-                for (int hh = 0; hh < kHeadsB; ++hh) {
-                    const int j = it * kHeadsB + hh;
-                    wait_abort(&ops_ready, j & 1, abort_p);
-                    tc_fence_after();
-                    const uint32_t aX = smem_u32(sX + hh * 16384), tMh = tM + hh * 64;
-                    for (int k = 0; k < 8; ++k) umma_bf16_ts(tY, tMh + 8 * k, desc_mnmajor(aX, k, 16384), id_km, k > 0);
+            }
+            __syncwarp();
+            for (int hh = 0; hh < kHeadsB; ++hh) {
+                const int j = it * kHeadsB + hh;
+                wait_abort(&ops_ready, j & 1, abort_p);
+                tc_fence_after();
+                const uint64_t dX = desc_add(dX0, hh * 16384);
+                const uint32_t tMh = tM + hh * 64;
+                if (elect_one()) {
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) umma_bf16_ts(tY, tMh + 8 * k, desc_add(dX, k * kMnStep), id_km, k > 0);
+#pragma unroll
                     for (int k = 0; k < 8; ++k)
-                        umma_bf16(tZ, desc_kmajor(aC, 128, k), desc_mnmajor(aH, k, 16384), id_km, k > 0);
+                        umma_bf16(tZ, desc_add(dCk, kmajor_step(128, k)), desc_add(dH, k * kMnStep), id_km, k > 0);
+#pragma unroll
                     for (int k = 0; k < 8; ++k)
-                        umma_bf16(tS, desc_mnmajor(aB, k, 16384), desc_mnmajor(aW, k, 16384), id_mm, k > 0);
+                        umma_bf16(tS, desc_add(dBm, k * kMnStep), desc_add(dW, k * kMnStep), id_mm, k > 0);
                     umma_commit(&mma_done);
                     if (hh == kHeadsB - 1) umma_commit(&empty_cb[st]);
                 }
+                __syncwarp();
             }
         }
     } else {
@@ -464,9 +482,16 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
 
         // Head e done: y rows (token r, this quarter's 16 columns) and the state
         // update h <- exp(Acum_end) h + S (state row r).
+        const float Dh2[kHeadsB] = {D[h0], D[h0 + 1]};
+        const int hc = cw & 1;                      // head whose decay this warpgroup scans (cw < 2)
+        const float bias_c = dt_bias[h0 + hc], A_c = A[h0 + hc];
+        if (cw == 0 && r == 0 && (!(A_c <= 0.f) || isinf(A_c) || !(A[h0 + 1] <= 0.f) || isinf(A[h0 + 1])))
+            latch_error(SSD_ERR_INVALID_ARG);
+        float dt_next = (cw < 2 && r < min(kTile, seg.len)) ? dt_raw[((int64_t)seg.start + r) * H + h0 + hc] : 0.f;
+
         auto drain = [&](int e, int64_t t0, int tl) {
-            const float et = exp2f(ac2[e][r]);
-            const float Dh = D[h0 + e];
+            const float et = fast_exp2(ac2[e][r]);
+            const float Dh = Dh2[e];
             const uint32_t xrow = smem_u32(sX + e * 16384);
             uint32_t ry[16], rz[16], rs[16];
             tmem_ld16(tY + lane_off + 16 * cw, ry);
@@ -492,7 +517,7 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
                 dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
             }
-            const float decay = exp2f(ac2[e][kTile - 1]);
+            const float decay = fast_exp2(ac2[e][kTile - 1]);
 #pragma unroll
             for (int j = 0; j < 16; ++j) h[e][j] = fmaf(decay, h[e][j], __uint_as_float(rs[j]));
         };
@@ -500,22 +525,24 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
         for (int it = 0; it < ntiles; ++it) {
             const int64_t t0 = seg.start + (int64_t)it * kTile;
             const int tl = min(kTile, seg.len - it * kTile);
-            // -------- dt and log2-scaled cumulative dt*A (head cw for cw < 2) and weights
+            // -------- dt and log2-scaled cumulative dt*A (warpgroup cw < 2 scans head cw)
             {
-                const int hh = cw & 1;
-                const float Ah = A[h0 + hh];
-                if (cw == 0 && r == 0 && it == 0 && (!(Ah <= 0.f) || isinf(Ah))) latch_error(SSD_ERR_INVALID_ARG);
-                const float dtv = r < tl ? softplus_f32(dt_raw[(t0 + r) * H + h0 + hh] + dt_bias[h0 + hh]) : 0.f;
+                const float zraw = dt_next;
+                if (it + 1 < ntiles && cw < 2) {
+                    const int tn = min(kTile, seg.len - (it + 1) * kTile);
+                    dt_next = r < tn ? dt_raw[(t0 + kTile + r) * H + h0 + hc] : 0.f;
+                }
+                const float dtv = (cw < 2 && r < tl) ? softplus_f32(zraw + bias_c) : 0.f;
                 compute_bar();              // previous tile's arrays no longer read
-                const float av = wg_scan(dtv * Ah, q, lane, part[cw]) * kLog2e;
+                const float av = wg_scan(dtv * A_c, q, lane, part[cw]) * kLog2e;
                 if (cw < kHeadsB) {
-                    ac2[hh][r] = av;
-                    dts[hh][r] = dtv;
+                    ac2[hc][r] = av;
+                    dts[hc][r] = dtv;
                 }
                 compute_bar();
                 if (cw < kHeadsB) {
-                    uw[hh][r] = exp2f(ac2[hh][(r | 31)] - av) * dtv;
-                    ww[hh][r] = exp2f(ac2[hh][kTile - 1] - av) * dtv;
+                    uw[hc][r] = fast_exp2(ac2[hc][(r | 31)] - av) * dtv;
+                    ww[hc][r] = fast_exp2(ac2[hc][kTile - 1] - av) * dtv;
                 }
                 compute_bar();
             }
@@ -539,7 +566,7 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                         tmem_ld32(tCB + lane_off + 32 * cw, rc);
                         tmem_wait_ld();
                         if (cw < bt) {
-                            const float v = exp2f(at - ac[32 * cw + 31]);
+                            const float v = fast_exp2(at - ac[32 * cw + 31]);
 #pragma unroll
                             for (int k = 0; k < 16; ++k) {
                                 const int s0 = 32 * cw + 2 * k;
@@ -550,8 +577,8 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
 #pragma unroll
                             for (int k = 0; k < 16; ++k) {
                                 const int s0 = 32 * cw + 2 * k;
-                                const float m0 = s0 <= r ? __uint_as_float(rc[2 * k]) * exp2f(at - ac[s0]) * dts[hh][s0] : 0.f;
-                                const float m1 = s0 + 1 <= r ? __uint_as_float(rc[2 * k + 1]) * exp2f(at - ac[s0 + 1]) * dts[hh][s0 + 1] : 0.f;
+                                const float m0 = s0 <= r ? __uint_as_float(rc[2 * k]) * fast_exp2(at - ac[s0]) * dts[hh][s0] : 0.f;
+                                const float m1 = s0 + 1 <= r ? __uint_as_float(rc[2 * k + 1]) * fast_exp2(at - ac[s0 + 1]) * dts[hh][s0 + 1] : 0.f;
                                 pk[k] = pack_bf16(m0, m1);
                             }
                         }

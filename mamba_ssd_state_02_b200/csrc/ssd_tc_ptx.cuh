@@ -222,6 +222,31 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_
            (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Descriptor advanced by `bytes` (start-address field, 16-byte units; no carry for
+// shared-memory addresses below 256 KB).
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
+// Byte offset of K-step k (16 elements) inside a K-major operand made of 64-column
+// sub-tiles of `rows` rows; MN-major operands advance 2048 bytes per K-step.
+__host__ __device__ constexpr uint32_t kmajor_step(int rows, int k) { return (k >> 2) * rows * 128 + (k & 3) * 32; }
+constexpr uint32_t kMnStep = 2048;
+
+// One lane of the (converged) warp returns true.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}\n"
+        : "=r"(pred));
+    return pred != 0;
+}
+
+// 2^x on the SFU (ex2.approx.ftz: relative error about 2^-22; x <= 0 here).
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // K-step `k` (16 elements) of a K-major operand stored as 64-column sub-tiles of
 // `rows` rows.
 __device__ __forceinline__ uint64_t desc_kmajor(uint32_t base, int rows, int k) {
