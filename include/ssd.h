@@ -130,6 +130,30 @@ ssd_status ssd_state_update(float* state, const void* x, const float* dt_raw, co
                             const ssd_dims* dims, ssd_stream_t stream);
 
 /*
+ * ssd_scan_fwd without any device allocation (the pages have no counterpart; this is a
+ * deployment convenience). Some callers cannot allocate device memory while they run:
+ * serving engines that reserve their whole memory budget at start-up and forbid later
+ * allocations, and latency-critical loops where a cudaMalloc/cudaFree (or a caching
+ * allocator's slow path) mid-step is unacceptable. This variant computes exactly what
+ * ssd_scan_fwd computes, with the same arguments, but takes its scratch from a 32 MiB
+ * array compiled into the library instead of dims->workspace (which must be NULL) or
+ * cudaMallocAsync. It calls no cudaMalloc, cudaFree or other allocating routine.
+ *   - Size limit: if the problem needs more scratch than 32 MiB (see
+ *     ssd_scan_fwd_workspace_size) it returns SSD_ERR_UNSUPPORTED and launches nothing.
+ *   - Every GPU that loads the library holds those 32 MiB until the process exits.
+ *   - The first call on each device looks up the array's device address (with that
+ *     device current); make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents: calls whose
+ *     work can overlap on the GPU (different streams, or different host threads on one
+ *     device) race on it and must be serialised by the caller. Nothing in it needs
+ *     clearing between calls: every slot a kernel reads is written earlier in the call.
+ */
+ssd_status ssd_scan_fwd_noalloc(const void* x, const float* dt_raw, const float* dt_bias, const float* A,
+                                const void* B, const void* C, const float* D, const float* init_state,
+                                const int32_t* cu_seqlens, void* y, float* final_state,
+                                const ssd_dims* dims, int chunk, ssd_stream_t stream);
+
+/*
  * Waits for `stream`, then reads and clears the device error word: SSD_OK, or the
  * first error a kernel latched since the last read (SSD_ERR_INVALID_ARG for bad
  * cu_seqlens or A > 0, SSD_ERR_TIMEOUT for an expired bounded wait). SSD_ERR_CUDA

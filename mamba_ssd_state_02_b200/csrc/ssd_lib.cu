@@ -603,3 +603,88 @@ int ssd_profile_read(ssd_kernel_time* out, int max, int* dropped) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------
+// Prefill without any allocation. Some callers cannot allocate device memory at call
+// time: serving engines that reserve their whole memory budget up front and forbid
+// later allocations, and latency-critical callers for which a cudaMalloc/cudaFree (or
+// a trip into a caching allocator) in the middle of a step is not acceptable. This
+// entry point takes its scratch from one array compiled into the library instead.
+namespace ssd {
+namespace {
+
+// Scratch compiled into the library: every GPU that loads libssd holds these 32 MiB
+// until the process exits. Host code must not pass the symbol itself to a kernel (on
+// the host it is only a stand-in); the device address is looked up once per device.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up on the first
+// call per device, with that device current).
+ssd_status noalloc_scratch(char** out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(SSD_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+        g_noalloc_addr[dev] = p;
+    }
+    *out = static_cast<char*>(g_noalloc_addr[dev]);
+    return SSD_OK;
+}
+
+}  // namespace
+}  // namespace ssd
+
+extern "C" ssd_status ssd_scan_fwd_noalloc(const void* x, const float* dt_raw, const float* dt_bias,
+                                           const float* A, const void* B, const void* C, const float* D,
+                                           const float* init_state, const int32_t* cu_seqlens, void* y,
+                                           float* final_state, const ssd_dims* dims, int chunk,
+                                           ssd_stream_t stream) {
+    Plan pl;
+    ssd_status s = make_plan(dims, chunk, cu_seqlens != nullptr, &pl);
+    if (s != SSD_OK) return s;
+    if (dims->workspace)
+        return fail(SSD_ERR_INVALID_ARG, "ssd_scan_fwd_noalloc uses its own scratch: dims->workspace must be NULL");
+    if (!dt_bias || !A || !D) return fail(SSD_ERR_INVALID_ARG, "dt_bias, A and D must be non-NULL");
+    if (pl.T > 0 && (!x || !dt_raw || !B || !C || !y))
+        return fail(SSD_ERR_INVALID_ARG, "x, dt_raw, B, C and y must be non-NULL");
+    if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(y, 16))
+        return fail(SSD_ERR_INVALID_ARG, "x, B, C and y must be 16-byte aligned");
+    if (!aligned(dt_raw, 4) || !aligned(dt_bias, 4) || !aligned(A, 4) || !aligned(D, 4) ||
+        !aligned(init_state, 16) || !aligned(final_state, 16) || !aligned(cu_seqlens, 4))
+        return fail(SSD_ERR_INVALID_ARG, "float/int arrays must be 4-byte aligned, states 16-byte");
+    if (pl.bytes > kNoAllocScratchBytes)
+        return fail(SSD_ERR_UNSUPPORTED,
+                    "problem needs %zu bytes of scratch; ssd_scan_fwd_noalloc has %zu (use ssd_scan_fwd)",
+                    pl.bytes, kNoAllocScratchBytes);
+    if (pl.nseq == 0) {
+        t_launches = 0;
+        t_last_error.clear();
+        return SSD_OK;
+    }
+    char* ws = nullptr;
+    s = noalloc_scratch(&ws);
+    if (s != SSD_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // Every slot of the scratch that a kernel reads is written earlier in the same call
+    // (chunk/segment table, then states), so nothing needs clearing between calls.
+    if (pl.tc)
+        s = launch_tc(pl, ws, x, dt_raw, dt_bias, A, B, C, D, init_state, cu_seqlens, y, final_state, st);
+    else if (pl.bf16)
+        s = dispatch_Q<__nv_bfloat16>(pl, ws, x, dt_raw, dt_bias, A, B, C, D, init_state, cu_seqlens, y,
+                                      final_state, st);
+    else
+        s = dispatch_Q<float>(pl, ws, x, dt_raw, dt_bias, A, B, C, D, init_state, cu_seqlens, y, final_state,
+                              st);
+    if (s == SSD_OK) t_last_error.clear();
+    return s;
+}

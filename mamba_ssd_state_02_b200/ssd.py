@@ -58,6 +58,9 @@ _lib.ssd_scan_fwd_workspace_size.restype = ctypes.c_int
 _lib.ssd_scan_fwd.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p,
                               ctypes.POINTER(SSDDims), ctypes.c_int, _p]
 _lib.ssd_scan_fwd.restype = ctypes.c_int
+_lib.ssd_scan_fwd_noalloc.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p,
+                                      ctypes.POINTER(SSDDims), ctypes.c_int, _p]
+_lib.ssd_scan_fwd_noalloc.restype = ctypes.c_int
 _lib.ssd_state_update.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, ctypes.POINTER(SSDDims), _p]
 _lib.ssd_state_update.restype = ctypes.c_int
 _lib.ssd_get_device_status.argtypes = [_p]
@@ -237,6 +240,53 @@ def scan_fwd(x, dt_raw, dt_bias, A, B, C, D, init_state=None, cu_seqlens=None, c
         _check(_lib.ssd_scan_fwd(_ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C),
                                  _ptr(D), _ptr(init_state), _ptr(cu_seqlens), _ptr(y),
                                  _ptr(final_state), ctypes.byref(dims), int(chunk), _stream(dev)))
+    return y, final_state
+
+
+def scan_fwd_noalloc(x, dt_raw, dt_bias, A, B, C, D, init_state=None, cu_seqlens=None, chunk=128,
+                     y=None, final_state=None):
+    """scan_fwd through ssd_scan_fwd_noalloc: the library's own 32 MiB scratch array, no
+    device allocation inside the call (y/final_state are allocated here only when the
+    caller passes none). For callers whose memory budget is fixed up front; calls that
+    overlap on the GPU share the scratch and must be serialised."""
+    dev = x.device
+    varlen = cu_seqlens is not None
+    if varlen:
+        T, H, P = x.shape
+        nseq = cu_seqlens.numel() - 1
+        tok = (T,)
+    else:
+        if x.dim() != 4:
+            raise ValueError("dense x must be [batch, L, H, P]")
+        bsz, L, H, P = x.shape
+        nseq = bsz
+        tok = (bsz, L)
+    G, N = B.shape[-2], B.shape[-1]
+    dt = x.dtype
+    _need(x, "x", tok + (H, P), dt, dev)
+    _need(dt_raw, "dt_raw", tok + (H,), torch.float32, dev)
+    _need(B, "B", tok + (G, N), dt, dev)
+    _need(C, "C", tok + (G, N), dt, dev)
+    for name, v in (("dt_bias", dt_bias), ("A", A), ("D", D)):
+        _need(v, name, (H,), torch.float32, dev)
+    if init_state is not None:
+        _need(init_state, "init_state", (nseq, H, P, N), torch.float32, dev)
+    if varlen:
+        _need(cu_seqlens, "cu_seqlens", (nseq + 1,), torch.int32, dev)
+    if y is None:
+        y = torch.empty_like(x)
+    _need(y, "y", tok + (H, P), dt, dev)
+    if final_state is None:
+        final_state = torch.empty(nseq, H, P, N, dtype=torch.float32, device=dev)
+    _need(final_state, "final_state", (nseq, H, P, N), torch.float32, dev)
+    if varlen:
+        dims = make_dims(x.shape[0], H, P, G, N, _dtype_code(x), nseq=nseq)
+    else:
+        dims = make_dims(bsz * L, H, P, G, N, _dtype_code(x), batch=bsz, seqlen=L)
+    with torch.cuda.device(dev):
+        _check(_lib.ssd_scan_fwd_noalloc(_ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C),
+                                         _ptr(D), _ptr(init_state), _ptr(cu_seqlens), _ptr(y),
+                                         _ptr(final_state), ctypes.byref(dims), int(chunk), _stream(dev)))
     return y, final_state
 
 
