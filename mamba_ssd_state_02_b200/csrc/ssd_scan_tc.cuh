@@ -39,44 +39,6 @@ constexpr int kN = 128;          // dstate
 constexpr int kHeads = 4;        // heads per CTA
 constexpr float kLog2e = 1.4426950408889634f;
 
-// Per-tile dt / cumulative decay for this CTA's 4 heads, computed by 128 threads
-// (thread s = token s of the tile). acs2[h][s] = log2(e) * sum_{r<=s} dt_r A[h];
-// dts[h][s] = dt_s (0 past the tile's valid length).
-__device__ __forceinline__ void tile_cumsum(const float* __restrict__ dt_raw, const float* __restrict__ dt_bias,
-                                            const float* __restrict__ A, int H, int h0, int64_t t0, int tl,
-                                            float (*acs2)[kTile], float (*dts)[kTile], float (*wsum)[kHeads]) {
-    const int s = threadIdx.x, lane = s & 31, warp = s >> 5;
-    float a[kHeads], dtv[kHeads];
-#pragma unroll
-    for (int hh = 0; hh < kHeads; ++hh) {
-        const float Ah = A[h0 + hh];
-        if (s == 0 && (!(Ah <= 0.f) || isinf(Ah))) latch_error(SSD_ERR_INVALID_ARG);
-        dtv[hh] = s < tl ? softplus_f32(dt_raw[(t0 + s) * H + h0 + hh] + dt_bias[h0 + hh]) : 0.f;
-        a[hh] = dtv[hh] * Ah;
-    }
-#pragma unroll
-    for (int hh = 0; hh < kHeads; ++hh) {
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const float v = __shfl_up_sync(0xffffffffu, a[hh], off);
-            if (lane >= off) a[hh] += v;
-        }
-    }
-    if (lane == 31) {
-#pragma unroll
-        for (int hh = 0; hh < kHeads; ++hh) wsum[warp][hh] = a[hh];
-    }
-    __syncthreads();
-#pragma unroll
-    for (int hh = 0; hh < kHeads; ++hh) {
-        float pre = 0.f;
-        for (int w = 0; w < warp; ++w) pre += wsum[w][hh];
-        acs2[hh][s] = (a[hh] + pre) * kLog2e;
-        dts[hh][s] = dtv[hh];
-    }
-    __syncthreads();
-}
-
 // ---------------------------------------------------------------------------------
 // Shared by both passes.
 constexpr int kRoleWarps = 2;                    // warp 0: TMA producer, warp 1: UMMA issuer
@@ -333,17 +295,24 @@ k_tc_segment_passing(float* __restrict__ seg_state, const float* __restrict__ se
 // ---------------------------------------------------------------------------------
 // Pass B: outputs y for one (segment, 2 heads), chunk by chunk.
 //
-// Warp 0 issues the TMA loads, warp 1 the UMMAs; the four compute warpgroups
-// (cw = 0..3) split every row's 64 columns in quarters (and the 128 source columns
-// of M in 32-wide blocks). Compute thread (cw, r) owns TMEM lane r = 32*(warp%4) +
-// lane and holds the FP32 running state h[head][n = r][p in its quarter].
-// Shared memory: two C/B stages (tile i+1 loads while tile i computes), a two-slot X
-// ring (one per head), one w*X and one bf16 h operand tile. TMEM: C B^T (128 cols),
-// two M buffers (A operands, bf16 pairs, 64 cols each), Y, Z, S (64 cols each). Per
-// head the compute warps build M for head hh while the UMMAs of head hh-1 run, then
-// drain head hh-1 (y rows, state update) and write the operands of head hh.
+// Warp 0 issues the TMA loads, warp 1 the UMMAs, and four compute warpgroups
+// (cw = 0..3) split every row's 64 columns in quarters (and the 128 source columns of
+// M in 32-wide blocks). Compute thread (cw, r) owns TMEM lane r = 32*(warp%4) + lane
+// and keeps the FP32 running state h[head][n = r][p in its quarter] in registers.
+//
+// Per chunk: CB = C B^T (UMMA) -> the compute warps build M for both heads into TMEM,
+// write w*X and bf16 h for both heads to shared memory -> one UMMA batch: Z = C [h0|h1]^T
+// and S = B^T [wX0|wX1] (N = 128 each, so C and B are read once for both heads), then
+// Y_hh = M_hh X_hh -> the compute warps drain y and update h. While that batch runs,
+// warpgroups 0 and 1 scan dt*A of the next chunk into the other half of a double
+// buffer, and x stays in registers from the w*X step to the D x term.
+// TMEM: Z (cols 0..127, first holds C B^T), S (128..255), Y0, Y1 (256..383), M0, M1
+// (384..511). Shared memory: one C/B stage (reloaded as soon as the Z/S UMMAs are done),
+// one X slot per head, bf16 h and w*X for both heads.
 constexpr int kHeadsB = 2;
-constexpr int kSmemB = 192 * 1024 + 1024;
+constexpr int kSmemB = 160 * 1024 + 1024;
+
+__device__ __forceinline__ void wg_bar(int cw) { asm volatile("bar.sync %0, 128;" ::"r"(2 + cw) : "memory"); }
 
 __global__ void __launch_bounds__(kThreadsTc, 1)
 k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
@@ -356,13 +325,15 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
     if (sg >= *nsegs) return;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sCB = sm;                      // stage st: C at st*65536 ([2][128 t][64 n]), B at +32768
-    uint8_t* sX = sm + 131072;              // slot hh: [128 s][64 p] at hh*16384
-    uint8_t* sW = sm + 163840;              // [128 s][64 p]  w * X
-    uint8_t* sH = sm + 180224;              // [128 n][64 p]  bf16 h_in
-    __shared__ float ac2[kHeadsB][kTile], dts[kHeadsB][kTile], uw[kHeadsB][kTile], ww[kHeadsB][kTile];
-    __shared__ float part[4][4];
-    __shared__ uint64_t full_cb[2], empty_cb[2], full_x[2], empty_x[2], cb_done, ops_ready, mma_done;
+    uint8_t* sC = sm;                       // [2][128 t][64 n]   K-major
+    uint8_t* sB = sm + 32768;               // [2][128 s][64 n]   K-major for C B^T, MN-major for B^T
+    uint8_t* sX = sm + 65536;               // head hh at hh*16384: [128 s][64 p]
+    uint8_t* sH = sm + 98304;               // head hh block at hh*16384: [128 n][64 p]  bf16 h_in
+    uint8_t* sW = sm + 131072;              // head hh block at hh*16384: [128 s][64 p]  w * X
+    __shared__ float ac2[2][kHeadsB][kTile], dts[2][kHeadsB][kTile], uw[2][kHeadsB][kTile], ww[2][kHeadsB][kTile];
+    __shared__ float part[kHeadsB][4];
+    __shared__ uint64_t full_cb, empty_cb, full_x[kHeadsB], empty_x[kHeadsB], cb_done, ops_ready, mma_done,
+        acc_free, dt_ready[2], dt_free[2];
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
 
@@ -372,15 +343,20 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
     const int ntiles = (seg.len + kTile - 1) / kTile;
 
     if (tid == 0) {
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&full_cb[i], 1);
-            mbar_init(&empty_cb[i], 1);
+        mbar_init(&full_cb, 1);
+        mbar_init(&empty_cb, 1);
+        for (int i = 0; i < kHeadsB; ++i) {
             mbar_init(&full_x[i], 1);
-            mbar_init(&empty_x[i], kComputeWarps);
+            mbar_init(&empty_x[i], 1 + kComputeWarps);
         }
         mbar_init(&cb_done, 1);
         mbar_init(&ops_ready, kComputeWarps);
         mbar_init(&mma_done, 1);
+        mbar_init(&acc_free, kComputeWarps);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&dt_ready[i], 8);
+            mbar_init(&dt_free[i], kComputeWarps);
+        }
         abort_flag = 0;
         fence_barrier_init();
         prefetch_tmap(&map_x);
@@ -395,21 +371,20 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = tmem_slot;
-    const uint32_t tCB = tbase, tM = tbase + 128, tY = tbase + 256, tZ = tbase + 320, tS = tbase + 384;
+    const uint32_t tZ = tbase, tCB = tbase, tS = tbase + 128, tY = tbase + 256, tM = tbase + 384;
     volatile int* abort_p = &abort_flag;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             for (int it = 0; it < ntiles; ++it) {
-                const int t0 = seg.start + it * kTile, st = it & 1;
-                if (it >= 2) wait_abort(&empty_cb[st], ((it - 2) >> 1) & 1, abort_p);
-                mbar_arrive_expect_tx(&full_cb[st], 65536);
-                uint8_t* cbuf = sCB + st * 65536;
-                tma_load_3d(cbuf, &map_c, &full_cb[st], 0, g, t0);
-                tma_load_3d(cbuf + 16384, &map_c, &full_cb[st], 64, g, t0);
-                tma_load_3d(cbuf + 32768, &map_b, &full_cb[st], 0, g, t0);
-                tma_load_3d(cbuf + 49152, &map_b, &full_cb[st], 64, g, t0);
+                const int t0 = seg.start + it * kTile;
+                if (it >= 1) wait_abort(&empty_cb, (it - 1) & 1, abort_p);
+                mbar_arrive_expect_tx(&full_cb, 65536);
+                tma_load_3d(sC, &map_c, &full_cb, 0, g, t0);
+                tma_load_3d(sC + 16384, &map_c, &full_cb, 64, g, t0);
+                tma_load_3d(sB, &map_b, &full_cb, 0, g, t0);
+                tma_load_3d(sB + 16384, &map_b, &full_cb, 64, g, t0);
                 for (int hh = 0; hh < kHeadsB; ++hh) {
                     if (it >= 1) wait_abort(&empty_x[hh], (it - 1) & 1, abort_p);
                     mbar_arrive_expect_tx(&full_x[hh], 16384);
@@ -420,17 +395,16 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
     } else if (warp == 1) {
         // ------------------------------------------------------------ UMMA issuer
         // The whole warp runs the loop (warp-uniform descriptors), one elected lane issues.
-        const uint32_t id_cb = idesc_bf16(128, 128, 0, 0);
-        const uint32_t id_km = idesc_bf16(128, 64, 0, 1), id_mm = idesc_bf16(128, 64, 1, 1);
-        const uint64_t dW = smem_desc(smem_u32(sW), 16384, 1024), dH = smem_desc(smem_u32(sH), 16384, 1024);
-        const uint64_t dX0 = smem_desc(smem_u32(sX), 16384, 1024);
+        const uint32_t id_cb = idesc_bf16(128, 128, 0, 0), id_z = idesc_bf16(128, 128, 0, 1);
+        const uint32_t id_s = idesc_bf16(128, 128, 1, 1), id_y = idesc_bf16(128, 64, 0, 1);
+        const uint64_t dCk = smem_desc(smem_u32(sC), 16, 1024), dBk = smem_desc(smem_u32(sB), 16, 1024);
+        const uint64_t dBm = smem_desc(smem_u32(sB), 16384, 1024);
+        const uint64_t dH = smem_desc(smem_u32(sH), 16384, 1024), dW = smem_desc(smem_u32(sW), 16384, 1024);
+        const uint64_t dX0 = smem_desc(smem_u32(sX), 16384, 1024), dX1 = desc_add(dX0, 16384);
         for (int it = 0; it < ntiles; ++it) {
-            const int st = it & 1;
-            wait_abort(&full_cb[st], (it >> 1) & 1, abort_p);
+            wait_abort(&full_cb, it & 1, abort_p);
+            if (it >= 1) wait_abort(&acc_free, (it - 1) & 1, abort_p);
             tc_fence_after();
-            const uint32_t aC = smem_u32(sCB + st * 65536);
-            const uint64_t dCk = smem_desc(aC, 16, 1024), dBk = smem_desc(aC + 32768, 16, 1024);
-            const uint64_t dBm = smem_desc(aC + 32768, 16384, 1024);
             if (elect_one()) {
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
@@ -438,26 +412,26 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 umma_commit(&cb_done);
             }
             __syncwarp();
-            for (int hh = 0; hh < kHeadsB; ++hh) {
-                const int j = it * kHeadsB + hh;
-                wait_abort(&ops_ready, j & 1, abort_p);
-                tc_fence_after();
-                const uint64_t dX = desc_add(dX0, hh * 16384);
-                const uint32_t tMh = tM + hh * 64;
-                if (elect_one()) {
+            wait_abort(&ops_ready, it & 1, abort_p);
+            tc_fence_after();
+            if (elect_one()) {
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) umma_bf16_ts(tY, tMh + 8 * k, desc_add(dX, k * kMnStep), id_km, k > 0);
+                for (int k = 0; k < 8; ++k)
+                    umma_bf16(tZ, desc_add(dCk, kmajor_step(128, k)), desc_add(dH, k * kMnStep), id_z, k > 0);
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        umma_bf16(tZ, desc_add(dCk, kmajor_step(128, k)), desc_add(dH, k * kMnStep), id_km, k > 0);
+                for (int k = 0; k < 8; ++k)
+                    umma_bf16(tS, desc_add(dBm, k * kMnStep), desc_add(dW, k * kMnStep), id_s, k > 0);
+                umma_commit(&empty_cb);
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        umma_bf16(tS, desc_add(dBm, k * kMnStep), desc_add(dW, k * kMnStep), id_mm, k > 0);
-                    umma_commit(&mma_done);
-                    if (hh == kHeadsB - 1) umma_commit(&empty_cb[st]);
-                }
-                __syncwarp();
+                for (int k = 0; k < 8; ++k) umma_bf16_ts(tY, tM + 8 * k, desc_add(dX0, k * kMnStep), id_y, k > 0);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    umma_bf16_ts(tY + 64, tM + 64 + 8 * k, desc_add(dX1, k * kMnStep), id_y, k > 0);
+                umma_commit(&mma_done);
+                umma_commit(&empty_x[0]);
+                umma_commit(&empty_x[1]);
             }
+            __syncwarp();
         }
     } else {
         // ------------------------------------------------------------ compute warpgroups
@@ -479,156 +453,164 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 h[hh][4 * j + 3] = v.w;
             }
         }
-
-        // Head e done: y rows (token r, this quarter's 16 columns) and the state
-        // update h <- exp(Acum_end) h + S (state row r).
-        const float Dh2[kHeadsB] = {D[h0], D[h0 + 1]};
-        const int hc = cw & 1;                      // head whose decay this warpgroup scans (cw < 2)
+        const float Dh0 = D[h0], Dh1 = D[h0 + 1];
+        const int hc = cw & 1;
         const float bias_c = dt_bias[h0 + hc], A_c = A[h0 + hc];
-        if (cw == 0 && r == 0 && (!(A_c <= 0.f) || isinf(A_c) || !(A[h0 + 1] <= 0.f) || isinf(A[h0 + 1])))
-            latch_error(SSD_ERR_INVALID_ARG);
-        float dt_next = (cw < 2 && r < min(kTile, seg.len)) ? dt_raw[((int64_t)seg.start + r) * H + h0 + hc] : 0.f;
+        if (cw < kHeadsB && r == 0 && (!(A_c <= 0.f) || isinf(A_c))) latch_error(SSD_ERR_INVALID_ARG);
 
-        auto drain = [&](int e, int64_t t0, int tl) {
-            const float et = fast_exp2(ac2[e][r]);
-            const float Dh = Dh2[e];
-            const uint32_t xrow = smem_u32(sX + e * 16384);
-            uint32_t ry[16], rz[16], rs[16];
-            tmem_ld16(tY + lane_off + 16 * cw, ry);
-            tmem_ld16(tZ + lane_off + 16 * cw, rz);
-            tmem_ld16(tS + lane_off + 16 * cw, rs);
-            tmem_wait_ld();
-            uint32_t o[8];
+        // dt, log2-scaled cumulative dt*A and the decay weights of chunk j (warpgroups 0
+        // and 1, one head each) into buffer j & 1.
+        auto scan_chunk = [&](int j) {
+            if (cw >= kHeadsB) return;
+            const int bf = j & 1;
+            if (j >= 2) wait_abort(&dt_free[bf], ((j - 2) >> 1) & 1, abort_p);
+            const int64_t tj = seg.start + (int64_t)j * kTile;
+            const int tlj = min(kTile, seg.len - j * kTile);
+            const float dtv = r < tlj ? softplus_f32(dt_raw[(tj + r) * H + h0 + cw] + bias_c) : 0.f;
+            float a = dtv * A_c;
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                const uint4 xv = ld_shared_v4(xrow + swz(r, 2 * cw + c));
-                const uint32_t xin[4] = {xv.x, xv.y, xv.z, xv.w};
-#pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const float2 xf = bf16x2_to_f2(xin[jj]);
-                    const int k0 = c * 8 + 2 * jj;
-                    const float v0 = fmaf(et, __uint_as_float(rz[k0]), __uint_as_float(ry[k0])) + Dh * xf.x;
-                    const float v1 = fmaf(et, __uint_as_float(rz[k0 + 1]), __uint_as_float(ry[k0 + 1])) + Dh * xf.y;
-                    o[c * 4 + jj] = pack_bf16(v0, v1);
-                }
+            for (int off = 1; off < 32; off <<= 1) {
+                const float v = __shfl_up_sync(0xffffffffu, a, off);
+                if (lane >= off) a += v;
             }
-            if (r < tl) {
-                uint4* dst = reinterpret_cast<uint4*>(y + ((t0 + r) * H + h0 + e) * kP + 16 * cw);
-                dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-                dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
-            }
-            const float decay = fast_exp2(ac2[e][kTile - 1]);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) h[e][j] = fmaf(decay, h[e][j], __uint_as_float(rs[j]));
+            if (lane == 31) part[cw][q] = a;
+            wg_bar(cw);
+            float pre = 0.f;
+            for (int w = 0; w < q; ++w) pre += part[cw][w];
+            const float av = (a + pre) * kLog2e;
+            ac2[bf][cw][r] = av;
+            dts[bf][cw][r] = dtv;
+            wg_bar(cw);
+            uw[bf][cw][r] = fast_exp2(ac2[bf][cw][r | 31] - av) * dtv;
+            ww[bf][cw][r] = fast_exp2(ac2[bf][cw][kTile - 1] - av) * dtv;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&dt_ready[bf]);
         };
 
+        scan_chunk(0);
         for (int it = 0; it < ntiles; ++it) {
             const int64_t t0 = seg.start + (int64_t)it * kTile;
             const int tl = min(kTile, seg.len - it * kTile);
-            // -------- dt and log2-scaled cumulative dt*A (warpgroup cw < 2 scans head cw)
-            {
-                const float zraw = dt_next;
-                if (it + 1 < ntiles && cw < 2) {
-                    const int tn = min(kTile, seg.len - (it + 1) * kTile);
-                    dt_next = r < tn ? dt_raw[(t0 + kTile + r) * H + h0 + hc] : 0.f;
-                }
-                const float dtv = (cw < 2 && r < tl) ? softplus_f32(zraw + bias_c) : 0.f;
-                compute_bar();              // previous tile's arrays no longer read
-                const float av = wg_scan(dtv * A_c, q, lane, part[cw]) * kLog2e;
-                if (cw < kHeadsB) {
-                    ac2[hc][r] = av;
-                    dts[hc][r] = dtv;
-                }
-                compute_bar();
-                if (cw < kHeadsB) {
-                    uw[hc][r] = fast_exp2(ac2[hc][(r | 31)] - av) * dtv;
-                    ww[hc][r] = fast_exp2(ac2[hc][kTile - 1] - av) * dtv;
-                }
-                compute_bar();
-            }
+            const int bf = it & 1;
+            wait_abort(&dt_ready[bf], (it >> 1) & 1, abort_p);
             wait_abort(&cb_done, it & 1, abort_p);
             tc_fence_after();
-
+            // -------- M[t][s] of both heads, t = r, s in source block cw -> TMEM
+            {
+                uint32_t rc[32];
+                const bool live = cw <= q;             // blocks above the diagonal are zero
+                if (live) {
+                    tmem_ld32(tCB + lane_off + 32 * cw, rc);
+                    tmem_wait_ld();
+                }
 #pragma unroll
-            for (int hh = 0; hh < kHeadsB; ++hh) {
-                const int j = it * kHeadsB + hh;
-                // -------- (c) M[t][s] for head hh, t = r, s in source block cw -> TMEM
-                {
-                    const float* ac = ac2[hh];
+                for (int hh = 0; hh < kHeadsB; ++hh) {
+                    const float* ac = ac2[bf][hh];
                     const float at = ac[r];
-                    const int bt = q;               // block of t = r >> 5
                     uint32_t pk[16];
-                    if (cw > bt) {
+                    if (!live) {
 #pragma unroll
                         for (int k = 0; k < 16; ++k) pk[k] = 0u;
+                    } else if (cw < q) {
+                        const float v = fast_exp2(at - ac[32 * cw + 31]);
+                        const float* u = uw[bf][hh] + 32 * cw;
+#pragma unroll
+                        for (int k = 0; k < 16; ++k)
+                            pk[k] = pack_bf16(__uint_as_float(rc[2 * k]) * v * u[2 * k],
+                                              __uint_as_float(rc[2 * k + 1]) * v * u[2 * k + 1]);
                     } else {
-                        uint32_t rc[32];
-                        tmem_ld32(tCB + lane_off + 32 * cw, rc);
-                        tmem_wait_ld();
-                        if (cw < bt) {
-                            const float v = fast_exp2(at - ac[32 * cw + 31]);
+                        const float* dv = dts[bf][hh] + 32 * cw;
+                        const float* as = ac + 32 * cw;
 #pragma unroll
-                            for (int k = 0; k < 16; ++k) {
-                                const int s0 = 32 * cw + 2 * k;
-                                pk[k] = pack_bf16(__uint_as_float(rc[2 * k]) * v * uw[hh][s0],
-                                                  __uint_as_float(rc[2 * k + 1]) * v * uw[hh][s0 + 1]);
-                            }
-                        } else {
-#pragma unroll
-                            for (int k = 0; k < 16; ++k) {
-                                const int s0 = 32 * cw + 2 * k;
-                                const float m0 = s0 <= r ? __uint_as_float(rc[2 * k]) * fast_exp2(at - ac[s0]) * dts[hh][s0] : 0.f;
-                                const float m1 = s0 + 1 <= r ? __uint_as_float(rc[2 * k + 1]) * fast_exp2(at - ac[s0 + 1]) * dts[hh][s0 + 1] : 0.f;
-                                pk[k] = pack_bf16(m0, m1);
-                            }
+                        for (int k = 0; k < 16; ++k) {
+                            const int s0 = 32 * cw + 2 * k;
+                            const float m0 = s0 <= r ? __uint_as_float(rc[2 * k]) * fast_exp2(at - as[2 * k]) * dv[2 * k] : 0.f;
+                            const float m1 = s0 + 1 <= r ? __uint_as_float(rc[2 * k + 1]) * fast_exp2(at - as[2 * k + 1]) * dv[2 * k + 1] : 0.f;
+                            pk[k] = pack_bf16(m0, m1);
                         }
                     }
                     tmem_st16(tM + hh * 64 + lane_off + 16 * cw, pk);
-                    tmem_wait_st();
                 }
-                // -------- drain head hh-1 (its UMMAs overlapped the M build above)
-                if (hh > 0) {
-                    wait_abort(&mma_done, (j - 1) & 1, abort_p);
-                    tc_fence_after();
-                    drain(hh - 1, t0, tl);
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&empty_x[hh - 1]);
-                }
-                // -------- (a) bf16 h_in of head hh, (b) w * X of head hh
-                {
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        uint32_t pk[4];
-#pragma unroll
-                        for (int jj = 0; jj < 4; ++jj) pk[jj] = pack_bf16(h[hh][8 * c + 2 * jj], h[hh][8 * c + 2 * jj + 1]);
-                        st_shared_v4(smem_u32(sH) + swz(r, 2 * cw + c), pk[0], pk[1], pk[2], pk[3]);
-                    }
-                    wait_abort(&full_x[hh], it & 1, abort_p);
-                    const float w = ww[hh][r];
-                    const uint32_t xrow = smem_u32(sX + hh * 16384);
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        const uint4 v = ld_shared_v4(xrow + swz(r, 2 * cw + c));
-                        const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-                        uint32_t o[4];
-#pragma unroll
-                        for (int jj = 0; jj < 4; ++jj) {
-                            const float2 f = bf16x2_to_f2(in[jj]);
-                            o[jj] = pack_bf16(f.x * w, f.y * w);
-                        }
-                        st_shared_v4(smem_u32(sW) + swz(r, 2 * cw + c), o[0], o[1], o[2], o[3]);
-                    }
-                }
-                fence_proxy_async_smem();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&ops_ready);
+                tmem_wait_st();
             }
-            wait_abort(&mma_done, (it * kHeadsB + kHeadsB - 1) & 1, abort_p);
-            tc_fence_after();
-            drain(kHeadsB - 1, t0, tl);
+            // -------- w*X and bf16 h of both heads; x kept for the D x term
+            uint32_t xk[kHeadsB][8];
+#pragma unroll
+            for (int hh = 0; hh < kHeadsB; ++hh) {
+                wait_abort(&full_x[hh], it & 1, abort_p);
+                const float w = ww[bf][hh][r];
+                const uint32_t xrow = smem_u32(sX + hh * 16384), wrow = smem_u32(sW + hh * 16384);
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const uint4 v = ld_shared_v4(xrow + swz(r, 2 * cw + c));
+                    xk[hh][4 * c] = v.x;
+                    xk[hh][4 * c + 1] = v.y;
+                    xk[hh][4 * c + 2] = v.z;
+                    xk[hh][4 * c + 3] = v.w;
+                    uint32_t o[4];
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const float2 f = bf16x2_to_f2(xk[hh][4 * c + jj]);
+                        o[jj] = pack_bf16(f.x * w, f.y * w);
+                    }
+                    st_shared_v4(wrow + swz(r, 2 * cw + c), o[0], o[1], o[2], o[3]);
+                }
+                const uint32_t hrow = smem_u32(sH + hh * 16384);
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) pk[jj] = pack_bf16(h[hh][8 * c + 2 * jj], h[hh][8 * c + 2 * jj + 1]);
+                    st_shared_v4(hrow + swz(r, 2 * cw + c), pk[0], pk[1], pk[2], pk[3]);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty_x[kHeadsB - 1]);
+            if (lane == 0) {
+                mbar_arrive(&ops_ready);
+                mbar_arrive(&empty_x[0]);
+                mbar_arrive(&empty_x[1]);
+            }
+            // -------- while the UMMAs run: scan the next chunk
+            if (it + 1 < ntiles) scan_chunk(it + 1);
+            // -------- drain: y rows and the state update, both heads
+            wait_abort(&mma_done, it & 1, abort_p);
+            tc_fence_after();
+#pragma unroll
+            for (int hh = 0; hh < kHeadsB; ++hh) {
+                const float et = fast_exp2(ac2[bf][hh][r]);
+                const float Dh = hh == 0 ? Dh0 : Dh1;
+                uint32_t ry[16], rz[16];
+                tmem_ld16(tY + hh * 64 + lane_off + 16 * cw, ry);
+                tmem_ld16(tZ + hh * 64 + lane_off + 16 * cw, rz);
+                tmem_wait_ld();
+                uint32_t o[8];
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    const float2 xf = bf16x2_to_f2(xk[hh][jj]);
+                    const float v0 = fmaf(et, __uint_as_float(rz[2 * jj]), __uint_as_float(ry[2 * jj])) + Dh * xf.x;
+                    const float v1 = fmaf(et, __uint_as_float(rz[2 * jj + 1]), __uint_as_float(ry[2 * jj + 1])) + Dh * xf.y;
+                    o[jj] = pack_bf16(v0, v1);
+                }
+                if (r < tl) {
+                    uint4* dst = reinterpret_cast<uint4*>(y + ((t0 + r) * H + h0 + hh) * kP + 16 * cw);
+                    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+                    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+                }
+                uint32_t rs[16];
+                tmem_ld16(tS + hh * 64 + lane_off + 16 * cw, rs);
+                tmem_wait_ld();
+                const float decay = fast_exp2(ac2[bf][hh][kTile - 1]);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) h[hh][j] = fmaf(decay, h[hh][j], __uint_as_float(rs[j]));
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&acc_free);
+                mbar_arrive(&dt_free[bf]);
+            }
         }
     }
     tc_fence_before();
