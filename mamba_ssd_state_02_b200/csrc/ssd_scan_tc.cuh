@@ -303,9 +303,11 @@ k_tc_segment_passing(float* __restrict__ seg_state, const float* __restrict__ se
 // Per chunk: CB = C B^T (UMMA) -> the compute warps build M for both heads into TMEM,
 // write w*X and bf16 h for both heads to shared memory -> one UMMA batch: Z = C [h0|h1]^T
 // and S = B^T [wX0|wX1] (N = 128 each, so C and B are read once for both heads), then
-// Y_hh = M_hh X_hh -> the compute warps drain y and update h. While that batch runs,
-// warpgroups 0 and 1 scan dt*A of the next chunk into the other half of a double
-// buffer, and x stays in registers from the w*X step to the D x term.
+// Y_hh = M_hh X_hh -> the compute warps drain y and update h. Once a batch is issued
+// the UMMA warp scans dt*A of the next chunk into the other half of a double buffer
+// (its dt_raw loads were issued a chunk earlier); x stays in registers from the w*X
+// step to the D x term; the compute warps release the C B^T / Z columns as soon as Z
+// is read, so the next chunk's C B^T overlaps the rest of the drain.
 // TMEM: Z (cols 0..127, first holds C B^T), S (128..255), Y0, Y1 (256..383), M0, M1
 // (384..511). Shared memory: one C/B stage (reloaded as soon as the Z/S UMMAs are done),
 // one X slot per head, bf16 h and w*X for both heads.
@@ -331,9 +333,8 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
     uint8_t* sH = sm + 98304;               // head hh block at hh*16384: [128 n][64 p]  bf16 h_in
     uint8_t* sW = sm + 131072;              // head hh block at hh*16384: [128 s][64 p]  w * X
     __shared__ float ac2[2][kHeadsB][kTile], dts[2][kHeadsB][kTile], uw[2][kHeadsB][kTile], ww[2][kHeadsB][kTile];
-    __shared__ float part[kHeadsB][4];
     __shared__ uint64_t full_cb, empty_cb, full_x[kHeadsB], empty_x[kHeadsB], cb_done, ops_ready, mma_done,
-        acc_free, dt_ready[2], dt_free[2];
+        z_free, dt_ready[2];
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
 
@@ -352,11 +353,8 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
         mbar_init(&cb_done, 1);
         mbar_init(&ops_ready, kComputeWarps);
         mbar_init(&mma_done, 1);
-        mbar_init(&acc_free, kComputeWarps);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&dt_ready[i], 8);
-            mbar_init(&dt_free[i], kComputeWarps);
-        }
+        mbar_init(&z_free, kComputeWarps);
+        for (int i = 0; i < 2; ++i) mbar_init(&dt_ready[i], 32);
         abort_flag = 0;
         fence_barrier_init();
         prefetch_tmap(&map_x);
@@ -401,9 +399,65 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
         const uint64_t dBm = smem_desc(smem_u32(sB), 16384, 1024);
         const uint64_t dH = smem_desc(smem_u32(sH), 16384, 1024), dW = smem_desc(smem_u32(sW), 16384, 1024);
         const uint64_t dX0 = smem_desc(smem_u32(sX), 16384, 1024), dX1 = desc_add(dX0, 16384);
+        // dt scan of one chunk by this warp: lane l owns tokens 4l..4l+3 of both heads.
+        const float bias0 = dt_bias[h0], bias1 = dt_bias[h0 + 1], A0 = A[h0], A1 = A[h0 + 1];
+        if (lane == 0 && (!(A0 <= 0.f) || isinf(A0) || !(A1 <= 0.f) || isinf(A1))) latch_error(SSD_ERR_INVALID_ARG);
+        float zr[kHeadsB][4];
+        auto load_dt = [&](int j) {
+            const int64_t tj = seg.start + (int64_t)j * kTile;
+            const int tlj = min(kTile, seg.len - j * kTile);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int t = 4 * lane + e;
+                zr[0][e] = t < tlj ? dt_raw[(tj + t) * H + h0] : 0.f;
+                zr[1][e] = t < tlj ? dt_raw[(tj + t) * H + h0 + 1] : 0.f;
+            }
+        };
+        auto scan_chunk = [&](int j) {
+            const int bf = j & 1;
+            const int tlj = min(kTile, seg.len - j * kTile);
+#pragma unroll
+            for (int hh = 0; hh < kHeadsB; ++hh) {
+                const float bias = hh ? bias1 : bias0, Ah = hh ? A1 : A0;
+                float dtv[4], cum[4], run = 0.f;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    dtv[e] = (4 * lane + e) < tlj ? softplus_f32(zr[hh][e] + bias) : 0.f;
+                    run += dtv[e] * Ah;
+                    cum[e] = run;
+                }
+                float incl = run;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float v = __shfl_up_sync(0xffffffffu, incl, off);
+                    if (lane >= off) incl += v;
+                }
+                const float excl = incl - run;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    ac2[bf][hh][4 * lane + e] = (excl + cum[e]) * kLog2e;
+                    dts[bf][hh][4 * lane + e] = dtv[e];
+                }
+            }
+            __syncwarp();
+#pragma unroll
+            for (int hh = 0; hh < kHeadsB; ++hh) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int t = 4 * lane + e;
+                    const float av = ac2[bf][hh][t];
+                    uw[bf][hh][t] = fast_exp2(ac2[bf][hh][t | 31] - av) * dts[bf][hh][t];
+                    ww[bf][hh][t] = fast_exp2(ac2[bf][hh][kTile - 1] - av) * dts[bf][hh][t];
+                }
+            }
+            mbar_arrive(&dt_ready[bf]);
+        };
+        load_dt(0);
+        scan_chunk(0);
+        if (ntiles > 1) load_dt(1);
         for (int it = 0; it < ntiles; ++it) {
             wait_abort(&full_cb, it & 1, abort_p);
-            if (it >= 1) wait_abort(&acc_free, (it - 1) & 1, abort_p);
+            if (it >= 1) wait_abort(&z_free, (it - 1) & 1, abort_p);
             tc_fence_after();
             if (elect_one()) {
 #pragma unroll
@@ -432,6 +486,12 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 umma_commit(&empty_x[1]);
             }
             __syncwarp();
+            // Chunk it+1's decay arrays: its buffer was last read by chunk it-1's drain,
+            // which finished before ops_ready(it) completed.
+            if (it + 1 < ntiles) {
+                scan_chunk(it + 1);
+                if (it + 2 < ntiles) load_dt(it + 2);
+            }
         }
     } else {
         // ------------------------------------------------------------ compute warpgroups
@@ -454,40 +514,7 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             }
         }
         const float Dh0 = D[h0], Dh1 = D[h0 + 1];
-        const int hc = cw & 1;
-        const float bias_c = dt_bias[h0 + hc], A_c = A[h0 + hc];
-        if (cw < kHeadsB && r == 0 && (!(A_c <= 0.f) || isinf(A_c))) latch_error(SSD_ERR_INVALID_ARG);
 
-        // dt, log2-scaled cumulative dt*A and the decay weights of chunk j (warpgroups 0
-        // and 1, one head each) into buffer j & 1.
-        auto scan_chunk = [&](int j) {
-            if (cw >= kHeadsB) return;
-            const int bf = j & 1;
-            if (j >= 2) wait_abort(&dt_free[bf], ((j - 2) >> 1) & 1, abort_p);
-            const int64_t tj = seg.start + (int64_t)j * kTile;
-            const int tlj = min(kTile, seg.len - j * kTile);
-            const float dtv = r < tlj ? softplus_f32(dt_raw[(tj + r) * H + h0 + cw] + bias_c) : 0.f;
-            float a = dtv * A_c;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float v = __shfl_up_sync(0xffffffffu, a, off);
-                if (lane >= off) a += v;
-            }
-            if (lane == 31) part[cw][q] = a;
-            wg_bar(cw);
-            float pre = 0.f;
-            for (int w = 0; w < q; ++w) pre += part[cw][w];
-            const float av = (a + pre) * kLog2e;
-            ac2[bf][cw][r] = av;
-            dts[bf][cw][r] = dtv;
-            wg_bar(cw);
-            uw[bf][cw][r] = fast_exp2(ac2[bf][cw][r | 31] - av) * dtv;
-            ww[bf][cw][r] = fast_exp2(ac2[bf][cw][kTile - 1] - av) * dtv;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&dt_ready[bf]);
-        };
-
-        scan_chunk(0);
         for (int it = 0; it < ntiles; ++it) {
             const int64_t t0 = seg.start + (int64_t)it * kTile;
             const int tl = min(kTile, seg.len - it * kTile);
@@ -497,39 +524,43 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             tc_fence_after();
             // -------- M[t][s] of both heads, t = r, s in source block cw -> TMEM
             {
-                uint32_t rc[32];
                 const bool live = cw <= q;             // blocks above the diagonal are zero
-                if (live) {
-                    tmem_ld32(tCB + lane_off + 32 * cw, rc);
-                    tmem_wait_ld();
-                }
 #pragma unroll
-                for (int hh = 0; hh < kHeadsB; ++hh) {
-                    const float* ac = ac2[bf][hh];
-                    const float at = ac[r];
-                    uint32_t pk[16];
-                    if (!live) {
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) pk[k] = 0u;
-                    } else if (cw < q) {
-                        const float v = fast_exp2(at - ac[32 * cw + 31]);
-                        const float* u = uw[bf][hh] + 32 * cw;
-#pragma unroll
-                        for (int k = 0; k < 16; ++k)
-                            pk[k] = pack_bf16(__uint_as_float(rc[2 * k]) * v * u[2 * k],
-                                              __uint_as_float(rc[2 * k + 1]) * v * u[2 * k + 1]);
-                    } else {
-                        const float* dv = dts[bf][hh] + 32 * cw;
-                        const float* as = ac + 32 * cw;
-#pragma unroll
-                        for (int k = 0; k < 16; ++k) {
-                            const int s0 = 32 * cw + 2 * k;
-                            const float m0 = s0 <= r ? __uint_as_float(rc[2 * k]) * fast_exp2(at - as[2 * k]) * dv[2 * k] : 0.f;
-                            const float m1 = s0 + 1 <= r ? __uint_as_float(rc[2 * k + 1]) * fast_exp2(at - as[2 * k + 1]) * dv[2 * k + 1] : 0.f;
-                            pk[k] = pack_bf16(m0, m1);
-                        }
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t rc[16];
+                    if (live) {
+                        tmem_ld16(tCB + lane_off + 32 * cw + 16 * half, rc);
+                        tmem_wait_ld();
                     }
-                    tmem_st16(tM + hh * 64 + lane_off + 16 * cw, pk);
+#pragma unroll
+                    for (int hh = 0; hh < kHeadsB; ++hh) {
+                        const float* ac = ac2[bf][hh];
+                        const float at = ac[r];
+                        const int sb = 32 * cw + 16 * half;    // first source column of this half
+                        uint32_t pk[8];
+                        if (!live) {
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) pk[k] = 0u;
+                        } else if (cw < q) {
+                            const float v = fast_exp2(at - ac[32 * cw + 31]);
+                            const float* u = uw[bf][hh] + sb;
+#pragma unroll
+                            for (int k = 0; k < 8; ++k)
+                                pk[k] = pack_bf16(__uint_as_float(rc[2 * k]) * v * u[2 * k],
+                                                  __uint_as_float(rc[2 * k + 1]) * v * u[2 * k + 1]);
+                        } else {
+                            const float* dv = dts[bf][hh] + sb;
+                            const float* as = ac + sb;
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) {
+                                const int s0 = sb + 2 * k;
+                                const float m0 = s0 <= r ? __uint_as_float(rc[2 * k]) * fast_exp2(at - as[2 * k]) * dv[2 * k] : 0.f;
+                                const float m1 = s0 + 1 <= r ? __uint_as_float(rc[2 * k + 1]) * fast_exp2(at - as[2 * k + 1]) * dv[2 * k + 1] : 0.f;
+                                pk[k] = pack_bf16(m0, m1);
+                            }
+                        }
+                        tmem_st8(tM + hh * 64 + lane_off + 16 * cw + 8 * half, pk);
+                    }
                 }
                 tmem_wait_st();
             }
@@ -572,9 +603,7 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 mbar_arrive(&empty_x[0]);
                 mbar_arrive(&empty_x[1]);
             }
-            // -------- while the UMMAs run: scan the next chunk
-            if (it + 1 < ntiles) scan_chunk(it + 1);
-            // -------- drain: y rows and the state update, both heads
+            // -------- drain: y rows (then release the Z columns), then the state update
             wait_abort(&mma_done, it & 1, abort_p);
             tc_fence_after();
 #pragma unroll
@@ -598,18 +627,18 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                     dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
                     dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
                 }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&z_free);
+#pragma unroll
+            for (int hh = 0; hh < kHeadsB; ++hh) {
                 uint32_t rs[16];
                 tmem_ld16(tS + hh * 64 + lane_off + 16 * cw, rs);
                 tmem_wait_ld();
                 const float decay = fast_exp2(ac2[bf][hh][kTile - 1]);
 #pragma unroll
                 for (int j = 0; j < 16; ++j) h[hh][j] = fmaf(decay, h[hh][j], __uint_as_float(rs[j]));
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&acc_free);
-                mbar_arrive(&dt_free[bf]);
             }
         }
     }
