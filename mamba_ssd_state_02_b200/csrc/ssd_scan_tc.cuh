@@ -305,16 +305,14 @@ k_tc_segment_passing(float* __restrict__ seg_state, const float* __restrict__ se
 // and S = B^T [wX0|wX1] (N = 128 each, so C and B are read once for both heads), then
 // Y_hh = M_hh X_hh -> the compute warps drain y and update h. Once a batch is issued
 // the UMMA warp scans dt*A of the next chunk into the other half of a double buffer
-// (its dt_raw loads were issued a chunk earlier); x stays in registers from the w*X
-// step to the D x term; the compute warps release the C B^T / Z columns as soon as Z
-// is read, so the next chunk's C B^T overlaps the rest of the drain.
+// (its dt_raw loads were issued a chunk earlier); the compute warps release the
+// C B^T / Z columns as soon as Z is read, so the next chunk's C B^T overlaps the rest
+// of the drain.
 // TMEM: Z (cols 0..127, first holds C B^T), S (128..255), Y0, Y1 (256..383), M0, M1
 // (384..511). Shared memory: one C/B stage (reloaded as soon as the Z/S UMMAs are done),
 // one X slot per head, bf16 h and w*X for both heads.
 constexpr int kHeadsB = 2;
 constexpr int kSmemB = 160 * 1024 + 1024;
-
-__device__ __forceinline__ void wg_bar(int cw) { asm volatile("bar.sync %0, 128;" ::"r"(2 + cw) : "memory"); }
 
 __global__ void __launch_bounds__(kThreadsTc, 1)
 k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
@@ -564,8 +562,7 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 }
                 tmem_wait_st();
             }
-            // -------- w*X and bf16 h of both heads; x kept for the D x term
-            uint32_t xk[kHeadsB][8];
+            // -------- w*X and bf16 h of both heads
 #pragma unroll
             for (int hh = 0; hh < kHeadsB; ++hh) {
                 wait_abort(&full_x[hh], it & 1, abort_p);
@@ -574,14 +571,11 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     const uint4 v = ld_shared_v4(xrow + swz(r, 2 * cw + c));
-                    xk[hh][4 * c] = v.x;
-                    xk[hh][4 * c + 1] = v.y;
-                    xk[hh][4 * c + 2] = v.z;
-                    xk[hh][4 * c + 3] = v.w;
+                    const uint32_t xin[4] = {v.x, v.y, v.z, v.w};
                     uint32_t o[4];
 #pragma unroll
                     for (int jj = 0; jj < 4; ++jj) {
-                        const float2 f = bf16x2_to_f2(xk[hh][4 * c + jj]);
+                        const float2 f = bf16x2_to_f2(xin[jj]);
                         o[jj] = pack_bf16(f.x * w, f.y * w);
                     }
                     st_shared_v4(wrow + swz(r, 2 * cw + c), o[0], o[1], o[2], o[3]);
@@ -598,11 +592,7 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&ops_ready);
-                mbar_arrive(&empty_x[0]);
-                mbar_arrive(&empty_x[1]);
-            }
+            if (lane == 0) mbar_arrive(&ops_ready);
             // -------- drain: y rows (then release the Z columns), then the state update
             wait_abort(&mma_done, it & 1, abort_p);
             tc_fence_after();
@@ -610,17 +600,23 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             for (int hh = 0; hh < kHeadsB; ++hh) {
                 const float et = fast_exp2(ac2[bf][hh][r]);
                 const float Dh = hh == 0 ? Dh0 : Dh1;
-                uint32_t ry[16], rz[16];
-                tmem_ld16(tY + hh * 64 + lane_off + 16 * cw, ry);
-                tmem_ld16(tZ + hh * 64 + lane_off + 16 * cw, rz);
-                tmem_wait_ld();
+                const uint32_t xrow = smem_u32(sX + hh * 16384);
                 uint32_t o[8];
 #pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
-                    const float2 xf = bf16x2_to_f2(xk[hh][jj]);
-                    const float v0 = fmaf(et, __uint_as_float(rz[2 * jj]), __uint_as_float(ry[2 * jj])) + Dh * xf.x;
-                    const float v1 = fmaf(et, __uint_as_float(rz[2 * jj + 1]), __uint_as_float(ry[2 * jj + 1])) + Dh * xf.y;
-                    o[jj] = pack_bf16(v0, v1);
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t ry[8], rz[8];
+                    tmem_ld8(tY + hh * 64 + lane_off + 16 * cw + 8 * half, ry);
+                    tmem_ld8(tZ + hh * 64 + lane_off + 16 * cw + 8 * half, rz);
+                    const uint4 xa = ld_shared_v4(xrow + swz(r, 2 * cw + half));
+                    const uint32_t xk[4] = {xa.x, xa.y, xa.z, xa.w};
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const float2 xf = bf16x2_to_f2(xk[jj]);
+                        const float v0 = fmaf(et, __uint_as_float(rz[2 * jj]), __uint_as_float(ry[2 * jj])) + Dh * xf.x;
+                        const float v1 = fmaf(et, __uint_as_float(rz[2 * jj + 1]), __uint_as_float(ry[2 * jj + 1])) + Dh * xf.y;
+                        o[4 * half + jj] = pack_bf16(v0, v1);
+                    }
                 }
                 if (r < tl) {
                     uint4* dst = reinterpret_cast<uint4*>(y + ((t0 + r) * H + h0 + hh) * kP + 16 * cw);
@@ -630,7 +626,11 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&z_free);
+            if (lane == 0) {
+                mbar_arrive(&z_free);
+                mbar_arrive(&empty_x[0]);          // x of both heads read for the last time
+                mbar_arrive(&empty_x[1]);
+            }
 #pragma unroll
             for (int hh = 0; hh < kHeadsB; ++hh) {
                 uint32_t rs[16];
