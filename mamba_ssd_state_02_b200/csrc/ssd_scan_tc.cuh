@@ -303,9 +303,9 @@ k_tc_segment_passing(float* __restrict__ seg_state, const float* __restrict__ se
 // Per chunk: CB = C B^T (UMMA) -> the compute warps build M for both heads into TMEM,
 // write w*X and bf16 h for both heads to shared memory -> one UMMA batch: Z = C [h0|h1]^T
 // and S = B^T [wX0|wX1] (N = 128 each, so C and B are read once for both heads), then
-// Y_hh = M_hh X_hh -> the compute warps drain y and update h. Once a batch is issued
-// the UMMA warp scans dt*A of the next chunk into the other half of a double buffer
-// (its dt_raw loads were issued a chunk earlier); the compute warps release the
+// Y_hh = M_hh X_hh -> the compute warps drain y and update h. While a batch runs,
+// warpgroups 0 and 1 scan dt*A of the next chunk into the other half of a double
+// buffer (its dt_raw was loaded a chunk earlier); the compute warps release the
 // C B^T / Z columns as soon as Z is read, so the next chunk's C B^T overlaps the rest
 // of the drain.
 // TMEM: Z (cols 0..127, first holds C B^T), S (128..255), Y0, Y1 (256..383), M0, M1
@@ -331,6 +331,7 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
     uint8_t* sH = sm + 98304;               // head hh block at hh*16384: [128 n][64 p]  bf16 h_in
     uint8_t* sW = sm + 131072;              // head hh block at hh*16384: [128 s][64 p]  w * X
     __shared__ float ac2[2][kHeadsB][kTile], dts[2][kHeadsB][kTile], uw[2][kHeadsB][kTile], ww[2][kHeadsB][kTile];
+    __shared__ float part[kHeadsB][4];
     __shared__ uint64_t full_cb, empty_cb, full_x[kHeadsB], empty_x[kHeadsB], cb_done, ops_ready, mma_done,
         z_free, dt_ready[2];
     __shared__ uint32_t tmem_slot;
@@ -352,7 +353,7 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
         mbar_init(&ops_ready, kComputeWarps);
         mbar_init(&mma_done, 1);
         mbar_init(&z_free, kComputeWarps);
-        for (int i = 0; i < 2; ++i) mbar_init(&dt_ready[i], 32);
+        for (int i = 0; i < 2; ++i) mbar_init(&dt_ready[i], 8);
         abort_flag = 0;
         fence_barrier_init();
         prefetch_tmap(&map_x);
@@ -397,62 +398,6 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
         const uint64_t dBm = smem_desc(smem_u32(sB), 16384, 1024);
         const uint64_t dH = smem_desc(smem_u32(sH), 16384, 1024), dW = smem_desc(smem_u32(sW), 16384, 1024);
         const uint64_t dX0 = smem_desc(smem_u32(sX), 16384, 1024), dX1 = desc_add(dX0, 16384);
-        // dt scan of one chunk by this warp: lane l owns tokens 4l..4l+3 of both heads.
-        const float bias0 = dt_bias[h0], bias1 = dt_bias[h0 + 1], A0 = A[h0], A1 = A[h0 + 1];
-        if (lane == 0 && (!(A0 <= 0.f) || isinf(A0) || !(A1 <= 0.f) || isinf(A1))) latch_error(SSD_ERR_INVALID_ARG);
-        float zr[kHeadsB][4];
-        auto load_dt = [&](int j) {
-            const int64_t tj = seg.start + (int64_t)j * kTile;
-            const int tlj = min(kTile, seg.len - j * kTile);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int t = 4 * lane + e;
-                zr[0][e] = t < tlj ? dt_raw[(tj + t) * H + h0] : 0.f;
-                zr[1][e] = t < tlj ? dt_raw[(tj + t) * H + h0 + 1] : 0.f;
-            }
-        };
-        auto scan_chunk = [&](int j) {
-            const int bf = j & 1;
-            const int tlj = min(kTile, seg.len - j * kTile);
-#pragma unroll
-            for (int hh = 0; hh < kHeadsB; ++hh) {
-                const float bias = hh ? bias1 : bias0, Ah = hh ? A1 : A0;
-                float dtv[4], cum[4], run = 0.f;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    dtv[e] = (4 * lane + e) < tlj ? softplus_f32(zr[hh][e] + bias) : 0.f;
-                    run += dtv[e] * Ah;
-                    cum[e] = run;
-                }
-                float incl = run;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const float v = __shfl_up_sync(0xffffffffu, incl, off);
-                    if (lane >= off) incl += v;
-                }
-                const float excl = incl - run;
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    ac2[bf][hh][4 * lane + e] = (excl + cum[e]) * kLog2e;
-                    dts[bf][hh][4 * lane + e] = dtv[e];
-                }
-            }
-            __syncwarp();
-#pragma unroll
-            for (int hh = 0; hh < kHeadsB; ++hh) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int t = 4 * lane + e;
-                    const float av = ac2[bf][hh][t];
-                    uw[bf][hh][t] = fast_exp2(ac2[bf][hh][t | 31] - av) * dts[bf][hh][t];
-                    ww[bf][hh][t] = fast_exp2(ac2[bf][hh][kTile - 1] - av) * dts[bf][hh][t];
-                }
-            }
-            mbar_arrive(&dt_ready[bf]);
-        };
-        load_dt(0);
-        scan_chunk(0);
-        if (ntiles > 1) load_dt(1);
         for (int it = 0; it < ntiles; ++it) {
             wait_abort(&full_cb, it & 1, abort_p);
             if (it >= 1) wait_abort(&z_free, (it - 1) & 1, abort_p);
@@ -484,12 +429,6 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 umma_commit(&empty_x[1]);
             }
             __syncwarp();
-            // Chunk it+1's decay arrays: its buffer was last read by chunk it-1's drain,
-            // which finished before ops_ready(it) completed.
-            if (it + 1 < ntiles) {
-                scan_chunk(it + 1);
-                if (it + 2 < ntiles) load_dt(it + 2);
-            }
         }
     } else {
         // ------------------------------------------------------------ compute warpgroups
@@ -512,6 +451,43 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             }
         }
         const float Dh0 = D[h0], Dh1 = D[h0 + 1];
+        const int hc = cw & 1;                      // head scanned by warpgroup cw (cw < 2)
+        const float bias_c = dt_bias[h0 + hc], A_c = A[h0 + hc];
+        if (cw < kHeadsB && r == 0 && (!(A_c <= 0.f) || isinf(A_c))) latch_error(SSD_ERR_INVALID_ARG);
+        auto load_dt = [&](int j) -> float {        // dt_raw of token r of chunk j, head cw
+            const int tlj = min(kTile, seg.len - j * kTile);
+            return (cw < kHeadsB && r < tlj) ? dt_raw[((int64_t)seg.start + (int64_t)j * kTile + r) * H + h0 + hc] : 0.f;
+        };
+        // dt, log2-scaled cumulative dt*A and the decay weights of chunk j into buffer
+        // j & 1 (warpgroups 0 and 1, one head each; named barrier 2 + cw).
+        auto scan_chunk = [&](int j, float z) {
+            const int bf = j & 1;
+            const int tlj = min(kTile, seg.len - j * kTile);
+            const float dtv = r < tlj ? softplus_f32(z + bias_c) : 0.f;
+            float a = dtv * A_c;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float v = __shfl_up_sync(0xffffffffu, a, off);
+                if (lane >= off) a += v;
+            }
+            if (lane == 31) part[cw][q] = a;
+            asm volatile("bar.sync %0, 128;" ::"r"(2 + cw) : "memory");
+            float pre = 0.f;
+            for (int w = 0; w < q; ++w) pre += part[cw][w];
+            const float av = (a + pre) * kLog2e;
+            ac2[bf][cw][r] = av;
+            dts[bf][cw][r] = dtv;
+            asm volatile("bar.sync %0, 128;" ::"r"(2 + cw) : "memory");
+            uw[bf][cw][r] = fast_exp2(ac2[bf][cw][r | 31] - av) * dtv;
+            ww[bf][cw][r] = fast_exp2(ac2[bf][cw][kTile - 1] - av) * dtv;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&dt_ready[bf]);
+        };
+        float zn = 0.f;                             // prefetched dt_raw of the next chunk to scan
+        if (cw < kHeadsB) {
+            scan_chunk(0, load_dt(0));
+            if (ntiles > 1) zn = load_dt(1);
+        }
 
         for (int it = 0; it < ntiles; ++it) {
             const int64_t t0 = seg.start + (int64_t)it * kTile;
@@ -593,6 +569,13 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&ops_ready);
+            // -------- while the UMMAs run: warpgroups 0/1 scan the next chunk. Its buffer
+            // was last read by chunk it-1's drain, done once ops_ready(it) has completed.
+            if (cw < kHeadsB && it + 1 < ntiles) {
+                wait_abort(&ops_ready, it & 1, abort_p);
+                scan_chunk(it + 1, zn);
+                if (it + 2 < ntiles) zn = load_dt(it + 2);
+            }
             // -------- drain: y rows (then release the Z columns), then the state update
             wait_abort(&mma_done, it & 1, abort_p);
             tc_fence_after();
