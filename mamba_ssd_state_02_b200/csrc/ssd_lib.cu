@@ -304,12 +304,13 @@ ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_ra
     }
     ++n;
     if (pl.max_segs > 0 && pl.T > 0) {
-        CUtensorMap mx, mb, mc;
+        CUtensorMap mx, mb, mc, my;
         const uint64_t T = (uint64_t)pl.T;
         if (!make_map3(&mx, x, tc::kP, H, T, (uint64_t)tc::kP * 2, (uint64_t)H * tc::kP * 2, 64, 1, tc::kTile) ||
             !make_map3(&mb, B, tc::kN, G, T, (uint64_t)tc::kN * 2, (uint64_t)G * tc::kN * 2, 64, 1, tc::kTile) ||
-            !make_map3(&mc, C, tc::kN, G, T, (uint64_t)tc::kN * 2, (uint64_t)G * tc::kN * 2, 64, 1, tc::kTile))
-            return fail(SSD_ERR_CUDA, "cuTensorMapEncodeTiled failed (x/B/C tensor maps)");
+            !make_map3(&mc, C, tc::kN, G, T, (uint64_t)tc::kN * 2, (uint64_t)G * tc::kN * 2, 64, 1, tc::kTile) ||
+            !make_map3(&my, y, tc::kP, H, T, (uint64_t)tc::kP * 2, (uint64_t)H * tc::kP * 2, 64, 1, tc::kTile))
+            return fail(SSD_ERR_CUDA, "cuTensorMapEncodeTiled failed (x/B/C/y tensor maps)");
         cudaError_t e = cudaFuncSetAttribute(tc::k_tc_segment_state, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              tc::kSmemA);
         if (e == cudaSuccess)
@@ -330,7 +331,7 @@ ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_ra
         ++n;
         {
             StageScope sc(ST_CHUNK_SCAN, st);
-            tc::k_tc_chunk_scan<<<(unsigned)(pl.max_segs * (H / tc::kHeadsB)), tc::kThreadsTc, tc::kSmemB, st>>>(mx, mb, mc, dt_raw, dt_bias, A, D, table, count, H,
+            tc::k_tc_chunk_scan<<<(unsigned)(pl.max_segs * (H / tc::kHeadsB)), tc::kThreadsTc, tc::kSmemB, st>>>(mx, mb, mc, my, dt_raw, dt_bias, A, D, table, count, H,
                                                                G, seg_state, (__nv_bfloat16*)y);
         }
         ++n;

@@ -295,31 +295,40 @@ k_tc_segment_passing(float* __restrict__ seg_state, const float* __restrict__ se
 // ---------------------------------------------------------------------------------
 // Pass B: outputs y for one (segment, 2 heads), chunk by chunk.
 //
-// Warp 0 issues the TMA loads, warp 1 the UMMAs, and four compute warpgroups
-// (cw = 0..3) split every row's 64 columns in quarters (and the 128 source columns of
-// M in 32-wide blocks). Compute thread (cw, r) owns TMEM lane r = 32*(warp%4) + lane
-// and keeps the FP32 running state h[head][n = r][p in its quarter] in registers.
+// Warp 0 issues the TMA loads and the y stores, warp 1 the UMMAs, and four compute
+// warpgroups (cw = 0..3) split every row's 64 columns in quarters. Compute thread
+// (cw, r) owns TMEM lane r = 32*(warp%4) + lane and keeps the FP32 running state
+// h[head][n = r][p in its quarter] in registers.
 //
 // Per chunk: CB = C B^T (UMMA) -> the compute warps build M for both heads into TMEM,
 // write w*X and bf16 h for both heads to shared memory -> one UMMA batch: Z = C [h0|h1]^T
 // and S = B^T [wX0|wX1] (N = 128 each, so C and B are read once for both heads), then
-// Y_hh = M_hh X_hh -> the compute warps drain y and update h. While a batch runs,
-// warpgroups 0 and 1 scan dt*A of the next chunk into the other half of a double
-// buffer (its dt_raw was loaded a chunk earlier); the compute warps release the
-// C B^T / Z columns as soon as Z is read, so the next chunk's C B^T overlaps the rest
-// of the drain.
+// Y_hh = M_hh X_hh -> the compute warps drain y into the chunk's X slot (full chunks)
+// and update h; warp 0 stores the y tile with one TMA store per head. While a batch
+// runs, warpgroups 0 and 1 scan dt*A of the next chunk into one of three buffers (its
+// dt_raw was loaded a chunk earlier); the compute warps release the C B^T / Z columns
+// as soon as Z is read, so the next chunk's C B^T overlaps the rest of the drain.
+//
+// M of row block q (TMEM lane quarter q) has source blocks 0..q-1 below the diagonal,
+// written as CB * exp2(Acum_t - Acum_e) * exp2(Acum_e - Acum_s) dt_s with e the last
+// row of the source block (both exponents <= 0), the diagonal block written directly,
+// and zeros above. Warp (cw, q) takes block cw when cw != q and one 16-source slice of
+// the diagonal block (head cw & 1), so the exp-heavy diagonal is shared by the four
+// warps that own lane quarter q.
+//
 // TMEM: Z (cols 0..127, first holds C B^T), S (128..255), Y0, Y1 (256..383), M0, M1
 // (384..511). Shared memory: one C/B stage (reloaded as soon as the Z/S UMMAs are done),
-// one X slot per head, bf16 h and w*X for both heads.
+// two X slots per head (chunk j uses slot j & 1; its y tile replaces x there), bf16 h
+// and w*X for both heads.
 constexpr int kHeadsB = 2;
-constexpr int kSmemB = 160 * 1024 + 1024;
+constexpr int kSmemB = 192 * 1024 + 1024;
 
 __global__ void __launch_bounds__(kThreadsTc, 1)
 k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
-                const __grid_constant__ CUtensorMap map_c, const float* __restrict__ dt_raw,
-                const float* __restrict__ dt_bias, const float* __restrict__ A, const float* __restrict__ D,
-                const ChunkEntry* __restrict__ segs, const int32_t* __restrict__ nsegs, int H, int G,
-                const float* __restrict__ hin, __nv_bfloat16* __restrict__ y) {
+                const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_y,
+                const float* __restrict__ dt_raw, const float* __restrict__ dt_bias, const float* __restrict__ A,
+                const float* __restrict__ D, const ChunkEntry* __restrict__ segs, const int32_t* __restrict__ nsegs,
+                int H, int G, const float* __restrict__ hin, __nv_bfloat16* __restrict__ y) {
     const int nhp = H / kHeadsB;
     const int sg = blockIdx.x / nhp;
     if (sg >= *nsegs) return;
@@ -327,13 +336,16 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sC = sm;                       // [2][128 t][64 n]   K-major
     uint8_t* sB = sm + 32768;               // [2][128 s][64 n]   K-major for C B^T, MN-major for B^T
-    uint8_t* sX = sm + 65536;               // head hh at hh*16384: [128 s][64 p]
-    uint8_t* sH = sm + 98304;               // head hh block at hh*16384: [128 n][64 p]  bf16 h_in
-    uint8_t* sW = sm + 131072;              // head hh block at hh*16384: [128 s][64 p]  w * X
-    __shared__ float ac2[2][kHeadsB][kTile], dts[2][kHeadsB][kTile], uw[2][kHeadsB][kTile], ww[2][kHeadsB][kTile];
+    uint8_t* sX = sm + 65536;               // slot sl, head hh at sl*32768 + hh*16384: [128 s][64 p]
+    uint8_t* sH = sm + 131072;              // head hh block at hh*16384: [128 n][64 p]  bf16 h_in
+    uint8_t* sW = sm + 163840;              // head hh block at hh*16384: [128 s][64 p]  w * X
+    __shared__ __align__(16) float ac2[3][kHeadsB][kTile];
+    __shared__ __align__(16) float dts[3][kHeadsB][kTile];
+    __shared__ __align__(16) float uw[3][kHeadsB][kTile];
+    __shared__ __align__(16) float ww[3][kHeadsB][kTile];
     __shared__ float part[kHeadsB][4];
-    __shared__ uint64_t full_cb, empty_cb, full_x[kHeadsB], empty_x[kHeadsB], cb_done, ops_ready, mma_done,
-        z_free, dt_ready[2];
+    __shared__ uint64_t full_cb, empty_cb, full_x[2][kHeadsB], empty_x[2][kHeadsB], cb_done, ops_ready, mma_done,
+        z_free, dt_ready[3];
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
 
@@ -345,20 +357,22 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
     if (tid == 0) {
         mbar_init(&full_cb, 1);
         mbar_init(&empty_cb, 1);
-        for (int i = 0; i < kHeadsB; ++i) {
-            mbar_init(&full_x[i], 1);
-            mbar_init(&empty_x[i], 1 + kComputeWarps);
-        }
+        for (int sl = 0; sl < 2; ++sl)
+            for (int i = 0; i < kHeadsB; ++i) {
+                mbar_init(&full_x[sl][i], 1);
+                mbar_init(&empty_x[sl][i], kComputeWarps);
+            }
         mbar_init(&cb_done, 1);
         mbar_init(&ops_ready, kComputeWarps);
         mbar_init(&mma_done, 1);
         mbar_init(&z_free, kComputeWarps);
-        for (int i = 0; i < 2; ++i) mbar_init(&dt_ready[i], 8);
+        for (int i = 0; i < 3; ++i) mbar_init(&dt_ready[i], 8);
         abort_flag = 0;
         fence_barrier_init();
         prefetch_tmap(&map_x);
         prefetch_tmap(&map_b);
         prefetch_tmap(&map_c);
+        prefetch_tmap(&map_y);
     }
     if (warp == 1) {
         tmem_alloc(&tmem_slot, 512);
@@ -374,6 +388,17 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
+            // y tile of chunk j: once the compute warps have staged it in the chunk's X
+            // slot (full chunks only; a partial last chunk is written by the threads).
+            auto store_y = [&](int j) {
+                const int sl = j & 1;
+                for (int hh = 0; hh < kHeadsB; ++hh) wait_abort(&empty_x[sl][hh], (j >> 1) & 1, abort_p);
+                if (seg.len - j * kTile >= kTile) {
+                    for (int hh = 0; hh < kHeadsB; ++hh)
+                        tma_store_3d(&map_y, sX + sl * 32768 + hh * 16384, 0, h0 + hh, seg.start + j * kTile);
+                    bulk_commit_group();
+                }
+            };
             for (int it = 0; it < ntiles; ++it) {
                 const int t0 = seg.start + it * kTile;
                 if (it >= 1) wait_abort(&empty_cb, (it - 1) & 1, abort_p);
@@ -382,12 +407,18 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 tma_load_3d(sC + 16384, &map_c, &full_cb, 64, g, t0);
                 tma_load_3d(sB, &map_b, &full_cb, 0, g, t0);
                 tma_load_3d(sB + 16384, &map_b, &full_cb, 64, g, t0);
+                const int sl = it & 1;
+                if (it >= 2) {
+                    store_y(it - 2);
+                    bulk_wait_read_all();           // the slot is free once the store has read it
+                }
                 for (int hh = 0; hh < kHeadsB; ++hh) {
-                    if (it >= 1) wait_abort(&empty_x[hh], (it - 1) & 1, abort_p);
-                    mbar_arrive_expect_tx(&full_x[hh], 16384);
-                    tma_load_3d(sX + hh * 16384, &map_x, &full_x[hh], 0, h0 + hh, t0);
+                    mbar_arrive_expect_tx(&full_x[sl][hh], 16384);
+                    tma_load_3d(sX + sl * 32768 + hh * 16384, &map_x, &full_x[sl][hh], 0, h0 + hh, t0);
                 }
             }
+            for (int j = ntiles >= 2 ? ntiles - 2 : 0; j < ntiles; ++j) store_y(j);
+            bulk_wait_all();
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ UMMA issuer
@@ -397,7 +428,7 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
         const uint64_t dCk = smem_desc(smem_u32(sC), 16, 1024), dBk = smem_desc(smem_u32(sB), 16, 1024);
         const uint64_t dBm = smem_desc(smem_u32(sB), 16384, 1024);
         const uint64_t dH = smem_desc(smem_u32(sH), 16384, 1024), dW = smem_desc(smem_u32(sW), 16384, 1024);
-        const uint64_t dX0 = smem_desc(smem_u32(sX), 16384, 1024), dX1 = desc_add(dX0, 16384);
+        const uint64_t dX = smem_desc(smem_u32(sX), 16384, 1024);
         for (int it = 0; it < ntiles; ++it) {
             wait_abort(&full_cb, it & 1, abort_p);
             if (it >= 1) wait_abort(&z_free, (it - 1) & 1, abort_p);
@@ -411,6 +442,7 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             __syncwarp();
             wait_abort(&ops_ready, it & 1, abort_p);
             tc_fence_after();
+            const uint64_t dX0 = desc_add(dX, (it & 1) * 32768), dX1 = desc_add(dX0, 16384);
             if (elect_one()) {
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
@@ -425,8 +457,6 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 for (int k = 0; k < 8; ++k)
                     umma_bf16_ts(tY + 64, tM + 64 + 8 * k, desc_add(dX1, k * kMnStep), id_y, k > 0);
                 umma_commit(&mma_done);
-                umma_commit(&empty_x[0]);
-                umma_commit(&empty_x[1]);
             }
             __syncwarp();
         }
@@ -459,9 +489,9 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             return (cw < kHeadsB && r < tlj) ? dt_raw[((int64_t)seg.start + (int64_t)j * kTile + r) * H + h0 + hc] : 0.f;
         };
         // dt, log2-scaled cumulative dt*A and the decay weights of chunk j into buffer
-        // j & 1 (warpgroups 0 and 1, one head each; named barrier 2 + cw).
+        // j % 3 (warpgroups 0 and 1, one head each; named barrier 2 + cw).
         auto scan_chunk = [&](int j, float z) {
-            const int bf = j & 1;
+            const int bf = j % 3;
             const int tlj = min(kTile, seg.len - j * kTile);
             const float dtv = r < tlj ? softplus_f32(z + bias_c) : 0.f;
             float a = dtv * A_c;
@@ -492,58 +522,73 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
         for (int it = 0; it < ntiles; ++it) {
             const int64_t t0 = seg.start + (int64_t)it * kTile;
             const int tl = min(kTile, seg.len - it * kTile);
-            const int bf = it & 1;
-            wait_abort(&dt_ready[bf], (it >> 1) & 1, abort_p);
+            const int bf = it % 3, sl = it & 1;
+            uint8_t* sXs = sX + sl * 32768;
+            wait_abort(&dt_ready[bf], (it / 3) & 1, abort_p);
             wait_abort(&cb_done, it & 1, abort_p);
             tc_fence_after();
-            // -------- M[t][s] of both heads, t = r, s in source block cw -> TMEM
-            {
-                const bool live = cw <= q;             // blocks above the diagonal are zero
+            // -------- M[t][s] of both heads, t = r -> TMEM
+            if (cw < q) {                          // below the diagonal: factorized
+                float v[kHeadsB];
+#pragma unroll
+                for (int hh = 0; hh < kHeadsB; ++hh) v[hh] = fast_exp2(ac2[bf][hh][r] - ac2[bf][hh][32 * cw + 31]);
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t rc[16];
-                    if (live) {
-                        tmem_ld16(tCB + lane_off + 32 * cw + 16 * half, rc);
-                        tmem_wait_ld();
-                    }
+                    tmem_ld16(tCB + lane_off + 32 * cw + 16 * half, rc);
+                    tmem_wait_ld();
 #pragma unroll
                     for (int hh = 0; hh < kHeadsB; ++hh) {
-                        const float* ac = ac2[bf][hh];
-                        const float at = ac[r];
-                        const int sb = 32 * cw + 16 * half;    // first source column of this half
+                        const float4* u4 = reinterpret_cast<const float4*>(&uw[bf][hh][32 * cw + 16 * half]);
                         uint32_t pk[8];
-                        if (!live) {
 #pragma unroll
-                            for (int k = 0; k < 8; ++k) pk[k] = 0u;
-                        } else if (cw < q) {
-                            const float v = fast_exp2(at - ac[32 * cw + 31]);
-                            const float* u = uw[bf][hh] + sb;
-#pragma unroll
-                            for (int k = 0; k < 8; ++k)
-                                pk[k] = pack_bf16(__uint_as_float(rc[2 * k]) * v * u[2 * k],
-                                                  __uint_as_float(rc[2 * k + 1]) * v * u[2 * k + 1]);
-                        } else {
-                            const float* dv = dts[bf][hh] + sb;
-                            const float* as = ac + sb;
-#pragma unroll
-                            for (int k = 0; k < 8; ++k) {
-                                const int s0 = sb + 2 * k;
-                                const float m0 = s0 <= r ? __uint_as_float(rc[2 * k]) * fast_exp2(at - as[2 * k]) * dv[2 * k] : 0.f;
-                                const float m1 = s0 + 1 <= r ? __uint_as_float(rc[2 * k + 1]) * fast_exp2(at - as[2 * k + 1]) * dv[2 * k + 1] : 0.f;
-                                pk[k] = pack_bf16(m0, m1);
-                            }
+                        for (int k4 = 0; k4 < 4; ++k4) {
+                            const float4 u = u4[k4];
+                            pk[2 * k4] = pack_bf16(__uint_as_float(rc[4 * k4]) * (v[hh] * u.x),
+                                                   __uint_as_float(rc[4 * k4 + 1]) * (v[hh] * u.y));
+                            pk[2 * k4 + 1] = pack_bf16(__uint_as_float(rc[4 * k4 + 2]) * (v[hh] * u.z),
+                                                       __uint_as_float(rc[4 * k4 + 3]) * (v[hh] * u.w));
                         }
                         tmem_st8(tM + hh * 64 + lane_off + 16 * cw + 8 * half, pk);
                     }
                 }
-                tmem_wait_st();
+            } else if (cw > q) {                   // above the diagonal: zero
+                const uint32_t zero[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll
+                for (int hh = 0; hh < kHeadsB; ++hh) {
+                    tmem_st8(tM + hh * 64 + lane_off + 16 * cw, zero);
+                    tmem_st8(tM + hh * 64 + lane_off + 16 * cw + 8, zero);
+                }
             }
+            {                                       // diagonal slice: head cw & 1, 16 sources
+                const int hd = cw & 1, sd = 32 * q + 16 * (cw >> 1);
+                uint32_t rc[16];
+                tmem_ld16(tCB + lane_off + sd, rc);
+                tmem_wait_ld();
+                const float at = ac2[bf][hd][r];
+                const float4* a4 = reinterpret_cast<const float4*>(&ac2[bf][hd][sd]);
+                const float4* d4 = reinterpret_cast<const float4*>(&dts[bf][hd][sd]);
+                uint32_t pk[8];
+#pragma unroll
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const float4 as = a4[k4], dv = d4[k4];
+                    const int s0 = sd + 4 * k4;
+                    const float m0 = s0 <= r ? __uint_as_float(rc[4 * k4]) * fast_exp2(at - as.x) * dv.x : 0.f;
+                    const float m1 = s0 + 1 <= r ? __uint_as_float(rc[4 * k4 + 1]) * fast_exp2(at - as.y) * dv.y : 0.f;
+                    const float m2 = s0 + 2 <= r ? __uint_as_float(rc[4 * k4 + 2]) * fast_exp2(at - as.z) * dv.z : 0.f;
+                    const float m3 = s0 + 3 <= r ? __uint_as_float(rc[4 * k4 + 3]) * fast_exp2(at - as.w) * dv.w : 0.f;
+                    pk[2 * k4] = pack_bf16(m0, m1);
+                    pk[2 * k4 + 1] = pack_bf16(m2, m3);
+                }
+                tmem_st8(tM + hd * 64 + lane_off + (sd >> 1), pk);
+            }
+            tmem_wait_st();
             // -------- w*X and bf16 h of both heads
 #pragma unroll
             for (int hh = 0; hh < kHeadsB; ++hh) {
-                wait_abort(&full_x[hh], it & 1, abort_p);
+                wait_abort(&full_x[sl][hh], (it >> 1) & 1, abort_p);
                 const float w = ww[bf][hh][r];
-                const uint32_t xrow = smem_u32(sX + hh * 16384), wrow = smem_u32(sW + hh * 16384);
+                const uint32_t xrow = smem_u32(sXs + hh * 16384), wrow = smem_u32(sW + hh * 16384);
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     const uint4 v = ld_shared_v4(xrow + swz(r, 2 * cw + c));
@@ -570,49 +615,61 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             __syncwarp();
             if (lane == 0) mbar_arrive(&ops_ready);
             // -------- while the UMMAs run: warpgroups 0/1 scan the next chunk. Its buffer
-            // was last read by chunk it-1's drain, done once ops_ready(it) has completed.
+            // (of three) was last read by chunk it-2's drain, which every warp finished
+            // before this warp could pass chunk it-1's mma_done wait.
             if (cw < kHeadsB && it + 1 < ntiles) {
-                wait_abort(&ops_ready, it & 1, abort_p);
                 scan_chunk(it + 1, zn);
                 if (it + 2 < ntiles) zn = load_dt(it + 2);
             }
-            // -------- drain: y rows (then release the Z columns), then the state update
+            // -------- drain: y rows (into the X slot for a full chunk, else straight to
+            // HBM), then release the Z columns and the slot, then the state update. The
+            // TMEM loads of the next 8-column piece are issued before the current one
+            // is consumed.
             wait_abort(&mma_done, it & 1, abort_p);
             tc_fence_after();
+            {
+                const bool staged = tl == kTile;
+                uint32_t ry[2][8], rz[2][8];
+                tmem_ld8(tY + lane_off + 16 * cw, ry[0]);
+                tmem_ld8(tZ + lane_off + 16 * cw, rz[0]);
+                const float et0 = fast_exp2(ac2[bf][0][r]), et1 = fast_exp2(ac2[bf][1][r]);
 #pragma unroll
-            for (int hh = 0; hh < kHeadsB; ++hh) {
-                const float et = fast_exp2(ac2[bf][hh][r]);
-                const float Dh = hh == 0 ? Dh0 : Dh1;
-                const uint32_t xrow = smem_u32(sX + hh * 16384);
-                uint32_t o[8];
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t ry[8], rz[8];
-                    tmem_ld8(tY + hh * 64 + lane_off + 16 * cw + 8 * half, ry);
-                    tmem_ld8(tZ + hh * 64 + lane_off + 16 * cw + 8 * half, rz);
-                    const uint4 xa = ld_shared_v4(xrow + swz(r, 2 * cw + half));
-                    const uint32_t xk[4] = {xa.x, xa.y, xa.z, xa.w};
+                for (int piece = 0; piece < 4; ++piece) {           // (head, half) = (piece/2, piece%2)
+                    const int hh = piece >> 1, half = piece & 1, cur = piece & 1;
                     tmem_wait_ld();
+                    if (piece < 3) {
+                        const int nh = (piece + 1) >> 1, nf = (piece + 1) & 1;
+                        tmem_ld8(tY + nh * 64 + lane_off + 16 * cw + 8 * nf, ry[cur ^ 1]);
+                        tmem_ld8(tZ + nh * 64 + lane_off + 16 * cw + 8 * nf, rz[cur ^ 1]);
+                    }
+                    const float et = hh ? et1 : et0;
+                    const float Dh = hh ? Dh1 : Dh0;
+                    const uint32_t xa = smem_u32(sXs + hh * 16384) + swz(r, 2 * cw + half);
+                    const uint4 xv = ld_shared_v4(xa);
+                    const uint32_t xk[4] = {xv.x, xv.y, xv.z, xv.w};
+                    uint32_t o[4];
 #pragma unroll
                     for (int jj = 0; jj < 4; ++jj) {
                         const float2 xf = bf16x2_to_f2(xk[jj]);
-                        const float v0 = fmaf(et, __uint_as_float(rz[2 * jj]), __uint_as_float(ry[2 * jj])) + Dh * xf.x;
-                        const float v1 = fmaf(et, __uint_as_float(rz[2 * jj + 1]), __uint_as_float(ry[2 * jj + 1])) + Dh * xf.y;
-                        o[4 * half + jj] = pack_bf16(v0, v1);
+                        const float v0 = fmaf(et, __uint_as_float(rz[cur][2 * jj]), __uint_as_float(ry[cur][2 * jj])) + Dh * xf.x;
+                        const float v1 = fmaf(et, __uint_as_float(rz[cur][2 * jj + 1]), __uint_as_float(ry[cur][2 * jj + 1])) + Dh * xf.y;
+                        o[jj] = pack_bf16(v0, v1);
+                    }
+                    if (staged) {
+                        st_shared_v4(xa, o[0], o[1], o[2], o[3]);
+                    } else if (r < tl) {
+                        *reinterpret_cast<uint4*>(y + ((t0 + r) * H + h0 + hh) * kP + 16 * cw + 8 * half) =
+                            make_uint4(o[0], o[1], o[2], o[3]);
                     }
                 }
-                if (r < tl) {
-                    uint4* dst = reinterpret_cast<uint4*>(y + ((t0 + r) * H + h0 + hh) * kP + 16 * cw);
-                    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-                    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
-                }
             }
+            fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(&z_free);
-                mbar_arrive(&empty_x[0]);          // x of both heads read for the last time
-                mbar_arrive(&empty_x[1]);
+                mbar_arrive(&empty_x[sl][0]);       // y staged, x of both heads read for the last time
+                mbar_arrive(&empty_x[sl][1]);
             }
 #pragma unroll
             for (int hh = 0; hh < kHeadsB; ++hh) {
