@@ -52,7 +52,7 @@ __device__ __forceinline__ void compute_bar() { asm volatile("bar.sync 1, 512;" 
 __device__ __forceinline__ void wait_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
     if (mbar_try_wait(bar, parity)) return;
     const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_sleep(bar, parity)) {
         if (*abort_flag) return;
         if (clock64() - t0 > kWaitBudgetCycles) {
             latch_error(SSD_ERR_TIMEOUT);
@@ -300,28 +300,30 @@ k_tc_segment_passing(float* __restrict__ seg_state, const float* __restrict__ se
 // (cw, r) owns TMEM lane r = 32*(warp%4) + lane and keeps the FP32 running state
 // h[head][n = r][p in its quarter] in registers.
 //
-// Per chunk: CB = C B^T (UMMA) -> the compute warps build M for both heads into TMEM,
-// write w*X and bf16 h for both heads to shared memory -> one UMMA batch: Z = C [h0|h1]^T
-// and S = B^T [wX0|wX1] (N = 128 each, so C and B are read once for both heads), then
-// Y_hh = M_hh X_hh -> the compute warps drain y into the chunk's X slot (full chunks)
-// and update h; warp 0 stores the y tile with one TMA store per head. While a batch
-// runs, warpgroups 0 and 1 scan dt*A of the next chunk into one of three buffers (its
-// dt_raw was loaded a chunk earlier); the compute warps release the C B^T / Z columns
-// as soon as Z is read, so the next chunk's C B^T overlaps the rest of the drain.
+// Per chunk: CB = C B^T (UMMA, into the M columns) -> the compute warps turn it into M
+// for both heads in place, write w*X and bf16 h for both heads to shared memory -> one
+// UMMA batch: Z = C [h0|h1]^T and S = B^T [wX0|wX1] (N = 128 each, so C and B are read
+// once for both heads), then Y_hh = M_hh X_hh -> the compute warps drain y into the
+// chunk's X slot (full chunks) and update h; warp 0 stores the y tile with one TMA
+// store per head. As soon as the Y UMMAs have read M, the UMMA warp issues the next
+// chunk's C B^T, which overlaps the drain. While a batch runs, warpgroups 0 and 1 scan
+// dt*A of the chunk after next into one of four buffers (its dt_raw was loaded a chunk
+// earlier), and warpgroups 2 and 3 tabulate the next chunk's diagonal-block decays.
 //
 // M of row block q (TMEM lane quarter q) has source blocks 0..q-1 below the diagonal,
 // written as CB * exp2(Acum_t - Acum_e) * exp2(Acum_e - Acum_s) dt_s with e the last
-// row of the source block (both exponents <= 0), the diagonal block written directly,
-// and zeros above. Warp (cw, q) takes block cw when cw != q and one 16-source slice of
-// the diagonal block (head cw & 1), so the exp-heavy diagonal is shared by the four
-// warps that own lane quarter q.
+// row of the source block (both exponents <= 0), the diagonal block as CB times the
+// tabulated exp2(Acum_t - Acum_s) dt_s (fp16, shared memory), and zeros above. Warp
+// (cw, q) takes block cw when cw != q and one 16-source slice of the diagonal block
+// (head cw & 1).
 //
-// TMEM: Z (cols 0..127, first holds C B^T), S (128..255), Y0, Y1 (256..383), M0, M1
-// (384..511). Shared memory: one C/B stage (reloaded as soon as the Z/S UMMAs are done),
-// two X slots per head (chunk j uses slot j & 1; its y tile replaces x there), bf16 h
-// and w*X for both heads.
+// TMEM: Z (cols 0..127), S (128..255), Y0, Y1 (256..383), C B^T then M (384..511; M of
+// head hh for sources 16k..16k+15 in columns 384 + 16k + 8hh). Shared memory: one C/B
+// stage (reloaded as soon as the Z/S UMMAs are done), two X slots per head (chunk j
+// uses slot j & 1; its y tile replaces x there), bf16 h and w*X for both heads, the
+// diagonal-block decay table (16 KB).
 constexpr int kHeadsB = 2;
-constexpr int kSmemB = 192 * 1024 + 1024;
+constexpr int kSmemB = 208 * 1024 + 1024;
 
 __global__ void __launch_bounds__(kThreadsTc, 1)
 k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
@@ -339,13 +341,14 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
     uint8_t* sX = sm + 65536;               // slot sl, head hh at sl*32768 + hh*16384: [128 s][64 p]
     uint8_t* sH = sm + 131072;              // head hh block at hh*16384: [128 n][64 p]  bf16 h_in
     uint8_t* sW = sm + 163840;              // head hh block at hh*16384: [128 s][64 p]  w * X
-    __shared__ __align__(16) float ac2[3][kHeadsB][kTile];
-    __shared__ __align__(16) float dts[3][kHeadsB][kTile];
-    __shared__ __align__(16) float uw[3][kHeadsB][kTile];
-    __shared__ __align__(16) float ww[3][kHeadsB][kTile];
+    uint8_t* sL = sm + 196608;              // head hh at hh*8192: [128 t][32] fp16 diagonal-block decays
+    __shared__ __align__(16) float ac2[4][kHeadsB][kTile];
+    __shared__ __align__(16) float dts[4][kHeadsB][kTile];
+    __shared__ __align__(16) float uw[4][kHeadsB][kTile];
+    __shared__ __align__(16) float ww[4][kHeadsB][kTile];
     __shared__ float part[kHeadsB][4];
     __shared__ uint64_t full_cb, empty_cb, full_x[2][kHeadsB], empty_x[2][kHeadsB], cb_done, ops_ready, mma_done,
-        z_free, dt_ready[3];
+        l_ready, dt_ready[4];
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
 
@@ -365,8 +368,8 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
         mbar_init(&cb_done, 1);
         mbar_init(&ops_ready, kComputeWarps);
         mbar_init(&mma_done, 1);
-        mbar_init(&z_free, kComputeWarps);
-        for (int i = 0; i < 3; ++i) mbar_init(&dt_ready[i], 8);
+        for (int i = 0; i < 4; ++i) mbar_init(&dt_ready[i], 8);
+        mbar_init(&l_ready, 8);
         abort_flag = 0;
         fence_barrier_init();
         prefetch_tmap(&map_x);
@@ -382,7 +385,7 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = tmem_slot;
-    const uint32_t tZ = tbase, tCB = tbase, tS = tbase + 128, tY = tbase + 256, tM = tbase + 384;
+    const uint32_t tZ = tbase, tS = tbase + 128, tY = tbase + 256, tM = tbase + 384;
     volatile int* abort_p = &abort_flag;
 
     if (warp == 0) {
@@ -429,17 +432,20 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
         const uint64_t dBm = smem_desc(smem_u32(sB), 16384, 1024);
         const uint64_t dH = smem_desc(smem_u32(sH), 16384, 1024), dW = smem_desc(smem_u32(sW), 16384, 1024);
         const uint64_t dX = smem_desc(smem_u32(sX), 16384, 1024);
-        for (int it = 0; it < ntiles; ++it) {
-            wait_abort(&full_cb, it & 1, abort_p);
-            if (it >= 1) wait_abort(&z_free, (it - 1) & 1, abort_p);
+        // C B^T of chunk j into the M columns (fp32), once its C/B tiles have landed.
+        auto issue_cb = [&](int j) {
+            wait_abort(&full_cb, j & 1, abort_p);
             tc_fence_after();
             if (elect_one()) {
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    umma_bf16(tCB, desc_add(dCk, kmajor_step(128, k)), desc_add(dBk, kmajor_step(128, k)), id_cb, k > 0);
+                    umma_bf16(tM, desc_add(dCk, kmajor_step(128, k)), desc_add(dBk, kmajor_step(128, k)), id_cb, k > 0);
                 umma_commit(&cb_done);
             }
             __syncwarp();
+        };
+        if (ntiles > 0) issue_cb(0);
+        for (int it = 0; it < ntiles; ++it) {
             wait_abort(&ops_ready, it & 1, abort_p);
             tc_fence_after();
             const uint64_t dX0 = desc_add(dX, (it & 1) * 32768), dX1 = desc_add(dX0, 16384);
@@ -451,14 +457,19 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 for (int k = 0; k < 8; ++k)
                     umma_bf16(tS, desc_add(dBm, k * kMnStep), desc_add(dW, k * kMnStep), id_s, k > 0);
                 umma_commit(&empty_cb);
+                // M of head hh, sources 16k..16k+15: TMEM columns 16k + 8hh of the M block.
 #pragma unroll
-                for (int k = 0; k < 8; ++k) umma_bf16_ts(tY, tM + 8 * k, desc_add(dX0, k * kMnStep), id_y, k > 0);
+                for (int k = 0; k < 8; ++k) umma_bf16_ts(tY, tM + 16 * k, desc_add(dX0, k * kMnStep), id_y, k > 0);
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    umma_bf16_ts(tY + 64, tM + 64 + 8 * k, desc_add(dX1, k * kMnStep), id_y, k > 0);
+                    umma_bf16_ts(tY + 64, tM + 16 * k + 8, desc_add(dX1, k * kMnStep), id_y, k > 0);
                 umma_commit(&mma_done);
             }
             __syncwarp();
+            if (it + 1 < ntiles) {
+                wait_abort(&mma_done, it & 1, abort_p);     // the Y UMMAs have read M
+                issue_cb(it + 1);
+            }
         }
     } else {
         // ------------------------------------------------------------ compute warpgroups
@@ -489,9 +500,9 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             return (cw < kHeadsB && r < tlj) ? dt_raw[((int64_t)seg.start + (int64_t)j * kTile + r) * H + h0 + hc] : 0.f;
         };
         // dt, log2-scaled cumulative dt*A and the decay weights of chunk j into buffer
-        // j % 3 (warpgroups 0 and 1, one head each; named barrier 2 + cw).
+        // j % 4 (warpgroups 0 and 1, one head each; named barrier 2 + cw).
         auto scan_chunk = [&](int j, float z) {
-            const int bf = j % 3;
+            const int bf = j % 4;
             const int tlj = min(kTile, seg.len - j * kTile);
             const float dtv = r < tlj ? softplus_f32(z + bias_c) : 0.f;
             float a = dtv * A_c;
@@ -513,29 +524,89 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             __syncwarp();
             if (lane == 0) mbar_arrive(&dt_ready[bf]);
         };
+        // Decays of the diagonal 32x32 blocks of chunk j, L[t][s] = exp2(Acum_t - Acum_s)
+        // dt_s for s <= t in t's block (fp16, row t = r of head cw - 2; warpgroups 2, 3).
+        // 16-byte chunk c of row t sits at chunk c ^ ((t >> 1) & 3).
+        auto diag_decays = [&](int j) {
+            const int bf = j % 4, hd = cw - kHeadsB;
+            wait_abort(&dt_ready[bf], (j / 4) & 1, abort_p);
+            const float at = ac2[bf][hd][r];
+            const float4* a4 = reinterpret_cast<const float4*>(&ac2[bf][hd][32 * q]);
+            const float4* d4 = reinterpret_cast<const float4*>(&dts[bf][hd][32 * q]);
+            const uint32_t row = smem_u32(sL + hd * 8192 + r * 64);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t o[4];
+#pragma unroll
+                for (int k2 = 0; k2 < 2; ++k2) {
+                    const float4 as = a4[2 * c + k2], dv = d4[2 * c + k2];
+                    const int s0 = 8 * c + 4 * k2;          // source offset within the block
+                    const float l0 = s0 <= lane ? fast_exp2(at - as.x) * dv.x : 0.f;
+                    const float l1 = s0 + 1 <= lane ? fast_exp2(at - as.y) * dv.y : 0.f;
+                    const float l2 = s0 + 2 <= lane ? fast_exp2(at - as.z) * dv.z : 0.f;
+                    const float l3 = s0 + 3 <= lane ? fast_exp2(at - as.w) * dv.w : 0.f;
+                    o[2 * k2] = pack_f16(l0, l1);
+                    o[2 * k2 + 1] = pack_f16(l2, l3);
+                }
+                st_shared_v4(row + ((c ^ ((r >> 1) & 3)) << 4), o[0], o[1], o[2], o[3]);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&l_ready);
+        };
         float zn = 0.f;                             // prefetched dt_raw of the next chunk to scan
         if (cw < kHeadsB) {
             scan_chunk(0, load_dt(0));
-            if (ntiles > 1) zn = load_dt(1);
+            if (ntiles > 1) scan_chunk(1, load_dt(1));
+            if (ntiles > 2) zn = load_dt(2);
+        } else {
+            diag_decays(0);
         }
 
         for (int it = 0; it < ntiles; ++it) {
             const int64_t t0 = seg.start + (int64_t)it * kTile;
             const int tl = min(kTile, seg.len - it * kTile);
-            const int bf = it % 3, sl = it & 1;
+            const int bf = it % 4, sl = it & 1;
             uint8_t* sXs = sX + sl * 32768;
-            wait_abort(&dt_ready[bf], (it / 3) & 1, abort_p);
+            wait_abort(&dt_ready[bf], (it / 4) & 1, abort_p);
+            wait_abort(&l_ready, it & 1, abort_p);
             wait_abort(&cb_done, it & 1, abort_p);
             tc_fence_after();
-            // -------- M[t][s] of both heads, t = r -> TMEM
-            if (cw < q) {                          // below the diagonal: factorized
-                float v[kHeadsB];
+            // -------- M[t][s] of both heads, t = r, in place over C B^T. Source block b
+            // (32 sources) keeps its 32 columns: half j (sources 16j..16j+15 of the
+            // block) becomes M of head 0 in its first 8 columns and of head 1 in the
+            // next 8. First the diagonal slice: head cw & 1, half cw >> 1 of block q;
+            // the four warps of lane quarter q read their C B^T slices before any of
+            // them overwrites the block (named barrier 4 + q).
+            {
+                const int hd = cw & 1, sd = 32 * q + 16 * (cw >> 1);
+                uint32_t rc[16];
+                tmem_ld16(tM + lane_off + sd, rc);
+                tmem_wait_ld();
+                asm volatile("bar.sync %0, 128;" ::"r"(4 + q) : "memory");
+                const uint32_t lrow = smem_u32(sL + hd * 8192 + r * 64);
+                const int c0 = 2 * (cw >> 1);
+                const uint4 la = ld_shared_v4(lrow + ((c0 ^ ((r >> 1) & 3)) << 4));
+                const uint4 lb = ld_shared_v4(lrow + (((c0 + 1) ^ ((r >> 1) & 3)) << 4));
+                const uint32_t lw[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
+                uint32_t pk[8];
 #pragma unroll
-                for (int hh = 0; hh < kHeadsB; ++hh) v[hh] = fast_exp2(ac2[bf][hh][r] - ac2[bf][hh][32 * cw + 31]);
+                for (int k = 0; k < 8; ++k)
+                    pk[k] = pack_bf16(fmul2(f16x2_to_f2(lw[k]),
+                                            make_float2(__uint_as_float(rc[2 * k]), __uint_as_float(rc[2 * k + 1]))));
+                tmem_st8(tM + lane_off + sd + 8 * hd, pk);
+            }
+            if (cw < q) {                          // below the diagonal: factorized
+                float2 v[kHeadsB];
+#pragma unroll
+                for (int hh = 0; hh < kHeadsB; ++hh) {
+                    const float vv = fast_exp2(ac2[bf][hh][r] - ac2[bf][hh][32 * cw + 31]);
+                    v[hh] = make_float2(vv, vv);
+                }
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
+                    const uint32_t col = lane_off + 32 * cw + 16 * half;
                     uint32_t rc[16];
-                    tmem_ld16(tCB + lane_off + 32 * cw + 16 * half, rc);
+                    tmem_ld16(tM + col, rc);
                     tmem_wait_ld();
 #pragma unroll
                     for (int hh = 0; hh < kHeadsB; ++hh) {
@@ -544,43 +615,20 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
 #pragma unroll
                         for (int k4 = 0; k4 < 4; ++k4) {
                             const float4 u = u4[k4];
-                            pk[2 * k4] = pack_bf16(__uint_as_float(rc[4 * k4]) * (v[hh] * u.x),
-                                                   __uint_as_float(rc[4 * k4 + 1]) * (v[hh] * u.y));
-                            pk[2 * k4 + 1] = pack_bf16(__uint_as_float(rc[4 * k4 + 2]) * (v[hh] * u.z),
-                                                       __uint_as_float(rc[4 * k4 + 3]) * (v[hh] * u.w));
+                            const float2 m01 = fmul2(make_float2(__uint_as_float(rc[4 * k4]), __uint_as_float(rc[4 * k4 + 1])),
+                                                     fmul2(v[hh], make_float2(u.x, u.y)));
+                            const float2 m23 = fmul2(make_float2(__uint_as_float(rc[4 * k4 + 2]), __uint_as_float(rc[4 * k4 + 3])),
+                                                     fmul2(v[hh], make_float2(u.z, u.w)));
+                            pk[2 * k4] = pack_bf16(m01);
+                            pk[2 * k4 + 1] = pack_bf16(m23);
                         }
-                        tmem_st8(tM + hh * 64 + lane_off + 16 * cw + 8 * half, pk);
+                        tmem_st8(tM + col + 8 * hh, pk);
                     }
                 }
             } else if (cw > q) {                   // above the diagonal: zero
                 const uint32_t zero[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
 #pragma unroll
-                for (int hh = 0; hh < kHeadsB; ++hh) {
-                    tmem_st8(tM + hh * 64 + lane_off + 16 * cw, zero);
-                    tmem_st8(tM + hh * 64 + lane_off + 16 * cw + 8, zero);
-                }
-            }
-            {                                       // diagonal slice: head cw & 1, 16 sources
-                const int hd = cw & 1, sd = 32 * q + 16 * (cw >> 1);
-                uint32_t rc[16];
-                tmem_ld16(tCB + lane_off + sd, rc);
-                tmem_wait_ld();
-                const float at = ac2[bf][hd][r];
-                const float4* a4 = reinterpret_cast<const float4*>(&ac2[bf][hd][sd]);
-                const float4* d4 = reinterpret_cast<const float4*>(&dts[bf][hd][sd]);
-                uint32_t pk[8];
-#pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
-                    const float4 as = a4[k4], dv = d4[k4];
-                    const int s0 = sd + 4 * k4;
-                    const float m0 = s0 <= r ? __uint_as_float(rc[4 * k4]) * fast_exp2(at - as.x) * dv.x : 0.f;
-                    const float m1 = s0 + 1 <= r ? __uint_as_float(rc[4 * k4 + 1]) * fast_exp2(at - as.y) * dv.y : 0.f;
-                    const float m2 = s0 + 2 <= r ? __uint_as_float(rc[4 * k4 + 2]) * fast_exp2(at - as.z) * dv.z : 0.f;
-                    const float m3 = s0 + 3 <= r ? __uint_as_float(rc[4 * k4 + 3]) * fast_exp2(at - as.w) * dv.w : 0.f;
-                    pk[2 * k4] = pack_bf16(m0, m1);
-                    pk[2 * k4 + 1] = pack_bf16(m2, m3);
-                }
-                tmem_st8(tM + hd * 64 + lane_off + (sd >> 1), pk);
+                for (int c8 = 0; c8 < 4; ++c8) tmem_st8(tM + lane_off + 32 * cw + 8 * c8, zero);
             }
             tmem_wait_st();
             // -------- w*X and bf16 h of both heads
@@ -588,18 +636,13 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             for (int hh = 0; hh < kHeadsB; ++hh) {
                 wait_abort(&full_x[sl][hh], (it >> 1) & 1, abort_p);
                 const float w = ww[bf][hh][r];
+                const uint32_t w2 = pack_bf16(w, w);
                 const uint32_t xrow = smem_u32(sXs + hh * 16384), wrow = smem_u32(sW + hh * 16384);
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     const uint4 v = ld_shared_v4(xrow + swz(r, 2 * cw + c));
-                    const uint32_t xin[4] = {v.x, v.y, v.z, v.w};
-                    uint32_t o[4];
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        const float2 f = bf16x2_to_f2(xin[jj]);
-                        o[jj] = pack_bf16(f.x * w, f.y * w);
-                    }
-                    st_shared_v4(wrow + swz(r, 2 * cw + c), o[0], o[1], o[2], o[3]);
+                    st_shared_v4(wrow + swz(r, 2 * cw + c), hmul2_bf16(v.x, w2), hmul2_bf16(v.y, w2),
+                                 hmul2_bf16(v.z, w2), hmul2_bf16(v.w, w2));
                 }
                 const uint32_t hrow = smem_u32(sH + hh * 16384);
 #pragma unroll
@@ -614,17 +657,23 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&ops_ready);
-            // -------- while the UMMAs run: warpgroups 0/1 scan the next chunk. Its buffer
-            // (of three) was last read by chunk it-2's drain, which every warp finished
-            // before this warp could pass chunk it-1's mma_done wait.
-            if (cw < kHeadsB && it + 1 < ntiles) {
-                scan_chunk(it + 1, zn);
-                if (it + 2 < ntiles) zn = load_dt(it + 2);
+            // -------- while the UMMAs run: warpgroups 0/1 scan chunk it+2. Its buffer (of
+            // four) was last read by chunk it-2's drain, which every warp finished before
+            // this warp could pass chunk it-1's mma_done wait. Warpgroups 2/3 write the
+            // diagonal-block decays of chunk it+1 once every warp has finished reading
+            // those of chunk it (ops_ready complete).
+            if (cw < kHeadsB) {
+                if (it + 2 < ntiles) {
+                    scan_chunk(it + 2, zn);
+                    if (it + 3 < ntiles) zn = load_dt(it + 3);
+                }
+            } else if (it + 1 < ntiles) {
+                wait_abort(&ops_ready, it & 1, abort_p);
+                diag_decays(it + 1);
             }
             // -------- drain: y rows (into the X slot for a full chunk, else straight to
-            // HBM), then release the Z columns and the slot, then the state update. The
-            // TMEM loads of the next 8-column piece are issued before the current one
-            // is consumed.
+            // HBM), then release the slot, then the state update. The TMEM loads of the
+            // next 8-column piece are issued before the current one is consumed.
             wait_abort(&mma_done, it & 1, abort_p);
             tc_fence_after();
             {
@@ -633,6 +682,8 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 tmem_ld8(tY + lane_off + 16 * cw, ry[0]);
                 tmem_ld8(tZ + lane_off + 16 * cw, rz[0]);
                 const float et0 = fast_exp2(ac2[bf][0][r]), et1 = fast_exp2(ac2[bf][1][r]);
+                const float2 e20 = make_float2(et0, et0), e21 = make_float2(et1, et1);
+                const float2 d20 = make_float2(Dh0, Dh0), d21 = make_float2(Dh1, Dh1);
 #pragma unroll
                 for (int piece = 0; piece < 4; ++piece) {           // (head, half) = (piece/2, piece%2)
                     const int hh = piece >> 1, half = piece & 1, cur = piece & 1;
@@ -642,8 +693,8 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                         tmem_ld8(tY + nh * 64 + lane_off + 16 * cw + 8 * nf, ry[cur ^ 1]);
                         tmem_ld8(tZ + nh * 64 + lane_off + 16 * cw + 8 * nf, rz[cur ^ 1]);
                     }
-                    const float et = hh ? et1 : et0;
-                    const float Dh = hh ? Dh1 : Dh0;
+                    const float2 et = hh ? e21 : e20;
+                    const float2 Dh = hh ? d21 : d20;
                     const uint32_t xa = smem_u32(sXs + hh * 16384) + swz(r, 2 * cw + half);
                     const uint4 xv = ld_shared_v4(xa);
                     const uint32_t xk[4] = {xv.x, xv.y, xv.z, xv.w};
@@ -651,9 +702,9 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
 #pragma unroll
                     for (int jj = 0; jj < 4; ++jj) {
                         const float2 xf = bf16x2_to_f2(xk[jj]);
-                        const float v0 = fmaf(et, __uint_as_float(rz[cur][2 * jj]), __uint_as_float(ry[cur][2 * jj])) + Dh * xf.x;
-                        const float v1 = fmaf(et, __uint_as_float(rz[cur][2 * jj + 1]), __uint_as_float(ry[cur][2 * jj + 1])) + Dh * xf.y;
-                        o[jj] = pack_bf16(v0, v1);
+                        const float2 zy = ffma2(et, make_float2(__uint_as_float(rz[cur][2 * jj]), __uint_as_float(rz[cur][2 * jj + 1])),
+                                                make_float2(__uint_as_float(ry[cur][2 * jj]), __uint_as_float(ry[cur][2 * jj + 1])));
+                        o[jj] = pack_bf16(ffma2(Dh, xf, zy));
                     }
                     if (staged) {
                         st_shared_v4(xa, o[0], o[1], o[2], o[3]);
@@ -667,7 +718,6 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&z_free);
                 mbar_arrive(&empty_x[sl][0]);       // y staged, x of both heads read for the last time
                 mbar_arrive(&empty_x[sl][1]);
             }
@@ -677,8 +727,14 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 tmem_ld16(tS + hh * 64 + lane_off + 16 * cw, rs);
                 tmem_wait_ld();
                 const float decay = fast_exp2(ac2[bf][hh][kTile - 1]);
+                const float2 dc = make_float2(decay, decay);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) h[hh][j] = fmaf(decay, h[hh][j], __uint_as_float(rs[j]));
+                for (int j = 0; j < 16; j += 2) {
+                    const float2 hn = ffma2(dc, make_float2(h[hh][j], h[hh][j + 1]),
+                                            make_float2(__uint_as_float(rs[j]), __uint_as_float(rs[j + 1])));
+                    h[hh][j] = hn.x;
+                    h[hh][j + 1] = hn.y;
+                }
             }
         }
     }
