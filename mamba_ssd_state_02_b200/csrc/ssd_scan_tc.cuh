@@ -191,7 +191,7 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
             {
                 const float Ah = A[h0 + cw];
                 if (r == 0 && k == 0 && (!(Ah <= 0.f) || isinf(Ah))) latch_error(SSD_ERR_INVALID_ARG);
-                const float dtv = r < tl ? softplus_f32(dt_raw[(t0 + r) * H + h0 + cw] + dt_bias[h0 + cw]) : 0.f;
+                const float dtv = r < tl ? softplus_fast(dt_raw[(t0 + r) * H + h0 + cw] + dt_bias[h0 + cw]) : 0.f;
                 compute_bar();              // previous tile's weights no longer read
                 const float incl = wg_scan(dtv * Ah, q, lane, part[cw]) * kLog2e;
                 if (r == kTile - 1) tile_tot[cw] = incl;
@@ -300,32 +300,36 @@ k_tc_segment_passing(float* __restrict__ seg_state, const float* __restrict__ se
 // (cw, r) owns TMEM lane r = 32*(warp%4) + lane and keeps the FP32 running state
 // h[head][n = r][p in its quarter] in registers.
 //
-// Per chunk: CB = C B^T (UMMA, into the M columns) -> the compute warps turn it into M
-// for both heads in place, write w*X and bf16 h for both heads to shared memory -> one
-// UMMA batch: Z = C [h0|h1]^T and S = B^T [wX0|wX1] (N = 128 each, so C and B are read
-// once for both heads), then Y_hh = M_hh X_hh -> the compute warps drain y into the
-// chunk's X slot (full chunks) and update h; warp 0 stores the y tile with one TMA
-// store per head. As soon as the Y UMMAs have read M, the UMMA warp issues the next
-// chunk's C B^T, which overlaps the drain. While a batch runs, warpgroups 0 and 1 scan
-// dt*A of the chunk after next into one of four buffers (its dt_raw was loaded a chunk
-// earlier), and warpgroups 2 and 3 tabulate the next chunk's diagonal-block decays.
+// Per chunk j: CB = C B^T (UMMA, into the M columns) -> the compute warps turn it into
+// M for both heads in place (D_h joins M on the diagonal, so y = M X + exp(Acum_t) Z
+// carries the skip term) -> UMMA batch: S = B^T [wX0|wX1] then Z = C [h0|h1]^T (N = 128
+// each, so C and B are read once for both heads), then Y_hh = M_hh X_hh. When S is done
+// the compute warps write w*X of chunk j+1; when Z is done they update h and write bf16
+// h of chunk j+1 (while the Y UMMAs run); when Y is done they drain y into the chunk's
+// X slot (full chunks) and warp 0 stores the tile with one TMA store per head, then
+// loads chunk j+2's X into the slot (prefetched into L2 a chunk earlier). The UMMA warp
+// issues chunk j+1's C B^T as soon as the Y UMMAs have read M, so it overlaps the
+// drain. Warp 18 scans dt*A up to four chunks ahead; while S and Z run, warpgroups 2
+// and 3 tabulate chunk j+1's diagonal-block decays.
 //
 // M of row block q (TMEM lane quarter q) has source blocks 0..q-1 below the diagonal,
 // written as CB * exp2(Acum_t - Acum_e) * exp2(Acum_e - Acum_s) dt_s with e the last
 // row of the source block (both exponents <= 0), the diagonal block as CB times the
 // tabulated exp2(Acum_t - Acum_s) dt_s (fp16, shared memory), and zeros above. Warp
-// (cw, q) takes block cw when cw != q and one 16-source slice of the diagonal block
-// (head cw & 1).
+// (cw, q) takes block cw when cw != q; the warps with cw >= q share the diagonal block
+// by 16-source halves.
 //
 // TMEM: Z (cols 0..127), S (128..255), Y0, Y1 (256..383), C B^T then M (384..511; M of
 // head hh for sources 16k..16k+15 in columns 384 + 16k + 8hh). Shared memory: one C/B
-// stage (reloaded as soon as the Z/S UMMAs are done), two X slots per head (chunk j
-// uses slot j & 1; its y tile replaces x there), bf16 h and w*X for both heads, the
-// diagonal-block decay table (16 KB).
+// stage (reloaded as soon as the Z/S UMMAs are done), two X slots (chunk j uses slot
+// j & 1; its y tile replaces x there), bf16 h and w*X for both heads, the diagonal-block
+// decay table (16 KB).
 constexpr int kHeadsB = 2;
 constexpr int kSmemB = 208 * 1024 + 1024;
+constexpr int kScanWarp = kRoleWarps + kComputeWarps;          // warp 18: dt scan
+constexpr int kThreadsB = 32 * (kScanWarp + 1);
 
-__global__ void __launch_bounds__(kThreadsTc, 1)
+__global__ void __launch_bounds__(kThreadsB, 1)
 k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
                 const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_y,
                 const float* __restrict__ dt_raw, const float* __restrict__ dt_bias, const float* __restrict__ A,
@@ -346,9 +350,8 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
     __shared__ __align__(16) float dts[4][kHeadsB][kTile];
     __shared__ __align__(16) float uw[4][kHeadsB][kTile];
     __shared__ __align__(16) float ww[4][kHeadsB][kTile];
-    __shared__ float part[kHeadsB][4];
-    __shared__ uint64_t full_cb, empty_cb, full_x[2][kHeadsB], empty_x[2][kHeadsB], cb_done, ops_ready, mma_done,
-        l_ready, dt_ready[4];
+    __shared__ uint64_t full_cb, s_done, zs_done, full_x[2], cb_done, ops_ready, mma_done, l_ready, dt_ready[4],
+        dt_free[4], y_staged;
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
 
@@ -359,16 +362,17 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
 
     if (tid == 0) {
         mbar_init(&full_cb, 1);
-        mbar_init(&empty_cb, 1);
-        for (int sl = 0; sl < 2; ++sl)
-            for (int i = 0; i < kHeadsB; ++i) {
-                mbar_init(&full_x[sl][i], 1);
-                mbar_init(&empty_x[sl][i], kComputeWarps);
-            }
+        mbar_init(&s_done, 1);
+        mbar_init(&zs_done, 1);
+        for (int sl = 0; sl < 2; ++sl) mbar_init(&full_x[sl], 1);
+        mbar_init(&y_staged, kComputeWarps);
         mbar_init(&cb_done, 1);
         mbar_init(&ops_ready, kComputeWarps);
         mbar_init(&mma_done, 1);
-        for (int i = 0; i < 4; ++i) mbar_init(&dt_ready[i], 8);
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(&dt_ready[i], 1);
+            mbar_init(&dt_free[i], kComputeWarps);
+        }
         mbar_init(&l_ready, 8);
         abort_flag = 0;
         fence_barrier_init();
@@ -391,36 +395,52 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            // y tile of chunk j: once the compute warps have staged it in the chunk's X
-            // slot (full chunks only; a partial last chunk is written by the threads).
-            auto store_y = [&](int j) {
+            auto load_x = [&](int j) {              // X of chunk j (both heads) into slot j & 1
                 const int sl = j & 1;
-                for (int hh = 0; hh < kHeadsB; ++hh) wait_abort(&empty_x[sl][hh], (j >> 1) & 1, abort_p);
-                if (seg.len - j * kTile >= kTile) {
-                    for (int hh = 0; hh < kHeadsB; ++hh)
-                        tma_store_3d(&map_y, sX + sl * 32768 + hh * 16384, 0, h0 + hh, seg.start + j * kTile);
-                    bulk_commit_group();
-                }
+                mbar_arrive_expect_tx(&full_x[sl], 32768);
+                for (int hh = 0; hh < kHeadsB; ++hh)
+                    tma_load_3d(sX + sl * 32768 + hh * 16384, &map_x, &full_x[sl], 0, h0 + hh, seg.start + j * kTile);
             };
-            for (int it = 0; it < ntiles; ++it) {
-                const int t0 = seg.start + it * kTile;
-                if (it >= 1) wait_abort(&empty_cb, (it - 1) & 1, abort_p);
+            // C and B of chunk j; those of chunk j+1 and X of chunk j+1 are prefetched into
+            // L2 meanwhile, so the loads that follow find them there.
+            auto load_cb = [&](int j) {
+                const int t0 = seg.start + j * kTile;
                 mbar_arrive_expect_tx(&full_cb, 65536);
                 tma_load_3d(sC, &map_c, &full_cb, 0, g, t0);
                 tma_load_3d(sC + 16384, &map_c, &full_cb, 64, g, t0);
                 tma_load_3d(sB, &map_b, &full_cb, 0, g, t0);
                 tma_load_3d(sB + 16384, &map_b, &full_cb, 64, g, t0);
-                const int sl = it & 1;
-                if (it >= 2) {
-                    store_y(it - 2);
-                    bulk_wait_read_all();           // the slot is free once the store has read it
+                if (j + 1 < ntiles) {
+                    tma_prefetch_3d(&map_c, 0, g, t0 + kTile);
+                    tma_prefetch_3d(&map_c, 64, g, t0 + kTile);
+                    tma_prefetch_3d(&map_b, 0, g, t0 + kTile);
+                    tma_prefetch_3d(&map_b, 64, g, t0 + kTile);
+                    for (int hh = 0; hh < kHeadsB; ++hh) tma_prefetch_3d(&map_x, 0, h0 + hh, t0 + kTile);
                 }
-                for (int hh = 0; hh < kHeadsB; ++hh) {
-                    mbar_arrive_expect_tx(&full_x[sl][hh], 16384);
-                    tma_load_3d(sX + sl * 32768 + hh * 16384, &map_x, &full_x[sl][hh], 0, h0 + hh, t0);
+            };
+            // y tile of chunk j, staged by the compute warps in the chunk's X slot (full
+            // chunks only; a partial last chunk is written by the threads).
+            auto store_y = [&](int j) {
+                wait_abort(&y_staged, j & 1, abort_p);
+                if (seg.len - j * kTile >= kTile) {
+                    for (int hh = 0; hh < kHeadsB; ++hh)
+                        tma_store_3d(&map_y, sX + (j & 1) * 32768 + hh * 16384, 0, h0 + hh, seg.start + j * kTile);
+                    bulk_commit_group();
+                }
+            };
+            if (ntiles > 0) load_x(0);
+            if (ntiles > 1) load_x(1);
+            if (ntiles > 0) load_cb(0);
+            for (int j = 1; j < ntiles; ++j) {
+                wait_abort(&zs_done, (j - 1) & 1, abort_p);         // C/B of chunk j-1 read
+                load_cb(j);
+                store_y(j - 1);
+                if (j + 1 < ntiles) {
+                    bulk_wait_read_all();                           // slot (j+1) & 1 read by the store
+                    load_x(j + 1);
                 }
             }
-            for (int j = ntiles >= 2 ? ntiles - 2 : 0; j < ntiles; ++j) store_y(j);
+            if (ntiles > 0) store_y(ntiles - 1);
             bulk_wait_all();
         }
     } else if (warp == 1) {
@@ -452,11 +472,12 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             if (elect_one()) {
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    umma_bf16(tZ, desc_add(dCk, kmajor_step(128, k)), desc_add(dH, k * kMnStep), id_z, k > 0);
+                    umma_bf16(tS, desc_add(dBm, k * kMnStep), desc_add(dW, k * kMnStep), id_s, k > 0);
+                umma_commit(&s_done);
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    umma_bf16(tS, desc_add(dBm, k * kMnStep), desc_add(dW, k * kMnStep), id_s, k > 0);
-                umma_commit(&empty_cb);
+                    umma_bf16(tZ, desc_add(dCk, kmajor_step(128, k)), desc_add(dH, k * kMnStep), id_z, k > 0);
+                umma_commit(&zs_done);
                 // M of head hh, sources 16k..16k+15: TMEM columns 16k + 8hh of the M block.
 #pragma unroll
                 for (int k = 0; k < 8; ++k) umma_bf16_ts(tY, tM + 16 * k, desc_add(dX0, k * kMnStep), id_y, k > 0);
@@ -470,6 +491,72 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 wait_abort(&mma_done, it & 1, abort_p);     // the Y UMMAs have read M
                 issue_cb(it + 1);
             }
+        }
+    } else if (warp == kScanWarp) {
+        // ------------------------------------------------------------ dt scan
+        // Chunk by chunk, up to four ahead of the compute warps: dt, the log2-scaled
+        // cumulative dt*A and the decay weights of both heads into buffer j % 4. Lane l
+        // holds tokens 4l..4l+3; the dt_raw of chunk j+1 is loaded while chunk j is scanned.
+        float bias[kHeadsB], Ah[kHeadsB];
+#pragma unroll
+        for (int hh = 0; hh < kHeadsB; ++hh) {
+            bias[hh] = dt_bias[h0 + hh];
+            Ah[hh] = A[h0 + hh];
+            if (lane == 0 && (!(Ah[hh] <= 0.f) || isinf(Ah[hh]))) latch_error(SSD_ERR_INVALID_ARG);
+        }
+        float z[kHeadsB][4], zn[kHeadsB][4];       // dt_raw of chunk j and of chunk j+1
+        auto load_dt = [&](int j, float (&zz)[kHeadsB][4]) {
+            const int tlj = min(kTile, seg.len - j * kTile);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int64_t row = ((int64_t)seg.start + (int64_t)j * kTile + 4 * lane + i) * H + h0;
+#pragma unroll
+                for (int hh = 0; hh < kHeadsB; ++hh) zz[hh][i] = 4 * lane + i < tlj ? dt_raw[row + hh] : 0.f;
+            }
+        };
+        if (ntiles > 0) load_dt(0, zn);
+        for (int j = 0; j < ntiles; ++j) {
+            const int bf = j % 4;
+#pragma unroll
+            for (int hh = 0; hh < kHeadsB; ++hh)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) z[hh][i] = zn[hh][i];
+            if (j + 1 < ntiles) load_dt(j + 1, zn);
+            if (j >= 4) wait_abort(&dt_free[bf], ((j >> 2) - 1) & 1, abort_p);
+            const int tlj = min(kTile, seg.len - j * kTile);
+#pragma unroll
+            for (int hh = 0; hh < kHeadsB; ++hh) {
+                float dtv[4], p[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    dtv[i] = 4 * lane + i < tlj ? softplus_fast(z[hh][i] + bias[hh]) : 0.f;
+                    p[i] = (i ? p[i - 1] : 0.f) + dtv[i] * Ah[hh];
+                }
+                float incl = p[3];
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float v = __shfl_up_sync(0xffffffffu, incl, off);
+                    if (lane >= off) incl += v;
+                }
+                const float excl = incl - p[3];
+                float av[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) av[i] = (excl + p[i]) * kLog2e;
+                const float a_blk = __shfl_sync(0xffffffffu, av[3], (lane & ~7) | 7);    // token 32b + 31
+                const float a_end = __shfl_sync(0xffffffffu, av[3], 31);                 // token 127
+                float u[4], w[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    u[i] = fast_exp2(a_blk - av[i]) * dtv[i];
+                    w[i] = fast_exp2(a_end - av[i]) * dtv[i];
+                }
+                *reinterpret_cast<float4*>(&ac2[bf][hh][4 * lane]) = make_float4(av[0], av[1], av[2], av[3]);
+                *reinterpret_cast<float4*>(&dts[bf][hh][4 * lane]) = make_float4(dtv[0], dtv[1], dtv[2], dtv[3]);
+                *reinterpret_cast<float4*>(&uw[bf][hh][4 * lane]) = make_float4(u[0], u[1], u[2], u[3]);
+                *reinterpret_cast<float4*>(&ww[bf][hh][4 * lane]) = make_float4(w[0], w[1], w[2], w[3]);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&dt_ready[bf]);
         }
     } else {
         // ------------------------------------------------------------ compute warpgroups
@@ -492,38 +579,6 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             }
         }
         const float Dh0 = D[h0], Dh1 = D[h0 + 1];
-        const int hc = cw & 1;                      // head scanned by warpgroup cw (cw < 2)
-        const float bias_c = dt_bias[h0 + hc], A_c = A[h0 + hc];
-        if (cw < kHeadsB && r == 0 && (!(A_c <= 0.f) || isinf(A_c))) latch_error(SSD_ERR_INVALID_ARG);
-        auto load_dt = [&](int j) -> float {        // dt_raw of token r of chunk j, head cw
-            const int tlj = min(kTile, seg.len - j * kTile);
-            return (cw < kHeadsB && r < tlj) ? dt_raw[((int64_t)seg.start + (int64_t)j * kTile + r) * H + h0 + hc] : 0.f;
-        };
-        // dt, log2-scaled cumulative dt*A and the decay weights of chunk j into buffer
-        // j % 4 (warpgroups 0 and 1, one head each; named barrier 2 + cw).
-        auto scan_chunk = [&](int j, float z) {
-            const int bf = j % 4;
-            const int tlj = min(kTile, seg.len - j * kTile);
-            const float dtv = r < tlj ? softplus_f32(z + bias_c) : 0.f;
-            float a = dtv * A_c;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float v = __shfl_up_sync(0xffffffffu, a, off);
-                if (lane >= off) a += v;
-            }
-            if (lane == 31) part[cw][q] = a;
-            asm volatile("bar.sync %0, 128;" ::"r"(2 + cw) : "memory");
-            float pre = 0.f;
-            for (int w = 0; w < q; ++w) pre += part[cw][w];
-            const float av = (a + pre) * kLog2e;
-            ac2[bf][cw][r] = av;
-            dts[bf][cw][r] = dtv;
-            asm volatile("bar.sync %0, 128;" ::"r"(2 + cw) : "memory");
-            uw[bf][cw][r] = fast_exp2(ac2[bf][cw][r | 31] - av) * dtv;
-            ww[bf][cw][r] = fast_exp2(ac2[bf][cw][kTile - 1] - av) * dtv;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&dt_ready[bf]);
-        };
         // Decays of the diagonal 32x32 blocks of chunk j, L[t][s] = exp2(Acum_t - Acum_s)
         // dt_s for s <= t in t's block (fp16, row t = r of head cw - 2; warpgroups 2, 3).
         // 16-byte chunk c of row t sits at chunk c ^ ((t >> 1) & 3).
@@ -553,20 +608,47 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             __syncwarp();
             if (lane == 0) mbar_arrive(&l_ready);
         };
-        float zn = 0.f;                             // prefetched dt_raw of the next chunk to scan
-        if (cw < kHeadsB) {
-            scan_chunk(0, load_dt(0));
-            if (ntiles > 1) scan_chunk(1, load_dt(1));
-            if (ntiles > 2) zn = load_dt(2);
-        } else {
-            diag_decays(0);
-        }
+        // w*X of chunk j for both heads into shared memory.
+        auto stage_wx = [&](int j) {
+            const int bf = j % 4, sl = j & 1;
+            wait_abort(&dt_ready[bf], (j / 4) & 1, abort_p);
+            wait_abort(&full_x[sl], (j >> 1) & 1, abort_p);
+#pragma unroll
+            for (int hh = 0; hh < kHeadsB; ++hh) {
+                const float w = ww[bf][hh][r];
+                const uint32_t w2 = pack_bf16(w, w);
+                const uint32_t xrow = smem_u32(sX + sl * 32768 + hh * 16384), wrow = smem_u32(sW + hh * 16384);
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const uint4 v = ld_shared_v4(xrow + swz(r, 2 * cw + c));
+                    st_shared_v4(wrow + swz(r, 2 * cw + c), hmul2_bf16(v.x, w2), hmul2_bf16(v.y, w2),
+                                 hmul2_bf16(v.z, w2), hmul2_bf16(v.w, w2));
+                }
+            }
+        };
+        // bf16 h (from the registers) for both heads into shared memory.
+        auto stage_h = [&]() {
+#pragma unroll
+            for (int hh = 0; hh < kHeadsB; ++hh) {
+                const uint32_t hrow = smem_u32(sH + hh * 16384);
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) pk[jj] = pack_bf16(h[hh][8 * c + 2 * jj], h[hh][8 * c + 2 * jj + 1]);
+                    st_shared_v4(hrow + swz(r, 2 * cw + c), pk[0], pk[1], pk[2], pk[3]);
+                }
+            }
+        };
+
+        if (cw >= kHeadsB) diag_decays(0);
+        stage_h();
+        stage_wx(0);
 
         for (int it = 0; it < ntiles; ++it) {
             const int64_t t0 = seg.start + (int64_t)it * kTile;
             const int tl = min(kTile, seg.len - it * kTile);
-            const int bf = it % 4, sl = it & 1;
-            uint8_t* sXs = sX + sl * 32768;
+            const int bf = it % 4;
             wait_abort(&dt_ready[bf], (it / 4) & 1, abort_p);
             wait_abort(&l_ready, it & 1, abort_p);
             wait_abort(&cb_done, it & 1, abort_p);
@@ -574,27 +656,38 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             // -------- M[t][s] of both heads, t = r, in place over C B^T. Source block b
             // (32 sources) keeps its 32 columns: half j (sources 16j..16j+15 of the
             // block) becomes M of head 0 in its first 8 columns and of head 1 in the
-            // next 8. First the diagonal slice: head cw & 1, half cw >> 1 of block q;
-            // the four warps of lane quarter q read their C B^T slices before any of
-            // them overwrites the block (named barrier 4 + q).
-            {
-                const int hd = cw & 1, sd = 32 * q + 16 * (cw >> 1);
+            // next 8. The diagonal block q is done half by half (both heads) by the warps
+            // of lane quarter q that have no block below the diagonal (cw >= q): warp
+            // cw takes the halves j = cw - q, cw - q + (4 - q), ... < 2. Each half is read
+            // and overwritten by one warp only.
+            auto diag_half = [&](int jh) {
+                const int sd = 32 * q + 16 * jh;
                 uint32_t rc[16];
                 tmem_ld16(tM + lane_off + sd, rc);
                 tmem_wait_ld();
-                asm volatile("bar.sync %0, 128;" ::"r"(4 + q) : "memory");
-                const uint32_t lrow = smem_u32(sL + hd * 8192 + r * 64);
-                const int c0 = 2 * (cw >> 1);
-                const uint4 la = ld_shared_v4(lrow + ((c0 ^ ((r >> 1) & 3)) << 4));
-                const uint4 lb = ld_shared_v4(lrow + (((c0 + 1) ^ ((r >> 1) & 3)) << 4));
-                const uint32_t lw[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
-                uint32_t pk[8];
+                const int jd = r - sd;              // D joins M on the diagonal (s = t)
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    pk[k] = pack_bf16(fmul2(f16x2_to_f2(lw[k]),
-                                            make_float2(__uint_as_float(rc[2 * k]), __uint_as_float(rc[2 * k + 1]))));
-                tmem_st8(tM + lane_off + sd + 8 * hd, pk);
-            }
+                for (int hd = 0; hd < kHeadsB; ++hd) {
+                    const uint32_t lrow = smem_u32(sL + hd * 8192 + r * 64);
+                    const int c0 = 2 * jh;
+                    const uint4 la = ld_shared_v4(lrow + ((c0 ^ ((r >> 1) & 3)) << 4));
+                    const uint4 lb = ld_shared_v4(lrow + (((c0 + 1) ^ ((r >> 1) & 3)) << 4));
+                    const uint32_t lw[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
+                    const float Dd = hd ? Dh1 : Dh0;
+                    uint32_t pk[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        float2 m = fmul2(f16x2_to_f2(lw[k]),
+                                         make_float2(__uint_as_float(rc[2 * k]), __uint_as_float(rc[2 * k + 1])));
+                        if (jd == 2 * k) m.x += Dd;
+                        if (jd == 2 * k + 1) m.y += Dd;
+                        pk[k] = pack_bf16(m);
+                    }
+                    tmem_st8(tM + lane_off + sd + 8 * hd, pk);
+                }
+            };
+            if (cw >= q && cw - q < 2) diag_half(cw - q);
+            if (q == 3 && cw == 3) diag_half(1);    // lane quarter 3: warp cw = 3 takes both halves
             if (cw < q) {                          // below the diagonal: factorized
                 float2 v[kHeadsB];
 #pragma unroll
@@ -631,96 +724,25 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 for (int c8 = 0; c8 < 4; ++c8) tmem_st8(tM + lane_off + 32 * cw + 8 * c8, zero);
             }
             tmem_wait_st();
-            // -------- w*X and bf16 h of both heads
-#pragma unroll
-            for (int hh = 0; hh < kHeadsB; ++hh) {
-                wait_abort(&full_x[sl][hh], (it >> 1) & 1, abort_p);
-                const float w = ww[bf][hh][r];
-                const uint32_t w2 = pack_bf16(w, w);
-                const uint32_t xrow = smem_u32(sXs + hh * 16384), wrow = smem_u32(sW + hh * 16384);
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    const uint4 v = ld_shared_v4(xrow + swz(r, 2 * cw + c));
-                    st_shared_v4(wrow + swz(r, 2 * cw + c), hmul2_bf16(v.x, w2), hmul2_bf16(v.y, w2),
-                                 hmul2_bf16(v.z, w2), hmul2_bf16(v.w, w2));
-                }
-                const uint32_t hrow = smem_u32(sH + hh * 16384);
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    uint32_t pk[4];
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) pk[jj] = pack_bf16(h[hh][8 * c + 2 * jj], h[hh][8 * c + 2 * jj + 1]);
-                    st_shared_v4(hrow + swz(r, 2 * cw + c), pk[0], pk[1], pk[2], pk[3]);
-                }
-            }
-            fence_proxy_async_smem();
+            fence_proxy_async_smem();              // bf16 h and w*X of this chunk
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&ops_ready);
-            // -------- while the UMMAs run: warpgroups 0/1 scan chunk it+2. Its buffer (of
-            // four) was last read by chunk it-2's drain, which every warp finished before
-            // this warp could pass chunk it-1's mma_done wait. Warpgroups 2/3 write the
-            // diagonal-block decays of chunk it+1 once every warp has finished reading
-            // those of chunk it (ops_ready complete).
-            if (cw < kHeadsB) {
-                if (it + 2 < ntiles) {
-                    scan_chunk(it + 2, zn);
-                    if (it + 3 < ntiles) zn = load_dt(it + 3);
-                }
-            } else if (it + 1 < ntiles) {
+            // -------- while S and Z run: warpgroups 2/3 tabulate chunk it+1's diagonal
+            // decays once every warp has read chunk it's (ops_ready complete).
+            if (cw >= kHeadsB && it + 1 < ntiles) {
                 wait_abort(&ops_ready, it & 1, abort_p);
                 diag_decays(it + 1);
             }
-            // -------- drain: y rows (into the X slot for a full chunk, else straight to
-            // HBM), then release the slot, then the state update. The TMEM loads of the
-            // next 8-column piece are issued before the current one is consumed.
-            wait_abort(&mma_done, it & 1, abort_p);
+            // -------- S done: w*X of the next chunk (its buffer was read by this chunk's S).
+            // Z done (the Y UMMAs may still run): state update, then bf16 h of the next
+            // chunk (its buffer was read by this chunk's Z).
+            if (it + 1 < ntiles) {
+                wait_abort(&s_done, it & 1, abort_p);
+                stage_wx(it + 1);
+            }
+            wait_abort(&zs_done, it & 1, abort_p);
             tc_fence_after();
-            {
-                const bool staged = tl == kTile;
-                uint32_t ry[2][8], rz[2][8];
-                tmem_ld8(tY + lane_off + 16 * cw, ry[0]);
-                tmem_ld8(tZ + lane_off + 16 * cw, rz[0]);
-                const float et0 = fast_exp2(ac2[bf][0][r]), et1 = fast_exp2(ac2[bf][1][r]);
-                const float2 e20 = make_float2(et0, et0), e21 = make_float2(et1, et1);
-                const float2 d20 = make_float2(Dh0, Dh0), d21 = make_float2(Dh1, Dh1);
-#pragma unroll
-                for (int piece = 0; piece < 4; ++piece) {           // (head, half) = (piece/2, piece%2)
-                    const int hh = piece >> 1, half = piece & 1, cur = piece & 1;
-                    tmem_wait_ld();
-                    if (piece < 3) {
-                        const int nh = (piece + 1) >> 1, nf = (piece + 1) & 1;
-                        tmem_ld8(tY + nh * 64 + lane_off + 16 * cw + 8 * nf, ry[cur ^ 1]);
-                        tmem_ld8(tZ + nh * 64 + lane_off + 16 * cw + 8 * nf, rz[cur ^ 1]);
-                    }
-                    const float2 et = hh ? e21 : e20;
-                    const float2 Dh = hh ? d21 : d20;
-                    const uint32_t xa = smem_u32(sXs + hh * 16384) + swz(r, 2 * cw + half);
-                    const uint4 xv = ld_shared_v4(xa);
-                    const uint32_t xk[4] = {xv.x, xv.y, xv.z, xv.w};
-                    uint32_t o[4];
-#pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        const float2 xf = bf16x2_to_f2(xk[jj]);
-                        const float2 zy = ffma2(et, make_float2(__uint_as_float(rz[cur][2 * jj]), __uint_as_float(rz[cur][2 * jj + 1])),
-                                                make_float2(__uint_as_float(ry[cur][2 * jj]), __uint_as_float(ry[cur][2 * jj + 1])));
-                        o[jj] = pack_bf16(ffma2(Dh, xf, zy));
-                    }
-                    if (staged) {
-                        st_shared_v4(xa, o[0], o[1], o[2], o[3]);
-                    } else if (r < tl) {
-                        *reinterpret_cast<uint4*>(y + ((t0 + r) * H + h0 + hh) * kP + 16 * cw + 8 * half) =
-                            make_uint4(o[0], o[1], o[2], o[3]);
-                    }
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&empty_x[sl][0]);       // y staged, x of both heads read for the last time
-                mbar_arrive(&empty_x[sl][1]);
-            }
 #pragma unroll
             for (int hh = 0; hh < kHeadsB; ++hh) {
                 uint32_t rs[16];
@@ -735,6 +757,49 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                     h[hh][j] = hn.x;
                     h[hh][j + 1] = hn.y;
                 }
+            }
+            if (it + 1 < ntiles) stage_h();
+            // -------- drain: y rows (into the chunk's X slot for a full chunk, else
+            // straight to HBM). The TMEM loads of the next 8-column piece are issued before the
+            // current one is consumed.
+            wait_abort(&mma_done, it & 1, abort_p);
+            tc_fence_after();
+            {
+                const bool staged = tl == kTile;
+                uint32_t ry[2][8], rz[2][8];
+                tmem_ld8(tY + lane_off + 16 * cw, ry[0]);
+                tmem_ld8(tZ + lane_off + 16 * cw, rz[0]);
+                const float et0 = fast_exp2(ac2[bf][0][r]), et1 = fast_exp2(ac2[bf][1][r]);
+                const float2 e20 = make_float2(et0, et0), e21 = make_float2(et1, et1);
+#pragma unroll
+                for (int piece = 0; piece < 4; ++piece) {           // (head, half) = (piece/2, piece%2)
+                    const int hh = piece >> 1, half = piece & 1, cur = piece & 1;
+                    tmem_wait_ld();
+                    if (piece < 3) {
+                        const int nh = (piece + 1) >> 1, nf = (piece + 1) & 1;
+                        tmem_ld8(tY + nh * 64 + lane_off + 16 * cw + 8 * nf, ry[cur ^ 1]);
+                        tmem_ld8(tZ + nh * 64 + lane_off + 16 * cw + 8 * nf, rz[cur ^ 1]);
+                    }
+                    const float2 et = hh ? e21 : e20;
+                    uint32_t o[4];
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj)
+                        o[jj] = pack_bf16(ffma2(et, make_float2(__uint_as_float(rz[cur][2 * jj]), __uint_as_float(rz[cur][2 * jj + 1])),
+                                                make_float2(__uint_as_float(ry[cur][2 * jj]), __uint_as_float(ry[cur][2 * jj + 1]))));
+                    if (staged) {
+                        st_shared_v4(smem_u32(sX + (it & 1) * 32768 + hh * 16384) + swz(r, 2 * cw + half), o[0], o[1],
+                                     o[2], o[3]);
+                    } else if (r < tl) {
+                        *reinterpret_cast<uint4*>(y + ((t0 + r) * H + h0 + hh) * kP + 16 * cw + 8 * half) =
+                            make_uint4(o[0], o[1], o[2], o[3]);
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&y_staged);
+                mbar_arrive(&dt_free[bf]);          // this chunk's dt buffer is no longer read
             }
         }
     }

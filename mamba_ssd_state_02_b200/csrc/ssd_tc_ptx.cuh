@@ -101,6 +101,14 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
+// Prefetch one box of a 3-D tiled tensor into L2 (no shared memory, no completion).
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+
 // 3-D tiled store of one box from shared memory (bulk-group completion). The source
 // must have been written through the async proxy or fenced with fence_proxy_async_smem.
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int c0, int c1, int c2) {
@@ -291,6 +299,24 @@ __device__ __forceinline__ float fast_exp2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+__device__ __forceinline__ float fast_log2(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// softplus(z) = max(z, 0) + log1p(e), e = exp(-|z|) <= 1, from the hardware base-2
+// exponential and logarithm. log1p uses Kahan's correction (Goldberg, "What every
+// computer scientist should know about floating-point arithmetic", 1991, Thm. 4):
+// with u = 1 + e rounded, log1p(e) = log(u) * e / (u - 1), exact division operand
+// u - 1, so the result keeps a few-ulp relative error even when e is tiny.
+__device__ __forceinline__ float softplus_fast(float z) {
+    const float e = fast_exp2(-fabsf(z) * 1.4426950408889634f);
+    const float u = 1.f + e;
+    const float l1p = u == 1.f ? e : fast_log2(u) * 0.6931471805599453f * __fdividef(e, u - 1.f);
+    return fmaxf(z, 0.f) + l1p;
 }
 
 // K-step `k` (16 elements) of a K-major operand stored as 64-column sub-tiles of
