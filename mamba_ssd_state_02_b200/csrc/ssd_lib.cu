@@ -318,7 +318,7 @@ ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_ra
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(tc kernels)");
         {
             StageScope sc(ST_CHUNK_STATE, st);
-            tc::k_tc_segment_state<<<(unsigned)(pl.max_segs * (H / tc::kHeads)), tc::kThreadsTc, tc::kSmemA,
+            tc::k_tc_segment_state<<<(unsigned)(pl.max_segs * (H / tc::kHeads)), tc::kThreadsA, tc::kSmemA,
                                      st>>>(mx, mb, dt_raw, dt_bias, A, table, count, H, G,
                                                                   seg_state, seg_acum);
         }

@@ -79,14 +79,26 @@ __device__ __forceinline__ float wg_scan(float a, int q, int lane, float* part) 
 
 // ---------------------------------------------------------------------------------
 // Pass A: zero-start segment states S_seg (fp32, layout [seg][H][N][P]) and the
-// segment's total sum of dt*A (seg_acum[seg][H]). One CTA per (segment, 4 heads);
-// compute warpgroup cw owns head cw for the decay weights and column quarter cw of
-// every w*X row. Tiles run from the segment end backwards so the decay to the end is
-// a running sum. Shared memory: two B stages, a four-slot X ring (one per head), two
-// w*X hi/lo buffer pairs. TMEM: S_seg of the 4 heads (64 columns each).
+// segment's total sum of dt*A (seg_acum[seg][H]). One CTA per (segment, 4 heads); the
+// chunks run from the segment end backwards so the decay to the end is a running sum.
+//
+// Warp 0 issues the TMA loads, warp 1 the UMMAs, warp 18 scans dt (up to four chunks
+// ahead; w_s = exp(sum_{r > s in seg} dt_r A) dt_s), and the 16 compute warps write
+// w*X as a bf16 hi/lo pair (hi in place over x, lo to its own buffer), so the product
+// keeps ~16 mantissa bits: the FP32 final state is held to 1e-3. Heads go in pairs:
+// per pair one batch of 8 hi + 8 lo UMMAs with N = 128 (both heads side by side, B^T
+// read once for the pair) accumulates S of the two heads in TMEM; while it runs the
+// compute warps prepare the other pair. Compute thread (cw, r) owns token row r and
+// column quarter cw of every head's w*X.
+//
+// Shared memory: two B stages, X of the 4 heads (one slot each; the pair's slots are
+// refilled as soon as its UMMAs are done), the lo buffers of the 4 heads. TMEM: S_seg
+// of the 4 heads (64 columns each; pair p at columns 128p).
 constexpr int kSmemA = 192 * 1024 + 1024;
+constexpr int kScanWarpA = kRoleWarps + kComputeWarps;         // warp 18: dt scan
+constexpr int kThreadsA = 32 * (kScanWarpA + 1);
 
-__global__ void __launch_bounds__(kThreadsTc, 1)
+__global__ void __launch_bounds__(kThreadsA, 1)
 k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
                    const float* __restrict__ dt_raw, const float* __restrict__ dt_bias,
                    const float* __restrict__ A, const ChunkEntry* __restrict__ segs,
@@ -98,11 +110,10 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sB = sm;                       // stage st at st*32768: [2][128 s][64 n]
-    uint8_t* sX = sm + 65536;               // slot hh at hh*16384: [128 s][64 p]
-    uint8_t* sWx = sm + 131072;             // buffer b at b*32768: hi [128 s][64 p], lo at +16384
-    __shared__ float wts[kHeads][kTile];
-    __shared__ float part[kHeads][4], tile_tot[kHeads];
-    __shared__ uint64_t full_b[2], empty_b[2], full_x[kHeads], empty_x[kHeads], ops_ready[2], mma_done[2];
+    uint8_t* sX = sm + 65536;               // head hh at hh*16384: [128 s][64 p]; x, then hi(w*x)
+    uint8_t* sLo = sm + 131072;             // head hh at hh*16384: [128 s][64 p]; lo(w*x)
+    __shared__ __align__(16) float wts[4][kHeads][kTile];
+    __shared__ uint64_t full_b[2], empty_b[2], full_x[2], pair_done[2], ops_ready[2], w_ready[4], w_free[4], all_done;
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
 
@@ -115,13 +126,15 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
         for (int i = 0; i < 2; ++i) {
             mbar_init(&full_b[i], 1);
             mbar_init(&empty_b[i], 1);
-            mbar_init(&ops_ready[i], kComputeWarps);
-            mbar_init(&mma_done[i], 1);
-        }
-        for (int i = 0; i < kHeads; ++i) {
             mbar_init(&full_x[i], 1);
-            mbar_init(&empty_x[i], kComputeWarps);
+            mbar_init(&pair_done[i], 1);
+            mbar_init(&ops_ready[i], kComputeWarps);
         }
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(&w_ready[i], 1);
+            mbar_init(&w_free[i], kComputeWarps);
+        }
+        mbar_init(&all_done, 1);
         abort_flag = 0;
         fence_barrier_init();
         prefetch_tmap(&map_x);
@@ -138,105 +151,159 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
     volatile int* abort_p = &abort_flag;
 
     if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            for (int k = 0; k < ntiles; ++k) {            // k-th tile processed = tile ntiles-1-k
-                const int t0 = seg.start + (ntiles - 1 - k) * kTile, st = k & 1;
+            auto t0_of = [&](int k) { return seg.start + (ntiles - 1 - k) * kTile; };   // k-th chunk processed
+            for (int k = 0; k < ntiles; ++k) {
+                const int t0 = t0_of(k), st = k & 1;
                 if (k >= 2) wait_abort(&empty_b[st], ((k - 2) >> 1) & 1, abort_p);
                 mbar_arrive_expect_tx(&full_b[st], 32768);
                 tma_load_3d(sB + st * 32768, &map_b, &full_b[st], 0, g, t0);
                 tma_load_3d(sB + st * 32768 + 16384, &map_b, &full_b[st], 64, g, t0);
-                for (int hh = 0; hh < kHeads; ++hh) {
-                    if (k >= 1) wait_abort(&empty_x[hh], (k - 1) & 1, abort_p);
-                    mbar_arrive_expect_tx(&full_x[hh], 16384);
-                    tma_load_3d(sX + hh * 16384, &map_x, &full_x[hh], 0, h0 + hh, t0);
+                if (k + 1 < ntiles) {               // next chunk's B and X into L2 meanwhile
+                    const int tn = t0_of(k + 1);
+                    tma_prefetch_3d(&map_b, 0, g, tn);
+                    tma_prefetch_3d(&map_b, 64, g, tn);
+                    for (int hh = 0; hh < kHeads; ++hh) tma_prefetch_3d(&map_x, 0, h0 + hh, tn);
+                }
+                for (int pr = 0; pr < 2; ++pr) {
+                    if (k >= 1) wait_abort(&pair_done[pr], (k - 1) & 1, abort_p);   // slots and lo free
+                    mbar_arrive_expect_tx(&full_x[pr], 32768);
+                    for (int hh = 2 * pr; hh < 2 * pr + 2; ++hh)
+                        tma_load_3d(sX + hh * 16384, &map_x, &full_x[pr], 0, h0 + hh, t0);
                 }
             }
         }
     } else if (warp == 1) {
-        // UMMA issuer: the whole warp runs the loop (warp-uniform descriptors), one
-        // elected lane issues.
-        const uint32_t idesc = idesc_bf16(128, 64, 1, 1);
-        const uint64_t dWx0 = smem_desc(smem_u32(sWx), 16384, 1024);
+        // ------------------------------------------------------------ UMMA issuer
+        // S[n][p] of a head pair += B^T (hi + lo): A = B^T (MN-major), B = [hi|lo] of the
+        // pair (MN-major, the two heads 16 KB apart), N = 128.
+        const uint32_t idesc = idesc_bf16(128, 128, 1, 1);
+        const uint64_t dHi = smem_desc(smem_u32(sX), 16384, 1024), dLo = smem_desc(smem_u32(sLo), 16384, 1024);
         for (int k = 0; k < ntiles; ++k) {
             const int st = k & 1;
             wait_abort(&full_b[st], (k >> 1) & 1, abort_p);
             const uint64_t dB = smem_desc(smem_u32(sB + st * 32768), 16384, 1024);
-            for (int hh = 0; hh < kHeads; ++hh) {
-                const int j = k * kHeads + hh, b = j & 1;
-                wait_abort(&ops_ready[b], (j >> 1) & 1, abort_p);
+            for (int pr = 0; pr < 2; ++pr) {
+                wait_abort(&ops_ready[pr], k & 1, abort_p);
                 tc_fence_after();
-                const uint64_t dHi = desc_add(dWx0, b * 32768), dLo = desc_add(dHi, 16384);
-                const uint32_t d = tS + hh * 64;
+                const uint32_t d = tS + pr * 128;
+                const uint64_t dh = desc_add(dHi, pr * 32768), dl = desc_add(dLo, pr * 32768);
                 if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        umma_bf16(d, desc_add(dB, kk * kMnStep), desc_add(dHi, kk * kMnStep), idesc, !(k == 0 && kk == 0));
+                        umma_bf16(d, desc_add(dB, kk * kMnStep), desc_add(dh, kk * kMnStep), idesc, !(k == 0 && kk == 0));
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        umma_bf16(d, desc_add(dB, kk * kMnStep), desc_add(dLo, kk * kMnStep), idesc, true);
-                    umma_commit(&mma_done[b]);
-                    if (hh == kHeads - 1) umma_commit(&empty_b[st]);
+                        umma_bf16(d, desc_add(dB, kk * kMnStep), desc_add(dl, kk * kMnStep), idesc, true);
+                    umma_commit(&pair_done[pr]);
+                    if (pr == 1) umma_commit(&empty_b[st]);
+                    if (pr == 1 && k == ntiles - 1) umma_commit(&all_done);
                 }
                 __syncwarp();
             }
         }
-    } else {
-        const int cw = (warp - kRoleWarps) >> 2, q = warp & 3, r = q * 32 + lane;
-        float suffix = 0.f;                 // log2-scaled sum of dt*A of head cw after this tile
-        for (int k = 0; k < ntiles; ++k) {
+    } else if (warp == kScanWarpA) {
+        // ------------------------------------------------------------ dt scan
+        // Lane l holds tokens 4l..4l+3 of a chunk; the dt_raw of the next chunk is loaded
+        // while this one is scanned. suf[hh] = sum of dt*A after the current chunk (log2).
+        float bias[kHeads], Ah[kHeads], suf[kHeads];
+#pragma unroll
+        for (int hh = 0; hh < kHeads; ++hh) {
+            bias[hh] = dt_bias[h0 + hh];
+            Ah[hh] = A[h0 + hh] * kLog2e;
+            suf[hh] = 0.f;
+            if (lane == 0 && (!(A[h0 + hh] <= 0.f) || isinf(A[h0 + hh]))) latch_error(SSD_ERR_INVALID_ARG);
+        }
+        float z[kHeads][4], zn[kHeads][4];
+        auto load_dt = [&](int k, float (&zz)[kHeads][4]) {
             const int it = ntiles - 1 - k;
-            const int64_t t0 = seg.start + (int64_t)it * kTile;
-            const int tl = min(kTile, seg.len - it * kTile);
-            // decay-to-segment-end weights of head cw: w_s = exp(sum_{r>s} dt_r A) dt_s
-            {
-                const float Ah = A[h0 + cw];
-                if (r == 0 && k == 0 && (!(Ah <= 0.f) || isinf(Ah))) latch_error(SSD_ERR_INVALID_ARG);
-                const float dtv = r < tl ? softplus_fast(dt_raw[(t0 + r) * H + h0 + cw] + dt_bias[h0 + cw]) : 0.f;
-                compute_bar();              // previous tile's weights no longer read
-                const float incl = wg_scan(dtv * Ah, q, lane, part[cw]) * kLog2e;
-                if (r == kTile - 1) tile_tot[cw] = incl;
-                compute_bar();
-                const float tot = tile_tot[cw];
-                wts[cw][r] = fast_exp2(suffix + tot - incl) * dtv;
-                suffix += tot;
-                compute_bar();
+            const int tlk = min(kTile, seg.len - it * kTile);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int64_t row = ((int64_t)seg.start + (int64_t)it * kTile + 4 * lane + i) * H + h0;
+#pragma unroll
+                for (int hh = 0; hh < kHeads; ++hh) zz[hh][i] = 4 * lane + i < tlk ? dt_raw[row + hh] : 0.f;
             }
+        };
+        load_dt(0, zn);
+        for (int k = 0; k < ntiles; ++k) {
+            const int bf = k % 4, it = ntiles - 1 - k;
+            const int tlk = min(kTile, seg.len - it * kTile);
+#pragma unroll
+            for (int hh = 0; hh < kHeads; ++hh)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) z[hh][i] = zn[hh][i];
+            if (k + 1 < ntiles) load_dt(k + 1, zn);
+            if (k >= 4) wait_abort(&w_free[bf], ((k >> 2) - 1) & 1, abort_p);
+#pragma unroll
             for (int hh = 0; hh < kHeads; ++hh) {
-                const int j = k * kHeads + hh, b = j & 1;
-                if (j >= 2) wait_abort(&mma_done[b], ((j - 2) >> 1) & 1, abort_p);
-                wait_abort(&full_x[hh], k & 1, abort_p);
-                const float w = wts[hh][r];
-                const uint32_t xrow = smem_u32(sX + hh * 16384);
-                const uint32_t hi = smem_u32(sWx + b * 32768), lo = hi + 16384;
+                float dtv[4], p[4];
 #pragma unroll
-                for (int c = 2 * cw; c < 2 * cw + 2; ++c) {
-                    const uint4 v = ld_shared_v4(xrow + swz(r, c));
-                    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-                    uint32_t oh[4], ol[4];
+                for (int i = 0; i < 4; ++i) {
+                    dtv[i] = 4 * lane + i < tlk ? softplus_fast(z[hh][i] + bias[hh]) : 0.f;
+                    p[i] = (i ? p[i - 1] : 0.f) + dtv[i] * Ah[hh];
+                }
+                float incl = p[3];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = bf16x2_to_f2(in[e]);
-                        const float p0 = f.x * w, p1 = f.y * w;
-                        const __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
-                        const float2 hf = __bfloat1622float2(hb);
-                        oh[e] = *reinterpret_cast<const uint32_t*>(&hb);
-                        ol[e] = pack_bf16(p0 - hf.x, p1 - hf.y);
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float v = __shfl_up_sync(0xffffffffu, incl, off);
+                    if (lane >= off) incl += v;
+                }
+                const float tot = __shfl_sync(0xffffffffu, incl, 31);
+                const float base = suf[hh] + tot - (incl - p[3]);   // decay exponent of token 4l, plus p[i] below
+                float w[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) w[i] = fast_exp2(base - p[i]) * dtv[i];
+                *reinterpret_cast<float4*>(&wts[bf][hh][4 * lane]) = make_float4(w[0], w[1], w[2], w[3]);
+                suf[hh] += tot;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&w_ready[bf]);
+        }
+        if (lane < kHeads) {
+            float v = suf[0];
+#pragma unroll
+            for (int hh = 1; hh < kHeads; ++hh) v = lane == hh ? suf[hh] : v;
+            seg_acum[(int64_t)sg * H + h0 + lane] = v / kLog2e;
+        }
+    } else {
+        // ------------------------------------------------------------ compute warps
+        const int cw = (warp - kRoleWarps) >> 2, q = warp & 3, r = q * 32 + lane;
+        for (int k = 0; k < ntiles; ++k) {
+            const int bf = k % 4;
+            wait_abort(&w_ready[bf], (k >> 2) & 1, abort_p);
+            for (int pr = 0; pr < 2; ++pr) {
+                wait_abort(&full_x[pr], k & 1, abort_p);
+#pragma unroll
+                for (int hh = 2 * pr; hh < 2 * pr + 2; ++hh) {
+                    const float w = wts[bf][hh][r];
+                    const float2 w2 = make_float2(w, w);
+                    const uint32_t xrow = smem_u32(sX + hh * 16384), lrow = smem_u32(sLo + hh * 16384);
+#pragma unroll
+                    for (int c = 2 * cw; c < 2 * cw + 2; ++c) {
+                        const uint4 v = ld_shared_v4(xrow + swz(r, c));
+                        const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+                        uint32_t oh[4], ol[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 pw = fmul2(bf16x2_to_f2(in[e]), w2);
+                            oh[e] = pack_bf16(pw);
+                            ol[e] = pack_bf16(fsub2(pw, bf16x2_to_f2(oh[e])));
+                        }
+                        st_shared_v4(xrow + swz(r, c), oh[0], oh[1], oh[2], oh[3]);     // hi in place of x
+                        st_shared_v4(lrow + swz(r, c), ol[0], ol[1], ol[2], ol[3]);
                     }
-                    st_shared_v4(hi + swz(r, c), oh[0], oh[1], oh[2], oh[3]);
-                    st_shared_v4(lo + swz(r, c), ol[0], ol[1], ol[2], ol[3]);
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&empty_x[hh]);
-                    mbar_arrive(&ops_ready[b]);
-                }
+                if (lane == 0) mbar_arrive(&ops_ready[pr]);
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&w_free[bf]);
         }
         // Wait for the last UMMAs, then write S_seg of head cw: thread = state row n.
-        const int jl = ntiles * kHeads - 1;
-        wait_abort(&mma_done[jl & 1], (jl >> 1) & 1, abort_p);
-        if (ntiles * kHeads >= 2) wait_abort(&mma_done[(jl - 1) & 1], ((jl - 1) >> 1) & 1, abort_p);
+        wait_abort(&all_done, 0, abort_p);
         tc_fence_after();
         float* dst = seg_state + (((int64_t)sg * H + h0 + cw) * kN + r) * kP;
         for (int half = 0; half < 2; ++half) {
@@ -249,7 +316,6 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
                 d4[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
                                     __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
         }
-        if (r == 0) seg_acum[(int64_t)sg * H + h0 + cw] = suffix / kLog2e;
     }
     tc_fence_before();
     __syncthreads();
