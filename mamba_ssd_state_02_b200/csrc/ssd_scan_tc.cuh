@@ -82,21 +82,22 @@ __device__ __forceinline__ float wg_scan(float a, int q, int lane, float* part) 
 // segment's total sum of dt*A (seg_acum[seg][H]). One CTA per (segment, 4 heads); the
 // chunks run from the segment end backwards so the decay to the end is a running sum.
 //
-// Warp 0 issues the TMA loads, warp 1 the UMMAs, warp 18 scans dt (up to four chunks
-// ahead; w_s = exp(sum_{r > s in seg} dt_r A) dt_s), and the 16 compute warps write
-// w*X as a bf16 hi/lo pair (hi in place over x, lo to its own buffer), so the product
-// keeps ~16 mantissa bits: the FP32 final state is held to 1e-3. Heads go in pairs:
-// per pair one batch of 8 hi + 8 lo UMMAs with N = 128 (both heads side by side, B^T
-// read once for the pair) accumulates S of the two heads in TMEM; while it runs the
-// compute warps prepare the other pair. Compute thread (cw, r) owns token row r and
-// column quarter cw of every head's w*X.
+// Warp 0 issues the TMA loads, warp 1 the UMMAs, warps 18 and 19 scan dt of heads
+// 0-1 and 2-3 (up to four chunks ahead; w_s = exp(sum_{r > s in seg} dt_r A) dt_s), and
+// the 16 compute warps write w*X as a bf16 hi/lo pair (hi in place over x, lo next to
+// it), so the product keeps ~16 mantissa bits: the FP32 final state is held to 1e-3.
+// Heads go in pairs: per pair one batch of 8 UMMAs with N = 256 ([hi|hi|lo|lo] of the
+// two heads side by side, B^T read once) accumulates S_hi and S_lo of the two heads in
+// TMEM; while it runs the compute warps prepare the other pair. At the end S = S_hi +
+// S_lo. Compute thread (cw, r) owns token row r and column quarter cw of every head's
+// w*X.
 //
-// Shared memory: two B stages, X of the 4 heads (one slot each; the pair's slots are
-// refilled as soon as its UMMAs are done), the lo buffers of the 4 heads. TMEM: S_seg
-// of the 4 heads (64 columns each; pair p at columns 128p).
+// Shared memory: two B stages; per head pair [x/hi h0 | x/hi h1 | lo h0 | lo h1] (the
+// pair's X is reloaded as soon as its UMMAs are done). TMEM: per pair p, columns 256p
+// + [S_hi h0 | S_hi h1 | S_lo h0 | S_lo h1] (64 each).
 constexpr int kSmemA = 192 * 1024 + 1024;
-constexpr int kScanWarpA = kRoleWarps + kComputeWarps;         // warp 18: dt scan
-constexpr int kThreadsA = 32 * (kScanWarpA + 1);
+constexpr int kScanWarpA = kRoleWarps + kComputeWarps;         // warps 18, 19: dt scan
+constexpr int kThreadsA = 32 * (kScanWarpA + 2);
 
 __global__ void __launch_bounds__(kThreadsA, 1)
 k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
@@ -110,8 +111,9 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sB = sm;                       // stage st at st*32768: [2][128 s][64 n]
-    uint8_t* sX = sm + 65536;               // head hh at hh*16384: [128 s][64 p]; x, then hi(w*x)
-    uint8_t* sLo = sm + 131072;             // head hh at hh*16384: [128 s][64 p]; lo(w*x)
+    uint8_t* sP = sm + 65536;               // pair p at p*65536: x/hi of its heads, then lo; [128 s][64 p] each
+    auto xs = [&](int hh) { return sP + (hh >> 1) * 65536 + (hh & 1) * 16384; };           // x, then hi
+    auto los = [&](int hh) { return sP + (hh >> 1) * 65536 + 32768 + (hh & 1) * 16384; };  // lo
     __shared__ __align__(16) float wts[4][kHeads][kTile];
     __shared__ uint64_t full_b[2], empty_b[2], full_x[2], pair_done[2], ops_ready[2], w_ready[4], w_free[4], all_done;
     __shared__ uint32_t tmem_slot;
@@ -131,7 +133,7 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
             mbar_init(&ops_ready[i], kComputeWarps);
         }
         for (int i = 0; i < 4; ++i) {
-            mbar_init(&w_ready[i], 1);
+            mbar_init(&w_ready[i], 2);
             mbar_init(&w_free[i], kComputeWarps);
         }
         mbar_init(&all_done, 1);
@@ -141,13 +143,13 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
         prefetch_tmap(&map_b);
     }
     if (warp == 1) {
-        tmem_alloc(&tmem_slot, 256);
+        tmem_alloc(&tmem_slot, 512);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tS = tmem_slot;          // head hh at columns [64 hh, 64 hh + 64)
+    const uint32_t tS = tmem_slot;
     volatile int* abort_p = &abort_flag;
 
     if (warp == 0) {
@@ -170,16 +172,16 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
                     if (k >= 1) wait_abort(&pair_done[pr], (k - 1) & 1, abort_p);   // slots and lo free
                     mbar_arrive_expect_tx(&full_x[pr], 32768);
                     for (int hh = 2 * pr; hh < 2 * pr + 2; ++hh)
-                        tma_load_3d(sX + hh * 16384, &map_x, &full_x[pr], 0, h0 + hh, t0);
+                        tma_load_3d(xs(hh), &map_x, &full_x[pr], 0, h0 + hh, t0);
                 }
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ UMMA issuer
-        // S[n][p] of a head pair += B^T (hi + lo): A = B^T (MN-major), B = [hi|lo] of the
-        // pair (MN-major, the two heads 16 KB apart), N = 128.
-        const uint32_t idesc = idesc_bf16(128, 128, 1, 1);
-        const uint64_t dHi = smem_desc(smem_u32(sX), 16384, 1024), dLo = smem_desc(smem_u32(sLo), 16384, 1024);
+        // [S_hi|S_lo] of a head pair += B^T [hi h0|hi h1|lo h0|lo h1]: A = B^T (MN-major),
+        // B MN-major with its four 64-column blocks 16 KB apart, N = 256.
+        const uint32_t idesc = idesc_bf16(128, 256, 1, 1);
+        const uint64_t dP = smem_desc(smem_u32(sP), 16384, 1024);
         for (int k = 0; k < ntiles; ++k) {
             const int st = k & 1;
             wait_abort(&full_b[st], (k >> 1) & 1, abort_p);
@@ -187,15 +189,12 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
             for (int pr = 0; pr < 2; ++pr) {
                 wait_abort(&ops_ready[pr], k & 1, abort_p);
                 tc_fence_after();
-                const uint32_t d = tS + pr * 128;
-                const uint64_t dh = desc_add(dHi, pr * 32768), dl = desc_add(dLo, pr * 32768);
+                const uint32_t d = tS + pr * 256;
+                const uint64_t dp = desc_add(dP, pr * 65536);
                 if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        umma_bf16(d, desc_add(dB, kk * kMnStep), desc_add(dh, kk * kMnStep), idesc, !(k == 0 && kk == 0));
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        umma_bf16(d, desc_add(dB, kk * kMnStep), desc_add(dl, kk * kMnStep), idesc, true);
+                        umma_bf16(d, desc_add(dB, kk * kMnStep), desc_add(dp, kk * kMnStep), idesc, !(k == 0 && kk == 0));
                     umma_commit(&pair_done[pr]);
                     if (pr == 1) umma_commit(&empty_b[st]);
                     if (pr == 1 && k == ntiles - 1) umma_commit(&all_done);
@@ -203,27 +202,29 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
                 __syncwarp();
             }
         }
-    } else if (warp == kScanWarpA) {
+    } else if (warp >= kScanWarpA) {
         // ------------------------------------------------------------ dt scan
-        // Lane l holds tokens 4l..4l+3 of a chunk; the dt_raw of the next chunk is loaded
-        // while this one is scanned. suf[hh] = sum of dt*A after the current chunk (log2).
-        float bias[kHeads], Ah[kHeads], suf[kHeads];
+        // Warp 18 + i scans heads 2i, 2i+1. Lane l holds tokens 4l..4l+3 of a chunk; the
+        // dt_raw of the next chunk is loaded while this one is scanned. suf[e] = sum of
+        // dt*A after the current chunk (log2 units).
+        const int hb = 2 * (warp - kScanWarpA);
+        float bias[2], Ah[2], suf[2];
 #pragma unroll
-        for (int hh = 0; hh < kHeads; ++hh) {
-            bias[hh] = dt_bias[h0 + hh];
-            Ah[hh] = A[h0 + hh] * kLog2e;
-            suf[hh] = 0.f;
-            if (lane == 0 && (!(A[h0 + hh] <= 0.f) || isinf(A[h0 + hh]))) latch_error(SSD_ERR_INVALID_ARG);
+        for (int e = 0; e < 2; ++e) {
+            bias[e] = dt_bias[h0 + hb + e];
+            Ah[e] = A[h0 + hb + e] * kLog2e;
+            suf[e] = 0.f;
+            if (lane == 0 && (!(A[h0 + hb + e] <= 0.f) || isinf(A[h0 + hb + e]))) latch_error(SSD_ERR_INVALID_ARG);
         }
-        float z[kHeads][4], zn[kHeads][4];
-        auto load_dt = [&](int k, float (&zz)[kHeads][4]) {
+        float z[2][4], zn[2][4];
+        auto load_dt = [&](int k, float (&zz)[2][4]) {
             const int it = ntiles - 1 - k;
             const int tlk = min(kTile, seg.len - it * kTile);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const int64_t row = ((int64_t)seg.start + (int64_t)it * kTile + 4 * lane + i) * H + h0;
+                const int64_t row = ((int64_t)seg.start + (int64_t)it * kTile + 4 * lane + i) * H + h0 + hb;
 #pragma unroll
-                for (int hh = 0; hh < kHeads; ++hh) zz[hh][i] = 4 * lane + i < tlk ? dt_raw[row + hh] : 0.f;
+                for (int e = 0; e < 2; ++e) zz[e][i] = 4 * lane + i < tlk ? dt_raw[row + e] : 0.f;
             }
         };
         load_dt(0, zn);
@@ -231,18 +232,18 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
             const int bf = k % 4, it = ntiles - 1 - k;
             const int tlk = min(kTile, seg.len - it * kTile);
 #pragma unroll
-            for (int hh = 0; hh < kHeads; ++hh)
+            for (int e = 0; e < 2; ++e)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) z[hh][i] = zn[hh][i];
+                for (int i = 0; i < 4; ++i) z[e][i] = zn[e][i];
             if (k + 1 < ntiles) load_dt(k + 1, zn);
             if (k >= 4) wait_abort(&w_free[bf], ((k >> 2) - 1) & 1, abort_p);
 #pragma unroll
-            for (int hh = 0; hh < kHeads; ++hh) {
+            for (int e = 0; e < 2; ++e) {
                 float dtv[4], p[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    dtv[i] = 4 * lane + i < tlk ? softplus_fast(z[hh][i] + bias[hh]) : 0.f;
-                    p[i] = (i ? p[i - 1] : 0.f) + dtv[i] * Ah[hh];
+                    dtv[i] = 4 * lane + i < tlk ? softplus_fast(z[e][i] + bias[e]) : 0.f;
+                    p[i] = (i ? p[i - 1] : 0.f) + dtv[i] * Ah[e];
                 }
                 float incl = p[3];
 #pragma unroll
@@ -251,22 +252,17 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
                     if (lane >= off) incl += v;
                 }
                 const float tot = __shfl_sync(0xffffffffu, incl, 31);
-                const float base = suf[hh] + tot - (incl - p[3]);   // decay exponent of token 4l, plus p[i] below
+                const float base = suf[e] + tot - (incl - p[3]);    // decay exponent of token 4l, plus p[i] below
                 float w[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) w[i] = fast_exp2(base - p[i]) * dtv[i];
-                *reinterpret_cast<float4*>(&wts[bf][hh][4 * lane]) = make_float4(w[0], w[1], w[2], w[3]);
-                suf[hh] += tot;
+                *reinterpret_cast<float4*>(&wts[bf][hb + e][4 * lane]) = make_float4(w[0], w[1], w[2], w[3]);
+                suf[e] += tot;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&w_ready[bf]);
         }
-        if (lane < kHeads) {
-            float v = suf[0];
-#pragma unroll
-            for (int hh = 1; hh < kHeads; ++hh) v = lane == hh ? suf[hh] : v;
-            seg_acum[(int64_t)sg * H + h0 + lane] = v / kLog2e;
-        }
+        if (lane < 2) seg_acum[(int64_t)sg * H + h0 + hb + lane] = (lane ? suf[1] : suf[0]) / kLog2e;
     } else {
         // ------------------------------------------------------------ compute warps
         const int cw = (warp - kRoleWarps) >> 2, q = warp & 3, r = q * 32 + lane;
@@ -279,7 +275,7 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
                 for (int hh = 2 * pr; hh < 2 * pr + 2; ++hh) {
                     const float w = wts[bf][hh][r];
                     const float2 w2 = make_float2(w, w);
-                    const uint32_t xrow = smem_u32(sX + hh * 16384), lrow = smem_u32(sLo + hh * 16384);
+                    const uint32_t xrow = smem_u32(xs(hh)), lrow = smem_u32(los(hh));
 #pragma unroll
                     for (int c = 2 * cw; c < 2 * cw + 2; ++c) {
                         const uint4 v = ld_shared_v4(xrow + swz(r, c));
@@ -306,20 +302,24 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
         wait_abort(&all_done, 0, abort_p);
         tc_fence_after();
         float* dst = seg_state + (((int64_t)sg * H + h0 + cw) * kN + r) * kP;
+        const uint32_t thi = tS + ((uint32_t)(q * 32) << 16) + (cw >> 1) * 256 + (cw & 1) * 64;
         for (int half = 0; half < 2; ++half) {
-            uint32_t v[32];
-            tmem_ld32(tS + ((uint32_t)(q * 32) << 16) + cw * 64 + half * 32, v);
+            uint32_t vh[32], vl[32];
+            tmem_ld32(thi + half * 32, vh);
+            tmem_ld32(thi + 128 + half * 32, vl);
             tmem_wait_ld();
             float4* d4 = reinterpret_cast<float4*>(dst + half * 32);
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-                d4[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                                    __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+                d4[e] = make_float4(__uint_as_float(vh[4 * e]) + __uint_as_float(vl[4 * e]),
+                                    __uint_as_float(vh[4 * e + 1]) + __uint_as_float(vl[4 * e + 1]),
+                                    __uint_as_float(vh[4 * e + 2]) + __uint_as_float(vl[4 * e + 2]),
+                                    __uint_as_float(vh[4 * e + 3]) + __uint_as_float(vl[4 * e + 3]));
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) tmem_dealloc(tS, 256);
+    if (warp == 1) tmem_dealloc(tS, 512);
 }
 
 // ---------------------------------------------------------------------------------
