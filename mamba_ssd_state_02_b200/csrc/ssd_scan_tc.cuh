@@ -416,8 +416,8 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
     __shared__ __align__(16) float dts[4][kHeadsB][kTile];
     __shared__ __align__(16) float uw[4][kHeadsB][kTile];
     __shared__ __align__(16) float ww[4][kHeadsB][kTile];
-    __shared__ uint64_t full_cb, s_done, zs_done, full_x[2], cb_done, ops_ready, mma_done, l_ready, dt_ready[4],
-        dt_free[4], y_staged;
+    __shared__ uint64_t full_b, full_c[2], s_done, zs_done, full_x[2], cb_done, ops_ready, y0_done, mma_done, l_ready,
+        dt_ready[4], dt_free[4], y_staged;
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
 
@@ -427,7 +427,10 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
     const int ntiles = (seg.len + kTile - 1) / kTile;
 
     if (tid == 0) {
-        mbar_init(&full_cb, 1);
+        mbar_init(&full_b, 1);
+        mbar_init(&full_c[0], 1);
+        mbar_init(&full_c[1], 1);
+        mbar_init(&y0_done, 1);
         mbar_init(&s_done, 1);
         mbar_init(&zs_done, 1);
         for (int sl = 0; sl < 2; ++sl) mbar_init(&full_x[sl], 1);
@@ -467,15 +470,21 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 for (int hh = 0; hh < kHeadsB; ++hh)
                     tma_load_3d(sX + sl * 32768 + hh * 16384, &map_x, &full_x[sl], 0, h0 + hh, seg.start + j * kTile);
             };
-            // C and B of chunk j; those of chunk j+1 and X of chunk j+1 are prefetched into
-            // L2 meanwhile, so the loads that follow find them there.
-            auto load_cb = [&](int j) {
+            // B of chunk j (once the S UMMAs of chunk j-1 are done) and the two halves of
+            // C (once Z is done), on separate barriers, so C B^T can start on the first
+            // half. B, C and X of chunk j+1 are prefetched into L2 meanwhile.
+            auto load_b = [&](int j) {
                 const int t0 = seg.start + j * kTile;
-                mbar_arrive_expect_tx(&full_cb, 65536);
-                tma_load_3d(sC, &map_c, &full_cb, 0, g, t0);
-                tma_load_3d(sC + 16384, &map_c, &full_cb, 64, g, t0);
-                tma_load_3d(sB, &map_b, &full_cb, 0, g, t0);
-                tma_load_3d(sB + 16384, &map_b, &full_cb, 64, g, t0);
+                mbar_arrive_expect_tx(&full_b, 32768);
+                tma_load_3d(sB, &map_b, &full_b, 0, g, t0);
+                tma_load_3d(sB + 16384, &map_b, &full_b, 64, g, t0);
+            };
+            auto load_c = [&](int j) {
+                const int t0 = seg.start + j * kTile;
+                for (int hf = 0; hf < 2; ++hf) {
+                    mbar_arrive_expect_tx(&full_c[hf], 16384);
+                    tma_load_3d(sC + hf * 16384, &map_c, &full_c[hf], 64 * hf, g, t0);
+                }
                 if (j + 1 < ntiles) {
                     tma_prefetch_3d(&map_c, 0, g, t0 + kTile);
                     tma_prefetch_3d(&map_c, 64, g, t0 + kTile);
@@ -494,12 +503,17 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                     bulk_commit_group();
                 }
             };
-            if (ntiles > 0) load_x(0);
-            if (ntiles > 1) load_x(1);
-            if (ntiles > 0) load_cb(0);
+            if (ntiles > 0) {
+                load_x(0);
+                if (ntiles > 1) load_x(1);
+                load_b(0);
+                load_c(0);
+            }
             for (int j = 1; j < ntiles; ++j) {
-                wait_abort(&zs_done, (j - 1) & 1, abort_p);         // C/B of chunk j-1 read
-                load_cb(j);
+                wait_abort(&s_done, (j - 1) & 1, abort_p);          // B of chunk j-1 read
+                load_b(j);
+                wait_abort(&zs_done, (j - 1) & 1, abort_p);         // C of chunk j-1 read
+                load_c(j);
                 store_y(j - 1);
                 if (j + 1 < ntiles) {
                     bulk_wait_read_all();                           // slot (j+1) & 1 read by the store
@@ -518,17 +532,23 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
         const uint64_t dBm = smem_desc(smem_u32(sB), 16384, 1024);
         const uint64_t dH = smem_desc(smem_u32(sH), 16384, 1024), dW = smem_desc(smem_u32(sW), 16384, 1024);
         const uint64_t dX = smem_desc(smem_u32(sX), 16384, 1024);
-        // C B^T of chunk j into the M columns (fp32), once its C/B tiles have landed.
+        // C B^T of chunk j into the M columns (fp32): dstate columns 0..63 once B and the
+        // first half of C have landed, 64..127 once the second half has.
         auto issue_cb = [&](int j) {
-            wait_abort(&full_cb, j & 1, abort_p);
-            tc_fence_after();
-            if (elect_one()) {
+            wait_abort(&full_b, j & 1, abort_p);
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    umma_bf16(tM, desc_add(dCk, kmajor_step(128, k)), desc_add(dBk, kmajor_step(128, k)), id_cb, k > 0);
-                umma_commit(&cb_done);
+            for (int hf = 0; hf < 2; ++hf) {
+                wait_abort(&full_c[hf], j & 1, abort_p);
+                tc_fence_after();
+                if (elect_one()) {
+#pragma unroll
+                    for (int k = 4 * hf; k < 4 * hf + 4; ++k)
+                        umma_bf16(tM, desc_add(dCk, kmajor_step(128, k)), desc_add(dBk, kmajor_step(128, k)), id_cb,
+                                  k > 0);
+                    if (hf == 1) umma_commit(&cb_done);
+                }
+                __syncwarp();
             }
-            __syncwarp();
         };
         if (ntiles > 0) issue_cb(0);
         for (int it = 0; it < ntiles; ++it) {
@@ -547,6 +567,7 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 // M of head hh, sources 16k..16k+15: TMEM columns 16k + 8hh of the M block.
 #pragma unroll
                 for (int k = 0; k < 8; ++k) umma_bf16_ts(tY, tM + 16 * k, desc_add(dX0, k * kMnStep), id_y, k > 0);
+                umma_commit(&y0_done);
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
                     umma_bf16_ts(tY + 64, tM + 16 * k + 8, desc_add(dX1, k * kMnStep), id_y, k > 0);
@@ -828,7 +849,7 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             // -------- drain: y rows (into the chunk's X slot for a full chunk, else
             // straight to HBM). The TMEM loads of the next 8-column piece are issued before the
             // current one is consumed.
-            wait_abort(&mma_done, it & 1, abort_p);
+            wait_abort(&y0_done, it & 1, abort_p);
             tc_fence_after();
             {
                 const bool staged = tl == kTile;
@@ -841,6 +862,10 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 for (int piece = 0; piece < 4; ++piece) {           // (head, half) = (piece/2, piece%2)
                     const int hh = piece >> 1, half = piece & 1, cur = piece & 1;
                     tmem_wait_ld();
+                    if (piece == 1) {                               // head 1's Y needs all Y UMMAs
+                        wait_abort(&mma_done, it & 1, abort_p);
+                        tc_fence_after();
+                    }
                     if (piece < 3) {
                         const int nh = (piece + 1) >> 1, nf = (piece + 1) & 1;
                         tmem_ld8(tY + nh * 64 + lane_off + 16 * cw + 8 * nf, ry[cur ^ 1]);
