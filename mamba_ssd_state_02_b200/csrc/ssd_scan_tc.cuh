@@ -375,8 +375,8 @@ k_tc_segment_passing(float* __restrict__ seg_state, const float* __restrict__ se
 // X slot (full chunks) and warp 0 stores the tile with one TMA store per head, then
 // loads chunk j+2's X into the slot (prefetched into L2 a chunk earlier). The UMMA warp
 // issues chunk j+1's C B^T as soon as the Y UMMAs have read M, so it overlaps the
-// drain. Warp 18 scans dt*A up to four chunks ahead; while S and Z run, warpgroups 2
-// and 3 tabulate chunk j+1's diagonal-block decays.
+// drain. Warp 18 scans dt*A up to four chunks ahead; while S and Z run, the compute
+// warps tabulate chunk j+1's diagonal-block decays.
 //
 // M of row block q (TMEM lane quarter q) has source blocks 0..q-1 below the diagonal,
 // written as CB * exp2(Acum_t - Acum_e) * exp2(Acum_e - Acum_s) dt_s with e the last
@@ -442,7 +442,7 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             mbar_init(&dt_ready[i], 1);
             mbar_init(&dt_free[i], kComputeWarps);
         }
-        mbar_init(&l_ready, 8);
+        mbar_init(&l_ready, kComputeWarps);
         abort_flag = 0;
         fence_barrier_init();
         prefetch_tmap(&map_x);
@@ -667,22 +667,23 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
         }
         const float Dh0 = D[h0], Dh1 = D[h0 + 1];
         // Decays of the diagonal 32x32 blocks of chunk j, L[t][s] = exp2(Acum_t - Acum_s)
-        // dt_s for s <= t in t's block (fp16, row t = r of head cw - 2; warpgroups 2, 3).
-        // 16-byte chunk c of row t sits at chunk c ^ ((t >> 1) & 3).
+        // dt_s for s <= t in t's block (fp16). Thread (cw, r) writes row t = r of head
+        // cw & 1, sources 16 (cw >> 1) .. +15 of the block. 16-byte chunk c of a row sits
+        // at chunk c ^ ((t >> 1) & 3).
         auto diag_decays = [&](int j) {
-            const int bf = j % 4, hd = cw - kHeadsB;
+            const int bf = j % 4, hd = cw & 1, c0 = 2 * (cw >> 1);
             wait_abort(&dt_ready[bf], (j / 4) & 1, abort_p);
             const float at = ac2[bf][hd][r];
-            const float4* a4 = reinterpret_cast<const float4*>(&ac2[bf][hd][32 * q]);
-            const float4* d4 = reinterpret_cast<const float4*>(&dts[bf][hd][32 * q]);
+            const float4* a4 = reinterpret_cast<const float4*>(&ac2[bf][hd][32 * q + 8 * c0]);
+            const float4* d4 = reinterpret_cast<const float4*>(&dts[bf][hd][32 * q + 8 * c0]);
             const uint32_t row = smem_u32(sL + hd * 8192 + r * 64);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
                 uint32_t o[4];
 #pragma unroll
                 for (int k2 = 0; k2 < 2; ++k2) {
                     const float4 as = a4[2 * c + k2], dv = d4[2 * c + k2];
-                    const int s0 = 8 * c + 4 * k2;          // source offset within the block
+                    const int s0 = 8 * (c0 + c) + 4 * k2;   // source offset within the block
                     const float l0 = s0 <= lane ? fast_exp2(at - as.x) * dv.x : 0.f;
                     const float l1 = s0 + 1 <= lane ? fast_exp2(at - as.y) * dv.y : 0.f;
                     const float l2 = s0 + 2 <= lane ? fast_exp2(at - as.z) * dv.z : 0.f;
@@ -690,7 +691,7 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                     o[2 * k2] = pack_f16(l0, l1);
                     o[2 * k2 + 1] = pack_f16(l2, l3);
                 }
-                st_shared_v4(row + ((c ^ ((r >> 1) & 3)) << 4), o[0], o[1], o[2], o[3]);
+                st_shared_v4(row + (((c0 + c) ^ ((r >> 1) & 3)) << 4), o[0], o[1], o[2], o[3]);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&l_ready);
@@ -728,7 +729,7 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             }
         };
 
-        if (cw >= kHeadsB) diag_decays(0);
+        diag_decays(0);
         stage_h();
         stage_wx(0);
 
@@ -815,9 +816,9 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&ops_ready);
-            // -------- while S and Z run: warpgroups 2/3 tabulate chunk it+1's diagonal
+            // -------- while S and Z run: all compute warps tabulate chunk it+1's diagonal
             // decays once every warp has read chunk it's (ops_ready complete).
-            if (cw >= kHeadsB && it + 1 < ntiles) {
+            if (it + 1 < ntiles) {
                 wait_abort(&ops_ready, it & 1, abort_p);
                 diag_decays(it + 1);
             }
