@@ -228,6 +228,58 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+class NvmlSampler:
+    """SM clock and clock-event reasons read through NVML (the library nvidia-smi
+    reports from) every ~2 ms on a background thread, so that a timed region of a few
+    milliseconds still gets several samples. Read-only: no setting is changed."""
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20, "sw_power_cap": 0x4}
+
+    def __init__(self, device):
+        self.samples, self.thread, self.ok = [], None, False
+        try:
+            import pynvml
+            self.nv = pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_flag:
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.time(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def start(self):
+        if not self.ok:
+            return
+        import threading
+        self.stop_flag = False
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def stop(self, window):
+        if not self.ok or self.thread is None:
+            return None
+        self.stop_flag = True
+        self.thread.join(timeout=2)
+        sel = [x for x in self.samples if window[0] <= x[0] <= window[1]]
+        if not sel:
+            return None
+        reasons = sorted({k for _, _, rs in sel for k, bit in self.REASONS.items() if rs & bit})
+        return {"sm_mhz": statistics.median([m for _, m, _ in sel]), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(sel), "source": "nvml"}
+
+
 # ------------------------------------------------------------------------------ oracle baseline
 def oracle_sample(w: W.Workload, tokens: int, heads: int, seed_rank: int = 0):
     """Time the FP64 oracle (as it stands) on the first `tokens` tokens of sequence 0
@@ -284,7 +336,9 @@ def bench_ours(args, rank, world, local_rank):
     stream = torch.cuda.current_stream(dev)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(dev)
+    nvml_clocks = NvmlSampler(dev)
     clocks.start()
+    nvml_clocks.start()
     time.sleep(0.3)
     barrier(dev)
     torch.cuda.synchronize(dev)
@@ -301,7 +355,8 @@ def bench_ours(args, rank, world, local_rank):
     kprof = ssd.profile_read()
     ssd.profile_enable(False)
     time.sleep(0.1)
-    clk = clocks.stop((t_wall0, t_wall1))
+    clk_smi = dict(clocks.stop((t_wall0, t_wall1)), source="nvidia-smi")
+    clk = nvml_clocks.stop((t_wall0, t_wall1)) or clk_smi
     ssd.device_status()
     ms_step = max_over_ranks(ms_total / args.steps, dev)
     value = world * w.total_tokens / (ms_step / 1e3)
