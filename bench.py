@@ -422,6 +422,32 @@ def bench_ours(args, rank, world, local_rank):
     del host, dbuf, inp, x, dtr, Bm, Cm, y, ws
     torch.cuda.empty_cache()
 
+    # ---- state snapshots every 2048 tokens on the same workload (prefix-cache reuse)
+    snap_every = 2048
+    n_snap = ssd.snapshot_count(dims, snap_every)
+    snaps = torch.empty(n_snap, w.nheads, w.headdim, w.dstate, dtype=torch.float32, device=dev)
+    ws_snap = torch.empty(ssd.snapshot_workspace_size(dims, w.chunk, snap_every), dtype=torch.uint8, device=dev)
+
+    def snap_step():
+        ssd.scan_fwd(x, dtr, inp["dt_bias"], inp["A"], Bm, Cm, inp["D"], init_state=inp["init_state"],
+                     chunk=w.chunk, y=y, final_state=fin, workspace=ws_snap, snapshot_tokens=snap_every,
+                     snapshots=snaps)
+
+    for _ in range(args.warmup):
+        snap_step()
+    ssd.device_status()
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        snap_step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    snap_ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dev)
+    snapshots = {"interval_tokens": snap_every, "snapshots_per_step": n_snap,
+                 "snapshot_bytes_per_step": snaps.numel() * 4, "ms_per_step": round(snap_ms, 4),
+                 "overhead_vs_plain": round(snap_ms / ms_step - 1.0, 4)}
+
     # ---- decode (256 sequences, FP32 states from a 2048-token prefill)
     decode = bench_decode(args, ssd, dev, rank, world, hbm, peak_src)
 
@@ -437,6 +463,7 @@ def bench_ours(args, rank, world, local_rank):
         "roofline": roofline, "path_roofline": path_roof, "kernels": kernels,
         "clocks": clk, "e2e": e2e, "gpu_launches": launches_per_call * args.steps,
         "decode": decode,
+        "snapshots": snapshots,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, threads, secs = oracle_sample(w, 16384, w.nheads)

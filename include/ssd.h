@@ -117,6 +117,40 @@ ssd_status ssd_scan_fwd(const void* x, const float* dt_raw, const float* dt_bias
                         const ssd_dims* dims, int chunk, ssd_stream_t stream);
 
 /*
+ * ssd_scan_fwd that also returns the state at fixed token intervals of every
+ * sequence: state snapshots for prefix-cache reuse and chunked prefill (RL-Kernel
+ * issue page: §1 names Mamba prefix-cache reuse as a serving feature, §7 and §8 Q4
+ * tie it to sequence-anchored chunk boundaries). Snapshot k (k = 1, 2, ...) of a sequence is its state after its first
+ * k * snapshot_tokens tokens, for every k with k * snapshot_tokens <= its length
+ * (the last one equals final_state when the length is a multiple).
+ *   snapshots: [n_snap,H,P,N] float32 output, 16-byte aligned, where n_snap is the
+ *     sum over sequences of floor(length / snapshot_tokens) (ssd_snapshot_count),
+ *     ordered by sequence, then by k.
+ *   snapshot_tokens: > 0; a multiple of 128 on the tensor-core pipeline (which then
+ *     uses segments that divide it), a multiple of `chunk` on the CUDA-core pipeline;
+ *     otherwise SSD_ERR_UNSUPPORTED.
+ *   dims->workspace, if given, must hold ssd_scan_fwd_snapshots_workspace_size bytes.
+ * Everything else is as in ssd_scan_fwd; y and final_state are the same.
+ */
+ssd_status ssd_scan_fwd_snapshots(const void* x, const float* dt_raw, const float* dt_bias, const float* A,
+                                  const void* B, const void* C, const float* D, const float* init_state,
+                                  const int32_t* cu_seqlens, void* y, float* final_state, float* snapshots,
+                                  int64_t snapshot_tokens, const ssd_dims* dims, int chunk,
+                                  ssd_stream_t stream);
+
+/* Workspace bytes for ssd_scan_fwd_snapshots (as ssd_scan_fwd_workspace_size). */
+ssd_status ssd_scan_fwd_snapshots_workspace_size(const ssd_dims* dims, int chunk, int64_t snapshot_tokens,
+                                                 size_t* bytes);
+
+/*
+ * Number of snapshots ssd_scan_fwd_snapshots writes, into *count. cu_seqlens_host is
+ * a HOST copy of cu_seqlens ([dims->nseq + 1]) for a varlen call, or NULL for a
+ * dense call (dims->batch sequences of dims->seqlen tokens).
+ */
+ssd_status ssd_snapshot_count(const ssd_dims* dims, const int32_t* cu_seqlens_host, int64_t snapshot_tokens,
+                              int64_t* count);
+
+/*
  * One decode step for nseq = dims->batch sequences (dims->seqlen must be 1; varlen
  * fields are ignored): per sequence and head, dt = softplus(dt_raw + dt_bias),
  * state <- exp(dt*A) * state + dt * x B^T in place, y = state . C + D * x.

@@ -68,6 +68,11 @@ struct Plan {
     int Ls = 0;
     int64_t max_segs = 0;
     size_t off_seg_acum = 0;
+    // state snapshots every `snap` tokens of each sequence (0: none), written to
+    // snap_out; per-sequence index of the first snapshot in the workspace
+    int64_t snap = 0;
+    size_t off_snap_first = 0;
+    float* snap_out = nullptr;
 };
 
 }  // namespace ssd

@@ -136,7 +136,7 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Validate dims/chunk and fill the plan (no pointers looked at here).
-ssd_status make_plan(const ssd_dims* d, int chunk, bool varlen, Plan* pl) {
+ssd_status make_plan(const ssd_dims* d, int chunk, bool varlen, Plan* pl, int64_t snap = 0) {
     if (!d) return fail(SSD_ERR_INVALID_ARG, "dims is NULL");
     if (d->nheads <= 0 || d->headdim <= 0 || d->ngroups <= 0 || d->dstate <= 0)
         return fail(SSD_ERR_INVALID_ARG, "nheads, headdim, ngroups and dstate must be positive");
@@ -199,9 +199,21 @@ ssd_status make_plan(const ssd_dims* d, int chunk, bool varlen, Plan* pl) {
             const int v = atoi(e);
             if (v >= tc::kTile && v % tc::kTile == 0 && v <= (1 << 20)) Ls = v;
         }
+        if (snap > 0) {                 // segment boundaries must fall on every snapshot
+            if (snap % tc::kTile != 0)
+                return fail(SSD_ERR_UNSUPPORTED, "snapshot_tokens (%lld) must be a multiple of %d here",
+                            (long long)snap, tc::kTile);
+            if (snap < Ls) Ls = (int)snap;
+            while (snap % Ls != 0) Ls -= tc::kTile;
+        }
         p.Ls = Ls;
         p.max_segs = segs_for(Ls);
     }
+    if (snap < 0) return fail(SSD_ERR_INVALID_ARG, "snapshot_tokens must be >= 0");
+    if (snap > 0 && !p.tc && snap % chunk != 0)
+        return fail(SSD_ERR_UNSUPPORTED, "snapshot_tokens (%lld) must be a multiple of chunk (%d) here",
+                    (long long)snap, chunk);
+    p.snap = snap;
     // Workspace carving (256-byte aligned pieces).
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -225,6 +237,7 @@ ssd_status make_plan(const ssd_dims* d, int chunk, bool varlen, Plan* pl) {
         p.off_acum = take(sizeof(float) * mc * p.H * p.Q);
         p.off_states = take(sizeof(float) * mc * p.H * p.P * p.N);
     }
+    if (snap > 0) p.off_snap_first = take(sizeof(int32_t) * ((size_t)p.nseq + 1));
     p.bytes = off;
     *pl = p;
     return SSD_OK;
@@ -247,7 +260,8 @@ ssd_status launch_simt(const Plan& pl, char* ws, const T* x, const float* dt_raw
     int n = 0;
     {
         StageScope sc(ST_TABLE, st);
-        k_chunk_table<<<1, kTableThreads, 0, st>>>(cu, pl.nseq, pl.T, pl.seqlen, Q, table, first, count);
+        k_chunk_table<<<1, kTableThreads, 0, st>>>(cu, pl.nseq, pl.T, pl.seqlen, Q, table, first, count, pl.snap,
+                                                   reinterpret_cast<int32_t*>(ws + pl.off_snap_first));
     }
     ++n;
     if (pl.max_chunks > 0) {
@@ -267,7 +281,8 @@ ssd_status launch_simt(const Plan& pl, char* ws, const T* x, const float* dt_raw
     if (pl.nseq > 0) {
         StageScope sc(ST_STATE_PASSING, st);
         k_state_passing<Q><<<dim3(pl.nseq, H, (P * N + 255) / 256), 256, 0, st>>>(
-            states, acum, table, first, init, fin, H, P * N);
+            states, acum, table, first, init, fin, H, P * N, pl.snap,
+            reinterpret_cast<const int32_t*>(ws + pl.off_snap_first), pl.snap_out);
         ++n;
     }
     if (pl.max_chunks > 0) {
@@ -300,7 +315,8 @@ ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_ra
     int n = 0;
     {
         StageScope sc(ST_TABLE, st);
-        k_chunk_table<<<1, kTableThreads, 0, st>>>(cu, pl.nseq, pl.T, pl.seqlen, pl.Ls, table, first, count);
+        k_chunk_table<<<1, kTableThreads, 0, st>>>(cu, pl.nseq, pl.T, pl.seqlen, pl.Ls, table, first, count,
+                                                   pl.snap, reinterpret_cast<int32_t*>(ws + pl.off_snap_first));
     }
     ++n;
     if (pl.max_segs > 0 && pl.T > 0) {
@@ -326,7 +342,8 @@ ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_ra
         {
             StageScope sc(ST_STATE_PASSING, st);
             tc::k_tc_segment_passing<<<dim3(pl.nseq, H, (tc::kP * tc::kN) / 256), 256, 0, st>>>(
-                seg_state, seg_acum, first, init, fin, H);
+                seg_state, seg_acum, first, init, fin, H, table, pl.snap,
+                reinterpret_cast<const int32_t*>(ws + pl.off_snap_first), pl.snap_out);
         }
         ++n;
         {
@@ -338,7 +355,8 @@ ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_ra
     } else {
         StageScope sc(ST_STATE_PASSING, st);
         tc::k_tc_segment_passing<<<dim3(pl.nseq, H, (tc::kP * tc::kN) / 256), 256, 0, st>>>(
-            seg_state, seg_acum, first, init, fin, H);
+            seg_state, seg_acum, first, init, fin, H, table, pl.snap,
+                reinterpret_cast<const int32_t*>(ws + pl.off_snap_first), pl.snap_out);
         ++n;
     }
     cudaError_t e = cudaGetLastError();
@@ -424,12 +442,18 @@ ssd_status ssd_scan_fwd_workspace_size(const ssd_dims* dims, int chunk, size_t* 
     return SSD_OK;
 }
 
-ssd_status ssd_scan_fwd(const void* x, const float* dt_raw, const float* dt_bias, const float* A,
-                        const void* B, const void* C, const float* D, const float* init_state,
-                        const int32_t* cu_seqlens, void* y, float* final_state,
-                        const ssd_dims* dims, int chunk, ssd_stream_t stream) {
+}  // extern "C"
+
+namespace ssd {
+namespace {
+
+// ssd_scan_fwd and ssd_scan_fwd_snapshots: validate, find scratch, launch.
+ssd_status scan_fwd_impl(const void* x, const float* dt_raw, const float* dt_bias, const float* A, const void* B,
+                         const void* C, const float* D, const float* init_state, const int32_t* cu_seqlens,
+                         void* y, float* final_state, float* snapshots, int64_t snapshot_tokens,
+                         const ssd_dims* dims, int chunk, ssd_stream_t stream) {
     Plan pl;
-    ssd_status s = make_plan(dims, chunk, cu_seqlens != nullptr, &pl);
+    ssd_status s = make_plan(dims, chunk, cu_seqlens != nullptr, &pl, snapshot_tokens);
     if (s != SSD_OK) return s;
     if (!dt_bias || !A || !D) return fail(SSD_ERR_INVALID_ARG, "dt_bias, A and D must be non-NULL");
     if (pl.T > 0 && (!x || !dt_raw || !B || !C || !y))
@@ -439,6 +463,9 @@ ssd_status ssd_scan_fwd(const void* x, const float* dt_raw, const float* dt_bias
     if (!aligned(dt_raw, 4) || !aligned(dt_bias, 4) || !aligned(A, 4) || !aligned(D, 4) ||
         !aligned(init_state, 16) || !aligned(final_state, 16) || !aligned(cu_seqlens, 4))
         return fail(SSD_ERR_INVALID_ARG, "float/int arrays must be 4-byte aligned, states 16-byte");
+    if (snapshot_tokens > 0 && (!snapshots || !aligned(snapshots, 16)))
+        return fail(SSD_ERR_INVALID_ARG, "snapshots must be a non-NULL 16-byte aligned array");
+    pl.snap_out = snapshots;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (pl.nseq == 0) {
         t_launches = 0;
@@ -471,6 +498,66 @@ ssd_status ssd_scan_fwd(const void* x, const float* dt_raw, const float* dt_bias
     }
     if (s == SSD_OK) t_last_error.clear();
     return s;
+}
+
+}  // namespace
+}  // namespace ssd
+
+extern "C" {
+
+ssd_status ssd_scan_fwd(const void* x, const float* dt_raw, const float* dt_bias, const float* A,
+                        const void* B, const void* C, const float* D, const float* init_state,
+                        const int32_t* cu_seqlens, void* y, float* final_state,
+                        const ssd_dims* dims, int chunk, ssd_stream_t stream) {
+    return scan_fwd_impl(x, dt_raw, dt_bias, A, B, C, D, init_state, cu_seqlens, y, final_state, nullptr, 0,
+                         dims, chunk, stream);
+}
+
+ssd_status ssd_scan_fwd_snapshots(const void* x, const float* dt_raw, const float* dt_bias, const float* A,
+                                  const void* B, const void* C, const float* D, const float* init_state,
+                                  const int32_t* cu_seqlens, void* y, float* final_state, float* snapshots,
+                                  int64_t snapshot_tokens, const ssd_dims* dims, int chunk,
+                                  ssd_stream_t stream) {
+    if (snapshot_tokens <= 0) return fail(SSD_ERR_INVALID_ARG, "snapshot_tokens must be > 0");
+    return scan_fwd_impl(x, dt_raw, dt_bias, A, B, C, D, init_state, cu_seqlens, y, final_state, snapshots,
+                         snapshot_tokens, dims, chunk, stream);
+}
+
+ssd_status ssd_scan_fwd_snapshots_workspace_size(const ssd_dims* dims, int chunk, int64_t snapshot_tokens,
+                                                 size_t* bytes) {
+    if (!bytes) return fail(SSD_ERR_INVALID_ARG, "bytes is NULL");
+    if (snapshot_tokens <= 0) return fail(SSD_ERR_INVALID_ARG, "snapshot_tokens must be > 0");
+    Plan dense, packed;
+    const ssd_status sd = make_plan(dims, chunk, false, &dense, snapshot_tokens);
+    const ssd_status sp = make_plan(dims, chunk, true, &packed, snapshot_tokens);
+    if (sd != SSD_OK && sp != SSD_OK) return sd;
+    size_t b = 0;
+    if (sd == SSD_OK) b = dense.bytes;
+    if (sp == SSD_OK && packed.bytes > b) b = packed.bytes;
+    t_last_error.clear();
+    *bytes = b;
+    return SSD_OK;
+}
+
+ssd_status ssd_snapshot_count(const ssd_dims* dims, const int32_t* cu_seqlens_host, int64_t snapshot_tokens,
+                              int64_t* count) {
+    if (!dims || !count) return fail(SSD_ERR_INVALID_ARG, "dims and count must be non-NULL");
+    if (snapshot_tokens <= 0) return fail(SSD_ERR_INVALID_ARG, "snapshot_tokens must be > 0");
+    int64_t n = 0;
+    if (cu_seqlens_host) {
+        if (dims->nseq < 0) return fail(SSD_ERR_INVALID_ARG, "nseq must be >= 0");
+        for (int32_t s = 0; s < dims->nseq; ++s) {
+            const int64_t len = (int64_t)cu_seqlens_host[s + 1] - cu_seqlens_host[s];
+            if (len < 0) return fail(SSD_ERR_INVALID_ARG, "cu_seqlens must be non-decreasing");
+            n += len / snapshot_tokens;
+        }
+    } else {
+        if (dims->batch < 0 || dims->seqlen < 0) return fail(SSD_ERR_INVALID_ARG, "batch and seqlen must be >= 0");
+        n = dims->batch * (dims->seqlen / snapshot_tokens);
+    }
+    t_last_error.clear();
+    *count = n;
+    return SSD_OK;
 }
 
 ssd_status ssd_state_update(float* state, const void* x, const float* dt_raw, const float* dt_bias,

@@ -30,7 +30,7 @@ constexpr int kTableThreads = 1024;
 __global__ void __launch_bounds__(kTableThreads)
 k_chunk_table(const int32_t* __restrict__ cu, int32_t nseq, int64_t T, int64_t seqlen, int Q,
               ChunkEntry* __restrict__ table, int32_t* __restrict__ first,
-              int32_t* __restrict__ count) {
+              int32_t* __restrict__ count, int64_t snap, int32_t* __restrict__ snap_first) {
     __shared__ int32_t part[kTableThreads];
     const int tid = threadIdx.x;
     const int per = (nseq + kTableThreads - 1) / kTableThreads;
@@ -80,6 +80,25 @@ k_chunk_table(const int32_t* __restrict__ cu, int32_t nseq, int64_t T, int64_t s
     if (tid == kTableThreads - 1) {
         first[nseq] = part[tid];
         *count = part[tid];
+    }
+    if (snap > 0) {                                       // snapshots: floor(len / snap) per sequence
+        __syncthreads();
+        int32_t nsnap = 0;
+        for (int s = s0; s < s1; ++s) nsnap += (int32_t)((seq_begin(s + 1) - seq_begin(s)) / snap);
+        part[tid] = nsnap;
+        __syncthreads();
+        for (int off = 1; off < kTableThreads; off <<= 1) {
+            int32_t v = tid >= off ? part[tid - off] : 0;
+            __syncthreads();
+            part[tid] += v;
+            __syncthreads();
+        }
+        int32_t r2 = part[tid] - nsnap;
+        for (int s = s0; s < s1; ++s) {
+            snap_first[s] = r2;
+            r2 += (int32_t)((seq_begin(s + 1) - seq_begin(s)) / snap);
+        }
+        if (tid == kTableThreads - 1) snap_first[nseq] = part[tid];
     }
 }
 
@@ -196,18 +215,25 @@ template <int Q>
 __global__ void __launch_bounds__(256)
 k_state_passing(float* __restrict__ states, const float* __restrict__ acum,
                 const ChunkEntry* __restrict__ table, const int32_t* __restrict__ first,
-                const float* __restrict__ init, float* __restrict__ final_state, int H, int PN) {
+                const float* __restrict__ init, float* __restrict__ final_state, int H, int PN,
+                int64_t snap, const int32_t* __restrict__ snap_first, float* __restrict__ snap_out) {
     const int s = blockIdx.x, h = blockIdx.y;
     const int i = blockIdx.z * 256 + threadIdx.x;
     if (i >= PN) return;
     float hv = init ? init[((int64_t)s * H + h) * PN + i] : 0.f;
     const int c0 = first[s], c1 = first[s + 1];
+    const int64_t seq0 = c1 > c0 ? table[c0].start : 0;
     for (int c = c0; c < c1; ++c) {
-        const float decay = expf(acum[((int64_t)c * H + h) * Q + table[c].len - 1]);
+        const ChunkEntry e = table[c];
+        const float decay = expf(acum[((int64_t)c * H + h) * Q + e.len - 1]);
         float* slot = states + ((int64_t)c * H + h) * PN + i;
         const float sv = *slot;
         *slot = hv;
         hv = fmaf(decay, hv, sv);
+        if (snap > 0) {                                   // state after a multiple of snap tokens
+            const int64_t end = (int64_t)e.start + e.len - seq0;
+            if (end % snap == 0) snap_out[((int64_t)(snap_first[s] + end / snap - 1) * H + h) * PN + i] = hv;
+        }
     }
     if (final_state) final_state[((int64_t)s * H + h) * PN + i] = hv;
 }

@@ -329,7 +329,8 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
 __global__ void __launch_bounds__(256)
 k_tc_segment_passing(float* __restrict__ seg_state, const float* __restrict__ seg_acum,
                      const int32_t* __restrict__ first, const float* __restrict__ init,
-                     float* __restrict__ final_state, int H) {
+                     float* __restrict__ final_state, int H, const ChunkEntry* __restrict__ segs,
+                     int64_t snap, const int32_t* __restrict__ snap_first, float* __restrict__ snap_out) {
     const int s = blockIdx.x, h = blockIdx.y;
     const int e = blockIdx.z * 256 + threadIdx.x;
     if (e >= kP * kN) return;
@@ -337,6 +338,7 @@ k_tc_segment_passing(float* __restrict__ seg_state, const float* __restrict__ se
     const int64_t api = (((int64_t)s * H + h) * kP + p) * kN + n;
     float hv = init ? init[api] : 0.f;
     const int c0 = first[s], c1 = first[s + 1];
+    const int64_t seq0 = c1 > c0 ? segs[c0].start : 0;
     constexpr int U = 4;
     for (int c = c0; c < c1; c += U) {
         float sv[U], dec[U];
@@ -352,6 +354,11 @@ k_tc_segment_passing(float* __restrict__ seg_state, const float* __restrict__ se
             if (c + u < c1) {
                 seg_state[((int64_t)(c + u) * H + h) * (kP * kN) + e] = hv;
                 hv = fmaf(dec[u], hv, sv[u]);
+                if (snap > 0) {                           // state after a multiple of snap tokens
+                    const int64_t end = (int64_t)segs[c + u].start + segs[c + u].len - seq0;
+                    if (end % snap == 0)
+                        snap_out[(((int64_t)(snap_first[s] + end / snap - 1) * H + h) * kP + p) * kN + n] = hv;
+                }
             }
         }
     }

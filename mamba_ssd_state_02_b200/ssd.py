@@ -58,6 +58,14 @@ _lib.ssd_scan_fwd_workspace_size.restype = ctypes.c_int
 _lib.ssd_scan_fwd.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p,
                               ctypes.POINTER(SSDDims), ctypes.c_int, _p]
 _lib.ssd_scan_fwd.restype = ctypes.c_int
+_lib.ssd_scan_fwd_snapshots.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p, ctypes.c_int64,
+                                        ctypes.POINTER(SSDDims), ctypes.c_int, _p]
+_lib.ssd_scan_fwd_snapshots.restype = ctypes.c_int
+_lib.ssd_scan_fwd_snapshots_workspace_size.argtypes = [ctypes.POINTER(SSDDims), ctypes.c_int, ctypes.c_int64,
+                                                       ctypes.POINTER(ctypes.c_size_t)]
+_lib.ssd_scan_fwd_snapshots_workspace_size.restype = ctypes.c_int
+_lib.ssd_snapshot_count.argtypes = [ctypes.POINTER(SSDDims), _p, ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)]
+_lib.ssd_snapshot_count.restype = ctypes.c_int
 _lib.ssd_scan_fwd_noalloc.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p,
                                       ctypes.POINTER(SSDDims), ctypes.c_int, _p]
 _lib.ssd_scan_fwd_noalloc.restype = ctypes.c_int
@@ -146,6 +154,26 @@ def workspace_size(dims: SSDDims, chunk: int) -> int:
     return int(b.value)
 
 
+def snapshot_workspace_size(dims: SSDDims, chunk: int, snapshot_tokens: int) -> int:
+    b = ctypes.c_size_t(0)
+    _check(_lib.ssd_scan_fwd_snapshots_workspace_size(ctypes.byref(dims), int(chunk), int(snapshot_tokens),
+                                                      ctypes.byref(b)))
+    return int(b.value)
+
+
+def snapshot_count(dims: SSDDims, snapshot_tokens: int, cu_seqlens_host=None) -> int:
+    """Snapshots ssd_scan_fwd_snapshots writes (cu_seqlens_host: CPU int32 tensor for varlen)."""
+    n = ctypes.c_int64(0)
+    cu = None
+    if cu_seqlens_host is not None:
+        cu = cu_seqlens_host.to(torch.int32).contiguous()
+        if cu.device.type != "cpu":
+            raise ValueError("cu_seqlens_host must be a CPU tensor")
+    _check(_lib.ssd_snapshot_count(ctypes.byref(dims), None if cu is None else ctypes.c_void_p(cu.data_ptr()),
+                                   int(snapshot_tokens), ctypes.byref(n)))
+    return int(n.value)
+
+
 def scan_variant(dims: SSDDims, chunk: int) -> str:
     return _lib.ssd_scan_fwd_variant(ctypes.byref(dims), int(chunk)).decode()
 
@@ -194,13 +222,17 @@ def device_status(device=None) -> None:
 
 
 def scan_fwd(x, dt_raw, dt_bias, A, B, C, D, init_state=None, cu_seqlens=None, chunk=128,
-             y=None, final_state=None, workspace=None, batch=None):
+             y=None, final_state=None, workspace=None, batch=None, snapshot_tokens=None, snapshots=None):
     """Chunked SSD prefill.
 
     Dense: x [batch, L, H, P], dt_raw [batch, L, H], B/C [batch, L, G, N].
     Packed varlen (cu_seqlens int32 [nseq+1] on the device): x [T, H, P],
     dt_raw [T, H], B/C [T, G, N].
     Returns (y, final_state); final_state [nseq, H, P, N] float32.
+    With snapshot_tokens (ssd_scan_fwd_snapshots) returns (y, final_state, snapshots),
+    snapshots [n_snap, H, P, N] float32: each sequence's state after every multiple of
+    snapshot_tokens tokens (allocated here when not given; for varlen that reads
+    cu_seqlens back to the host to count them).
     """
     dev = x.device
     varlen = cu_seqlens is not None
@@ -236,6 +268,19 @@ def scan_fwd(x, dt_raw, dt_bias, A, B, C, D, init_state=None, cu_seqlens=None, c
         dims = make_dims(x.shape[0], H, P, G, N, _dtype_code(x), nseq=nseq, workspace=workspace)
     else:
         dims = make_dims(bsz * L, H, P, G, N, _dtype_code(x), batch=bsz, seqlen=L, workspace=workspace)
+    if snapshot_tokens is not None:
+        if snapshots is None:
+            n_snap = snapshot_count(dims, snapshot_tokens, cu_seqlens.cpu() if varlen else None)
+            snapshots = torch.empty(n_snap, H, P, N, dtype=torch.float32, device=dev)
+        if snapshots.dtype != torch.float32 or snapshots.device != dev or not snapshots.is_contiguous() or \
+                tuple(snapshots.shape[1:]) != (H, P, N):
+            raise ValueError("snapshots must be a contiguous float32 [n_snap, H, P, N] tensor on x's device")
+        with torch.cuda.device(dev):
+            _check(_lib.ssd_scan_fwd_snapshots(_ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C),
+                                               _ptr(D), _ptr(init_state), _ptr(cu_seqlens), _ptr(y),
+                                               _ptr(final_state), _ptr(snapshots), int(snapshot_tokens),
+                                               ctypes.byref(dims), int(chunk), _stream(dev)))
+        return y, final_state, snapshots
     with torch.cuda.device(dev):
         _check(_lib.ssd_scan_fwd(_ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C),
                                  _ptr(D), _ptr(init_state), _ptr(cu_seqlens), _ptr(y),

@@ -40,6 +40,9 @@ def lib():
         L.oracle_ssd_scan.argtypes = [i64, p, i32, i32, i32, i32, i32, p, p, p, p, p, p, p, p,
                                       i64, p, p, p, p, i32]
         L.oracle_ssd_scan.restype = i32
+        L.oracle_ssd_scan_snapshots.argtypes = [i64, p, i32, i32, i32, i32, i32, p, p, p, p, p, p, p, p,
+                                                i64, p, p, p, p, i64, p, p, i32]
+        L.oracle_ssd_scan_snapshots.restype = i32
         L.oracle_state_update.argtypes = [i64, i32, i32, i32, i32, i32, p, p, p, p, p, p, p, p, p]
         L.oracle_state_update.restype = i32
         L.oracle_closed_form.argtypes = [i32, i32, i32, i32, i32, i32, p, p, p, p, p, p, p, p, p, p]
@@ -95,7 +98,7 @@ def seq_offsets(T: int, cu_seqlens=None, batch: int | None = None) -> np.ndarray
 
 
 def ssd_scan(x, dt_raw, dt_bias, A, B, C, D, init_state=None, cu_seqlens=None, batch=None,
-             pairs=None, want_y=True, nthreads=None):
+             pairs=None, want_y=True, nthreads=None, snapshot_tokens=None):
     """Run the recurrence.
 
     x [T,H,P], dt_raw [T,H], B/C [T,G,N] (packed tokens), dt_bias/A/D [H];
@@ -104,6 +107,9 @@ def ssd_scan(x, dt_raw, dt_bias, A, B, C, D, init_state=None, cu_seqlens=None, b
 
     pairs=None: returns (y [T,H,P] float64, final [nseq,H,P,N] float64).
     pairs=[(s,h), ...]: returns (list of y blocks [len_s,P], final [npairs,P,N]).
+    snapshot_tokens=I adds a third result, the state after every I tokens of each
+    sequence: [n_snap,H,P,N] ordered by sequence, then position (pairs=None), or a list
+    of [len_s // I, P, N] blocks (pairs given).
     """
     x, B, C = _cpu(x), _cpu(B), _cpu(C)
     dtype = _dtype_code(x)
@@ -126,16 +132,26 @@ def ssd_scan(x, dt_raw, dt_bias, A, B, C, D, init_state=None, cu_seqlens=None, b
         yoff[1:] = np.cumsum(lens[:-1] * P)
     ybuf = np.zeros(int(lens.sum()) * P if want_y else 1, dtype=np.float64)
     fin = np.zeros((len(pr), P, N), dtype=np.float64)
-    rc = lib().oracle_ssd_scan(
+    I = int(snapshot_tokens or 0)
+    nsn = lens // I if I > 0 else np.zeros(len(pr), np.int64)
+    soff = np.zeros(len(pr), dtype=np.int64)
+    if len(pr) > 1:
+        soff[1:] = np.cumsum(nsn[:-1] * P * N)
+    sbuf = np.zeros(max(1, int(nsn.sum()) * P * N), dtype=np.float64)
+    rc = lib().oracle_ssd_scan_snapshots(
         nseq, off.ctypes.data_as(ctypes.c_void_p), H, P, G, N, dtype, _ptr(x), _ptr(dt_raw),
         _ptr(dt_bias), _ptr(A_), _ptr(B), _ptr(C), _ptr(D_), _ptr(init), len(pr),
         pr.ctypes.data_as(ctypes.c_void_p), yoff.ctypes.data_as(ctypes.c_void_p),
         ybuf.ctypes.data_as(ctypes.c_void_p) if want_y else None,
-        fin.ctypes.data_as(ctypes.c_void_p), nthreads or _threads())
+        fin.ctypes.data_as(ctypes.c_void_p), I, soff.ctypes.data_as(ctypes.c_void_p),
+        sbuf.ctypes.data_as(ctypes.c_void_p), nthreads or _threads())
     if rc != 0:
         raise ValueError("oracle_ssd_scan rejected its arguments")
     blocks = [ybuf[o:o + l * P].reshape(l, P) for o, l in zip(yoff, lens)] if want_y else None
+    sblocks = [sbuf[o:o + n * P * N].reshape(n, P, N) for o, n in zip(soff, nsn)] if I > 0 else None
     if not all_pairs:
+        if I > 0:
+            return blocks, torch.from_numpy(fin), [torch.from_numpy(b) for b in sblocks]
         return blocks, torch.from_numpy(fin)
     y = None
     if want_y:
@@ -143,7 +159,15 @@ def ssd_scan(x, dt_raw, dt_bias, A, B, C, D, init_state=None, cu_seqlens=None, b
         for (s, h), blk in zip(pr, blocks):
             y[off[s]:off[s + 1], h, :] = blk
         y = torch.from_numpy(y)
-    return y, torch.from_numpy(fin.reshape(nseq, H, P, N))
+    fin_t = torch.from_numpy(fin.reshape(nseq, H, P, N))
+    if I > 0:
+        per_seq = (off[1:] - off[:-1]) // I
+        snaps = np.zeros((int(per_seq.sum()), H, P, N), dtype=np.float64)
+        first = np.concatenate([[0], np.cumsum(per_seq)])
+        for (s, h), blk in zip(pr, sblocks):
+            snaps[first[s]:first[s + 1], h] = blk
+        return y, fin_t, torch.from_numpy(snaps)
+    return y, fin_t
 
 
 def state_update(state, x, dt_raw, dt_bias, A, B, C, D):

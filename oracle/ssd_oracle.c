@@ -94,6 +94,9 @@ typedef struct {
     const int64_t* y_off;    /* [npairs] offset (in doubles) of each pair's y block */
     double* y;               /* per pair: [len][P] */
     double* final_state;     /* per pair: [P][N], or NULL */
+    int64_t snap;            /* snapshot interval in tokens (0: none) */
+    const int64_t* snap_off; /* per pair: where its [len/snap][P][N] snapshots start in snaps */
+    double* snaps;
     /* threading */
     int64_t next;
     pthread_mutex_t lock;
@@ -137,6 +140,10 @@ static void scan_pair(const scan_job* j, int64_t k)
                 yo[(t - t0) * P + p] = acc;
             }
         }
+        /* snapshot: the state after the first m * snap tokens of the sequence */
+        if (j->snap > 0 && (t - t0 + 1) % j->snap == 0)
+            memcpy(j->snaps + j->snap_off[k] + ((t - t0 + 1) / j->snap - 1) * (int64_t)P * N, st,
+                   (size_t)P * N * sizeof(double));
     }
     if (j->final_state) memcpy(j->final_state + k * (int64_t)P * N, st, (size_t)P * N * sizeof(double));
     free(st);
@@ -163,20 +170,24 @@ static void* scan_worker(void* arg)
  *   init: [nseq,H,P,N] doubles or NULL (zero initial state).
  *   y_off[k]: where pair k's [len][P] output block starts in y (NULL y: skip y).
  *   final_state: [npairs][P][N] or NULL.
- * Returns 0, or -1 on a bad argument.
+ *   snap, snap_off, snaps: if snap > 0, pair k's state after the first m * snap tokens
+ *     of its sequence (m = 1 .. len / snap) goes to snaps + snap_off[k] + (m-1)*P*N.
+ * Returns 0, or -1 on a bad argument. oracle_ssd_scan is the same without snapshots.
  */
-int oracle_ssd_scan(int64_t nseq, const int64_t* seq_off, int H, int P, int G, int N, int dtype,
-                    const void* x, const float* dt_raw, const float* dt_bias, const float* A,
-                    const void* B, const void* C, const float* D, const double* init,
-                    int64_t npairs, const int64_t* pairs, const int64_t* y_off, double* y,
-                    double* final_state, int nthreads)
+int oracle_ssd_scan_snapshots(int64_t nseq, const int64_t* seq_off, int H, int P, int G, int N, int dtype,
+                              const void* x, const float* dt_raw, const float* dt_bias, const float* A,
+                              const void* B, const void* C, const float* D, const double* init,
+                              int64_t npairs, const int64_t* pairs, const int64_t* y_off, double* y,
+                              double* final_state, int64_t snap, const int64_t* snap_off, double* snaps,
+                              int nthreads)
 {
-    if (H <= 0 || G <= 0 || H % G != 0 || P <= 0 || N <= 0 || nseq < 0) return -1;
+    if (H <= 0 || G <= 0 || H % G != 0 || P <= 0 || N <= 0 || nseq < 0 || snap < 0) return -1;
+    if (snap > 0 && (!snap_off || !snaps)) return -1;
     for (int64_t k = 0; k < npairs; k++)
         if (pairs[2 * k] < 0 || pairs[2 * k] >= nseq || pairs[2 * k + 1] < 0 || pairs[2 * k + 1] >= H)
             return -1;
     scan_job j = {nseq, seq_off, H, P, G, N, dtype, x, dt_raw, dt_bias, A, B, C, D, init,
-                  npairs, pairs, y_off, y, final_state, 0};
+                  npairs, pairs, y_off, y, final_state, snap, snap_off, snaps, 0};
     pthread_mutex_init(&j.lock, NULL);
     if (nthreads < 1) nthreads = 1;
     if (nthreads > 256) nthreads = 256;
@@ -185,6 +196,16 @@ int oracle_ssd_scan(int64_t nseq, const int64_t* seq_off, int H, int P, int G, i
     for (int i = 0; i < nthreads; i++) pthread_join(th[i], NULL);
     pthread_mutex_destroy(&j.lock);
     return 0;
+}
+
+int oracle_ssd_scan(int64_t nseq, const int64_t* seq_off, int H, int P, int G, int N, int dtype,
+                    const void* x, const float* dt_raw, const float* dt_bias, const float* A,
+                    const void* B, const void* C, const float* D, const double* init,
+                    int64_t npairs, const int64_t* pairs, const int64_t* y_off, double* y,
+                    double* final_state, int nthreads)
+{
+    return oracle_ssd_scan_snapshots(nseq, seq_off, H, P, G, N, dtype, x, dt_raw, dt_bias, A, B, C, D, init,
+                                     npairs, pairs, y_off, y, final_state, 0, NULL, NULL, nthreads);
 }
 
 /*

@@ -94,3 +94,28 @@ def test_workspace_size_grows_with_tokens(ssd):
 def test_variant_names(ssd):
     assert ssd.scan_variant(_dims(ssd), 128) in ("tc", "simt")
     assert ssd.scan_variant(_dims(ssd, dtype_code=ssd.SSD_DTYPE_F32, P=16, N=16, H=4, G=1), 64) == "simt"
+
+
+def test_snapshot_count_and_workspace(ssd):
+    import torch
+    dense = _dims(ssd, T=1000, batch=2, seqlen=500)
+    assert ssd.snapshot_count(dense, 128) == 2 * (500 // 128)
+    assert ssd.snapshot_count(dense, 1000) == 0
+    packed = ssd.make_dims(1217, 8, 64, 2, 128, ssd.SSD_DTYPE_BF16, nseq=3)
+    cu = torch.tensor([0, 300, 317, 1217], dtype=torch.int32)
+    assert ssd.snapshot_count(packed, 128, cu) == 300 // 128 + 0 + 900 // 128
+    assert ssd.snapshot_workspace_size(dense, 128, 256) >= ssd.workspace_size(dense, 128)
+
+
+@pytest.mark.parametrize("snap,dims_kw,chunk,status", [
+    (0, {}, 128, "INVALID_ARG"),
+    (-128, {}, 128, "INVALID_ARG"),
+    (200, {}, 128, "UNSUPPORTED"),                                       # tensor-core path: multiple of 128
+    (96, dict(dtype_code=1 - 1, P=16, N=16, H=4, G=1), 64, "UNSUPPORTED"),  # CUDA-core path: multiple of chunk
+])
+def test_bad_snapshot_interval_fails_closed(ssd, snap, dims_kw, chunk, status):
+    kw = dict(dims_kw)
+    if "dtype_code" in kw:
+        kw["dtype_code"] = ssd.SSD_DTYPE_F32
+    with pytest.raises(ssd.SSDError, match=status):
+        ssd.snapshot_workspace_size(_dims(ssd, **kw), chunk, snap)

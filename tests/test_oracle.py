@@ -24,6 +24,7 @@ import pytest
 import torch
 
 from oracle import oracle as O
+from mamba_ssd_state_02_b200 import workloads as W
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 LN2 = math.log(2.0)
@@ -257,3 +258,30 @@ def test_oracle_rejects_bad_dims():
     with pytest.raises(ValueError):
         O.ssd_scan(d["x"], d["dt_raw"], d["dt_bias"], d["A"], d["B"].expand(4, 2, 2).contiguous(),
                    d["C"].expand(4, 2, 2).contiguous(), d["D"])   # H=3 not divisible by G=2
+
+
+def test_snapshots_equal_prefix_final_states():
+    """A snapshot (state after the first m*I tokens of a sequence) is, by definition, the
+    final state of the same sequence cut after m*I tokens; the last one of a sequence
+    whose length is a multiple of I is its final state."""
+    w = W.Workload("snap", nheads=4, headdim=8, ngroups=2, dstate=8, chunk=64, dtype=torch.float32,
+                   seqlens=[300, 17, 256], varlen=True, init="normal", seed=5)
+    d = W.make_all(w)
+    I = 64
+    y, fin, sn = O.ssd_scan(d["x"], d["dt_raw"], d["dt_bias"], d["A"], d["B"], d["C"], d["D"],
+                            init_state=d["init_state"], cu_seqlens=d["cu_seqlens"], snapshot_tokens=I)
+    per = [300 // I, 17 // I, 256 // I]
+    assert sn.shape == (sum(per), 4, 8, 8)
+    cu = d["cu_seqlens"].tolist()
+    first = [0, per[0], per[0] + per[1]]
+    for s in range(3):
+        for m in range(1, per[s] + 1):
+            sl = slice(cu[s], cu[s] + m * I)
+            _, f2 = O.ssd_scan(d["x"][sl], d["dt_raw"][sl], d["dt_bias"], d["A"], d["B"][sl], d["C"][sl],
+                               d["D"], init_state=d["init_state"][s:s + 1], batch=1)
+            assert torch.equal(sn[first[s] + m - 1], f2[0])
+    assert torch.equal(sn[-1], fin[2])                       # 256 = 4 * 64: the final state
+    # Without snapshots the results are unchanged.
+    y0, fin0 = O.ssd_scan(d["x"], d["dt_raw"], d["dt_bias"], d["A"], d["B"], d["C"], d["D"],
+                          init_state=d["init_state"], cu_seqlens=d["cu_seqlens"])
+    assert torch.equal(y0, y) and torch.equal(fin0, fin)
