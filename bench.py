@@ -419,8 +419,6 @@ def bench_ours(args, rank, world, local_rank):
     e2e = {"value": world * w.total_tokens / (e2e_ms / 1e3), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3),
            "steps": e2e_steps}
-    del host, dbuf, inp, x, dtr, Bm, Cm, y, ws
-    torch.cuda.empty_cache()
 
     # ---- state snapshots every 2048 tokens on the same workload (prefix-cache reuse)
     snap_every = 2048
@@ -448,6 +446,58 @@ def bench_ours(args, rank, world, local_rank):
                  "snapshot_bytes_per_step": snaps.numel() * 4, "ms_per_step": round(snap_ms, 4),
                  "overhead_vs_plain": round(snap_ms / ms_step - 1.0, 4)}
 
+    # ---- conv1d prologue (width 4) over the same tokens: xBC = H*P + 2*G*N channels
+    K = 4
+    ci = W.make_conv_inputs(w, K, init=True, device=dev)
+    Dc = W.conv_channels(w)
+    cx = ci["xbc"].view(w.nseq, L, Dc)
+    cst_out = torch.empty_like(ci["conv_state"])
+    cxo, cbo, cco = torch.empty_like(x), torch.empty_like(Bm), torch.empty_like(Cm)
+
+    def conv_step():
+        ssd.conv1d_fwd(cx, ci["weight"], ci["bias"], w.nheads, w.headdim, w.ngroups, w.dstate,
+                       conv_state=ci["conv_state"], x=cxo, B=cbo, C=cco, conv_state_out=cst_out)
+
+    for _ in range(args.warmup):
+        conv_step()
+    ssd.device_status()
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        conv_step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    conv_ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dev)
+    esz = 2 if w.dtype == torch.bfloat16 else 4
+    conv_bytes = (2 * w.total_tokens * Dc * esz + Dc * K * 4 + Dc * 4
+                  + 2 * w.nseq * Dc * (K - 1) * esz)
+    # decode step of the conv for 256 sequences
+    nd = 256
+    dst = torch.zeros(nd, Dc, K - 1, dtype=w.dtype, device=dev)
+    dx = ci["xbc"][:nd].contiguous()
+    xo = torch.empty(nd, w.nheads, w.headdim, dtype=w.dtype, device=dev)
+    bo = torch.empty(nd, w.ngroups, w.dstate, dtype=w.dtype, device=dev)
+    co = torch.empty_like(bo)
+    for _ in range(args.warmup):
+        ssd.conv1d_update(dst, dx, ci["weight"], ci["bias"], w.nheads, w.headdim, w.ngroups, w.dstate, x=xo, B=bo, C=co)
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    nrep = 100
+    for _ in range(nrep):
+        ssd.conv1d_update(dst, dx, ci["weight"], ci["bias"], w.nheads, w.headdim, w.ngroups, w.dstate, x=xo, B=bo, C=co)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    ssd.device_status()
+    conv_upd_us = ev0.elapsed_time(ev1) / nrep * 1e3
+    conv1d = {"workload": f"conv1d_width{K}_{w.total_tokens}tok_D{Dc}", "ms_per_call": round(conv_ms, 4),
+              "bytes_per_call": conv_bytes, "achieved_gbs": round(conv_bytes / conv_ms / 1e6, 1),
+              "peak_gbs": hbm, "frac": round(conv_bytes / conv_ms / 1e6 / hbm, 4),
+              "decode_256seq_us_per_step": round(conv_upd_us, 2)}
+    del ci, cx, cst_out, cxo, cbo, cco
+    del host, dbuf, inp, x, dtr, Bm, Cm, y, ws, snaps, ws_snap
+    torch.cuda.empty_cache()
+
     # ---- decode (256 sequences, FP32 states from a 2048-token prefill)
     decode = bench_decode(args, ssd, dev, rank, world, hbm, peak_src)
 
@@ -464,6 +514,7 @@ def bench_ours(args, rank, world, local_rank):
         "clocks": clk, "e2e": e2e, "gpu_launches": launches_per_call * args.steps,
         "decode": decode,
         "snapshots": snapshots,
+        "conv1d": conv1d,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, threads, secs = oracle_sample(w, 16384, w.nheads)

@@ -164,6 +164,37 @@ ssd_status ssd_state_update(float* state, const void* x, const float* dt_raw, co
                             const ssd_dims* dims, ssd_stream_t stream);
 
 /*
+ * Causal depthwise conv1d + bias + SiLU over the xBC channels, the stage that feeds the
+ * scan in a Mamba-2 block (RL-Kernel issue page, Figure 2, and §1 item 2: a conv state
+ * per sequence; width 4 in the JAX Nemotron 3 Nano page's configuration). With
+ * D = H*P + 2*G*N channels, width K and each sequence's previous K-1 inputs in front of
+ * its first token (conv_state_in, or zeros):
+ *   out[t][c] = silu(bias[c] + sum_{k<K} weight[c][k] * in[t-(K-1)+k][c]),
+ * written split into the scan's inputs: channels [0,H*P) -> x [T,H,P], [H*P,H*P+G*N)
+ * -> B [T,G,N], the rest -> C [T,G,N].
+ *   xbc: [T,D] (dims->dtype), packed like the scan's inputs (dense batch or cu_seqlens).
+ *   weight: [D,K] float32; bias: [D] float32 or NULL (both 16-byte aligned).
+ *   conv_state_in: [nseq,D,K-1] (dims->dtype, oldest input first) or NULL for zeros.
+ *   conv_state_out: [nseq,D,K-1] output or NULL: each sequence's last K-1 inputs
+ *     (taken from conv_state_in where the sequence is shorter than K-1).
+ *   width: K in {2,3,4}. The convolution never crosses a sequence boundary.
+ * Supported: the scan's head/group geometry; xbc/x/B/C 16-byte aligned. The states may
+ * not overlap each other or xbc.
+ */
+ssd_status ssd_conv1d_fwd(const void* xbc, const float* weight, const float* bias, const void* conv_state_in,
+                          const int32_t* cu_seqlens, void* x, void* B, void* C, void* conv_state_out,
+                          const ssd_dims* dims, int width, ssd_stream_t stream);
+
+/*
+ * One decode step of the conv1d above for nseq = dims->batch sequences (seqlen 1):
+ * conv_state [nseq,D,K-1] (16-byte aligned) is read and shifted in place (the new
+ * input appended), xbc [nseq,D] in, x [nseq,H,P], B/C [nseq,G,N] out (dims->dtype).
+ * A step gives the same bits as ssd_conv1d_fwd on one token from the same state.
+ */
+ssd_status ssd_conv1d_update(void* conv_state, const void* xbc, const float* weight, const float* bias, void* x,
+                             void* B, void* C, const ssd_dims* dims, int width, ssd_stream_t stream);
+
+/*
  * ssd_scan_fwd without any device allocation (the pages have no counterpart; this is a
  * deployment convenience). Some callers cannot allocate device memory while they run:
  * serving engines that reserve their whole memory budget at start-up and forbid later

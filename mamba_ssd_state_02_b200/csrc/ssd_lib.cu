@@ -17,6 +17,7 @@
 
 #include "ssd.h"
 #include "ssd_common.cuh"
+#include "ssd_conv.cuh"
 #include "ssd_decode.cuh"
 #include "ssd_scan_simt.cuh"
 #include "ssd_scan_tc.cuh"
@@ -45,9 +46,9 @@ ssd_status cuda_fail(cudaError_t e, const char* what) {
 // ---------------------------------------------------------------------------------
 // Per-kernel event timing (ssd_profile_enable / ssd_profile_read).
 enum Stage { ST_TABLE, ST_CUMSUM, ST_CHUNK_STATE, ST_STATE_PASSING, ST_CHUNK_SCAN, ST_STATE_UPDATE,
-             ST_COUNT };
+             ST_CONV, ST_CONV_UPDATE, ST_COUNT };
 const char* const kStageName[ST_COUNT] = {"ssd_chunk_table", "ssd_chunk_cumsum", "ssd_chunk_state",
-                                          "ssd_state_passing", "ssd_chunk_scan", "ssd_state_update"};
+                                          "ssd_state_passing", "ssd_chunk_scan", "ssd_state_update", "ssd_conv1d", "ssd_conv1d_update"};
 constexpr size_t kMaxRecords = 65536;
 
 struct Profiler {
@@ -775,4 +776,148 @@ extern "C" ssd_status ssd_scan_fwd_noalloc(const void* x, const float* dt_raw, c
                               st);
     if (s == SSD_OK) t_last_error.clear();
     return s;
+}
+
+// ---------------------------------------------------------------------------------
+// Causal conv1d prologue (prefill and decode).
+namespace ssd {
+namespace {
+
+struct ConvShape {
+    int64_t T = 0, seqlen = 0;
+    int32_t nseq = 0;
+    int Dc = 0, HP = 0, GN = 0;
+    bool bf16 = false;
+};
+
+ssd_status conv_shape(const ssd_dims* d, bool varlen, int width, ConvShape* cs) {
+    if (!d) return fail(SSD_ERR_INVALID_ARG, "dims is NULL");
+    if (d->nheads <= 0 || d->headdim <= 0 || d->ngroups <= 0 || d->dstate <= 0)
+        return fail(SSD_ERR_INVALID_ARG, "nheads, headdim, ngroups and dstate must be positive");
+    if (d->nheads % d->ngroups != 0) return fail(SSD_ERR_UNSUPPORTED, "nheads must be a multiple of ngroups");
+    if (!pow2_in(d->headdim, 16, 128) || !pow2_in(d->dstate, 16, 128))
+        return fail(SSD_ERR_UNSUPPORTED, "headdim and dstate must be in {16,32,64,128}");
+    if (width < 2 || width > 4) return fail(SSD_ERR_UNSUPPORTED, "conv width %d not in {2,3,4}", width);
+    if (d->dtype != SSD_DTYPE_F32 && d->dtype != SSD_DTYPE_BF16)
+        return fail(SSD_ERR_INVALID_ARG, "unknown dtype %d", (int)d->dtype);
+    ConvShape c;
+    c.HP = d->nheads * d->headdim;
+    c.GN = d->ngroups * d->dstate;
+    c.Dc = c.HP + 2 * c.GN;
+    c.bf16 = d->dtype == SSD_DTYPE_BF16;
+    if (varlen) {
+        if (d->nseq < 0 || d->total_tokens < 0) return fail(SSD_ERR_INVALID_ARG, "nseq and total_tokens must be >= 0");
+        c.nseq = d->nseq;
+        c.T = d->total_tokens;
+    } else {
+        if (d->batch < 0 || d->seqlen < 0) return fail(SSD_ERR_INVALID_ARG, "batch and seqlen must be >= 0");
+        if (d->batch > INT32_MAX) return fail(SSD_ERR_UNSUPPORTED, "batch too large");
+        if (d->seqlen > 0 && d->batch > INT64_MAX / d->seqlen) return fail(SSD_ERR_INVALID_ARG, "batch*seqlen overflows");
+        c.nseq = (int32_t)d->batch;
+        c.seqlen = d->seqlen;
+        c.T = d->batch * d->seqlen;
+    }
+    if (c.T >= INT32_MAX) return fail(SSD_ERR_UNSUPPORTED, "more than 2^31-1 tokens in one call");
+    *cs = c;
+    return SSD_OK;
+}
+
+template <typename T, int K>
+void launch_conv(const ConvShape& c, const void* in, const float* w, const float* bias, const void* st_in,
+                 const int32_t* cu, void* x, void* B, void* C, void* st_out, cudaStream_t st) {
+    const unsigned cx = (unsigned)((c.Dc / 8 + kConvThreads - 1) / kConvThreads);
+    if (c.T > 0) {
+        StageScope sc(ST_CONV, st);
+        k_conv1d_fwd<T, K><<<dim3((unsigned)((c.T + kConvTokens - 1) / kConvTokens), cx), kConvThreads, 0, st>>>(
+            (const T*)in, w, bias, (const T*)st_in, cu, c.nseq, c.T, c.seqlen, c.Dc, c.HP, c.GN, (T*)x, (T*)B, (T*)C,
+            (T*)st_out);
+    }
+    if (st_out && c.nseq > 0) {
+        const int64_t n = (int64_t)c.nseq * c.Dc;
+        k_conv1d_empty<T, K><<<(unsigned)((n + 255) / 256), 256, 0, st>>>((const T*)st_in, cu, c.nseq, c.seqlen, c.Dc,
+                                                                          (T*)st_out);
+    }
+}
+
+template <typename T, int K>
+void launch_conv_update(const ConvShape& c, void* state, const void* in, const float* w, const float* bias, void* x,
+                        void* B, void* C, cudaStream_t st) {
+    StageScope sc(ST_CONV_UPDATE, st);
+    const unsigned cx = (unsigned)((c.Dc / 8 + kConvThreads - 1) / kConvThreads);
+    k_conv1d_update<T, K><<<dim3(cx, (unsigned)((c.nseq + kConvSeqs - 1) / kConvSeqs)), kConvThreads, 0, st>>>(
+        (T*)state, (const T*)in, w, bias, c.nseq, c.Dc, c.HP, c.GN, (T*)x, (T*)B, (T*)C);
+}
+
+}  // namespace
+}  // namespace ssd
+
+extern "C" ssd_status ssd_conv1d_fwd(const void* xbc, const float* weight, const float* bias,
+                                     const void* conv_state_in, const int32_t* cu_seqlens, void* x, void* B,
+                                     void* C, void* conv_state_out, const ssd_dims* dims, int width,
+                                     ssd_stream_t stream) {
+    ConvShape c;
+    ssd_status s = conv_shape(dims, cu_seqlens != nullptr, width, &c);
+    if (s != SSD_OK) return s;
+    if (c.T > 0 && (!xbc || !weight || !x || !B || !C))
+        return fail(SSD_ERR_INVALID_ARG, "xbc, weight, x, B and C must be non-NULL");
+    if (!aligned(xbc, 16) || !aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16))
+        return fail(SSD_ERR_INVALID_ARG, "xbc, x, B and C must be 16-byte aligned");
+    if (!aligned(weight, 16) || !aligned(bias, 16) || !aligned(cu_seqlens, 4) || !aligned(conv_state_in, 4) ||
+        !aligned(conv_state_out, 4))
+        return fail(SSD_ERR_INVALID_ARG, "weight and bias must be 16-byte aligned, cu_seqlens and conv states 4-byte");
+    if (c.nseq == 0) {
+        t_launches = 0;
+        t_last_error.clear();
+        return SSD_OK;
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+#define SSD_CONV_CASE(TT, KK)                                                                          \
+    if (width == KK) launch_conv<TT, KK>(c, xbc, weight, bias, conv_state_in, cu_seqlens, x, B, C, conv_state_out, st);
+    if (c.bf16) {
+        SSD_CONV_CASE(__nv_bfloat16, 2) SSD_CONV_CASE(__nv_bfloat16, 3) SSD_CONV_CASE(__nv_bfloat16, 4)
+    } else {
+        SSD_CONV_CASE(float, 2) SSD_CONV_CASE(float, 3) SSD_CONV_CASE(float, 4)
+    }
+#undef SSD_CONV_CASE
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch (conv1d)");
+    t_launches = (c.T > 0 ? 1 : 0) + (conv_state_out ? 1 : 0);
+    t_last_error.clear();
+    return SSD_OK;
+}
+
+extern "C" ssd_status ssd_conv1d_update(void* conv_state, const void* xbc, const float* weight, const float* bias,
+                                        void* x, void* B, void* C, const ssd_dims* dims, int width,
+                                        ssd_stream_t stream) {
+    if (!dims) return fail(SSD_ERR_INVALID_ARG, "dims is NULL");
+    if (dims->seqlen != 1) return fail(SSD_ERR_INVALID_ARG, "decode takes seqlen == 1 (got %lld)", (long long)dims->seqlen);
+    ConvShape c;
+    ssd_status s = conv_shape(dims, false, width, &c);
+    if (s != SSD_OK) return s;
+    if (c.nseq == 0) {
+        t_launches = 0;
+        t_last_error.clear();
+        return SSD_OK;
+    }
+    if (c.nseq > 65535LL * kConvSeqs) return fail(SSD_ERR_UNSUPPORTED, "too many sequences in one decode call");
+    if (!conv_state || !xbc || !weight || !x || !B || !C)
+        return fail(SSD_ERR_INVALID_ARG, "conv_state, xbc, weight, x, B and C must be non-NULL");
+    if (!aligned(xbc, 16) || !aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16))
+        return fail(SSD_ERR_INVALID_ARG, "xbc, x, B and C must be 16-byte aligned");
+    if (!aligned(weight, 16) || !aligned(bias, 16) || !aligned(conv_state, 16))
+        return fail(SSD_ERR_INVALID_ARG, "weight, bias and conv_state must be 16-byte aligned");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+#define SSD_CONV_CASE(TT, KK) \
+    if (width == KK) launch_conv_update<TT, KK>(c, conv_state, xbc, weight, bias, x, B, C, st);
+    if (c.bf16) {
+        SSD_CONV_CASE(__nv_bfloat16, 2) SSD_CONV_CASE(__nv_bfloat16, 3) SSD_CONV_CASE(__nv_bfloat16, 4)
+    } else {
+        SSD_CONV_CASE(float, 2) SSD_CONV_CASE(float, 3) SSD_CONV_CASE(float, 4)
+    }
+#undef SSD_CONV_CASE
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch (conv1d update)");
+    t_launches = 1;
+    t_last_error.clear();
+    return SSD_OK;
 }

@@ -66,6 +66,10 @@ _lib.ssd_scan_fwd_snapshots_workspace_size.argtypes = [ctypes.POINTER(SSDDims), 
 _lib.ssd_scan_fwd_snapshots_workspace_size.restype = ctypes.c_int
 _lib.ssd_snapshot_count.argtypes = [ctypes.POINTER(SSDDims), _p, ctypes.c_int64, ctypes.POINTER(ctypes.c_int64)]
 _lib.ssd_snapshot_count.restype = ctypes.c_int
+_lib.ssd_conv1d_fwd.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, ctypes.POINTER(SSDDims), ctypes.c_int, _p]
+_lib.ssd_conv1d_fwd.restype = ctypes.c_int
+_lib.ssd_conv1d_update.argtypes = [_p, _p, _p, _p, _p, _p, _p, ctypes.POINTER(SSDDims), ctypes.c_int, _p]
+_lib.ssd_conv1d_update.restype = ctypes.c_int
 _lib.ssd_scan_fwd_noalloc.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p,
                                       ctypes.POINTER(SSDDims), ctypes.c_int, _p]
 _lib.ssd_scan_fwd_noalloc.restype = ctypes.c_int
@@ -357,3 +361,83 @@ def state_update(state, x, dt_raw, dt_bias, A, B, C, D, y=None):
                                      _ptr(B), _ptr(C), _ptr(D), _ptr(y), ctypes.byref(dims),
                                      _stream(dev)))
     return y
+
+
+def conv1d_fwd(xbc, weight, bias, nheads, headdim, ngroups, dstate, conv_state=None, cu_seqlens=None,
+               x=None, B=None, C=None, conv_state_out=None, return_state=True):
+    """Causal conv1d + bias + SiLU prologue (ssd_conv1d_fwd).
+
+    Dense: xbc [batch, L, D]; packed varlen (cu_seqlens int32 [nseq+1]): xbc [T, D],
+    D = nheads*headdim + 2*ngroups*dstate. weight [D, K] float32, bias [D] float32 or
+    None, conv_state [nseq, D, K-1] (xbc's dtype) or None.
+    Returns (x, B, C, conv_state_out): x [..., H, P], B/C [..., G, N] in the scan's
+    layouts, conv_state_out [nseq, D, K-1] (None if return_state is False)."""
+    dev = xbc.device
+    varlen = cu_seqlens is not None
+    H, P, G, N = int(nheads), int(headdim), int(ngroups), int(dstate)
+    Dc = H * P + 2 * G * N
+    if varlen:
+        T = xbc.shape[0]
+        nseq = cu_seqlens.numel() - 1
+        tok = (T,)
+    else:
+        if xbc.dim() != 3:
+            raise ValueError("dense xbc must be [batch, L, D]")
+        bsz, L = xbc.shape[0], xbc.shape[1]
+        nseq = bsz
+        tok = (bsz, L)
+    dt = xbc.dtype
+    _need(xbc, "xbc", tok + (Dc,), dt, dev)
+    if weight.dim() != 2 or weight.shape[0] != Dc:
+        raise ValueError(f"weight must be [D={Dc}, K]")
+    K = weight.shape[1]
+    _need(weight, "weight", (Dc, K), torch.float32, dev)
+    if bias is not None:
+        _need(bias, "bias", (Dc,), torch.float32, dev)
+    if conv_state is not None:
+        _need(conv_state, "conv_state", (nseq, Dc, K - 1), dt, dev)
+    if varlen:
+        _need(cu_seqlens, "cu_seqlens", (nseq + 1,), torch.int32, dev)
+    x = torch.empty(*tok, H, P, dtype=dt, device=dev) if x is None else x
+    B = torch.empty(*tok, G, N, dtype=dt, device=dev) if B is None else B
+    C = torch.empty(*tok, G, N, dtype=dt, device=dev) if C is None else C
+    _need(x, "x", tok + (H, P), dt, dev)
+    _need(B, "B", tok + (G, N), dt, dev)
+    _need(C, "C", tok + (G, N), dt, dev)
+    if return_state and conv_state_out is None:
+        conv_state_out = torch.empty(nseq, Dc, K - 1, dtype=dt, device=dev)
+    if conv_state_out is not None:
+        _need(conv_state_out, "conv_state_out", (nseq, Dc, K - 1), dt, dev)
+    if varlen:
+        dims = make_dims(T, H, P, G, N, _dtype_code(xbc), nseq=nseq)
+    else:
+        dims = make_dims(bsz * L, H, P, G, N, _dtype_code(xbc), batch=bsz, seqlen=L)
+    with torch.cuda.device(dev):
+        _check(_lib.ssd_conv1d_fwd(_ptr(xbc), _ptr(weight), _ptr(bias), _ptr(conv_state), _ptr(cu_seqlens),
+                                   _ptr(x), _ptr(B), _ptr(C), _ptr(conv_state_out), ctypes.byref(dims), int(K),
+                                   _stream(dev)))
+    return x, B, C, conv_state_out
+
+
+def conv1d_update(conv_state, xbc, weight, bias, nheads, headdim, ngroups, dstate, x=None, B=None, C=None):
+    """One decode step of the conv1d prologue (ssd_conv1d_update): conv_state [nseq, D, K-1]
+    updated in place, xbc [nseq, D]. Returns (x [nseq,H,P], B [nseq,G,N], C [nseq,G,N])."""
+    dev = xbc.device
+    H, P, G, N = int(nheads), int(headdim), int(ngroups), int(dstate)
+    Dc = H * P + 2 * G * N
+    nseq = xbc.shape[0]
+    dt = xbc.dtype
+    _need(xbc, "xbc", (nseq, Dc), dt, dev)
+    K = weight.shape[1]
+    _need(weight, "weight", (Dc, K), torch.float32, dev)
+    if bias is not None:
+        _need(bias, "bias", (Dc,), torch.float32, dev)
+    _need(conv_state, "conv_state", (nseq, Dc, K - 1), dt, dev)
+    x = torch.empty(nseq, H, P, dtype=dt, device=dev) if x is None else x
+    B = torch.empty(nseq, G, N, dtype=dt, device=dev) if B is None else B
+    C = torch.empty(nseq, G, N, dtype=dt, device=dev) if C is None else C
+    dims = make_dims(nseq, H, P, G, N, _dtype_code(xbc), batch=nseq, seqlen=1)
+    with torch.cuda.device(dev):
+        _check(_lib.ssd_conv1d_update(_ptr(conv_state), _ptr(xbc), _ptr(weight), _ptr(bias), _ptr(x), _ptr(B),
+                                      _ptr(C), ctypes.byref(dims), int(K), _stream(dev)))
+    return x, B, C

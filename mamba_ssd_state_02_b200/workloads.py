@@ -62,6 +62,7 @@ def _splitmix64(z: torch.Tensor) -> torch.Tensor:
 STREAM = {
     "x": 1, "dt_raw": 2, "dt0": 3, "A": 4, "B": 5, "C": 6, "D": 7, "init_state": 8,
     "lengths": 15,
+    "xbc": 20, "conv_w": 21, "conv_b": 22, "conv_state": 23,
 }
 
 _CHUNK = 1 << 22
@@ -236,3 +237,25 @@ def make_all(w: Workload, device="cpu") -> dict:
     d["init_state"] = make_init_state(w, device)
     d["cu_seqlens"] = cu_seqlens(w, device) if w.varlen else None
     return d
+
+
+def conv_channels(w: Workload) -> int:
+    """Channels of the conv1d prologue's input: x, B and C side by side."""
+    return w.nheads * w.headdim + 2 * w.ngroups * w.dstate
+
+
+def make_conv_inputs(w: Workload, width: int = 4, init: bool = True, device="cpu") -> dict:
+    """Inputs of the conv1d prologue for workload w: xbc [T, D] ~ N(0,1) (w.dtype),
+    weight [D, width] ~ U(-1, 1)/sqrt(width) and bias [D] ~ U(-0.5, 0.5) (float32), and a
+    conv state [nseq, D, width-1] ~ N(0,1) (w.dtype) or None."""
+    Dc = conv_channels(w)
+    T = w.total_tokens
+    xbc = to_input_dtype(normal(w.seed, STREAM["xbc"], T * Dc, device=device), w.dtype).view(T, Dc)
+    weight = ((uniform(w.seed, STREAM["conv_w"], Dc * width, device=device) * 2 - 1) / math.sqrt(width))
+    bias = uniform(w.seed, STREAM["conv_b"], Dc, device=device) - 0.5
+    st = None
+    if init:
+        st = to_input_dtype(normal(w.seed, STREAM["conv_state"], w.nseq * Dc * (width - 1), device=device),
+                            w.dtype).view(w.nseq, Dc, width - 1)
+    return {"xbc": xbc, "weight": weight.to(torch.float32).view(Dc, width), "bias": bias.to(torch.float32),
+            "conv_state": st, "cu_seqlens": cu_seqlens(w, device) if w.varlen else None}

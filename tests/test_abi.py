@@ -14,7 +14,8 @@ def declared_functions():
     names = []
     for f in sorted(os.listdir(os.path.join(ROOT, "include"))):
         if f.endswith(".h"):
-            src = open(os.path.join(ROOT, "include", f)).read()
+            with open(os.path.join(ROOT, "include", f)) as fh:
+                src = fh.read()
             src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
             names += re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(ssd_\w+)\s*\(", src, flags=re.M)
     return sorted(set(names))

@@ -35,7 +35,7 @@ def _worker(rank, world, port, out):
 def test_two_gloo_ranks_max_time_and_distinct_problems():
     world = 2
     port = _free_port()
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()          # no fork of this (threaded) process
     out = mgr.dict()
     mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
     assert out[0][0] == out[1][0] == pytest.approx(2.5)
