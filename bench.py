@@ -495,6 +495,29 @@ def bench_ours(args, rank, world, local_rank):
               "peak_gbs": hbm, "frac": round(conv_bytes / conv_ms / 1e6 / hbm, 4),
               "decode_256seq_us_per_step": round(conv_upd_us, 2)}
     del ci, cx, cst_out, cxo, cbo, cco
+
+    # ---- gated group RMSNorm (group 512) over the scan's output and a z branch
+    HPc = w.nheads * w.headdim
+    yz = y.view(w.total_tokens, HPc)
+    zb = W.to_input_dtype(W.normal(w.seed, 30, w.total_tokens * HPc, device=dev), w.dtype).view(w.total_tokens, HPc)
+    nw = (W.uniform(w.seed, 32, HPc, device=dev) + 0.5).to(torch.float32)
+    nout = torch.empty_like(yz)
+    for _ in range(args.warmup):
+        ssd.gated_rmsnorm(yz, zb, nw, group_size=512, eps=1e-6, out=nout)
+    ssd.device_status()
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        ssd.gated_rmsnorm(yz, zb, nw, group_size=512, eps=1e-6, out=nout)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    norm_ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dev)
+    norm_bytes = 3 * yz.numel() * yz.element_size() + HPc * 4
+    gated_norm = {"workload": f"gated_rmsnorm_group512_{w.total_tokens}tok_C{HPc}", "ms_per_call": round(norm_ms, 4),
+                  "bytes_per_call": norm_bytes, "achieved_gbs": round(norm_bytes / norm_ms / 1e6, 1),
+                  "peak_gbs": hbm, "frac": round(norm_bytes / norm_ms / 1e6 / hbm, 4)}
+    del zb, nout, yz
     del host, dbuf, inp, x, dtr, Bm, Cm, y, ws, snaps, ws_snap
     torch.cuda.empty_cache()
 
@@ -515,6 +538,7 @@ def bench_ours(args, rank, world, local_rank):
         "decode": decode,
         "snapshots": snapshots,
         "conv1d": conv1d,
+        "gated_rmsnorm": gated_norm,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, threads, secs = oracle_sample(w, 16384, w.nheads)

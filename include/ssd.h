@@ -195,6 +195,20 @@ ssd_status ssd_conv1d_update(void* conv_state, const void* xbc, const float* wei
                              void* B, void* C, const ssd_dims* dims, int width, ssd_stream_t stream);
 
 /*
+ * Gated group RMSNorm, the stage after the scan in a Mamba-2 block (RL-Kernel issue page,
+ * Figure 2: y gated by SiLU of the z branch, normalised over groups of 512 channels; the
+ * JAX Nemotron 3 Nano page's configuration gives the RMSNorm epsilon, 1e-6). Per token t
+ * and channel c of its group:
+ *   g = y[t][c] * silu(z[t][c]);  out[t][c] = g * rsqrt(mean over the group of g^2 + eps) * weight[c]
+ * in FP32, rounded to `dtype`.
+ *   y, z, out: [ntok, channels] (dtype; y is the scan's output viewed as [T, H*P]).
+ *   weight: [channels] float32. All four 16-byte aligned; out may alias y.
+ *   group_size: 256, 512 or 1024, dividing channels; eps >= 0.
+ */
+ssd_status ssd_gated_rmsnorm(const void* y, const void* z, const float* weight, void* out, int64_t ntok,
+                             int channels, int group_size, float eps, ssd_dtype dtype, ssd_stream_t stream);
+
+/*
  * ssd_scan_fwd without any device allocation (the pages have no counterpart; this is a
  * deployment convenience). Some callers cannot allocate device memory while they run:
  * serving engines that reserve their whole memory budget at start-up and forbid later

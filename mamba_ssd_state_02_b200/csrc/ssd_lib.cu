@@ -18,6 +18,7 @@
 #include "ssd.h"
 #include "ssd_common.cuh"
 #include "ssd_conv.cuh"
+#include "ssd_norm.cuh"
 #include "ssd_decode.cuh"
 #include "ssd_scan_simt.cuh"
 #include "ssd_scan_tc.cuh"
@@ -46,9 +47,10 @@ ssd_status cuda_fail(cudaError_t e, const char* what) {
 // ---------------------------------------------------------------------------------
 // Per-kernel event timing (ssd_profile_enable / ssd_profile_read).
 enum Stage { ST_TABLE, ST_CUMSUM, ST_CHUNK_STATE, ST_STATE_PASSING, ST_CHUNK_SCAN, ST_STATE_UPDATE,
-             ST_CONV, ST_CONV_UPDATE, ST_COUNT };
+             ST_CONV, ST_CONV_UPDATE, ST_NORM, ST_COUNT };
 const char* const kStageName[ST_COUNT] = {"ssd_chunk_table", "ssd_chunk_cumsum", "ssd_chunk_state",
-                                          "ssd_state_passing", "ssd_chunk_scan", "ssd_state_update", "ssd_conv1d", "ssd_conv1d_update"};
+                                          "ssd_state_passing", "ssd_chunk_scan", "ssd_state_update", "ssd_conv1d", "ssd_conv1d_update",
+                                          "ssd_gated_rmsnorm"};
 constexpr size_t kMaxRecords = 65536;
 
 struct Profiler {
@@ -917,6 +919,50 @@ extern "C" ssd_status ssd_conv1d_update(void* conv_state, const void* xbc, const
 #undef SSD_CONV_CASE
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch (conv1d update)");
+    t_launches = 1;
+    t_last_error.clear();
+    return SSD_OK;
+}
+
+// ---------------------------------------------------------------------------------
+// Gated group RMSNorm (epilogue stage).
+extern "C" ssd_status ssd_gated_rmsnorm(const void* y, const void* z, const float* weight, void* out, int64_t ntok,
+                                        int channels, int group_size, float eps, ssd_dtype dtype,
+                                        ssd_stream_t stream) {
+    if (ntok < 0 || channels <= 0) return fail(SSD_ERR_INVALID_ARG, "ntok must be >= 0 and channels > 0");
+    if (group_size != 256 && group_size != 512 && group_size != 1024)
+        return fail(SSD_ERR_UNSUPPORTED, "group_size %d not in {256,512,1024}", group_size);
+    if (channels % group_size != 0)
+        return fail(SSD_ERR_UNSUPPORTED, "channels (%d) must be a multiple of group_size (%d)", channels, group_size);
+    if (dtype != SSD_DTYPE_F32 && dtype != SSD_DTYPE_BF16) return fail(SSD_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+    if (!(eps >= 0.f)) return fail(SSD_ERR_INVALID_ARG, "eps must be >= 0");
+    if (ntok > 0 && (!y || !z || !weight || !out)) return fail(SSD_ERR_INVALID_ARG, "y, z, weight and out must be non-NULL");
+    if (!aligned(y, 16) || !aligned(z, 16) || !aligned(weight, 16) || !aligned(out, 16))
+        return fail(SSD_ERR_INVALID_ARG, "y, z, weight and out must be 16-byte aligned");
+    if (ntok == 0) {
+        t_launches = 0;
+        t_last_error.clear();
+        return SSD_OK;
+    }
+    const int64_t warps = (ntok + kNormTokens - 1) / kNormTokens * (channels / group_size);
+    const int64_t blocks = (warps + kNormWarps - 1) / kNormWarps;
+    if (blocks > INT32_MAX) return fail(SSD_ERR_UNSUPPORTED, "too many tokens in one call");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    {
+        StageScope sc(ST_NORM, st);
+#define SSD_NORM_CASE(TT, VV)                                                                              \
+    if (group_size == 256 * VV)                                                                            \
+        k_gated_rmsnorm<TT, VV><<<(unsigned)blocks, 32 * kNormWarps, 0, st>>>((const TT*)y, (const TT*)z, weight, \
+                                                                           (TT*)out, ntok, channels, eps);
+        if (dtype == SSD_DTYPE_BF16) {
+            SSD_NORM_CASE(__nv_bfloat16, 1) SSD_NORM_CASE(__nv_bfloat16, 2) SSD_NORM_CASE(__nv_bfloat16, 4)
+        } else {
+            SSD_NORM_CASE(float, 1) SSD_NORM_CASE(float, 2) SSD_NORM_CASE(float, 4)
+        }
+#undef SSD_NORM_CASE
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch (gated rmsnorm)");
     t_launches = 1;
     t_last_error.clear();
     return SSD_OK;

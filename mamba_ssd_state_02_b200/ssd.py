@@ -70,6 +70,9 @@ _lib.ssd_conv1d_fwd.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, ctypes.POINT
 _lib.ssd_conv1d_fwd.restype = ctypes.c_int
 _lib.ssd_conv1d_update.argtypes = [_p, _p, _p, _p, _p, _p, _p, ctypes.POINTER(SSDDims), ctypes.c_int, _p]
 _lib.ssd_conv1d_update.restype = ctypes.c_int
+_lib.ssd_gated_rmsnorm.argtypes = [_p, _p, _p, _p, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+                                   ctypes.c_int, _p]
+_lib.ssd_gated_rmsnorm.restype = ctypes.c_int
 _lib.ssd_scan_fwd_noalloc.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, _p, _p,
                                       ctypes.POINTER(SSDDims), ctypes.c_int, _p]
 _lib.ssd_scan_fwd_noalloc.restype = ctypes.c_int
@@ -441,3 +444,21 @@ def conv1d_update(conv_state, xbc, weight, bias, nheads, headdim, ngroups, dstat
         _check(_lib.ssd_conv1d_update(_ptr(conv_state), _ptr(xbc), _ptr(weight), _ptr(bias), _ptr(x), _ptr(B),
                                       _ptr(C), ctypes.byref(dims), int(K), _stream(dev)))
     return x, B, C
+
+
+def gated_rmsnorm(y, z, weight, group_size=512, eps=1e-6, out=None):
+    """Gated group RMSNorm (ssd_gated_rmsnorm): out = rmsnorm_group(y * silu(z)) * weight.
+    y, z: [..., channels] (bf16 or float32, same shape); weight [channels] float32."""
+    dev = y.device
+    channels = y.shape[-1]
+    ntok = y.numel() // channels if channels else 0
+    _need(y, "y", tuple(y.shape), y.dtype, dev)
+    _need(z, "z", tuple(y.shape), y.dtype, dev)
+    _need(weight, "weight", (channels,), torch.float32, dev)
+    if out is None:
+        out = torch.empty_like(y)
+    _need(out, "out", tuple(y.shape), y.dtype, dev)
+    with torch.cuda.device(dev):
+        _check(_lib.ssd_gated_rmsnorm(_ptr(y), _ptr(z), _ptr(weight), _ptr(out), int(ntok), int(channels),
+                                      int(group_size), float(eps), _dtype_code(y), _stream(dev)))
+    return out
