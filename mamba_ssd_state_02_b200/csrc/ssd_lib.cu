@@ -189,11 +189,12 @@ ssd_status make_plan(const ssd_dims* d, int chunk, bool varlen, Plan* pl, int64_
         return varlen ? p.T / Ls + p.nseq : (int64_t)p.nseq * ((p.seqlen + Ls - 1) / Ls);
     };
     if (p.tc) {
-        // Segment length: the longest of 2048/1024/512/256 tokens that still gives at least
-        // two work units (segment x 4 heads) per SM of a 148-SM B200.
+        // Segment length: the longest of 8192/4096/.../512/256 tokens whose chunk-scan grid
+        // (segment x 2 heads) still fills one wave of a 148-SM B200. Longer segments carry
+        // fewer inter-segment states through HBM; below one wave SMs sit idle.
         int Ls = 256;
-        for (int cand : {2048, 1024, 512}) {
-            if (segs_for(cand) * (p.H / tc::kHeads) >= 2 * 148) {
+        for (int cand : {8192, 4096, 2048, 1024, 512}) {
+            if (segs_for(cand) * (p.H / tc::kHeadsB) >= 148) {
                 Ls = cand;
                 break;
             }
