@@ -233,6 +233,79 @@ ssd_status ssd_scan_fwd_noalloc(const void* x, const float* dt_raw, const float*
                                 const ssd_dims* dims, int chunk, ssd_stream_t stream);
 
 /*
+ * Strict mode: bitwise split invariance (RL-Kernel issue page, §4.1: a token's output is
+ * bitwise the same whether it came from a full-sequence pass, a prefill of any length or a
+ * decode at any step after any chunk-aligned prefill split; §7: prefill and decode share
+ * device functions, the decode emulates the chunked arithmetic, and strict mode fails
+ * closed where chunks cannot stay sequence-anchored).
+ *
+ * Both entry points below evaluate the chunked algorithm (chunks of `chunk` tokens
+ * anchored at each sequence start) with one set of FP32 device functions, every sum and
+ * dot product taken left to right over its index and every operation correctly rounded
+ * (no contraction, no reassociation):
+ *   dt_s = softplus(dt_raw_s + dt_bias);  Acum_s = Acum_{s-1} + dt_s A  (in-chunk, from 0)
+ *   y_t  = D x_t + exp(Acum_t) (C_t . h_in) + sum_{s<=t} (C_t . B_s) exp(Acum_t - Acum_s) dt_s x_s
+ *   h_in(next chunk) = exp(Acum_last) h_in + sum_s exp(Acum_last - Acum_s) dt_s x_s B_s^T
+ * The decode keeps each sequence's open (partial) chunk in a chunk cache and computes a
+ * new token's y as the prefill computes that chunk position; when the chunk fills, it
+ * folds the chunk into the cached state as the prefill does. So for any split of a
+ * sequence into a strict prefill followed by strict decode steps, or into strict prefills
+ * at chunk boundaries, every y and every cached state is bit-identical to a single strict
+ * prefill over the whole sequence, and no result depends on batch size or position.
+ * Strict results agree with ssd_scan_fwd to within rounding but not bitwise.
+ *
+ * The chunk cache, per sequence (Q = chunk; all arrays device memory owned by the caller):
+ *   state [nseq,H,P,N] float32: the state entering the sequence's open chunk (16-byte aligned)
+ *   x     [nseq,H,Q,P] dtype:   x of the open chunk's tokens, rows 0..len-1 (16-byte aligned)
+ *   B     [nseq,G,Q,N] dtype:   B of the open chunk's tokens (16-byte aligned)
+ *   dt    [nseq,H,Q]   float32: their dt;  acum [nseq,H,Q] float32: their Acum
+ *   len   [nseq,H]     int32:   tokens in the open chunk, 0..Q-1 (equal across a sequence's heads)
+ * Rows at or past len are never read. Only these entry points should write a cache.
+ */
+typedef struct {
+    float* state;
+    void* x;
+    void* B;
+    float* dt;
+    float* acum;
+    int32_t* len;
+} ssd_chunk_cache;
+
+/* Workspace bytes for ssd_strict_scan_fwd (as ssd_scan_fwd_workspace_size). */
+ssd_status ssd_strict_scan_fwd_workspace_size(const ssd_dims* dims, int chunk, size_t* bytes);
+
+/*
+ * Strict chunked prefill. Arguments as ssd_scan_fwd, except:
+ *   cache: required; written on return with each sequence's open chunk (the tokens of a
+ *     partial last chunk, len = length mod chunk) and the state entering it.
+ *   resume: 0 starts every sequence from a zero state; 1 starts from cache->state, which
+ *     must have an empty open chunk (len == 0 for every sequence and head: the previous
+ *     strict call ended on a chunk boundary). Otherwise the kernel latches
+ *     SSD_ERR_UNSUPPORTED (fail closed) and the results are not valid.
+ *   final_state: optional, the state after each sequence's last token.
+ * Supported: fp32 or bf16 x/B/C, P and N in {16, 32, 64, 128}, chunk in {64, 128, 256};
+ * the CUDA-core kernels are used for every geometry (no tensor cores: their summation
+ * order is not the decode's).
+ */
+ssd_status ssd_strict_scan_fwd(const void* x, const float* dt_raw, const float* dt_bias, const float* A,
+                               const void* B, const void* C, const float* D, const int32_t* cu_seqlens,
+                               void* y, float* final_state, const ssd_chunk_cache* cache, int resume,
+                               const ssd_dims* dims, int chunk, ssd_stream_t stream);
+
+/*
+ * Chunk-emulating decode step for nseq = dims->batch sequences (dims->seqlen must be 1),
+ * continuing the caches that ssd_strict_scan_fwd or earlier steps wrote with the same
+ * dims and chunk. Per sequence and head the token becomes position len of the open
+ * chunk: y is that position's strict prefill output, the token is appended, and when the
+ * chunk is full it is folded into cache->state (len back to 0). A len outside [0, chunk)
+ * latches SSD_ERR_INVALID_ARG. x [nseq,H,P], B/C [nseq,G,N], dt_raw [nseq,H], y out
+ * [nseq,H,P], as ssd_state_update.
+ */
+ssd_status ssd_strict_state_update(const ssd_chunk_cache* cache, const void* x, const float* dt_raw,
+                                   const float* dt_bias, const float* A, const void* B, const void* C,
+                                   const float* D, void* y, const ssd_dims* dims, int chunk, ssd_stream_t stream);
+
+/*
  * Waits for `stream`, then reads and clears the device error word: SSD_OK, or the
  * first error a kernel latched since the last read (SSD_ERR_INVALID_ARG for bad
  * cu_seqlens or A > 0, SSD_ERR_TIMEOUT for an expired bounded wait). SSD_ERR_CUDA

@@ -21,6 +21,7 @@
 #include "ssd_norm.cuh"
 #include "ssd_decode.cuh"
 #include "ssd_scan_simt.cuh"
+#include "ssd_strict.cuh"
 #include "ssd_scan_tc.cuh"
 #include "ssd_tc_selftest.cuh"
 
@@ -47,10 +48,13 @@ ssd_status cuda_fail(cudaError_t e, const char* what) {
 // ---------------------------------------------------------------------------------
 // Per-kernel event timing (ssd_profile_enable / ssd_profile_read).
 enum Stage { ST_TABLE, ST_CUMSUM, ST_CHUNK_STATE, ST_STATE_PASSING, ST_CHUNK_SCAN, ST_STATE_UPDATE,
-             ST_CONV, ST_CONV_UPDATE, ST_NORM, ST_COUNT };
+             ST_CONV, ST_CONV_UPDATE, ST_NORM, ST_STRICT_CUMSUM, ST_STRICT_STATE, ST_STRICT_PASSING,
+             ST_STRICT_SCAN, ST_STRICT_CACHE, ST_STRICT_UPDATE, ST_COUNT };
 const char* const kStageName[ST_COUNT] = {"ssd_chunk_table", "ssd_chunk_cumsum", "ssd_chunk_state",
                                           "ssd_state_passing", "ssd_chunk_scan", "ssd_state_update", "ssd_conv1d", "ssd_conv1d_update",
-                                          "ssd_gated_rmsnorm"};
+                                          "ssd_gated_rmsnorm", "ssd_strict_cumsum", "ssd_strict_chunk_state",
+                                          "ssd_strict_state_passing", "ssd_strict_chunk_scan",
+                                          "ssd_strict_cache_fill", "ssd_strict_state_update"};
 constexpr size_t kMaxRecords = 65536;
 
 struct Profiler {
@@ -139,7 +143,7 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Validate dims/chunk and fill the plan (no pointers looked at here).
-ssd_status make_plan(const ssd_dims* d, int chunk, bool varlen, Plan* pl, int64_t snap = 0) {
+ssd_status make_plan(const ssd_dims* d, int chunk, bool varlen, Plan* pl, int64_t snap = 0, bool strict = false) {
     if (!d) return fail(SSD_ERR_INVALID_ARG, "dims is NULL");
     if (d->nheads <= 0 || d->headdim <= 0 || d->ngroups <= 0 || d->dstate <= 0)
         return fail(SSD_ERR_INVALID_ARG, "nheads, headdim, ngroups and dstate must be positive");
@@ -184,7 +188,7 @@ ssd_status make_plan(const ssd_dims* d, int chunk, bool varlen, Plan* pl, int64_
     if (p.T * (int64_t)p.H * p.P >= (int64_t)1 << 40)
         return fail(SSD_ERR_UNSUPPORTED, "x has more than 2^40 elements");
     // Tensor-core pipeline: bf16, headdim 64, dstate 128, heads per group a multiple of 4.
-    p.tc = p.bf16 && p.P == tc::kP && p.N == tc::kN && (p.H / p.G) % tc::kHeads == 0;
+    p.tc = !strict && p.bf16 && p.P == tc::kP && p.N == tc::kN && (p.H / p.G) % tc::kHeads == 0;
     auto segs_for = [&](int64_t Ls) -> int64_t {
         return varlen ? p.T / Ls + p.nseq : (int64_t)p.nseq * ((p.seqlen + Ls - 1) / Ls);
     };
@@ -964,6 +968,201 @@ extern "C" ssd_status ssd_gated_rmsnorm(const void* y, const void* z, const floa
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch (gated rmsnorm)");
+    t_launches = 1;
+    t_last_error.clear();
+    return SSD_OK;
+}
+
+// ---------------------------------------------------------------------------------
+// Strict mode: bitwise split-invariant prefill and the chunk-emulating decode step.
+namespace ssd {
+namespace {
+
+ssd_status check_cache(const ssd_chunk_cache* cc) {
+    if (!cc) return fail(SSD_ERR_INVALID_ARG, "cache is NULL");
+    if (!cc->state || !cc->x || !cc->B || !cc->dt || !cc->acum || !cc->len)
+        return fail(SSD_ERR_INVALID_ARG, "every cache array must be non-NULL");
+    if (!aligned(cc->state, 16) || !aligned(cc->x, 16) || !aligned(cc->B, 16) || !aligned(cc->dt, 4) ||
+        !aligned(cc->acum, 4) || !aligned(cc->len, 4))
+        return fail(SSD_ERR_INVALID_ARG, "cache state/x/B must be 16-byte aligned, dt/acum/len 4-byte");
+    return SSD_OK;
+}
+
+template <typename T>
+ssd_status launch_strict(const Plan& pl, char* ws, const T* x, const float* dt_raw, const float* dt_bias,
+                         const float* A, const T* B, const T* C, const float* D, const int32_t* cu, T* y,
+                         float* fin, const ssd_chunk_cache& cc, int resume, cudaStream_t st) {
+    using namespace strict;
+    auto* table = reinterpret_cast<ChunkEntry*>(ws + pl.off_table);
+    auto* first = reinterpret_cast<int32_t*>(ws + pl.off_first);
+    auto* count = reinterpret_cast<int32_t*>(ws + pl.off_count);
+    auto* dtc = reinterpret_cast<float*>(ws + pl.off_dt);
+    auto* acum = reinterpret_cast<float*>(ws + pl.off_acum);
+    auto* states = reinterpret_cast<float*>(ws + pl.off_states);
+    const int H = pl.H, G = pl.G, P = pl.P, N = pl.N, Q = pl.Q;
+    const size_t scan_smem = chunk_scan_smem(P, N, Q);
+    cudaError_t e = cudaFuncSetAttribute(k_strict_chunk_scan<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)scan_smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(strict chunk scan)");
+    int n = 0;
+    {
+        StageScope sc(ST_TABLE, st);
+        k_chunk_table<<<1, kTableThreads, 0, st>>>(cu, pl.nseq, pl.T, pl.seqlen, Q, table, first, count, 0,
+                                                   nullptr);
+    }
+    ++n;
+    const unsigned mc = (unsigned)pl.max_chunks;
+    if (mc > 0) {
+        {
+            StageScope sc(ST_STRICT_CUMSUM, st);
+            k_strict_cumsum<<<dim3(mc, (H + 127) / 128), 128, 0, st>>>(dt_raw, dt_bias, A, table, count, H, Q,
+                                                                       dtc, acum);
+        }
+        {
+            StageScope sc(ST_STRICT_STATE, st);
+            k_strict_chunk_state<T><<<dim3(mc, H), kThreads, chunk_state_smem(P, N, Q), st>>>(
+                x, B, dtc, acum, table, count, H, G, P, N, Q, states);
+        }
+        n += 2;
+    }
+    {
+        StageScope sc(ST_STRICT_PASSING, st);
+        k_strict_passing<<<dim3(pl.nseq, H, (P * N + kThreads - 1) / kThreads), kThreads, 0, st>>>(
+            states, acum, table, first, resume, cc.state, cc.len, fin, H, P * N, Q);
+    }
+    ++n;
+    if (mc > 0) {
+        StageScope sc(ST_STRICT_SCAN, st);
+        k_strict_chunk_scan<T><<<dim3(mc, H, Q / 32), kThreads, scan_smem, st>>>(
+            x, B, C, D, dtc, acum, states, table, count, H, G, P, N, Q, y);
+        ++n;
+    }
+    {
+        StageScope sc(ST_STRICT_CACHE, st);
+        k_strict_cache_fill<T><<<dim3(pl.nseq, H), kThreads, 0, st>>>(
+            x, B, dtc, acum, table, first, H, G, P, N, Q, static_cast<T*>(cc.x), static_cast<T*>(cc.B), cc.dt,
+            cc.acum, cc.len);
+    }
+    ++n;
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch (strict scan)");
+    t_launches = n;
+    return SSD_OK;
+}
+
+}  // namespace
+}  // namespace ssd
+
+extern "C" ssd_status ssd_strict_scan_fwd_workspace_size(const ssd_dims* dims, int chunk, size_t* bytes) {
+    if (!bytes) return fail(SSD_ERR_INVALID_ARG, "bytes is NULL");
+    Plan dense, packed;
+    const ssd_status sd = make_plan(dims, chunk, false, &dense, 0, true);
+    const ssd_status sp = make_plan(dims, chunk, true, &packed, 0, true);
+    if (sd != SSD_OK && sp != SSD_OK) return sd;
+    size_t b = 0;
+    if (sd == SSD_OK) b = dense.bytes;
+    if (sp == SSD_OK && packed.bytes > b) b = packed.bytes;
+    t_last_error.clear();
+    *bytes = b;
+    return SSD_OK;
+}
+
+extern "C" ssd_status ssd_strict_scan_fwd(const void* x, const float* dt_raw, const float* dt_bias, const float* A,
+                                          const void* B, const void* C, const float* D, const int32_t* cu_seqlens,
+                                          void* y, float* final_state, const ssd_chunk_cache* cache, int resume,
+                                          const ssd_dims* dims, int chunk, ssd_stream_t stream) {
+    Plan pl;
+    ssd_status s = make_plan(dims, chunk, cu_seqlens != nullptr, &pl, 0, true);
+    if (s != SSD_OK) return s;
+    s = check_cache(cache);
+    if (s != SSD_OK) return s;
+    if (!dt_bias || !A || !D) return fail(SSD_ERR_INVALID_ARG, "dt_bias, A and D must be non-NULL");
+    if (pl.T > 0 && (!x || !dt_raw || !B || !C || !y))
+        return fail(SSD_ERR_INVALID_ARG, "x, dt_raw, B, C and y must be non-NULL");
+    if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(y, 16))
+        return fail(SSD_ERR_INVALID_ARG, "x, B, C and y must be 16-byte aligned");
+    if (!aligned(dt_raw, 4) || !aligned(dt_bias, 4) || !aligned(A, 4) || !aligned(D, 4) ||
+        !aligned(final_state, 16) || !aligned(cu_seqlens, 4))
+        return fail(SSD_ERR_INVALID_ARG, "float/int arrays must be 4-byte aligned, states 16-byte");
+    if (resume != 0 && resume != 1) return fail(SSD_ERR_INVALID_ARG, "resume must be 0 or 1");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (pl.nseq == 0) {
+        t_launches = 0;
+        t_last_error.clear();
+        return SSD_OK;
+    }
+    char* ws = static_cast<char*>(dims->workspace);
+    bool owned = false;
+    if (ws) {
+        if (dims->workspace_bytes < pl.bytes)
+            return fail(SSD_ERR_INVALID_ARG, "workspace_bytes %zu < required %zu", dims->workspace_bytes,
+                        pl.bytes);
+        if (!aligned(ws, 256)) return fail(SSD_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    } else {
+        cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&ws), pl.bytes, st);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(workspace)");
+        owned = true;
+    }
+    if (pl.bf16)
+        s = launch_strict<__nv_bfloat16>(pl, ws, static_cast<const __nv_bfloat16*>(x), dt_raw, dt_bias, A,
+                                         static_cast<const __nv_bfloat16*>(B), static_cast<const __nv_bfloat16*>(C),
+                                         D, cu_seqlens, static_cast<__nv_bfloat16*>(y), final_state, *cache,
+                                         resume, st);
+    else
+        s = launch_strict<float>(pl, ws, static_cast<const float*>(x), dt_raw, dt_bias, A,
+                                 static_cast<const float*>(B), static_cast<const float*>(C), D, cu_seqlens,
+                                 static_cast<float*>(y), final_state, *cache, resume, st);
+    if (owned) {
+        cudaError_t e = cudaFreeAsync(ws, st);
+        if (e != cudaSuccess && s == SSD_OK) return cuda_fail(e, "cudaFreeAsync(workspace)");
+    }
+    if (s == SSD_OK) t_last_error.clear();
+    return s;
+}
+
+extern "C" ssd_status ssd_strict_state_update(const ssd_chunk_cache* cache, const void* x, const float* dt_raw,
+                                              const float* dt_bias, const float* A, const void* B, const void* C,
+                                              const float* D, void* y, const ssd_dims* dims, int chunk,
+                                              ssd_stream_t stream) {
+    if (!dims) return fail(SSD_ERR_INVALID_ARG, "dims is NULL");
+    ssd_dims d = *dims;
+    if (d.seqlen != 1) return fail(SSD_ERR_INVALID_ARG, "decode takes seqlen == 1 (got %lld)", (long long)d.seqlen);
+    Plan pl;
+    ssd_status s = make_plan(&d, chunk, false, &pl, 0, true);
+    if (s != SSD_OK) return s;
+    if (pl.nseq == 0) {
+        t_launches = 0;
+        t_last_error.clear();
+        return SSD_OK;
+    }
+    s = check_cache(cache);
+    if (s != SSD_OK) return s;
+    if (!x || !dt_raw || !dt_bias || !A || !B || !C || !D || !y)
+        return fail(SSD_ERR_INVALID_ARG, "all decode pointers must be non-NULL");
+    if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(y, 16))
+        return fail(SSD_ERR_INVALID_ARG, "x, B, C and y must be 16-byte aligned");
+    if (!aligned(dt_raw, 4) || !aligned(dt_bias, 4) || !aligned(A, 4) || !aligned(D, 4))
+        return fail(SSD_ERR_INVALID_ARG, "float arrays must be 4-byte aligned");
+    if ((int64_t)pl.nseq * pl.H >= INT32_MAX) return fail(SSD_ERR_UNSUPPORTED, "nseq*nheads too large");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t smem = strict::decode_smem(pl.P, pl.N, pl.Q);
+    const unsigned grid = (unsigned)(pl.nseq * pl.H);
+    {
+        StageScope sc(ST_STRICT_UPDATE, st);
+        if (pl.bf16)
+            strict::k_strict_decode<__nv_bfloat16><<<grid, strict::kThreads, smem, st>>>(
+                cache->state, static_cast<__nv_bfloat16*>(cache->x), static_cast<__nv_bfloat16*>(cache->B),
+                cache->dt, cache->acum, cache->len, static_cast<const __nv_bfloat16*>(x), dt_raw, dt_bias, A,
+                static_cast<const __nv_bfloat16*>(B), static_cast<const __nv_bfloat16*>(C), D,
+                static_cast<__nv_bfloat16*>(y), pl.H, pl.G, pl.P, pl.N, pl.Q);
+        else
+            strict::k_strict_decode<float><<<grid, strict::kThreads, smem, st>>>(
+                cache->state, static_cast<float*>(cache->x), static_cast<float*>(cache->B), cache->dt, cache->acum,
+                cache->len, static_cast<const float*>(x), dt_raw, dt_bias, A, static_cast<const float*>(B),
+                static_cast<const float*>(C), D, static_cast<float*>(y), pl.H, pl.G, pl.P, pl.N, pl.Q);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch (strict state update)");
     t_launches = 1;
     t_last_error.clear();
     return SSD_OK;

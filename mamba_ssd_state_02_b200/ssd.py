@@ -10,6 +10,7 @@ Functions mirror the C entry points:
   scan_fwd(x, dt_raw, dt_bias, A, B, C, D, init_state=None, cu_seqlens=None,
            chunk=128, y=None, final_state=None, workspace=None)
   state_update(state, x, dt_raw, dt_bias, A, B, C, D, y=None)
+  ChunkCache.empty(...), strict_scan_fwd(...), strict_state_update(...)  (strict mode)
   device_status(), scan_variant(...), workspace_size(...), last_launch_count()
 """
 from __future__ import annotations
@@ -86,6 +87,23 @@ _lib.ssd_scan_fwd_variant.argtypes = [ctypes.POINTER(SSDDims), ctypes.c_int]
 _lib.ssd_scan_fwd_variant.restype = ctypes.c_char_p
 _lib.ssd_scan_fwd_segment_tokens.argtypes = [ctypes.POINTER(SSDDims), ctypes.c_int]
 _lib.ssd_scan_fwd_segment_tokens.restype = ctypes.c_int
+
+
+class SSDChunkCache(ctypes.Structure):
+    """Mirror of ``ssd_chunk_cache``."""
+    _fields_ = [("state", ctypes.c_void_p), ("x", ctypes.c_void_p), ("B", ctypes.c_void_p),
+                ("dt", ctypes.c_void_p), ("acum", ctypes.c_void_p), ("len", ctypes.c_void_p)]
+
+
+_lib.ssd_strict_scan_fwd_workspace_size.argtypes = [ctypes.POINTER(SSDDims), ctypes.c_int,
+                                                    ctypes.POINTER(ctypes.c_size_t)]
+_lib.ssd_strict_scan_fwd_workspace_size.restype = ctypes.c_int
+_lib.ssd_strict_scan_fwd.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _p, _p, ctypes.POINTER(SSDChunkCache),
+                                     ctypes.c_int, ctypes.POINTER(SSDDims), ctypes.c_int, _p]
+_lib.ssd_strict_scan_fwd.restype = ctypes.c_int
+_lib.ssd_strict_state_update.argtypes = [ctypes.POINTER(SSDChunkCache), _p, _p, _p, _p, _p, _p, _p, _p,
+                                         ctypes.POINTER(SSDDims), ctypes.c_int, _p]
+_lib.ssd_strict_state_update.restype = ctypes.c_int
 _lib.ssd_last_launch_count.argtypes = []
 _lib.ssd_last_launch_count.restype = ctypes.c_int
 
@@ -462,3 +480,119 @@ def gated_rmsnorm(y, z, weight, group_size=512, eps=1e-6, out=None):
         _check(_lib.ssd_gated_rmsnorm(_ptr(y), _ptr(z), _ptr(weight), _ptr(out), int(ntok), int(channels),
                                       int(group_size), float(eps), _dtype_code(y), _stream(dev)))
     return out
+
+
+# ---------------------------------------------------------------------------------
+# Strict mode (ssd_strict_scan_fwd / ssd_strict_state_update): bitwise split invariance
+# between a chunked prefill and the chunk-emulating decode.
+class ChunkCache:
+    """Per-sequence chunk cache of strict mode (``ssd_chunk_cache``): the state entering
+    each sequence's open chunk and that chunk's tokens. Tensors are owned here; the
+    library only reads and writes them."""
+
+    def __init__(self, state, x, B, dt, acum, length, chunk):
+        self.state, self.x, self.B, self.dt, self.acum, self.len = state, x, B, dt, acum, length
+        self.chunk = int(chunk)
+
+    @classmethod
+    def empty(cls, nseq, H, P, G, N, chunk, dtype, device):
+        f32 = dict(dtype=torch.float32, device=device)
+        return cls(torch.zeros(nseq, H, P, N, **f32), torch.zeros(nseq, H, chunk, P, dtype=dtype, device=device),
+                   torch.zeros(nseq, G, chunk, N, dtype=dtype, device=device), torch.zeros(nseq, H, chunk, **f32),
+                   torch.zeros(nseq, H, chunk, **f32), torch.zeros(nseq, H, dtype=torch.int32, device=device),
+                   chunk)
+
+    def clone(self):
+        return ChunkCache(self.state.clone(), self.x.clone(), self.B.clone(), self.dt.clone(), self.acum.clone(),
+                          self.len.clone(), self.chunk)
+
+    def _check(self, nseq, H, P, G, N, dtype, device):
+        Q = self.chunk
+        _need(self.state, "cache.state", (nseq, H, P, N), torch.float32, device)
+        _need(self.x, "cache.x", (nseq, H, Q, P), dtype, device)
+        _need(self.B, "cache.B", (nseq, G, Q, N), dtype, device)
+        _need(self.dt, "cache.dt", (nseq, H, Q), torch.float32, device)
+        _need(self.acum, "cache.acum", (nseq, H, Q), torch.float32, device)
+        _need(self.len, "cache.len", (nseq, H), torch.int32, device)
+
+    def _c(self):
+        return SSDChunkCache(_ptr(self.state), _ptr(self.x), _ptr(self.B), _ptr(self.dt), _ptr(self.acum),
+                             _ptr(self.len))
+
+
+def strict_workspace_size(dims: SSDDims, chunk: int) -> int:
+    b = ctypes.c_size_t(0)
+    _check(_lib.ssd_strict_scan_fwd_workspace_size(ctypes.byref(dims), int(chunk), ctypes.byref(b)))
+    return int(b.value)
+
+
+def strict_scan_fwd(x, dt_raw, dt_bias, A, B, C, D, cache: ChunkCache, resume=False, cu_seqlens=None,
+                    y=None, final_state=None, workspace=None):
+    """Strict chunked prefill (ssd_strict_scan_fwd). Shapes as scan_fwd; the chunk length
+    is the cache's. resume=True starts from cache.state (its open chunks must be empty).
+    Writes the cache in place; returns (y, final_state)."""
+    dev = x.device
+    varlen = cu_seqlens is not None
+    if varlen:
+        T, H, P = x.shape
+        nseq = cu_seqlens.numel() - 1
+        tok = (T,)
+    else:
+        if x.dim() != 4:
+            raise ValueError("dense x must be [batch, L, H, P]")
+        bsz, L, H, P = x.shape
+        nseq = bsz
+        tok = (bsz, L)
+    G, N = B.shape[-2], B.shape[-1]
+    dt = x.dtype
+    _need(x, "x", tok + (H, P), dt, dev)
+    _need(dt_raw, "dt_raw", tok + (H,), torch.float32, dev)
+    _need(B, "B", tok + (G, N), dt, dev)
+    _need(C, "C", tok + (G, N), dt, dev)
+    for name, v in (("dt_bias", dt_bias), ("A", A), ("D", D)):
+        _need(v, name, (H,), torch.float32, dev)
+    if varlen:
+        _need(cu_seqlens, "cu_seqlens", (nseq + 1,), torch.int32, dev)
+    cache._check(nseq, H, P, G, N, dt, dev)
+    if y is None:
+        y = torch.empty_like(x)
+    _need(y, "y", tok + (H, P), dt, dev)
+    if final_state is None:
+        final_state = torch.empty(nseq, H, P, N, dtype=torch.float32, device=dev)
+    _need(final_state, "final_state", (nseq, H, P, N), torch.float32, dev)
+    if varlen:
+        dims = make_dims(x.shape[0], H, P, G, N, _dtype_code(x), nseq=nseq, workspace=workspace)
+    else:
+        dims = make_dims(bsz * L, H, P, G, N, _dtype_code(x), batch=bsz, seqlen=L, workspace=workspace)
+    cc = cache._c()
+    with torch.cuda.device(dev):
+        _check(_lib.ssd_strict_scan_fwd(_ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                        _ptr(cu_seqlens), _ptr(y), _ptr(final_state), ctypes.byref(cc),
+                                        1 if resume else 0, ctypes.byref(dims), cache.chunk, _stream(dev)))
+    return y, final_state
+
+
+def strict_state_update(cache: ChunkCache, x, dt_raw, dt_bias, A, B, C, D, y=None):
+    """Chunk-emulating decode step (ssd_strict_state_update). x [nseq,H,P], dt_raw
+    [nseq,H], B/C [nseq,G,N]; updates the cache in place and returns y [nseq,H,P]."""
+    dev = x.device
+    nseq, H, P = x.shape
+    G, N = B.shape[-2], B.shape[-1]
+    dt = x.dtype
+    _need(x, "x", (nseq, H, P), dt, dev)
+    _need(dt_raw, "dt_raw", (nseq, H), torch.float32, dev)
+    _need(B, "B", (nseq, G, N), dt, dev)
+    _need(C, "C", (nseq, G, N), dt, dev)
+    for name, v in (("dt_bias", dt_bias), ("A", A), ("D", D)):
+        _need(v, name, (H,), torch.float32, dev)
+    cache._check(nseq, H, P, G, N, dt, dev)
+    if y is None:
+        y = torch.empty_like(x)
+    _need(y, "y", (nseq, H, P), dt, dev)
+    dims = make_dims(nseq, H, P, G, N, _dtype_code(x), batch=nseq, seqlen=1)
+    cc = cache._c()
+    with torch.cuda.device(dev):
+        _check(_lib.ssd_strict_state_update(ctypes.byref(cc), _ptr(x), _ptr(dt_raw), _ptr(dt_bias), _ptr(A), _ptr(B),
+                                            _ptr(C), _ptr(D), _ptr(y), ctypes.byref(dims), cache.chunk,
+                                            _stream(dev)))
+    return y

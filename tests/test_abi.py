@@ -120,3 +120,24 @@ def test_bad_snapshot_interval_fails_closed(ssd, snap, dims_kw, chunk, status):
         kw["dtype_code"] = ssd.SSD_DTYPE_F32
     with pytest.raises(ssd.SSDError, match=status):
         ssd.snapshot_workspace_size(_dims(ssd, **kw), chunk, snap)
+
+
+def test_strict_entry_points_fail_closed_on_host(ssd):
+    """Strict mode rejects bad chunk lengths and missing caches before any CUDA work."""
+    d = _dims(ssd)
+    b = ctypes.c_size_t(0)
+    assert ssd._lib.ssd_strict_scan_fwd_workspace_size(ctypes.byref(d), 96, ctypes.byref(b)) == \
+        ssd.SSD_ERR_UNSUPPORTED
+    assert ssd._lib.ssd_strict_scan_fwd_workspace_size(ctypes.byref(d), 128, ctypes.byref(b)) == ssd.SSD_OK
+    assert b.value > 0
+    rc = ssd._lib.ssd_strict_scan_fwd(None, None, None, None, None, None, None, None, None, None, None, 0,
+                                      ctypes.byref(d), 128, None)
+    assert rc == ssd.SSD_ERR_INVALID_ARG and "cache" in ssd._lib.ssd_last_error().decode()
+    empty = ssd.SSDChunkCache()
+    dd = _dims(ssd, T=1, batch=1, seqlen=1)
+    rc = ssd._lib.ssd_strict_state_update(ctypes.byref(empty), None, None, None, None, None, None, None, None,
+                                          ctypes.byref(dd), 128, None)
+    assert rc == ssd.SSD_ERR_INVALID_ARG
+    rc = ssd._lib.ssd_strict_state_update(ctypes.byref(empty), None, None, None, None, None, None, None, None,
+                                          ctypes.byref(dd), 100, None)
+    assert rc == ssd.SSD_ERR_UNSUPPORTED
