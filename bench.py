@@ -518,6 +518,36 @@ def bench_ours(args, rank, world, local_rank):
                   "bytes_per_call": norm_bytes, "achieved_gbs": round(norm_bytes / norm_ms / 1e6, 1),
                   "peak_gbs": hbm, "frac": round(norm_bytes / norm_ms / 1e6 / hbm, 4)}
     del zb, nout, yz
+
+    # ---- strict mode (bitwise split-invariant CUDA-core prefill) on the same workload
+    scache = ssd.ChunkCache.empty(w.nseq, w.nheads, w.headdim, w.ngroups, w.dstate, w.chunk, w.dtype, dev)
+    ws_strict = torch.empty(ssd.strict_workspace_size(dims, w.chunk), dtype=torch.uint8, device=dev)
+
+    def strict_step():
+        ssd.strict_scan_fwd(x, dtr, inp["dt_bias"], inp["A"], Bm, Cm, inp["D"], scache, y=y, final_state=fin,
+                            workspace=ws_strict)
+
+    strict_steps = max(3, min(args.steps, 5))
+    for _ in range(2):
+        strict_step()
+    ssd.device_status()
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    ssd.profile_enable(True)
+    ev0.record(stream)
+    for _ in range(strict_steps):
+        strict_step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    sprof = ssd.profile_read()
+    ssd.profile_enable(False)
+    strict_ms = max_over_ranks(ev0.elapsed_time(ev1) / strict_steps, dev)
+    strict = {"workload": w.name, "prefill_ms_per_step": round(strict_ms, 3),
+              "prefill_tokens_per_s": world * w.total_tokens / (strict_ms / 1e3),
+              "slowdown_vs_default_path": round(strict_ms / ms_step, 2), "steps_timed": strict_steps,
+              "kernels_ms_per_launch": {k: round(v[1] / max(1, v[0]), 4) for k, v in sprof.items()
+                                        if not k.startswith("_")}}
+    del scache, ws_strict
     del host, dbuf, inp, x, dtr, Bm, Cm, y, ws, snaps, ws_snap
     torch.cuda.empty_cache()
 
@@ -539,6 +569,7 @@ def bench_ours(args, rank, world, local_rank):
         "snapshots": snapshots,
         "conv1d": conv1d,
         "gated_rmsnorm": gated_norm,
+        "strict": strict,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, threads, secs = oracle_sample(w, 16384, w.nheads)
@@ -593,13 +624,41 @@ def bench_decode(args, ssd, dev, rank, world, hbm, peak_src):
     ms = max_over_ranks(ev0.elapsed_time(ev1) / steps_timed, dev)
     sb = decode_step_bytes(nseq, H, P, G, N)
     achieved = sb / (ms / 1e3) / 1e9
+
+    # Chunk-emulating (strict) decode from the same state: whole chunk cycles, so the
+    # steps that fold a full chunk into the state are included at their share.
+    scache = ssd.ChunkCache.empty(nseq, H, P, G, N, w.chunk, w.dtype, dev)
+    scache.state.copy_(state)
+
+    def sstep():
+        i = k[0] % nstep_inputs
+        ssd.strict_state_update(scache, xs[i], dts[i], par["dt_bias"], par["A"], Bs[i], Cs[i], par["D"], y=y)
+        k[0] += 1
+
+    for _ in range(w.chunk):
+        sstep()
+    ssd.device_status()
+    barrier(dev)
+    torch.cuda.synchronize(dev)
+    s_steps = 2 * w.chunk
+    ev0.record(stream)
+    for _ in range(s_steps):
+        sstep()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    ssd.device_status()
+    s_ms = max_over_ranks(ev0.elapsed_time(ev1) / s_steps, dev)
+    strict = {"ms_per_step": round(s_ms, 4), "steps_timed": s_steps, "fold_every_steps": w.chunk,
+              "overhead_vs_plain_decode": round(s_ms / ms - 1.0, 4)}
+    del scache
     return {"workload": w.name, "steps_per_s": 1e3 / ms, "replicas": world,
             "tokens_per_s": world * nseq * 1e3 / ms, "ms_per_step": round(ms, 4),
             "steps_timed": steps_timed,
             "roofline": {"bound": "hbm", "kernel": "ssd_state_update", "achieved": round(achieved, 1),
                          "peak": hbm, "peak_source": peak_src, "unit": "GB/s",
                          "frac": round(achieved / hbm, 4), "bytes_per_launch": sb,
-                         "traffic": ncu_traffic("ssd_state_update", w.name)}}
+                         "traffic": ncu_traffic("ssd_state_update", w.name)},
+            "strict_chunk_emulating": strict}
 
 
 # ------------------------------------------------------------------------------ reference arm

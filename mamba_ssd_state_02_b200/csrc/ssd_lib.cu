@@ -49,12 +49,13 @@ ssd_status cuda_fail(cudaError_t e, const char* what) {
 // Per-kernel event timing (ssd_profile_enable / ssd_profile_read).
 enum Stage { ST_TABLE, ST_CUMSUM, ST_CHUNK_STATE, ST_STATE_PASSING, ST_CHUNK_SCAN, ST_STATE_UPDATE,
              ST_CONV, ST_CONV_UPDATE, ST_NORM, ST_STRICT_CUMSUM, ST_STRICT_STATE, ST_STRICT_PASSING,
-             ST_STRICT_SCAN, ST_STRICT_CACHE, ST_STRICT_UPDATE, ST_COUNT };
+             ST_STRICT_SCAN, ST_STRICT_CACHE, ST_STRICT_UPDATE, ST_STRICT_FOLD, ST_COUNT };
 const char* const kStageName[ST_COUNT] = {"ssd_chunk_table", "ssd_chunk_cumsum", "ssd_chunk_state",
                                           "ssd_state_passing", "ssd_chunk_scan", "ssd_state_update", "ssd_conv1d", "ssd_conv1d_update",
                                           "ssd_gated_rmsnorm", "ssd_strict_cumsum", "ssd_strict_chunk_state",
                                           "ssd_strict_state_passing", "ssd_strict_chunk_scan",
-                                          "ssd_strict_cache_fill", "ssd_strict_state_update"};
+                                          "ssd_strict_cache_fill", "ssd_strict_state_update",
+                                          "ssd_strict_fold"};
 constexpr size_t kMaxRecords = 65536;
 
 struct Profiler {
@@ -1001,8 +1002,16 @@ ssd_status launch_strict(const Plan& pl, char* ws, const T* x, const float* dt_r
     auto* states = reinterpret_cast<float*>(ws + pl.off_states);
     const int H = pl.H, G = pl.G, P = pl.P, N = pl.N, Q = pl.Q;
     const size_t scan_smem = chunk_scan_smem(P, N, Q);
-    cudaError_t e = cudaFuncSetAttribute(k_strict_chunk_scan<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)scan_smem);
+    void (*scan_kernel)(const T*, const T*, const T*, const float*, const float*, const float*, const float*,
+                        const ChunkEntry*, const int32_t*, int, int, int, int, T*) = nullptr;
+    switch (P) {
+        case 16: scan_kernel = k_strict_chunk_scan<T, 16>; break;
+        case 32: scan_kernel = k_strict_chunk_scan<T, 32>; break;
+        case 64: scan_kernel = k_strict_chunk_scan<T, 64>; break;
+        case 128: scan_kernel = k_strict_chunk_scan<T, 128>; break;
+        default: return fail(SSD_ERR_UNSUPPORTED, "headdim %d", P);
+    }
+    cudaError_t e = cudaFuncSetAttribute(scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)scan_smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(strict chunk scan)");
     int n = 0;
     {
@@ -1020,8 +1029,17 @@ ssd_status launch_strict(const Plan& pl, char* ws, const T* x, const float* dt_r
         }
         {
             StageScope sc(ST_STRICT_STATE, st);
-            k_strict_chunk_state<T><<<dim3(mc, H), kThreads, chunk_state_smem(P, N, Q), st>>>(
-                x, B, dtc, acum, table, count, H, G, P, N, Q, states);
+            const dim3 grid(mc, H);
+            const size_t sm = chunk_state_smem(P, N, Q);
+            switch (P * N / kThreads) {
+#define SSD_NOUT(V)                                                                                        \
+                case V: k_strict_chunk_state<T, V><<<grid, kThreads, sm, st>>>(x, B, dtc, acum, table, count, \
+                                                                              H, G, P, N, Q, states);        \
+                    break;
+                SSD_NOUT(1) SSD_NOUT(2) SSD_NOUT(4) SSD_NOUT(8) SSD_NOUT(16) SSD_NOUT(32) SSD_NOUT(64)
+#undef SSD_NOUT
+                default: return fail(SSD_ERR_UNSUPPORTED, "headdim*dstate");
+            }
         }
         n += 2;
     }
@@ -1033,8 +1051,8 @@ ssd_status launch_strict(const Plan& pl, char* ws, const T* x, const float* dt_r
     ++n;
     if (mc > 0) {
         StageScope sc(ST_STRICT_SCAN, st);
-        k_strict_chunk_scan<T><<<dim3(mc, H, Q / 32), kThreads, scan_smem, st>>>(
-            x, B, C, D, dtc, acum, states, table, count, H, G, P, N, Q, y);
+        scan_kernel<<<dim3(mc, G, Q / 32), kThreads, scan_smem, st>>>(x, B, C, D, dtc, acum, states, table,
+                                                                      count, H, G, N, Q, y);
         ++n;
     }
     {
@@ -1047,6 +1065,38 @@ ssd_status launch_strict(const Plan& pl, char* ws, const T* x, const float* dt_r
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch (strict scan)");
     t_launches = n;
+    return SSD_OK;
+}
+
+// Chunk-emulating decode: the step kernel, then the fold of chunks it filled.
+template <typename T>
+ssd_status launch_strict_decode(const Plan& pl, const ssd_chunk_cache& cc, const void* x, const float* dt_raw,
+                                const float* dt_bias, const float* A, const void* B, const void* C, const float* D,
+                                void* y, cudaStream_t st) {
+    using namespace strict;
+    const unsigned grid = (unsigned)(pl.nseq * pl.H);
+    const int H = pl.H, G = pl.G, P = pl.P, N = pl.N, Q = pl.Q;
+    {
+        StageScope sc(ST_STRICT_UPDATE, st);
+        k_strict_decode<T><<<grid, kDecThreads, decode_smem(N, Q), st>>>(
+            cc.state, static_cast<T*>(cc.x), static_cast<T*>(cc.B), cc.dt, cc.acum, cc.len, static_cast<const T*>(x),
+            dt_raw, dt_bias, A, static_cast<const T*>(B), static_cast<const T*>(C), D, static_cast<T*>(y), H, G, P,
+            N, Q);
+    }
+    {
+        StageScope sc(ST_STRICT_FOLD, st);
+        const size_t sm = fold_smem(P, N, Q);
+        switch (P * N / kThreads) {
+#define SSD_NOUT(V)                                                                                              \
+            case V: k_strict_fold<T, V><<<grid, kThreads, sm, st>>>(cc.state, static_cast<const T*>(cc.x),      \
+                                                                    static_cast<const T*>(cc.B), cc.dt, cc.acum, \
+                                                                    cc.len, H, G, P, N, Q);                     \
+                break;
+            SSD_NOUT(1) SSD_NOUT(2) SSD_NOUT(4) SSD_NOUT(8) SSD_NOUT(16) SSD_NOUT(32) SSD_NOUT(64)
+#undef SSD_NOUT
+            default: return fail(SSD_ERR_UNSUPPORTED, "headdim*dstate");
+        }
+    }
     return SSD_OK;
 }
 
@@ -1145,25 +1195,14 @@ extern "C" ssd_status ssd_strict_state_update(const ssd_chunk_cache* cache, cons
         return fail(SSD_ERR_INVALID_ARG, "float arrays must be 4-byte aligned");
     if ((int64_t)pl.nseq * pl.H >= INT32_MAX) return fail(SSD_ERR_UNSUPPORTED, "nseq*nheads too large");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const size_t smem = strict::decode_smem(pl.P, pl.N, pl.Q);
-    const unsigned grid = (unsigned)(pl.nseq * pl.H);
-    {
-        StageScope sc(ST_STRICT_UPDATE, st);
-        if (pl.bf16)
-            strict::k_strict_decode<__nv_bfloat16><<<grid, strict::kThreads, smem, st>>>(
-                cache->state, static_cast<__nv_bfloat16*>(cache->x), static_cast<__nv_bfloat16*>(cache->B),
-                cache->dt, cache->acum, cache->len, static_cast<const __nv_bfloat16*>(x), dt_raw, dt_bias, A,
-                static_cast<const __nv_bfloat16*>(B), static_cast<const __nv_bfloat16*>(C), D,
-                static_cast<__nv_bfloat16*>(y), pl.H, pl.G, pl.P, pl.N, pl.Q);
-        else
-            strict::k_strict_decode<float><<<grid, strict::kThreads, smem, st>>>(
-                cache->state, static_cast<float*>(cache->x), static_cast<float*>(cache->B), cache->dt, cache->acum,
-                cache->len, static_cast<const float*>(x), dt_raw, dt_bias, A, static_cast<const float*>(B),
-                static_cast<const float*>(C), D, static_cast<float*>(y), pl.H, pl.G, pl.P, pl.N, pl.Q);
-    }
+    if (pl.bf16)
+        s = launch_strict_decode<__nv_bfloat16>(pl, *cache, x, dt_raw, dt_bias, A, B, C, D, y, st);
+    else
+        s = launch_strict_decode<float>(pl, *cache, x, dt_raw, dt_bias, A, B, C, D, y, st);
+    if (s != SSD_OK) return s;
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch (strict state update)");
-    t_launches = 1;
+    t_launches = 2;
     t_last_error.clear();
     return SSD_OK;
 }

@@ -68,6 +68,24 @@ __device__ __forceinline__ bool bad_A(float a) { return !(a <= 0.f) || isinf(a);
 
 constexpr int kThreads = 256;
 
+// acc[k] += xr[k] * bv for k < NOUT (one source row of a chunk state), 16-byte shared loads.
+template <int NOUT>
+__device__ __forceinline__ void state_row(float (&acc)[NOUT], const float* xr, float bv) {
+    if constexpr (NOUT % 4 == 0) {
+#pragma unroll
+        for (int k = 0; k < NOUT; k += 4) {
+            const float4 v = *reinterpret_cast<const float4*>(xr + k);
+            acc[k] = state_step(acc[k], v.x, bv);
+            acc[k + 1] = state_step(acc[k + 1], v.y, bv);
+            acc[k + 2] = state_step(acc[k + 2], v.z, bv);
+            acc[k + 3] = state_step(acc[k + 3], v.w, bv);
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < NOUT; ++k) acc[k] = state_step(acc[k], xr[k], bv);
+    }
+}
+
 // ---------------------------------------------------------------------------------
 // Prefill stage 1: dt and Acum per (chunk, head), left to right, [chunk][H][Q] (zero past
 // the chunk's end). One thread per (chunk, head).
@@ -96,8 +114,9 @@ k_strict_cumsum(const float* __restrict__ dt_raw, const float* __restrict__ dt_b
 
 // ---------------------------------------------------------------------------------
 // Prefill stage 2: chunk states S_c[p][n] (zero-start state at the chunk's last token).
-// One block per (chunk, head); thread owns column n = tid % N and rows tid / N + k (256 / N).
-template <typename T>
+// One block per (chunk, head); thread owns column n = tid % N and the NOUT consecutive
+// rows (tid / N) * NOUT + k (NOUT = P N / 256).
+template <typename T, int NOUT>
 __global__ void __launch_bounds__(kThreads)
 k_strict_chunk_state(const T* __restrict__ x, const T* __restrict__ B, const float* __restrict__ dtc,
                      const float* __restrict__ acum, const ChunkEntry* __restrict__ table,
@@ -115,11 +134,10 @@ k_strict_chunk_state(const T* __restrict__ x, const T* __restrict__ B, const flo
     const float* dv = dtc + ((int64_t)c * H + h) * Q;
     const float last = ac[e.len - 1];
     for (int s = tid; s < e.len; s += kThreads) w[s] = src_weight(last, ac[s], dv[s]);
-    const int n = tid % N, p0 = tid / N, pstep = kThreads / N;
-    const int nout = P * N / kThreads;   // 1..64
-    float acc[64];
+    const int n = tid % N, pb = (tid / N) * NOUT;
+    float acc[NOUT];
 #pragma unroll
-    for (int k = 0; k < 64; ++k) acc[k] = 0.f;
+    for (int k = 0; k < NOUT; ++k) acc[k] = 0.f;
     __syncthreads();
     for (int s0 = 0; s0 < e.len; s0 += 32) {
         const int rows = min(32, e.len - s0);
@@ -134,18 +152,12 @@ k_strict_chunk_state(const T* __restrict__ x, const T* __restrict__ B, const flo
             bs[r * N + nn] = to_f32(B[(t * G + g) * N + nn]);
         }
         __syncthreads();
-        for (int r = 0; r < rows; ++r) {
-            const float bv = bs[r * N + n];
-#pragma unroll
-            for (int k = 0; k < 64; ++k)
-                if (k < nout) acc[k] = state_step(acc[k], xs[r * P + p0 + k * pstep], bv);
-        }
+        for (int r = 0; r < rows; ++r) state_row<NOUT>(acc, xs + r * P + pb, bs[r * N + n]);
         __syncthreads();
     }
     float* out = states + ((int64_t)c * H + h) * P * N;
 #pragma unroll
-    for (int k = 0; k < 64; ++k)
-        if (k < nout) out[(p0 + k * pstep) * N + n] = acc[k];
+    for (int k = 0; k < NOUT; ++k) out[(pb + k) * N + n] = acc[k];
 }
 
 // ---------------------------------------------------------------------------------
@@ -183,116 +195,180 @@ k_strict_passing(float* __restrict__ states, const float* __restrict__ acum, con
 }
 
 // ---------------------------------------------------------------------------------
-// Prefill stage 4: y for 32 rows of one (chunk, head). Thread owns column p = tid % P and
-// rows tid / P + k (256 / P).
-template <typename T>
+// Prefill stage 4: y for 32 rows of one chunk and every head of one group. One block per
+// (chunk, group, 32-row tile), 256 threads:
+//   1. C_t . B_s for the tile's rows and every source s <= t, once for the group
+//      (2x2 (t, s) pairs per thread, 16-byte shared loads along n);
+//   2. per head: the coefficients (C_t . B_s) w(t, s); the incoming-state term
+//      C_t . h_in[p] (TA x TB (t, p) outputs per thread, 16-byte loads along n); the
+//      sources s = 0..t left to right; D x_t; store.
+// Thread (rg, pg) owns rows rg*TA + i and columns pg + j*PG (PG = P / TB).
+template <int P> struct ScanTile;
+template <> struct ScanTile<16> { static constexpr int TA = 2, TB = 1; };
+template <> struct ScanTile<32> { static constexpr int TA = 2, TB = 2; };
+template <> struct ScanTile<64> { static constexpr int TA = 4, TB = 2; };
+template <> struct ScanTile<128> { static constexpr int TA = 4, TB = 4; };
+
+constexpr int kHPad = 36;    // row stride of the h_in slice [P][32 + 4]
+
+__host__ __device__ inline int scan_cb_region(int N, int Q) { return 32 * (Q > N + 4 ? Q : N + 4); }
+
+template <typename T, int P>
 __global__ void __launch_bounds__(kThreads)
 k_strict_chunk_scan(const T* __restrict__ x, const T* __restrict__ B, const T* __restrict__ C,
                     const float* __restrict__ D, const float* __restrict__ dtc, const float* __restrict__ acum,
                     const float* __restrict__ hin, const ChunkEntry* __restrict__ table,
-                    const int32_t* __restrict__ count, int H, int G, int P, int N, int Q, T* __restrict__ y) {
-    extern __shared__ float sm[];
-    const int NP = N + 1;
-    float* acs = sm;                      // [Q]
+                    const int32_t* __restrict__ count, int H, int G, int N, int Q, T* __restrict__ y) {
+    constexpr int TA = ScanTile<P>::TA, TB = ScanTile<P>::TB, PG = P / TB;
+    static_assert((32 / TA) * PG == kThreads, "tile covers 32 rows x P columns");
+    extern __shared__ __align__(16) float sm[];
+    const int NS = N + 4;                 // row stride of C and B tiles
+    float* cs = sm;                       // [32][N+4]   C rows of the tile
+    float* ms = cs + 32 * NS;             // [32][Q] coefficients (aliases the B slice [32][N+4])
+    float* bs = ms;
+    float* cbm = ms + scan_cb_region(N, Q);   // [32][Q]  C_t . B_s
+    float* acs = cbm + 32 * Q;            // [Q]
     float* dts = acs + Q;                 // [Q]
-    float* cs = dts + Q;                  // [32][N+1]
-    float* bs = cs + 32 * NP;             // [32][N+1]
-    float* xs = bs + 32 * NP;             // [32][P]
-    float* ms = xs + 32 * P;              // [32][33]
-    float* hs = ms + 32 * 33;             // [P][33]
+    float* hs = dts + Q;                  // [P][36]
+    float* xs = hs + P * kHPad;           // [32][P]
     const int c = blockIdx.x;
     if (c >= *count) return;
     const ChunkEntry e = table[c];
     const int t0 = blockIdx.z * 32;
     if (t0 >= e.len) return;
-    const int h = blockIdx.y, g = h / (H / G), tid = threadIdx.x;
-    const int64_t cbase = ((int64_t)c * H + h) * Q;
-    for (int i = tid; i < Q; i += kThreads) {
-        acs[i] = acum[cbase + i];
-        dts[i] = dtc[cbase + i];
-    }
+    const int g = blockIdx.y, hpg = H / G, tid = threadIdx.x;
     const int rows = min(32, e.len - t0);
     for (int i = tid; i < 32 * N; i += kThreads) {
         const int r = i / N, nn = i % N;
-        cs[r * NP + nn] = r < rows ? to_f32(C[((int64_t)(e.start + t0 + r) * G + g) * N + nn]) : 0.f;
+        cs[r * NS + nn] = r < rows ? to_f32(C[((int64_t)(e.start + t0 + r) * G + g) * N + nn]) : 0.f;
     }
-    const int p = tid % P, r0 = tid / P, tstep = kThreads / P;
-    const int nout = 32 * P / kThreads;   // 2..16
-    float acc[16];
-#pragma unroll
-    for (int k = 0; k < 16; ++k) acc[k] = 0.f;
-    __syncthreads();
 
-    // (1) C_t . h_in[p], left to right over n (in slices of 32 columns).
-    const float* hp = hin + ((int64_t)c * H + h) * P * N;
-    for (int n0 = 0; n0 < N; n0 += 32) {
-        const int cols = min(32, N - n0);
-        for (int i = tid; i < P * 32; i += kThreads) {
-            const int pp = i / 32, j = i % 32;
-            hs[pp * 33 + j] = j < cols ? hp[pp * N + n0 + j] : 0.f;
-        }
-        __syncthreads();
-        for (int j = 0; j < cols; ++j) {
-            const float hv = hs[p * 33 + j];
-#pragma unroll
-            for (int k = 0; k < 16; ++k)
-                if (k < nout) acc[k] = dot_step(acc[k], cs[(r0 + k * tstep) * NP + n0 + j], hv);
-        }
-        __syncthreads();
-    }
-#pragma unroll
-    for (int k = 0; k < 16; ++k)
-        if (k < nout) acc[k] = y_begin(acc[k], acs[min(t0 + r0 + k * tstep, Q - 1)]);
-
-    // (2) sources s = 0..t, left to right, in 32-token slices.
-    for (int s0 = 0; s0 <= t0; s0 += 32) {
-        const int srows = min(32, e.len - s0);
-        for (int i = tid; i < 32 * N; i += kThreads) {
-            const int r = i / N, nn = i % N;
-            bs[r * NP + nn] = r < srows ? to_f32(B[((int64_t)(e.start + s0 + r) * G + g) * N + nn]) : 0.f;
-        }
-        for (int i = tid; i < 32 * P; i += kThreads) {
-            const int r = i / P, pp = i % P;
-            xs[r * P + pp] = r < srows ? to_f32(x[((int64_t)(e.start + s0 + r) * H + h) * P + pp]) : 0.f;
-        }
-        __syncthreads();
-        for (int q = tid; q < 32 * 32; q += kThreads) {
-            const int tt = q >> 5, ss = q & 31;
-            const int ta = t0 + tt, sa = s0 + ss;
-            float v = 0.f;
-            if (sa <= ta && ss < srows && tt < rows) {
-                float dot = 0.f;
-                for (int nn = 0; nn < N; ++nn) dot = dot_step(dot, cs[tt * NP + nn], bs[ss * NP + nn]);
-                v = mix_coef(dot, acs[ta], acs[sa], dts[sa]);
+    // (1) C_t . B_s, left to right over n, for s <= t (source slices of 32).
+    {
+        const int ti = 2 * (tid >> 4), sj = tid & 15;     // rows ti, ti+1; sources sj, sj+16
+        for (int s0 = 0; s0 <= t0; s0 += 32) {
+            const int srows = min(32, e.len - s0);
+            __syncthreads();
+            for (int i = tid; i < 32 * N; i += kThreads) {
+                const int r = i / N, nn = i % N;
+                bs[r * NS + nn] = r < srows ? to_f32(B[((int64_t)(e.start + s0 + r) * G + g) * N + nn]) : 0.f;
             }
-            ms[tt * 33 + ss] = v;
-        }
-        __syncthreads();
+            __syncthreads();
+            float d[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+            for (int n = 0; n < N; n += 4) {
+                const float4 c0 = *reinterpret_cast<const float4*>(cs + ti * NS + n);
+                const float4 c1 = *reinterpret_cast<const float4*>(cs + (ti + 1) * NS + n);
+                const float4 b0 = *reinterpret_cast<const float4*>(bs + sj * NS + n);
+                const float4 b1 = *reinterpret_cast<const float4*>(bs + (sj + 16) * NS + n);
+                const float cv[2][4] = {{c0.x, c0.y, c0.z, c0.w}, {c1.x, c1.y, c1.z, c1.w}};
+                const float bv[2][4] = {{b0.x, b0.y, b0.z, b0.w}, {b1.x, b1.y, b1.z, b1.w}};
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            if (k >= nout) break;
-            const int tt = r0 + k * tstep;
-            const int smax = min(min(31, t0 + tt - s0), srows - 1);
-            for (int ss = 0; ss <= smax; ++ss) acc[k] = y_step(acc[k], ms[tt * 33 + ss], xs[ss * P + p]);
+                for (int k = 0; k < 4; ++k)
+#pragma unroll
+                    for (int a = 0; a < 2; ++a)
+#pragma unroll
+                        for (int b = 0; b < 2; ++b) d[a][b] = dot_step(d[a][b], cv[a][k], bv[b][k]);
+            }
+#pragma unroll
+            for (int a = 0; a < 2; ++a)
+#pragma unroll
+                for (int b = 0; b < 2; ++b) cbm[(ti + a) * Q + s0 + sj + 16 * b] = d[a][b];
         }
-        __syncthreads();
     }
-
-    // (3) D skip and store.
-    const float Dh = D[h];
+    const int rg = tid / PG, pg = tid % PG;
+    const float* hbase = hin + (int64_t)c * H * P * N;
+    for (int hh = 0; hh < hpg; ++hh) {
+        const int h = g * hpg + hh;
+        const int64_t cbase = ((int64_t)c * H + h) * Q;
+        __syncthreads();                  // previous head done with ms, xs, hs, acs
+        for (int i = tid; i < Q; i += kThreads) {
+            acs[i] = acum[cbase + i];
+            dts[i] = dtc[cbase + i];
+        }
+        __syncthreads();
+        // (2a) coefficients of the tile's rows (only s <= t, s < len are used).
+        for (int i = tid; i < 32 * (t0 + 32); i += kThreads) {
+            const int tt = i / (t0 + 32), sa = i % (t0 + 32), ta = t0 + tt;
+            if (sa <= ta && sa < e.len && tt < rows) ms[tt * Q + sa] = mix_coef(cbm[tt * Q + sa], acs[ta], acs[sa], dts[sa]);
+        }
+        // (2b) C_t . h_in[p], left to right over n, in slices of 32 columns.
+        float acc[TA][TB];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-        if (k >= nout) break;
-        const int tt = r0 + k * tstep;
-        if (tt < rows) {
-            const int64_t o = ((int64_t)(e.start + t0 + tt) * H + h) * P + p;
-            y[o] = from_f32<T>(y_end(acc[k], Dh, to_f32(x[o])));
+        for (int i = 0; i < TA; ++i)
+#pragma unroll
+            for (int j = 0; j < TB; ++j) acc[i][j] = 0.f;
+        const float* hp = hbase + (int64_t)h * P * N;
+        for (int n0 = 0; n0 < N; n0 += 32) {
+            const int cols = min(32, N - n0);
+            __syncthreads();
+            for (int i = tid; i < P * 32; i += kThreads) {
+                const int pp = i / 32, jj = i % 32;
+                hs[pp * kHPad + jj] = jj < cols ? hp[(int64_t)pp * N + n0 + jj] : 0.f;
+            }
+            __syncthreads();
+            for (int q = 0; q < cols; q += 4) {
+                float cv[TA][4], hv[TB][4];
+#pragma unroll
+                for (int i = 0; i < TA; ++i) {
+                    const float4 v = *reinterpret_cast<const float4*>(cs + (rg * TA + i) * NS + n0 + q);
+                    cv[i][0] = v.x; cv[i][1] = v.y; cv[i][2] = v.z; cv[i][3] = v.w;
+                }
+#pragma unroll
+                for (int j = 0; j < TB; ++j) {
+                    const float4 v = *reinterpret_cast<const float4*>(hs + (pg + j * PG) * kHPad + q);
+                    hv[j][0] = v.x; hv[j][1] = v.y; hv[j][2] = v.z; hv[j][3] = v.w;
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+#pragma unroll
+                    for (int i = 0; i < TA; ++i)
+#pragma unroll
+                        for (int j = 0; j < TB; ++j) acc[i][j] = dot_step(acc[i][j], cv[i][k], hv[j][k]);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < TA; ++i)
+#pragma unroll
+            for (int j = 0; j < TB; ++j) acc[i][j] = y_begin(acc[i][j], acs[t0 + rg * TA + i]);
+
+        // (2c) sources s = 0..t, left to right, in 32-token slices.
+        for (int s0 = 0; s0 <= t0; s0 += 32) {
+            const int srows = min(32, e.len - s0);
+            __syncthreads();
+            for (int i = tid; i < 32 * P; i += kThreads) {
+                const int r = i / P, pp = i % P;
+                xs[i] = r < srows ? to_f32(x[((int64_t)(e.start + s0 + r) * H + h) * P + pp]) : 0.f;
+            }
+            __syncthreads();
+#pragma unroll
+            for (int i = 0; i < TA; ++i) {
+                const int tt = rg * TA + i;
+                const int smax = min(min(31, t0 + tt - s0), srows - 1);
+                for (int ss = 0; ss <= smax; ++ss) {
+                    const float cf = ms[tt * Q + s0 + ss];
+#pragma unroll
+                    for (int j = 0; j < TB; ++j) acc[i][j] = y_step(acc[i][j], cf, xs[ss * P + pg + j * PG]);
+                }
+            }
+        }
+
+        // (2d) D skip and store.
+        const float Dh = D[h];
+#pragma unroll
+        for (int i = 0; i < TA; ++i) {
+            const int tt = rg * TA + i;
+            if (tt >= rows) continue;
+#pragma unroll
+            for (int j = 0; j < TB; ++j) {
+                const int64_t o = ((int64_t)(e.start + t0 + tt) * H + h) * P + pg + j * PG;
+                y[o] = from_f32<T>(y_end(acc[i][j], Dh, to_f32(x[o])));
+            }
         }
     }
 }
 
 inline size_t chunk_scan_smem(int P, int N, int Q) {
-    return sizeof(float) * (2 * Q + 2 * 32 * (N + 1) + 32 * P + 32 * 33 + P * 33);
+    return sizeof(float) * (32 * (N + 4) + scan_cb_region(N, Q) + 32 * Q + 2 * Q + P * kHPad + 32 * P);
 }
 inline size_t chunk_state_smem(int P, int N, int Q) { return sizeof(float) * (Q + 32 * P + 32 * N); }
 
@@ -334,25 +410,54 @@ k_strict_cache_fill(const T* __restrict__ x, const T* __restrict__ B, const floa
 
 // ---------------------------------------------------------------------------------
 // Chunk-emulating decode step. One block per (sequence, head). With j = the open chunk's
-// length, the new token is position j of the open chunk:
-//   y   = the prefill's y_t for t = j over sources 0..j (cached 0..j-1, the new token j),
-//   the new token is appended to the cache, and when j = Q-1 the full chunk is folded into
-//   the cache state with the prefill's chunk-state and passing arithmetic (length -> 0).
-// Shared memory: C_t [N], coefficients [Q], and for the fold w(last,s) x_s [32][P] and
-// B_s [32][N] slices.
+// length, the new token is position j of the open chunk: y is the prefill's y_t for t = j
+// over sources 0..j (cached 0..j-1, the new token j), and the token is appended to the
+// cache (len -> j + 1). A chunk that this fills (len == Q) is folded into the state by
+// k_strict_fold, launched right after in the same call.
+constexpr int kDecThreads = 128;
+
+// Left-to-right dot of the float row c[0..N) with the row b[0..N) of T, 16-byte loads.
 template <typename T>
-__global__ void __launch_bounds__(kThreads)
-k_strict_decode(float* __restrict__ cstate, T* __restrict__ cx, T* __restrict__ cB, float* __restrict__ cdt,
+__device__ __forceinline__ float row_dot(const float* c, const T* b, int N);
+template <>
+__device__ __forceinline__ float row_dot<__nv_bfloat16>(const float* c, const __nv_bfloat16* b, int N) {
+    float d = 0.f;
+    for (int n = 0; n < N; n += 8) {
+        const uint4 u = *reinterpret_cast<const uint4*>(b + n);
+        d = dot_step(d, c[n], __uint_as_float(u.x << 16));
+        d = dot_step(d, c[n + 1], __uint_as_float(u.x & 0xffff0000u));
+        d = dot_step(d, c[n + 2], __uint_as_float(u.y << 16));
+        d = dot_step(d, c[n + 3], __uint_as_float(u.y & 0xffff0000u));
+        d = dot_step(d, c[n + 4], __uint_as_float(u.z << 16));
+        d = dot_step(d, c[n + 5], __uint_as_float(u.z & 0xffff0000u));
+        d = dot_step(d, c[n + 6], __uint_as_float(u.w << 16));
+        d = dot_step(d, c[n + 7], __uint_as_float(u.w & 0xffff0000u));
+    }
+    return d;
+}
+template <>
+__device__ __forceinline__ float row_dot<float>(const float* c, const float* b, int N) {
+    float d = 0.f;
+    for (int n = 0; n < N; n += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(b + n);
+        d = dot_step(d, c[n], v.x);
+        d = dot_step(d, c[n + 1], v.y);
+        d = dot_step(d, c[n + 2], v.z);
+        d = dot_step(d, c[n + 3], v.w);
+    }
+    return d;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kDecThreads)
+k_strict_decode(const float* __restrict__ cstate, T* __restrict__ cx, T* __restrict__ cB, float* __restrict__ cdt,
                 float* __restrict__ cacum, int32_t* __restrict__ clen, const T* __restrict__ x,
                 const float* __restrict__ dt_raw, const float* __restrict__ dt_bias, const float* __restrict__ A,
                 const T* __restrict__ B, const T* __restrict__ C, const float* __restrict__ D, T* __restrict__ y,
                 int H, int G, int P, int N, int Q) {
     extern __shared__ float sm[];
-    float* cs = sm;                       // [N]
+    float* cs = sm;                       // [N]  C_t
     float* coef = cs + N;                 // [Q]
-    float* wv = coef + Q;                 // [Q]  w(last, s) for the fold
-    float* xs = wv + Q;                   // [32][P]
-    float* bs = xs + 32 * P;              // [32][N]
     __shared__ float s_dt, s_acum;
     const int bid = blockIdx.x;
     const int s = bid / H, h = bid % H, g = h / (H / G), tid = threadIdx.x;
@@ -374,15 +479,13 @@ k_strict_decode(float* __restrict__ cstate, T* __restrict__ cx, T* __restrict__ 
     const T* Ct = C + ((int64_t)s * G + g) * N;
     const T* xrow = cx + sh * Q * P;                       // cached x rows [Q][P]
     const T* brow = cB + ((int64_t)s * G + g) * Q * N;     // cached B rows [Q][N]
-    for (int n = tid; n < N; n += kThreads) cs[n] = to_f32(Ct[n]);
+    for (int n = tid; n < N; n += kDecThreads) cs[n] = to_f32(Ct[n]);
     __syncthreads();
     const float dtj = s_dt, acj = s_acum;
 
     // Coefficients of sources 0..j: (C_t . B_s) w(j, s).
-    for (int sidx = tid; sidx <= j; sidx += kThreads) {
-        const T* bsrc = sidx < j ? brow + (int64_t)sidx * N : Bt;
-        float dot = 0.f;
-        for (int n = 0; n < N; ++n) dot = dot_step(dot, cs[n], to_f32(bsrc[n]));
+    for (int sidx = tid; sidx <= j; sidx += kDecThreads) {
+        const float dot = row_dot<T>(cs, sidx < j ? brow + (int64_t)sidx * N : Bt, N);
         const float acs = sidx < j ? cacum[sh * Q + sidx] : acj;
         const float dts = sidx < j ? cdt[sh * Q + sidx] : dtj;
         coef[sidx] = mix_coef(dot, acj, acs, dts);
@@ -391,18 +494,20 @@ k_strict_decode(float* __restrict__ cstate, T* __restrict__ cx, T* __restrict__ 
 
     // y[p]: incoming-state term, sources left to right, D skip.
     const float* hrow = cstate + sh * P * N;
-    for (int p = tid; p < P; p += kThreads) {
-        float dot = 0.f;
-        const float* hp = hrow + (int64_t)p * N;
-        for (int n = 0; n < N; n += 4) {
-            const float4 v = *reinterpret_cast<const float4*>(hp + n);
-            dot = dot_step(dot, cs[n], v.x);
-            dot = dot_step(dot, cs[n + 1], v.y);
-            dot = dot_step(dot, cs[n + 2], v.z);
-            dot = dot_step(dot, cs[n + 3], v.w);
-        }
+    for (int p = tid; p < P; p += kDecThreads) {
+        const float dot = row_dot<float>(cs, hrow + (int64_t)p * N, N);
         float acc = y_begin(dot, acj);
-        for (int sidx = 0; sidx < j; ++sidx) acc = y_step(acc, coef[sidx], to_f32(xrow[(int64_t)sidx * P + p]));
+        const T* xp = xrow + p;
+        int sidx = 0;
+        for (; sidx + 4 <= j; sidx += 4) {
+            const float x0 = to_f32(xp[(int64_t)sidx * P]), x1 = to_f32(xp[(int64_t)(sidx + 1) * P]);
+            const float x2 = to_f32(xp[(int64_t)(sidx + 2) * P]), x3 = to_f32(xp[(int64_t)(sidx + 3) * P]);
+            acc = y_step(acc, coef[sidx], x0);
+            acc = y_step(acc, coef[sidx + 1], x1);
+            acc = y_step(acc, coef[sidx + 2], x2);
+            acc = y_step(acc, coef[sidx + 3], x3);
+        }
+        for (; sidx < j; ++sidx) acc = y_step(acc, coef[sidx], to_f32(xp[(int64_t)sidx * P]));
         const float xv = to_f32(xt[p]);
         acc = y_step(acc, coef[j], xv);
         y[sh * P + p] = from_f32<T>(y_end(acc, D[h], xv));
@@ -410,63 +515,71 @@ k_strict_decode(float* __restrict__ cstate, T* __restrict__ cx, T* __restrict__ 
 
     // Append the token to the open chunk.
     T* xdst = cx + (sh * Q + j) * P;
-    for (int p = tid; p < P; p += kThreads) xdst[p] = xt[p];
+    for (int p = tid; p < P; p += kDecThreads) xdst[p] = xt[p];
     if (h % (H / G) == 0) {
         T* bdst = cB + (((int64_t)s * G + g) * Q + j) * N;
-        for (int n = tid; n < N; n += kThreads) bdst[n] = Bt[n];
+        for (int n = tid; n < N; n += kDecThreads) bdst[n] = Bt[n];
     }
     if (tid == 0) {
         cdt[sh * Q + j] = dtj;
         cacum[sh * Q + j] = acj;
+        clen[sh] = j + 1;
     }
-    if (j + 1 < Q) {
-        if (tid == 0) clen[sh] = j + 1;
-        return;
-    }
+}
 
-    // The chunk is full: fold it into the cache state (the prefill's chunk-state and
-    // passing arithmetic, sources left to right), then empty the open chunk.
-    for (int sidx = tid; sidx < Q; sidx += kThreads) {
-        const float acs = sidx < j ? cacum[sh * Q + sidx] : acj;
-        const float dts = sidx < j ? cdt[sh * Q + sidx] : dtj;
-        wv[sidx] = src_weight(acj, acs, dts);
-    }
-    const int n = tid % N, p0 = tid / N, pstep = kThreads / N;
-    const int nout = P * N / kThreads;
-    float acc[64];
+inline size_t decode_smem(int N, int Q) { return sizeof(float) * (N + Q); }
+
+// ---------------------------------------------------------------------------------
+// Fold of a full open chunk (len == Q) into the cache state: the prefill's chunk-state
+// and passing arithmetic, sources left to right; then len -> 0. Blocks whose chunk is
+// not full return at once. One block per (sequence, head); thread owns column
+// n = tid % N and the NOUT consecutive rows (tid / N) * NOUT + k.
+template <typename T, int NOUT>
+__global__ void __launch_bounds__(kThreads)
+k_strict_fold(float* __restrict__ cstate, const T* __restrict__ cx, const T* __restrict__ cB,
+              const float* __restrict__ cdt, const float* __restrict__ cacum, int32_t* __restrict__ clen, int H,
+              int G, int P, int N, int Q) {
+    extern __shared__ float sm[];
+    float* wv = sm;                       // [Q]      w(last, s)
+    float* xs = wv + Q;                   // [32][P]  w(last, s) x_s
+    float* bs = xs + 32 * P;              // [32][N]
+    const int bid = blockIdx.x;
+    const int s = bid / H, h = bid % H, g = h / (H / G), tid = threadIdx.x;
+    const int64_t sh = (int64_t)s * H + h;
+    if (clen[sh] != Q) return;
+    const T* xrow = cx + sh * Q * P;
+    const T* brow = cB + ((int64_t)s * G + g) * Q * N;
+    const float last = cacum[sh * Q + Q - 1];
+    for (int sidx = tid; sidx < Q; sidx += kThreads)
+        wv[sidx] = src_weight(last, cacum[sh * Q + sidx], cdt[sh * Q + sidx]);
+    const int n = tid % N, pb = (tid / N) * NOUT;
+    float acc[NOUT];
 #pragma unroll
-    for (int k = 0; k < 64; ++k) acc[k] = 0.f;
+    for (int k = 0; k < NOUT; ++k) acc[k] = 0.f;
     __syncthreads();
     for (int s0 = 0; s0 < Q; s0 += 32) {
         for (int i = tid; i < 32 * P; i += kThreads) {
-            const int r = i / P, pp = i % P, sidx = s0 + r;
-            const float xv = sidx < j ? to_f32(xrow[(int64_t)sidx * P + pp]) : to_f32(xt[pp]);
-            xs[r * P + pp] = state_src(wv[sidx], xv);
+            const int r = i / P, pp = i % P;
+            xs[r * P + pp] = state_src(wv[s0 + r], to_f32(xrow[(int64_t)(s0 + r) * P + pp]));
         }
         for (int i = tid; i < 32 * N; i += kThreads) {
-            const int r = i / N, nn = i % N, sidx = s0 + r;
-            bs[r * N + nn] = sidx < j ? to_f32(brow[(int64_t)sidx * N + nn]) : to_f32(Bt[nn]);
+            const int r = i / N, nn = i % N;
+            bs[r * N + nn] = to_f32(brow[(int64_t)(s0 + r) * N + nn]);
         }
         __syncthreads();
-        for (int r = 0; r < 32; ++r) {
-            const float bv = bs[r * N + n];
-#pragma unroll
-            for (int k = 0; k < 64; ++k)
-                if (k < nout) acc[k] = state_step(acc[k], xs[r * P + p0 + k * pstep], bv);
-        }
+        for (int r = 0; r < 32; ++r) state_row<NOUT>(acc, xs + r * P + pb, bs[r * N + n]);
         __syncthreads();
     }
     float* hout = cstate + sh * P * N;
 #pragma unroll
-    for (int k = 0; k < 64; ++k)
-        if (k < nout) {
-            const int64_t o = (int64_t)(p0 + k * pstep) * N + n;
-            hout[o] = pass(hout[o], acj, acc[k]);
-        }
+    for (int k = 0; k < NOUT; ++k) {
+        const int64_t o = (int64_t)(pb + k) * N + n;
+        hout[o] = pass(hout[o], last, acc[k]);
+    }
     if (tid == 0) clen[sh] = 0;
 }
 
-inline size_t decode_smem(int P, int N, int Q) { return sizeof(float) * (N + 2 * Q + 32 * P + 32 * N); }
+inline size_t fold_smem(int P, int N, int Q) { return sizeof(float) * (Q + 32 * P + 32 * N); }
 
 }  // namespace strict
 }  // namespace ssd
