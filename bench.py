@@ -641,15 +641,20 @@ def bench_decode(args, ssd, dev, rank, world, hbm, peak_src):
     barrier(dev)
     torch.cuda.synchronize(dev)
     s_steps = 2 * w.chunk
+    ssd.profile_enable(True)
     ev0.record(stream)
     for _ in range(s_steps):
         sstep()
     ev1.record(stream)
     torch.cuda.synchronize(dev)
+    sprof = ssd.profile_read()
+    ssd.profile_enable(False)
     ssd.device_status()
     s_ms = max_over_ranks(ev0.elapsed_time(ev1) / s_steps, dev)
     strict = {"ms_per_step": round(s_ms, 4), "steps_timed": s_steps, "fold_every_steps": w.chunk,
-              "overhead_vs_plain_decode": round(s_ms / ms - 1.0, 4)}
+              "overhead_vs_plain_decode": round(s_ms / ms - 1.0, 4),
+              "kernels_ms_per_launch": {k: round(v[1] / max(1, v[0]), 4) for k, v in sprof.items()
+                                        if not k.startswith("_")}}
     del scache
     return {"workload": w.name, "steps_per_s": 1e3 / ms, "replicas": world,
             "tokens_per_s": world * nseq * 1e3 / ms, "ms_per_step": round(ms, 4),

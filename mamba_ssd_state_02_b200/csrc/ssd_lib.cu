@@ -1076,9 +1076,10 @@ ssd_status launch_strict_decode(const Plan& pl, const ssd_chunk_cache& cc, const
     using namespace strict;
     const unsigned grid = (unsigned)(pl.nseq * pl.H);
     const int H = pl.H, G = pl.G, P = pl.P, N = pl.N, Q = pl.Q;
+    const size_t dsm = decode_smem(N, Q);
     {
         StageScope sc(ST_STRICT_UPDATE, st);
-        k_strict_decode<T><<<grid, kDecThreads, decode_smem(N, Q), st>>>(
+        k_strict_decode<T><<<grid, kDecThreads, dsm, st>>>(
             cc.state, static_cast<T*>(cc.x), static_cast<T*>(cc.B), cc.dt, cc.acum, cc.len, static_cast<const T*>(x),
             dt_raw, dt_bias, A, static_cast<const T*>(B), static_cast<const T*>(C), D, static_cast<T*>(y), H, G, P,
             N, Q);

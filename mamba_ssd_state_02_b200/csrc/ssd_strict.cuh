@@ -340,14 +340,30 @@ k_strict_chunk_scan(const T* __restrict__ x, const T* __restrict__ B, const T* _
                 xs[i] = r < srows ? to_f32(x[((int64_t)(e.start + s0 + r) * H + h) * P + pp]) : 0.f;
             }
             __syncthreads();
+            if (s0 < t0) {                // every row of the tile sees all 32 sources
+                for (int ss = 0; ss < 32; ++ss) {
+                    float xv[TB];
 #pragma unroll
-            for (int i = 0; i < TA; ++i) {
-                const int tt = rg * TA + i;
-                const int smax = min(min(31, t0 + tt - s0), srows - 1);
-                for (int ss = 0; ss <= smax; ++ss) {
-                    const float cf = ms[tt * Q + s0 + ss];
+                    for (int j = 0; j < TB; ++j) xv[j] = xs[ss * P + pg + j * PG];
 #pragma unroll
-                    for (int j = 0; j < TB; ++j) acc[i][j] = y_step(acc[i][j], cf, xs[ss * P + pg + j * PG]);
+                    for (int i = 0; i < TA; ++i) {
+                        const float cf = ms[(rg * TA + i) * Q + s0 + ss];
+#pragma unroll
+                        for (int j = 0; j < TB; ++j) acc[i][j] = y_step(acc[i][j], cf, xv[j]);
+                    }
+                }
+            } else {                      // diagonal slice: sources s <= t, s < len
+                for (int ss = 0; ss < srows; ++ss) {
+                    float xv[TB];
+#pragma unroll
+                    for (int j = 0; j < TB; ++j) xv[j] = xs[ss * P + pg + j * PG];
+#pragma unroll
+                    for (int i = 0; i < TA; ++i) {
+                        if (ss > rg * TA + i) continue;
+                        const float cf = ms[(rg * TA + i) * Q + s0 + ss];
+#pragma unroll
+                        for (int j = 0; j < TB; ++j) acc[i][j] = y_step(acc[i][j], cf, xv[j]);
+                    }
                 }
             }
         }
