@@ -135,10 +135,29 @@ def decode_step_bytes(nseq, H, P, G, N, e=2) -> int:
     return 2 * nseq * H * P * N * 4 + 2 * nseq * H * P * e + 2 * nseq * G * N * e + nseq * H * 4
 
 
-def source_hash() -> str:
+# Sources that determine each kernel's code and launch (the plan, grid and segment length
+# live in ssd_lib.cu), by the stage name the library reports.
+_KERNEL_SOURCES = {
+    "tc": ["ssd_lib.cu", "ssd_common.cuh", "ssd_scan_tc.cuh", "ssd_tc_ptx.cuh", "ssd_scan_simt.cuh"],
+    "ssd_state_update": ["ssd_lib.cu", "ssd_common.cuh", "ssd_decode.cuh"],
+    "strict": ["ssd_lib.cu", "ssd_common.cuh", "ssd_scan_simt.cuh", "ssd_strict.cuh"],
+}
+
+
+def kernel_sources(kernel: str) -> list:
+    if kernel.startswith("ssd_strict"):
+        return _KERNEL_SOURCES["strict"]
+    if kernel in _KERNEL_SOURCES:
+        return _KERNEL_SOURCES[kernel]
+    return _KERNEL_SOURCES["tc"]
+
+
+def source_hash(kernel: str | None = None) -> str:
+    """Hash of the kernel's sources (all of csrc when kernel is None)."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "mamba_ssd_state_02_b200", "csrc")
-    for f in sorted(os.listdir(d)):
+    names = sorted(os.listdir(d)) if kernel is None else sorted(kernel_sources(kernel))
+    for f in names:
         with open(os.path.join(d, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -146,14 +165,14 @@ def source_hash() -> str:
 
 def ncu_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the
-    current kernel sources; else None."""
+    kernel's current sources; else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     e = d.get(workload, {}).get(kernel)
-    if not e or e.get("source_hash") != source_hash():
+    if not e or e.get("source_hash") != source_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -572,10 +591,10 @@ def bench_ours(args, rank, world, local_rank):
         "strict": strict,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, threads, secs = oracle_sample(w, 16384, w.nheads)
+        v, threads, secs = oracle_sample(w, w.total_tokens, w.nheads)
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                                "sample": f"all {w.nheads} heads of the first 16384 tokens "
-                                          f"({secs:.1f} s wall)"}
+                                "sample": f"the whole step: all {w.nheads} heads of all {w.total_tokens} tokens "
+                                          f"({secs:.1f} s wall on {threads} threads)"}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -699,7 +718,9 @@ def bench_reference(args, rank, world):
 def ncu_case(args):
     """Small fixed workloads for ncu captures (no timing, no JSON): `decode` runs
     W + K decode steps of 256 sequences on a random 512 MiB FP32 state; `prefill`
-    runs W + K prefill calls of the long-context workload."""
+    runs W + K prefill calls of the long-context workload; `strict` runs W + K strict
+    prefill calls of the long-context workload, then W + K chunk-emulating decode
+    steps of 256 sequences with half-full open chunks."""
     from mamba_ssd_state_02_b200 import build
     build.build()
     from mamba_ssd_state_02_b200 import ssd
@@ -717,6 +738,38 @@ def ncu_case(args):
         for _ in range(args.warmup + args.steps):
             ssd.state_update(state, tok["x"], tok["dt_raw"], par["dt_bias"], par["A"], tok["B"], tok["C"],
                              par["D"], y=y)
+    elif args.ncu_case == "strict":
+        # strict prefill of the long-context workload, then chunk-emulating decode steps of
+        # 256 sequences whose open chunks hold 64 tokens
+        w = W.config(PREFILL_CONFIG)
+        inp = W.make_all(w, device=dev)
+        L = w.seqlens[0]
+        r4 = lambda t: t.view(w.nseq, L, *t.shape[1:])
+        y = torch.empty_like(r4(inp["x"]))
+        cache = ssd.ChunkCache.empty(w.nseq, w.nheads, w.headdim, w.ngroups, w.dstate, w.chunk, w.dtype, dev)
+        for _ in range(args.warmup + args.steps):
+            ssd.strict_scan_fwd(r4(inp["x"]), r4(inp["dt_raw"]), inp["dt_bias"], inp["A"], r4(inp["B"]),
+                                r4(inp["C"]), inp["D"], cache, y=y)
+        del inp, y, cache
+        wd = W.config(DECODE_CONFIG)
+        nseq, H, P, G, N, Q = wd.nseq, wd.nheads, wd.headdim, wd.ngroups, wd.dstate, wd.chunk
+        par = W.make_params(wd, device=dev)
+        dc = ssd.ChunkCache.empty(nseq, H, P, G, N, Q, wd.dtype, dev)
+        dc.state.copy_((W.normal(wd.seed, W.STREAM["init_state"], nseq * H * P * N, 0, dev) * 0.1)
+                       .float().view(nseq, H, P, N))
+        open_rows = torch.arange(nseq * Q, device=dev, dtype=torch.int64)
+        tk = W.make_tokens(wd, 0, 0, rows=open_rows)
+        dc.x.copy_(tk["x"].view(nseq, Q, H, P).transpose(1, 2))
+        dc.B.copy_(tk["B"].view(nseq, Q, G, N).transpose(1, 2))
+        dc.dt.fill_(0.01)
+        dc.acum.copy_(-0.01 * torch.arange(1, Q + 1, device=dev, dtype=torch.float32).expand(nseq, H, Q))
+        dc.len.fill_(Q // 2)
+        rows = torch.arange(nseq, device=dev, dtype=torch.int64)
+        tok = W.make_tokens(wd, 0, 0, rows=rows)
+        yd = torch.empty(nseq, H, P, dtype=wd.dtype, device=dev)
+        for _ in range(args.warmup + args.steps):
+            ssd.strict_state_update(dc, tok["x"], tok["dt_raw"], par["dt_bias"], par["A"], tok["B"], tok["C"],
+                                    par["D"], y=yd)
     else:
         w = W.config(PREFILL_CONFIG)
         inp = W.make_all(w, device=dev)
@@ -738,7 +791,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ncu-case", choices=["decode", "prefill"], default=None,
+    ap.add_argument("--ncu-case", choices=["decode", "prefill", "strict"], default=None,
                     help="run a small fixed workload for an ncu capture instead of the benchmark")
     args = ap.parse_args(argv)
     if args.ncu_case:

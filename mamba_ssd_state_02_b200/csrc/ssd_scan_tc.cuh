@@ -11,18 +11,18 @@
 //       accumulated over the segment's chunks in TMEM by UMMA (A = B^T from the TMA
 //       tile, B = w*X written by the threads as a bf16 hi/lo pair, so the product
 //       keeps ~16 mantissa bits: the FP32 final state is held to 1e-3). dt =
-//       softplus(dt_raw + dt_bias) and the in-chunk cumulative sums of dt*A
-//       (ssd_chunk_cumsum) are computed in the same kernel.
+//       softplus(dt_raw + dt_bias) and the cumulative sums of dt*A (ssd_chunk_cumsum)
+//       are computed in the same kernel.
 //   ssd_state_passing (chain): per (sequence, head, state element), sequentially over
 //       the sequence's segments, h_in(seg+1) = exp(sum_seg dt*A) h_in(seg) + S_seg,
 //       starting from the initial state; the last value is the final state.
-//   ssd_chunk_scan (pass B): per (segment, 4 heads), chunk by chunk, starting from
-//       h_in(seg) held in TMEM (FP32):
-//         CB   = C B^T                                  (UMMA, once per chunk)
-//         M    = CB o exp(Acum_t - Acum_s) dt_s, s <= t (threads, bf16 to smem)
-//         Y    = M X,  Z = C h^T                        (UMMA)
-//         y_t  = Y_t + exp(Acum_t) Z_t + D x_t          (threads, bf16 to HBM)
-//         h   <- exp(Acum_end) h + B^T (w X)            (TMEM rescale + UMMA accumulate)
+//   ssd_chunk_scan (pass B): per (segment, 2 heads), chunk by chunk, starting from
+//       h_in(seg) held in the compute threads' registers (FP32):
+//         CB   = C B^T                                      (UMMA, once per chunk)
+//         M    = CB o exp(Acum_t - Acum_s) dt_s, s <= t, + D on the diagonal
+//                                                           (threads, bf16 in TMEM)
+//         Y    = M X + exp(Acum_t) C h^T                    (UMMA; scaled sum by threads)
+//         h   <- exp(Acum_end) h + B^T (w X)                (UMMA + threads)
 //
 // All exponents are <= 0 since A <= 0. TMA boxes that run past a sequence's end read
 // the next sequence's rows: their dt is forced to 0 and their y rows are not stored.
