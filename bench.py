@@ -647,7 +647,7 @@ def bench_decode(args, ssd, dev, rank, world, hbm, peak_src):
     # Chunk-emulating (strict) decode from the same state: whole chunk cycles, so the
     # steps that fold a full chunk into the state are included at their share.
     scache = ssd.ChunkCache.empty(nseq, H, P, G, N, w.chunk, w.dtype, dev)
-    scache.state.copy_(state)
+    scache.set_state(state)
 
     def sstep():
         i = k[0] % nstep_inputs
@@ -755,8 +755,8 @@ def ncu_case(args):
         nseq, H, P, G, N, Q = wd.nseq, wd.nheads, wd.headdim, wd.ngroups, wd.dstate, wd.chunk
         par = W.make_params(wd, device=dev)
         dc = ssd.ChunkCache.empty(nseq, H, P, G, N, Q, wd.dtype, dev)
-        dc.state.copy_((W.normal(wd.seed, W.STREAM["init_state"], nseq * H * P * N, 0, dev) * 0.1)
-                       .float().view(nseq, H, P, N))
+        dc.set_state((W.normal(wd.seed, W.STREAM["init_state"], nseq * H * P * N, 0, dev) * 0.1)
+                     .float().view(nseq, H, P, N))
         open_rows = torch.arange(nseq * Q, device=dev, dtype=torch.int64)
         tk = W.make_tokens(wd, 0, 0, rows=open_rows)
         dc.x.copy_(tk["x"].view(nseq, Q, H, P).transpose(1, 2))

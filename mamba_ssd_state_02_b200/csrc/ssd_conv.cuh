@@ -13,10 +13,12 @@
 //
 // HBM-bound: every input is read once and every output written once. A thread owns 8
 // consecutive channels (one 16-byte bf16 vector) over a run of tokens and keeps the
-// sliding window in registers.
+// sliding window in registers; the taps run as paired FP32 FMAs (two channels per
+// instruction) and SiLU costs one special-function operation per bf16 output.
 #pragma once
 
 #include "ssd_common.cuh"
+#include "ssd_tc_ptx.cuh"
 
 namespace ssd {
 
@@ -50,13 +52,57 @@ __device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&v)[8]) {
     *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// silu(v) = v * sigmoid(v), with the hardware base-2 exponential and reciprocal
-// (a few ulp; the outputs are rounded to the input dtype).
-__device__ __forceinline__ float silu_f32(float v) {
-    float e, r;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-v * 1.4426950408889634f));
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.f + e));
-    return v * r;
+// silu(v) = v * sigmoid(v). For float outputs: v * 1 / (1 + 2^(-v log2 e)) with the
+// hardware base-2 exponential and reciprocal (a few ulp). For bf16 outputs: sigmoid(v) =
+// (1 + tanh(v / 2)) / 2 with the hardware tanh (relative error about 2^-11, below the
+// bf16 rounding of the result), one special-function operation instead of two. The
+// prefill and decode kernels use the same operations in the same order, paired or not,
+// so a decode step and a one-token prefill give the same bits.
+__device__ __forceinline__ float conv_ex2(float v) {
+    float e;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(v));
+    return e;
+}
+__device__ __forceinline__ float conv_rcp(float v) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+    return r;
+}
+__device__ __forceinline__ float conv_tanh(float v) {
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(v));
+    return t;
+}
+constexpr float kNegLog2e = -1.4426950408889634f;
+
+template <typename T>
+__device__ __forceinline__ float silu(float v);
+template <>
+__device__ __forceinline__ float silu<float>(float v) {
+    const float e = conv_ex2(__fmul_rn(v, kNegLog2e));
+    return __fmul_rn(v, conv_rcp(__fadd_rn(e, 1.f)));
+}
+template <>
+__device__ __forceinline__ float silu<__nv_bfloat16>(float v) {
+    const float t = conv_tanh(__fmul_rn(v, 0.5f));
+    return __fmul_rn(v, __fmaf_rn(t, 0.5f, 0.5f));
+}
+// The same for a pair of channels with paired FP32 instructions.
+template <typename T>
+__device__ __forceinline__ float2 silu2(float2 v);
+template <>
+__device__ __forceinline__ float2 silu2<float>(float2 v) {
+    const float2 a = tc::fmul2(v, make_float2(kNegLog2e, kNegLog2e));
+    const float2 d = tc::ffma2(make_float2(conv_ex2(a.x), conv_ex2(a.y)), make_float2(1.f, 1.f),
+                               make_float2(1.f, 1.f));
+    return tc::fmul2(v, make_float2(conv_rcp(d.x), conv_rcp(d.y)));
+}
+template <>
+__device__ __forceinline__ float2 silu2<__nv_bfloat16>(float2 v) {
+    const float2 a = tc::fmul2(v, make_float2(0.5f, 0.5f));
+    const float2 sg = tc::ffma2(make_float2(conv_tanh(a.x), conv_tanh(a.y)), make_float2(0.5f, 0.5f),
+                                make_float2(0.5f, 0.5f));
+    return tc::fmul2(v, sg);
 }
 
 // Weights of channels c0..c0+7 of thread `tid` (w [D][K]). A lane's 8 rows are 32*K
@@ -110,6 +156,8 @@ k_conv1d_fwd(const T* __restrict__ in, const float* __restrict__ w, const float*
     load_taps<K>(w, cbase, min(kConvThreads * 8, Dc - cbase), sw, wk);
     if (c0 >= Dc || t0 >= T_) return;
     const int64_t t1 = t0 + kConvTokens < T_ ? t0 + kConvTokens : T_;
+    T* const dst = conv_dst((int64_t)0, c0, HP, GN, x, B, C);   // row 0 of this thread's output
+    const int64_t dstride = c0 < HP ? HP : GN;                   // elements per token row
     auto seq_begin = [&](int s) -> int64_t { return cu ? (int64_t)cu[s] : (int64_t)s * seqlen; };
     // Sequence of token t0: the last s with seq_begin(s) <= t0 and a non-empty range.
     int lo = 0, hi = nseq;                      // invariant: seq_begin(lo) <= t0 < seq_begin(hi)
@@ -152,13 +200,19 @@ k_conv1d_fwd(const T* __restrict__ in, const float* __restrict__ w, const float*
     auto step = [&](int64_t t, const float (&cur)[8]) {
         float o[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            float acc = bv[j] + wk[K - 1][j] * cur[j];
+        for (int i = 0; i < 4; ++i) {
+            const int j = 2 * i;
+            float2 acc = tc::ffma2(make_float2(wk[K - 1][j], wk[K - 1][j + 1]), make_float2(cur[j], cur[j + 1]),
+                                   make_float2(bv[j], bv[j + 1]));
 #pragma unroll
-            for (int k = 1; k < K; ++k) acc = fmaf(wk[K - 1 - k][j], win[k][j], acc);
-            o[j] = silu_f32(acc);
+            for (int k = 1; k < K; ++k)
+                acc = tc::ffma2(make_float2(wk[K - 1 - k][j], wk[K - 1 - k][j + 1]),
+                                make_float2(win[k][j], win[k][j + 1]), acc);
+            const float2 v = silu2<T>(acc);
+            o[j] = v.x;
+            o[j + 1] = v.y;
         }
-        store8(conv_dst(t, c0, HP, GN, x, B, C), o);
+        store8(dst + t * dstride, o);
 #pragma unroll
         for (int k = K - 1; k >= 2; --k)
 #pragma unroll
@@ -249,12 +303,12 @@ k_conv1d_update(T* __restrict__ state, const T* __restrict__ in, const float* __
     float o[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-        float acc = bv[j] + wk[K - 1][j] * cur[j];
+        float acc = __fmaf_rn(wk[K - 1][j], cur[j], bv[j]);
         // newest previous input first: the prefill kernel's order, so a decode step and
         // a one-token prefill give the same bits
 #pragma unroll
-        for (int k = K - 2; k >= 0; --k) acc = fmaf(wk[k][j], sv[j * (K - 1) + k], acc);
-        o[j] = silu_f32(acc);
+        for (int k = K - 2; k >= 0; --k) acc = __fmaf_rn(wk[k][j], sv[j * (K - 1) + k], acc);
+        o[j] = silu<T>(acc);
     }
     store8(conv_dst((int64_t)s, c0, HP, GN, x, B, C), o);
     // shift: drop the oldest input of each channel, append the new one

@@ -487,8 +487,9 @@ def gated_rmsnorm(y, z, weight, group_size=512, eps=1e-6, out=None):
 # between a chunked prefill and the chunk-emulating decode.
 class ChunkCache:
     """Per-sequence chunk cache of strict mode (``ssd_chunk_cache``): the state entering
-    each sequence's open chunk and that chunk's tokens. Tensors are owned here; the
-    library only reads and writes them."""
+    each sequence's open chunk ([nseq, H, P, N]) and that chunk's tokens (x [nseq, H, Q, P],
+    B [nseq, G, Q, N], dt and Acum [nseq, H, Q], len [nseq, H]). Tensors are owned here;
+    the library only reads and writes them."""
 
     def __init__(self, state, x, B, dt, acum, length, chunk):
         self.state, self.x, self.B, self.dt, self.acum, self.len = state, x, B, dt, acum, length
@@ -501,6 +502,15 @@ class ChunkCache:
                    torch.zeros(nseq, G, chunk, N, dtype=dtype, device=device), torch.zeros(nseq, H, chunk, **f32),
                    torch.zeros(nseq, H, chunk, **f32), torch.zeros(nseq, H, dtype=torch.int32, device=device),
                    chunk)
+
+    def state_pn(self):
+        """The cached states, [nseq, H, P, N]."""
+        return self.state
+
+    def set_state(self, states):
+        """Set the cached states from [nseq, H, P, N] (the layout of init/final states);
+        the open chunks are left as they are."""
+        self.state.copy_(states)
 
     def clone(self):
         return ChunkCache(self.state.clone(), self.x.clone(), self.B.clone(), self.dt.clone(), self.acum.clone(),

@@ -40,7 +40,7 @@ def assert_same_bits(a, b, what):
 def _cache(ssd, w, dev, init=None):
     c = ssd.ChunkCache.empty(w.nseq, w.nheads, w.headdim, w.ngroups, w.dstate, w.chunk, w.dtype, dev)
     if init is not None:
-        c.state.copy_(init)
+        c.set_state(init)
     return c
 
 
@@ -98,7 +98,7 @@ def test_strict_prefill_matches_oracle(ssd, cuda_dev, dtype, chunk, P, N):
         full = L // chunk
         ref_state.append(snaps[k + full - 1] if full > 0 else cpu["init_state"][s].double())
         k += full
-    assert rel_err(cache.state, torch.stack(ref_state)) <= TOL_STATE
+    assert rel_err(cache.state_pn(), torch.stack(ref_state)) <= TOL_STATE
     assert cache.len[:, 0].tolist() == [L % chunk for L in w.seqlens]
     assert bool((cache.len == cache.len[:, :1]).all())
 
@@ -129,7 +129,7 @@ def test_strict_decode_matches_oracle(ssd, cuda_dev, dtype):
     assert cache.len[:, 0].tolist() == [(L1 + K) % 128] * w.nseq
     _, _, snaps = O.ssd_scan(cpu["x"], cpu["dt_raw"], cpu["dt_bias"], cpu["A"], cpu["B"], cpu["C"], cpu["D"],
                              init_state=cpu["init_state"], cu_seqlens=cpu["cu_seqlens"], snapshot_tokens=128)
-    assert rel_err(cache.state, snaps.view(w.nseq, 2, *snaps.shape[1:])[:, 1]) <= TOL_STATE
+    assert rel_err(cache.state_pn(), snaps.view(w.nseq, 2, *snaps.shape[1:])[:, 1]) <= TOL_STATE
 
 
 # --------------------------------------------------------------------------------------
