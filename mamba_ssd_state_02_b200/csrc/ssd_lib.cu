@@ -194,14 +194,35 @@ ssd_status make_plan(const ssd_dims* d, int chunk, bool varlen, Plan* pl, int64_
         return varlen ? p.T / Ls + p.nseq : (int64_t)p.nseq * ((p.seqlen + Ls - 1) / Ls);
     };
     if (p.tc) {
-        // Segment length: the longest of 8192/4096/.../512/256 tokens whose chunk-scan grid
-        // (segment x 2 heads) still fills one wave of a 148-SM B200. Longer segments carry
-        // fewer inter-segment states through HBM; below one wave SMs sit idle.
         int Ls = 256;
-        for (int cand : {8192, 4096, 2048, 1024, 512}) {
-            if (segs_for(cand) * (p.H / tc::kHeadsB) >= 148) {
-                Ls = cand;
-                break;
+        if (!varlen) {
+            // Dense batch: the segment length, any multiple of 128 tokens up to 16384, that
+            // minimises the estimated time of the two tensor-core passes. Each pass runs its
+            // CTAs (segment x 2 heads for the chunk scan, segment x 4 heads for the segment
+            // states) in waves of 148; a CTA costs (chunks per segment + 2) chunk steps, the
+            // 2 standing for its prologue and epilogue; a segment-state chunk step costs
+            // about 0.76 of a chunk-scan one. Ties go to the longer segment (fewer states).
+            const int64_t nch = (p.seqlen + tc::kTile - 1) / tc::kTile;
+            const int64_t mmax = nch < 2 ? 2 : (nch < 128 ? nch : 128);
+            double best = 0.0;
+            for (int64_t m = 2; m <= mmax; ++m) {
+                const int64_t segs = (int64_t)p.nseq * ((nch + m - 1) / m);
+                const int64_t wB = (segs * (p.H / tc::kHeadsB) + 147) / 148;
+                const int64_t wA = (segs * (p.H / tc::kHeads) + 147) / 148;
+                const double cost = ((double)wB + 0.76 * (double)wA) * (double)(m + 2);
+                if (m == 2 || cost <= best) {
+                    best = cost;
+                    Ls = (int)(m * tc::kTile);
+                }
+            }
+        } else {
+            // Packed varlen (segment counts known only as an upper bound): the longest of
+            // 8192/.../512/256 tokens whose chunk-scan grid still fills one wave.
+            for (int cand : {8192, 4096, 2048, 1024, 512}) {
+                if (segs_for(cand) * (p.H / tc::kHeadsB) >= 148) {
+                    Ls = cand;
+                    break;
+                }
             }
         }
         if (const char* e = getenv("SSD_SEGMENT_TOKENS")) {

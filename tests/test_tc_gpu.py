@@ -58,7 +58,7 @@ def test_tc_short_segments(ssd, cuda_dev, seg, monkeypatch):
     _check(ssd, cuda_dev, _tc_wl([1500, 700], True, seed=43, dt_range=(1e-4, 0.5)))
 
 
-@pytest.mark.parametrize("seg", ["2048", "4096", "8192"])
+@pytest.mark.parametrize("seg", ["2048", "4096", "7296", "8192"])
 def test_tc_long_segments(ssd, cuda_dev, seg, monkeypatch):
     # Segments of 16 to 64 chunks with ragged last segments and a sequence shorter than one.
     monkeypatch.setenv("SSD_SEGMENT_TOKENS", seg)

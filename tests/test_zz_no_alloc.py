@@ -59,9 +59,9 @@ def test_noalloc_matches_scan_fwd_on_two_calls_in_a_row(ssd, cuda_dev):
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(ssd, cuda_dev):
-    # 8 x 32768 tokens, 64 heads: 32 segments of 8192 tokens, whose states alone need
-    # 64 MiB > 32 MiB.
-    d = ssd.make_dims(8 * 32768, 64, 64, 8, 128, ssd.SSD_DTYPE_BF16, batch=8, seqlen=32768)
+    # 32 x 32768 tokens, 64 heads: at least 64 segments (at most 16384 tokens each), whose
+    # states alone need at least 128 MiB > 32 MiB.
+    d = ssd.make_dims(32 * 32768, 64, 64, 8, 128, ssd.SSD_DTYPE_BF16, batch=32, seqlen=32768)
     assert ssd.workspace_size(d, 256) > 32 << 20
     p = 1 << 20                                  # never dereferenced: rejected on the host
     rc = ssd._lib.ssd_scan_fwd_noalloc(p, p, p, p, p, p, p, None, None, p, None, ctypes.byref(d), 256,
