@@ -68,6 +68,7 @@ struct Plan {
     int Ls = 0;
     int64_t max_segs = 0;
     size_t off_seg_acum = 0;
+    size_t off_order = 0;     // packed varlen: CTA order over the segments, longest first
     // state snapshots every `snap` tokens of each sequence (0: none), written to
     // snap_out; per-sequence index of the first snapshot in the workspace
     int64_t snap = 0;

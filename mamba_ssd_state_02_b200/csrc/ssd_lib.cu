@@ -258,6 +258,7 @@ ssd_status make_plan(const ssd_dims* d, int chunk, bool varlen, Plan* pl, int64_
         p.off_count = take(sizeof(int32_t));
         p.off_states = take(sizeof(float) * ms * p.H * p.P * p.N);
         p.off_seg_acum = take(sizeof(float) * ms * p.H);
+        p.off_order = take(sizeof(int32_t) * (ms > 0 ? ms : 1));
     } else {
         const size_t mc = (size_t)p.max_chunks;
         p.off_table = take(sizeof(ChunkEntry) * (mc > 0 ? mc : 1));
@@ -341,12 +342,14 @@ ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_ra
     auto* count = reinterpret_cast<int32_t*>(ws + pl.off_count);
     auto* seg_state = reinterpret_cast<float*>(ws + pl.off_states);
     auto* seg_acum = reinterpret_cast<float*>(ws + pl.off_seg_acum);
+    int32_t* order = pl.varlen ? reinterpret_cast<int32_t*>(ws + pl.off_order) : nullptr;
     const int H = pl.H, G = pl.G;
     int n = 0;
     {
         StageScope sc(ST_TABLE, st);
         k_chunk_table<<<1, kTableThreads, 0, st>>>(cu, pl.nseq, pl.T, pl.seqlen, pl.Ls, table, first, count,
-                                                   pl.snap, reinterpret_cast<int32_t*>(ws + pl.off_snap_first));
+                                                   pl.snap, reinterpret_cast<int32_t*>(ws + pl.off_snap_first),
+                                                   order);
     }
     ++n;
     if (pl.max_segs > 0 && pl.T > 0) {
@@ -366,7 +369,7 @@ ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_ra
             StageScope sc(ST_CHUNK_STATE, st);
             tc::k_tc_segment_state<<<(unsigned)(pl.max_segs * (H / tc::kHeads)), tc::kThreadsA, tc::kSmemA,
                                      st>>>(mx, mb, dt_raw, dt_bias, A, table, count, H, G,
-                                                                  seg_state, seg_acum);
+                                                                  seg_state, seg_acum, order);
         }
         ++n;
         {
@@ -379,7 +382,7 @@ ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_ra
         {
             StageScope sc(ST_CHUNK_SCAN, st);
             tc::k_tc_chunk_scan<<<(unsigned)(pl.max_segs * (H / tc::kHeadsB)), tc::kThreadsB, tc::kSmemB, st>>>(mx, mb, mc, my, dt_raw, dt_bias, A, D, table, count, H,
-                                                               G, seg_state, (__nv_bfloat16*)y);
+                                                               G, seg_state, (__nv_bfloat16*)y, order);
         }
         ++n;
     } else {

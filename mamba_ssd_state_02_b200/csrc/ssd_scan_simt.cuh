@@ -25,12 +25,16 @@ namespace ssd {
 // first chunk of sequence s (first[nseq] = number of chunks). Packed mode validates
 // cu_seqlens (cu[0] == 0, non-decreasing, cu[nseq] == T); on failure it latches
 // SSD_ERR_INVALID_ARG and emits an empty table, so later kernels touch nothing.
+// With `order` (entries of at most 128 chunks of 128 tokens), order[k] is the entry the
+// k-th CTA of a pass takes: longest entries first (by 128-token chunks), so that CTAs of
+// unequal length finish together (longest-processing-time-first scheduling).
 constexpr int kTableThreads = 1024;
 
 __global__ void __launch_bounds__(kTableThreads)
 k_chunk_table(const int32_t* __restrict__ cu, int32_t nseq, int64_t T, int64_t seqlen, int Q,
               ChunkEntry* __restrict__ table, int32_t* __restrict__ first,
-              int32_t* __restrict__ count, int64_t snap, int32_t* __restrict__ snap_first) {
+              int32_t* __restrict__ count, int64_t snap, int32_t* __restrict__ snap_first,
+              int32_t* __restrict__ order = nullptr) {
     __shared__ int32_t part[kTableThreads];
     const int tid = threadIdx.x;
     const int per = (nseq + kTableThreads - 1) / kTableThreads;
@@ -80,6 +84,26 @@ k_chunk_table(const int32_t* __restrict__ cu, int32_t nseq, int64_t T, int64_t s
     if (tid == kTableThreads - 1) {
         first[nseq] = part[tid];
         *count = part[tid];
+    }
+    if (order) {                                          // counting sort by chunks, descending
+        __shared__ int32_t hist[129];
+        __syncthreads();                                  // every entry is written
+        const int32_t n = part[kTableThreads - 1];
+        for (int b = tid; b < 129; b += kTableThreads) hist[b] = 0;
+        __syncthreads();
+        for (int32_t i = tid; i < n; i += kTableThreads) atomicAdd(&hist[min(128, (table[i].len + 127) / 128)], 1);
+        __syncthreads();
+        if (tid == 0) {
+            int32_t r = 0;
+            for (int b = 128; b >= 0; --b) {
+                const int32_t c = hist[b];
+                hist[b] = r;
+                r += c;
+            }
+        }
+        __syncthreads();
+        for (int32_t i = tid; i < n; i += kTableThreads)
+            order[atomicAdd(&hist[min(128, (table[i].len + 127) / 128)], 1)] = i;
     }
     if (snap > 0) {                                       // snapshots: floor(len / snap) per sequence
         __syncthreads();

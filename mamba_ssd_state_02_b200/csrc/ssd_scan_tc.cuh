@@ -104,10 +104,10 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
                    const float* __restrict__ dt_raw, const float* __restrict__ dt_bias,
                    const float* __restrict__ A, const ChunkEntry* __restrict__ segs,
                    const int32_t* __restrict__ nsegs, int H, int G, float* __restrict__ seg_state,
-                   float* __restrict__ seg_acum) {
+                   float* __restrict__ seg_acum, const int32_t* __restrict__ order) {
     const int nq = H / kHeads;
-    const int sg = blockIdx.x / nq;
-    if (sg >= *nsegs) return;
+    if ((int)(blockIdx.x / nq) >= *nsegs) return;
+    const int sg = order ? order[blockIdx.x / nq] : (int)(blockIdx.x / nq);   // longest segments first
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sB = sm;                       // stage st at st*32768: [2][128 s][64 n]
@@ -407,10 +407,11 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_y,
                 const float* __restrict__ dt_raw, const float* __restrict__ dt_bias, const float* __restrict__ A,
                 const float* __restrict__ D, const ChunkEntry* __restrict__ segs, const int32_t* __restrict__ nsegs,
-                int H, int G, const float* __restrict__ hin, __nv_bfloat16* __restrict__ y) {
+                int H, int G, const float* __restrict__ hin, __nv_bfloat16* __restrict__ y,
+                const int32_t* __restrict__ order) {
     const int nhp = H / kHeadsB;
-    const int sg = blockIdx.x / nhp;
-    if (sg >= *nsegs) return;
+    if ((int)(blockIdx.x / nhp) >= *nsegs) return;
+    const int sg = order ? order[blockIdx.x / nhp] : (int)(blockIdx.x / nhp);   // longest segments first
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sC = sm;                       // [2][128 t][64 n]   K-major
