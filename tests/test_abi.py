@@ -141,3 +141,24 @@ def test_strict_entry_points_fail_closed_on_host(ssd):
     rc = ssd._lib.ssd_strict_state_update(ctypes.byref(empty), None, None, None, None, None, None, None, None,
                                           ctypes.byref(dd), 100, None)
     assert rc == ssd.SSD_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("batch,seqlen,H,G,expect", [
+    (1, 65536, 64, 8, 7296),      # 9 segments of 57 chunks: 288 chunk-scan CTAs, about two full waves
+    (4, 4096, 64, 8, 2048),       # 8 segments: 256 chunk-scan CTAs, 128 segment-state CTAs
+    (256, 2048, 64, 8, 2048),     # one segment per sequence
+    (1, 2049, 8, 2, 256),         # small problem: shortest segments, every CTA in one wave
+])
+def test_dense_segment_planner(ssd, batch, seqlen, H, G, expect):
+    """The tensor-core segment length chosen for dense batches (host logic, no GPU)."""
+    d = ssd.make_dims(batch * seqlen, H, 64, G, 128, ssd.SSD_DTYPE_BF16, batch=batch, seqlen=seqlen)
+    assert ssd.scan_variant(d, 256) == "tc"
+    assert ssd.segment_tokens(d, 256) == expect
+
+
+def test_varlen_segment_planner(ssd):
+    """Packed calls: the longest power-of-two segment whose chunk-scan grid fills a wave."""
+    d = ssd.make_dims(68177, 64, 64, 8, 128, ssd.SSD_DTYPE_BF16, nseq=16)
+    assert ssd.segment_tokens(d, 128) == 8192
+    d = ssd.make_dims(3000, 64, 64, 8, 128, ssd.SSD_DTYPE_BF16, nseq=2)
+    assert ssd.segment_tokens(d, 128) == 512
