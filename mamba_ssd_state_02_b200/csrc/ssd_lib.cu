@@ -374,7 +374,7 @@ ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_ra
         ++n;
         {
             StageScope sc(ST_STATE_PASSING, st);
-            tc::k_tc_segment_passing<<<dim3(pl.nseq, H, (tc::kP * tc::kN) / 256), 256, 0, st>>>(
+            tc::k_tc_segment_passing<<<dim3(pl.nseq, H, tc::kN / tc::kPassN), 256, 0, st>>>(
                 seg_state, seg_acum, first, init, fin, H, table, pl.snap,
                 reinterpret_cast<const int32_t*>(ws + pl.off_snap_first), pl.snap_out);
         }
@@ -387,7 +387,7 @@ ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_ra
         ++n;
     } else {
         StageScope sc(ST_STATE_PASSING, st);
-        tc::k_tc_segment_passing<<<dim3(pl.nseq, H, (tc::kP * tc::kN) / 256), 256, 0, st>>>(
+        tc::k_tc_segment_passing<<<dim3(pl.nseq, H, tc::kN / tc::kPassN), 256, 0, st>>>(
             seg_state, seg_acum, first, init, fin, H, table, pl.snap,
                 reinterpret_cast<const int32_t*>(ws + pl.off_snap_first), pl.snap_out);
         ++n;

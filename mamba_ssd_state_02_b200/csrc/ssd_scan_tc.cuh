@@ -323,46 +323,93 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
 }
 
 // ---------------------------------------------------------------------------------
-// Chain over segments. Element e = n*P + p of head h; seg_state slots are replaced
-// by the state entering each segment (h_in, layout [seg][H][N][P]); final_state and
-// init use the API layout [nseq][H][P][N].
+// Chain over segments. seg_state slots are replaced by the state entering each segment
+// (h_in, layout [seg][H][N][P]); init, final_state and the snapshots use the API layout
+// [nseq][H][P][N]. A CTA owns kPassN = 8 state rows (n) x all P columns of one (sequence,
+// head); thread t walks elements t and t + 256 of that tile ([N][P] order, coalesced)
+// down the segments, four segments' loads in flight. API-layout reads and writes go
+// through a shared-memory transpose, so a warp touches 32-byte sectors it uses whole.
+constexpr int kPassN = 8;
+
 __global__ void __launch_bounds__(256)
 k_tc_segment_passing(float* __restrict__ seg_state, const float* __restrict__ seg_acum,
                      const int32_t* __restrict__ first, const float* __restrict__ init,
                      float* __restrict__ final_state, int H, const ChunkEntry* __restrict__ segs,
                      int64_t snap, const int32_t* __restrict__ snap_first, float* __restrict__ snap_out) {
-    const int s = blockIdx.x, h = blockIdx.y;
-    const int e = blockIdx.z * 256 + threadIdx.x;
-    if (e >= kP * kN) return;
-    const int n = e / kP, p = e % kP;
-    const int64_t api = (((int64_t)s * H + h) * kP + p) * kN + n;
-    float hv = init ? init[api] : 0.f;
+    constexpr int E = kP * kPassN / 256;                   // elements per thread (2)
+    __shared__ float tile[kP][kPassN + 1];
+    const int s = blockIdx.x, h = blockIdx.y, n0 = blockIdx.z * kPassN, tid = threadIdx.x;
+    const int64_t api0 = ((int64_t)s * H + h) * kP * kN + n0;   // (p, n0 + nn) at api0 + p*kN + nn
+    // element i of thread tid: idx = tid + 256 i, n = n0 + idx / kP, p = idx % kP
+    auto api_load = [&](const float* src, float (&v)[E]) {
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+            const int idx = tid + 256 * i, p = idx / kPassN, nn = idx % kPassN;
+            tile[p][nn] = src[(int64_t)p * kN + nn];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+            const int idx = tid + 256 * i;
+            v[i] = tile[idx % kP][idx / kP];
+        }
+    };
+    auto api_store = [&](float* dst, const float (&v)[E]) {
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+            const int idx = tid + 256 * i;
+            tile[idx % kP][idx / kP] = v[i];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+            const int idx = tid + 256 * i, p = idx / kPassN, nn = idx % kPassN;
+            dst[(int64_t)p * kN + nn] = tile[p][nn];
+        }
+    };
+    float hv[E];
+    if (init) {
+        api_load(init + api0, hv);
+    } else {
+#pragma unroll
+        for (int i = 0; i < E; ++i) hv[i] = 0.f;
+    }
     const int c0 = first[s], c1 = first[s + 1];
     const int64_t seq0 = c1 > c0 ? segs[c0].start : 0;
+    const int64_t eoff = (int64_t)n0 * kP + tid;
     constexpr int U = 4;
     for (int c = c0; c < c1; c += U) {
-        float sv[U], dec[U];
+        float sv[U][E], dec[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             if (c + u < c1) {
-                sv[u] = seg_state[((int64_t)(c + u) * H + h) * (kP * kN) + e];
+                const float* slot = seg_state + ((int64_t)(c + u) * H + h) * (kP * kN) + eoff;
+#pragma unroll
+                for (int i = 0; i < E; ++i) sv[u][i] = slot[256 * i];
                 dec[u] = expf(seg_acum[(int64_t)(c + u) * H + h]);
             }
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             if (c + u < c1) {
-                seg_state[((int64_t)(c + u) * H + h) * (kP * kN) + e] = hv;
-                hv = fmaf(dec[u], hv, sv[u]);
+                float* slot = seg_state + ((int64_t)(c + u) * H + h) * (kP * kN) + eoff;
+#pragma unroll
+                for (int i = 0; i < E; ++i) {
+                    slot[256 * i] = hv[i];
+                    hv[i] = fmaf(dec[u], hv[i], sv[u][i]);
+                }
                 if (snap > 0) {                           // state after a multiple of snap tokens
                     const int64_t end = (int64_t)segs[c + u].start + segs[c + u].len - seq0;
                     if (end % snap == 0)
-                        snap_out[(((int64_t)(snap_first[s] + end / snap - 1) * H + h) * kP + p) * kN + n] = hv;
+                        api_store(snap_out + ((int64_t)(snap_first[s] + end / snap - 1) * H + h) * kP * kN + n0,
+                                  hv);
                 }
             }
         }
     }
-    if (final_state) final_state[api] = hv;
+    if (final_state) api_store(final_state + api0, hv);
 }
 
 // ---------------------------------------------------------------------------------
