@@ -141,12 +141,18 @@ _KERNEL_SOURCES = {
     "tc": ["ssd_lib.cu", "ssd_common.cuh", "ssd_scan_tc.cuh", "ssd_tc_ptx.cuh", "ssd_scan_simt.cuh"],
     "ssd_state_update": ["ssd_lib.cu", "ssd_common.cuh", "ssd_decode.cuh"],
     "strict": ["ssd_lib.cu", "ssd_common.cuh", "ssd_scan_simt.cuh", "ssd_strict.cuh"],
+    "conv": ["ssd_lib.cu", "ssd_common.cuh", "ssd_tc_ptx.cuh", "ssd_conv.cuh"],
+    "norm": ["ssd_lib.cu", "ssd_common.cuh", "ssd_norm.cuh"],
 }
 
 
 def kernel_sources(kernel: str) -> list:
     if kernel.startswith("ssd_strict"):
         return _KERNEL_SOURCES["strict"]
+    if kernel.startswith("ssd_conv1d"):
+        return _KERNEL_SOURCES["conv"]
+    if kernel == "ssd_gated_rmsnorm":
+        return _KERNEL_SOURCES["norm"]
     if kernel in _KERNEL_SOURCES:
         return _KERNEL_SOURCES[kernel]
     return _KERNEL_SOURCES["tc"]
@@ -512,6 +518,7 @@ def bench_ours(args, rank, world, local_rank):
     conv1d = {"workload": f"conv1d_width{K}_{w.total_tokens}tok_D{Dc}", "ms_per_call": round(conv_ms, 4),
               "bytes_per_call": conv_bytes, "achieved_gbs": round(conv_bytes / conv_ms / 1e6, 1),
               "peak_gbs": hbm, "frac": round(conv_bytes / conv_ms / 1e6 / hbm, 4),
+              "traffic": ncu_traffic("ssd_conv1d", w.name),
               "decode_256seq_us_per_step": round(conv_upd_us, 2)}
     del ci, cx, cst_out, cxo, cbo, cco
 
@@ -720,7 +727,8 @@ def ncu_case(args):
     W + K decode steps of 256 sequences on a random 512 MiB FP32 state; `prefill`
     runs W + K prefill calls of the long-context workload; `strict` runs W + K strict
     prefill calls of the long-context workload, then W + K chunk-emulating decode
-    steps of 256 sequences with half-full open chunks."""
+    steps of 256 sequences with half-full open chunks; `conv` runs W + K conv1d prologue
+    calls over the long-context workload's tokens."""
     from mamba_ssd_state_02_b200 import build
     build.build()
     from mamba_ssd_state_02_b200 import ssd
@@ -738,6 +746,21 @@ def ncu_case(args):
         for _ in range(args.warmup + args.steps):
             ssd.state_update(state, tok["x"], tok["dt_raw"], par["dt_bias"], par["A"], tok["B"], tok["C"],
                              par["D"], y=y)
+    elif args.ncu_case == "conv":
+        # conv1d prologue (width 4) over the long-context workload's tokens
+        w = W.config(PREFILL_CONFIG)
+        K = 4
+        ci = W.make_conv_inputs(w, K, init=True, device=dev)
+        L = w.seqlens[0]
+        Dc = W.conv_channels(w)
+        cx = ci["xbc"].view(w.nseq, L, Dc)
+        xo = torch.empty(w.nseq, L, w.nheads, w.headdim, dtype=w.dtype, device=dev)
+        bo = torch.empty(w.nseq, L, w.ngroups, w.dstate, dtype=w.dtype, device=dev)
+        co = torch.empty_like(bo)
+        so = torch.empty_like(ci["conv_state"])
+        for _ in range(args.warmup + args.steps):
+            ssd.conv1d_fwd(cx, ci["weight"], ci["bias"], w.nheads, w.headdim, w.ngroups, w.dstate,
+                           conv_state=ci["conv_state"], x=xo, B=bo, C=co, conv_state_out=so)
     elif args.ncu_case == "strict":
         # strict prefill of the long-context workload, then chunk-emulating decode steps of
         # 256 sequences whose open chunks hold 64 tokens
@@ -791,7 +814,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ncu-case", choices=["decode", "prefill", "strict"], default=None,
+    ap.add_argument("--ncu-case", choices=["decode", "prefill", "strict", "conv"], default=None,
                     help="run a small fixed workload for an ncu capture instead of the benchmark")
     args = ap.parse_args(argv)
     if args.ncu_case:
