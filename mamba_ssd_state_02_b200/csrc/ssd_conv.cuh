@@ -132,6 +132,25 @@ __device__ __forceinline__ void load_taps(const float* __restrict__ w, int cbase
         for (int k = 0; k < K; ++k) wk[k][j] = r[j * K + k];
 }
 
+// Token ring of the prefill kernel. Once the taps are in registers, the tap staging
+// buffer holds, per thread, the next R token vectors of its 8 channels (slot k of thread
+// tid at element (k * kConvThreads + tid) * 8), filled by 16-byte asynchronous copies
+// (cp.async), so R tokens per thread are in flight without holding registers. R is the
+// largest power of two (at most 8) whose slots fit the thread's tap row.
+template <typename T, int K>
+constexpr int conv_ring() {
+    constexpr int cap = kTapRow(K) * 4 / (8 * (int)sizeof(T));
+    return cap >= 8 ? 8 : (cap >= 4 ? 4 : (cap >= 2 ? 2 : 1));
+}
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 // Destination of channel vector c0 (8 channels) of one token row: x, B or C.
 template <typename T>
 __device__ __forceinline__ T* conv_dst(int64_t row, int c0, int HP, int GN, T* x, T* B, T* C) {
@@ -143,7 +162,7 @@ __device__ __forceinline__ T* conv_dst(int64_t row, int c0, int HP, int GN, T* x
 // Prefill: block (token tile of kConvTokens, channel tile). seq_begin(s) gives packed
 // token offsets (cu_seqlens, or s * seqlen for a dense batch).
 template <typename T, int K>
-__global__ void __launch_bounds__(kConvThreads)
+__global__ void __launch_bounds__(kConvThreads, 3)
 k_conv1d_fwd(const T* __restrict__ in, const float* __restrict__ w, const float* __restrict__ bias,
              const T* __restrict__ st_in, const int32_t* __restrict__ cu, int32_t nseq, int64_t T_,
              int64_t seqlen, int Dc, int HP, int GN, T* __restrict__ x, T* __restrict__ B,
@@ -154,6 +173,7 @@ k_conv1d_fwd(const T* __restrict__ in, const float* __restrict__ w, const float*
     const int64_t t0 = (int64_t)blockIdx.x * kConvTokens;
     float wk[K][8];
     load_taps<K>(w, cbase, min(kConvThreads * 8, Dc - cbase), sw, wk);
+    __syncthreads();                             // taps are in registers: sw becomes the token ring
     if (c0 >= Dc || t0 >= T_) return;
     const int64_t t1 = t0 + kConvTokens < T_ ? t0 + kConvTokens : T_;
     T* const dst = conv_dst((int64_t)0, c0, HP, GN, x, B, C);   // row 0 of this thread's output
@@ -227,23 +247,34 @@ k_conv1d_fwd(const T* __restrict__ in, const float* __restrict__ w, const float*
                     st_out[((int64_t)s * Dc + c0 + j) * (K - 1) + (K - 1 - k)] = from_f32<T>(win[k][j]);
         }
     };
-    constexpr int U = 4;                         // tokens loaded ahead of their use
-    for (int64_t t = t0; t < t1; t += U) {
-        float cur[U][8];
+    constexpr int R = conv_ring<T, K>();
+    T* const ring = reinterpret_cast<T*>(sw);
+    auto slot = [&](int k) { return ring + ((int64_t)k * kConvThreads + threadIdx.x) * 8; };
+    auto issue = [&](int64_t t, int k) {         // token t's 8 channels into slot k
+        const char* src = reinterpret_cast<const char*>(in + t * Dc + c0);
+        char* d = reinterpret_cast<char*>(slot(k));
 #pragma unroll
-        for (int u = 0; u < U; ++u)
-            if (t + u < t1) load8(in + (t + u) * Dc + c0, cur[u]);
+        for (int q = 0; q < (int)(8 * sizeof(T) / 16); ++q) cp_async16(d + 16 * q, src + 16 * q);
+    };
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            if (t + u >= t1) break;
-            while (t + u >= se) {                // next sequence (skipping empty ones)
-                ++s;
-                sb = seq_begin(s);
-                se = seq_begin(s + 1);
-                load_state(s);
-            }
-            step(t + u, cur[u]);
+    for (int k = 0; k < R; ++k) {                // one commit group per token, in token order
+        if (t0 + k < t1) issue(t0 + k, k);
+        cp_async_commit();
+    }
+    for (int64_t t = t0; t < t1; ++t) {
+        const int k = (int)(t - t0) & (R - 1);
+        cp_async_wait<R - 1>();                  // token t's group (the oldest pending) is done
+        float cur[8];
+        load8(slot(k), cur);
+        while (t >= se) {                        // next sequence (skipping empty ones)
+            ++s;
+            sb = seq_begin(s);
+            se = seq_begin(s + 1);
+            load_state(s);
         }
+        step(t, cur);                            // consumes slot k before it is refilled
+        if (t + R < t1) issue(t + R, k);
+        cp_async_commit();
     }
 }
 
