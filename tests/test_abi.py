@@ -162,3 +162,21 @@ def test_varlen_segment_planner(ssd):
     assert ssd.segment_tokens(d, 128) == 8192
     d = ssd.make_dims(3000, 64, 64, 8, 128, ssd.SSD_DTYPE_BF16, nseq=2)
     assert ssd.segment_tokens(d, 128) == 512
+
+
+def test_strict_binding_checks_before_the_library(ssd):
+    """The strict-mode binding validates cache shapes and devices on the host (no GPU)."""
+    import torch
+    c = ssd.ChunkCache.empty(2, 8, 64, 2, 128, 128, torch.bfloat16, "cpu")
+    assert tuple(c.state.shape) == (2, 8, 64, 128) and tuple(c.B.shape) == (2, 2, 128, 128)
+    assert c.state_pn() is c.state
+    x = torch.zeros(2, 8, 64, dtype=torch.bfloat16)
+    dt = torch.zeros(2, 8)
+    B = torch.zeros(2, 2, 128, dtype=torch.bfloat16)
+    h = torch.zeros(8)
+    with pytest.raises(ValueError, match="must be on"):
+        ssd.strict_state_update(c, x, dt, h, h, B, B, h)
+    bad = ssd.ChunkCache.empty(2, 8, 64, 2, 128, 64, torch.bfloat16, "cpu")
+    bad.len = torch.zeros(3, 8, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        bad._check(2, 8, 64, 2, 128, torch.bfloat16, torch.device("cpu"))
