@@ -266,3 +266,32 @@ def test_strict_is_within_tolerance_of_fast_path(ssd, cuda_dev):
     ssd.device_status()
     assert rel_err(ys, yf) <= 1e-2
     assert rel_err(fs, ff) <= 1e-3
+
+
+# --------------------------------------------------------------------------------------
+# Full size: the long-context workload (1 x 65536 tokens, 64 heads, chunk 256) in strict
+# mode against the oracle on one head of every group; its cache ends on a chunk boundary.
+GROUP_HEADS = [0, 9, 18, 27, 36, 45, 54, 63]
+
+
+@pytest.mark.slow
+def test_strict_long_context_full_size(ssd, cuda_dev):
+    w = W.config(2)
+    inp = W.make_all(w, device=cuda_dev)
+    L = w.seqlens[0]
+    r4 = lambda t: t.view(w.nseq, L, *t.shape[1:])
+    cache = _cache(ssd, w, cuda_dev, inp["init_state"])
+    y, fin = ssd.strict_scan_fwd(r4(inp["x"]), r4(inp["dt_raw"]), inp["dt_bias"], inp["A"], r4(inp["B"]),
+                                 r4(inp["C"]), inp["D"], cache, resume=inp["init_state"] is not None)
+    ssd.device_status()
+    pairs = [(0, h) for h in GROUP_HEADS]
+    cpu = {k: (None if v is None else v.cpu()) for k, v in inp.items()}
+    blocks, fin_ref = O.ssd_scan(cpu["x"], cpu["dt_raw"], cpu["dt_bias"], cpu["A"], cpu["B"], cpu["C"], cpu["D"],
+                                 init_state=cpu["init_state"], batch=1, pairs=pairs)
+    yc = y.view(L, w.nheads, w.headdim)
+    got = torch.stack([yc[:, h, :] for _, h in pairs])
+    ref = torch.stack([torch.from_numpy(b) for b in blocks])
+    assert rel_err(got, ref) <= TOL_Y[w.dtype]
+    assert rel_err(torch.stack([fin[0, h] for _, h in pairs]), fin_ref) <= TOL_STATE
+    assert int(cache.len.max()) == 0                      # 65536 is a multiple of the chunk
+    assert_same_bits(cache.state, fin, "cache state = final state on a chunk boundary")
