@@ -144,24 +144,38 @@ def test_strict_entry_points_fail_closed_on_host(ssd):
 
 
 @pytest.mark.parametrize("batch,seqlen,H,G,expect", [
-    (1, 65536, 64, 8, 7296),      # 9 segments of 57 chunks: 288 chunk-scan CTAs, about two full waves
-    (4, 4096, 64, 8, 2048),       # 8 segments: 256 chunk-scan CTAs, 128 segment-state CTAs
+    (1, 65536, 64, 8, 2048),      # 32 segments x 48 items: over six items per SM, L2-sized segments
+    (4, 4096, 64, 8, 512),        # 2048 would give 8 segments (384 items, under six per SM)
     (256, 2048, 64, 8, 2048),     # one segment per sequence
-    (1, 2049, 8, 2, 256),         # small problem: shortest segments, every CTA in one wave
+    (1, 2049, 8, 2, 256),         # small problem: shortest segments
 ])
 def test_dense_segment_planner(ssd, batch, seqlen, H, G, expect):
-    """The tensor-core segment length chosen for dense batches (host logic, no GPU)."""
+    """The tensor-core segment length chosen for dense batches (host logic, no GPU; 148 SMs
+    assumed when no device answers)."""
     d = ssd.make_dims(batch * seqlen, H, 64, G, 128, ssd.SSD_DTYPE_BF16, batch=batch, seqlen=seqlen)
     assert ssd.scan_variant(d, 256) == "tc"
     assert ssd.segment_tokens(d, 256) == expect
 
 
 def test_varlen_segment_planner(ssd):
-    """Packed calls: the longest power-of-two segment whose chunk-scan grid fills a wave."""
+    """Packed calls: the same rule on the upper bound of the segment count."""
     d = ssd.make_dims(68177, 64, 64, 8, 128, ssd.SSD_DTYPE_BF16, nseq=16)
-    assert ssd.segment_tokens(d, 128) == 8192
+    assert ssd.segment_tokens(d, 128) == 2048
     d = ssd.make_dims(3000, 64, 64, 8, 128, ssd.SSD_DTYPE_BF16, nseq=2)
-    assert ssd.segment_tokens(d, 128) == 512
+    assert ssd.segment_tokens(d, 128) == 256
+
+
+def test_segment_override(ssd):
+    """ssd_set_segment_tokens forces the segment length and 0 restores the planner."""
+    d = ssd.make_dims(65536, 64, 64, 8, 128, ssd.SSD_DTYPE_BF16, batch=1, seqlen=65536)
+    try:
+        ssd.set_segment_tokens(384)
+        assert ssd.segment_tokens(d, 256) == 384
+        ssd.set_segment_tokens(100)        # not a multiple of 128: planner again
+        assert ssd.segment_tokens(d, 256) == 2048
+    finally:
+        ssd.set_segment_tokens(0)
+    assert ssd.segment_tokens(d, 256) == 2048
 
 
 def test_strict_binding_checks_before_the_library(ssd):

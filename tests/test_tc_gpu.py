@@ -52,16 +52,23 @@ def test_tc_varlen_ragged(ssd, cuda_dev, seqlens):
     _check(ssd, cuda_dev, _tc_wl(seqlens, True))
 
 
-@pytest.mark.parametrize("seg", ["128", "256", "384"])
-def test_tc_short_segments(ssd, cuda_dev, seg, monkeypatch):
-    monkeypatch.setenv("SSD_SEGMENT_TOKENS", seg)
+@pytest.fixture
+def segment_tokens(ssd):
+    """Force the tensor-core segment length for one test, then restore the planner."""
+    yield ssd.set_segment_tokens
+    ssd.set_segment_tokens(0)
+
+
+@pytest.mark.parametrize("seg", [128, 256, 384])
+def test_tc_short_segments(ssd, cuda_dev, seg, segment_tokens):
+    segment_tokens(seg)
     _check(ssd, cuda_dev, _tc_wl([1500, 700], True, seed=43, dt_range=(1e-4, 0.5)))
 
 
-@pytest.mark.parametrize("seg", ["2048", "4096", "7296", "8192"])
-def test_tc_long_segments(ssd, cuda_dev, seg, monkeypatch):
+@pytest.mark.parametrize("seg", [2048, 4096, 7296, 8192])
+def test_tc_long_segments(ssd, cuda_dev, seg, segment_tokens):
     # Segments of 16 to 64 chunks with ragged last segments and a sequence shorter than one.
-    monkeypatch.setenv("SSD_SEGMENT_TOKENS", seg)
+    segment_tokens(seg)
     _check(ssd, cuda_dev, _tc_wl([9000, 4500, 130], True, seed=46, dt_range=(1e-4, 0.5)))
 
 
@@ -71,3 +78,33 @@ def test_tc_dense_heads_per_group_16(ssd, cuda_dev):
 
 def test_tc_zero_init_wide_dt(ssd, cuda_dev):
     _check(ssd, cuda_dev, _tc_wl([2049], False, init="zero", seed=45, dt_range=(1e-4, 0.5)))
+
+
+@pytest.mark.parametrize("seqlens,H,G,seg", [
+    ([3000, 2000, 1], 8, 2, 128),      # 41 segments x 6 items: every CTA runs several items
+    ([1024, 1000], 64, 8, 128),        # 16 segments x 48 items, both item kinds back to back
+    ([4096] * 4, 64, 8, 512),          # the batched workload's shape and planner choice
+])
+def test_tc_many_items_per_cta(ssd, cuda_dev, seqlens, H, G, seg, segment_tokens):
+    """More work items than CTAs: each persistent CTA runs state and scan items in turn,
+    reusing its barriers, shared memory and TMEM between them."""
+    segment_tokens(seg)
+    _check(ssd, cuda_dev, _tc_wl(seqlens, len(set(seqlens)) > 1, H=H, G=G, seed=48))
+
+
+def test_flag_wait_timeout_fails_closed(ssd, cuda_dev, segment_tokens):
+    """Segment states that are never published: every wait for one runs out after a short
+    bound, the call reports SSD_ERR_TIMEOUT through ssd_get_device_status (no hang, no
+    fault), and the next call, with the defaults restored, is correct again."""
+    w = _tc_wl([3000, 2000], True, seed=49)
+    segment_tokens(256)
+    inp = W.make_all(w)
+    try:
+        ssd.test_flag_waits(200_000, publish=False)        # about 0.1 ms per wait
+        run_gpu_scan(ssd, w, inp, cuda_dev)
+        with pytest.raises(ssd.SSDError, match="TIMEOUT"):
+            ssd.device_status()
+    finally:
+        ssd.test_flag_waits(0, publish=True)
+    ssd.device_status()                                    # the error word was cleared
+    _check(ssd, cuda_dev, w)
