@@ -224,9 +224,8 @@ ssd_status ssd_gated_rmsnorm(const void* y, const void* z, const float* weight, 
  *     device current); make that first call before any stream capture.
  *   - All calls share the one array and it keeps the last call's contents: calls whose
  *     work can overlap on the GPU (different streams, or different host threads on one
- *     device) race on it and must be serialised by the caller. The call clears what
- *     must start at zero (the tensor-core pipeline's ticket counter and flags) itself;
- *     every other slot a kernel reads is written earlier in the same call.
+ *     device) race on it and must be serialised by the caller. Nothing in it needs
+ *     clearing between calls: every slot a kernel reads is written earlier in the call.
  */
 ssd_status ssd_scan_fwd_noalloc(const void* x, const float* dt_raw, const float* dt_bias, const float* A,
                                 const void* B, const void* C, const float* D, const float* init_state,
@@ -335,30 +334,11 @@ int ssd_scan_fwd_segment_tokens(const ssd_dims* dims, int chunk);
  * Tuning and testing knob (process-wide): force the tensor-core pipeline's segment
  * length to `tokens` (a multiple of 128, at most 2^20) for every later call; 0 or any
  * other value restores the planner's choice. Results do not depend on it beyond
- * rounding; the workspace size does (query it after setting).
+ * rounding; the workspace size does (query it after setting). Snapshot calls still
+ * shorten the segment to a divisor of the snapshot interval.
  */
 void ssd_set_segment_tokens(int tokens);
 
-/*
- * Tuning knob (process-wide): how far, in blocks of work items, the tensor-core
- * prefill's chunk-scan items trail the segment-state items they depend on (1..64;
- * any other value restores the default, 2). Results do not depend on it.
- */
-void ssd_set_ticket_lag(int blocks);
-
-/*
- * Test hook for the fail-closed path (RL-Kernel issue page, §4.1 and §7: fail closed).
- * The tensor-core prefill passes segment states between CTAs through flags, and every
- * wait for a flag is bounded. This sets, on the current device and for later calls,
- * the bound in SM cycles (0 or less: the default, about 2 s) and whether flags are
- * published at all (publish = 0: never, so every wait for one runs out). A wait that
- * runs out latches SSD_ERR_TIMEOUT (read with ssd_get_device_status); its CTA finishes
- * its current work item on the data it has, leaving no copy or MMA in flight, and all
- * CTAs then stop taking items, so the call ends with y and the final state undefined.
- * Call ssd_test_flag_waits(0, 1) to restore the defaults. Returns SSD_ERR_CUDA if the
- * device settings cannot be written.
- */
-ssd_status ssd_test_flag_waits(int64_t budget_cycles, int publish);
 
 /* Number of kernels the last successful call on this host thread enqueued. */
 int ssd_last_launch_count(void);

@@ -67,8 +67,8 @@ struct Plan {
     bool tc = false;
     int Ls = 0;
     int64_t max_segs = 0;
-    size_t off_flags = 0;     // per (segment, 4 heads): the segment's end state is published
-    size_t off_sched = 0;     // ticket counter and abort word of the persistent kernel
+    size_t off_seg_acum = 0;
+    size_t off_order = 0;     // packed varlen: CTA order over the segments, longest first
     // state snapshots every `snap` tokens of each sequence (0: none), written to
     // snap_out; per-sequence index of the first snapshot in the workspace
     int64_t snap = 0;

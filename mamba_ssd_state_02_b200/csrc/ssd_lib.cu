@@ -50,15 +50,13 @@ ssd_status cuda_fail(cudaError_t e, const char* what) {
 // Per-kernel event timing (ssd_profile_enable / ssd_profile_read).
 enum Stage { ST_TABLE, ST_CUMSUM, ST_CHUNK_STATE, ST_STATE_PASSING, ST_CHUNK_SCAN, ST_STATE_UPDATE,
              ST_CONV, ST_CONV_UPDATE, ST_NORM, ST_STRICT_CUMSUM, ST_STRICT_STATE, ST_STRICT_PASSING,
-             ST_STRICT_SCAN, ST_STRICT_CACHE, ST_STRICT_UPDATE, ST_STRICT_FOLD, ST_PREPARE, ST_PREFILL,
-             ST_EMPTY_FINAL, ST_COUNT };
+             ST_STRICT_SCAN, ST_STRICT_CACHE, ST_STRICT_UPDATE, ST_STRICT_FOLD, ST_COUNT };
 const char* const kStageName[ST_COUNT] = {"ssd_chunk_table", "ssd_chunk_cumsum", "ssd_chunk_state",
                                           "ssd_state_passing", "ssd_chunk_scan", "ssd_state_update", "ssd_conv1d", "ssd_conv1d_update",
                                           "ssd_gated_rmsnorm", "ssd_strict_cumsum", "ssd_strict_chunk_state",
                                           "ssd_strict_state_passing", "ssd_strict_chunk_scan",
                                           "ssd_strict_cache_fill", "ssd_strict_state_update",
-                                          "ssd_strict_fold", "ssd_prefill_prepare", "ssd_prefill_fused",
-                                          "ssd_empty_final"};
+                                          "ssd_strict_fold"};
 constexpr size_t kMaxRecords = 65536;
 
 struct Profiler {
@@ -153,10 +151,8 @@ int sm_count() {
     return n;
 }
 
-// Segment length forced by ssd_set_segment_tokens (0: the planner chooses), and the lag
-// (in ticket blocks) of the persistent kernel's scan items behind its state items.
+// Segment length forced by ssd_set_segment_tokens (0: the planner chooses).
 std::atomic<int> g_segment_override{0};
-std::atomic<int> g_ticket_lag{2};
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -213,17 +209,37 @@ ssd_status make_plan(const ssd_dims* d, int chunk, bool varlen, Plan* pl, int64_
         return varlen ? p.T / Ls + p.nseq : (int64_t)p.nseq * ((p.seqlen + Ls - 1) / Ls);
     };
     if (p.tc) {
-        // Segment length: the longest of 2048/1024/512/256 tokens that gives the persistent
-        // kernel at least six items per SM (items = segments x (H/4 state + H/2 scan)), so
-        // the CTAs stay busy to the end; 2048 at most, so that the x and B tiles of the few
-        // segments in flight stay in L2 between their state and scan items.
-        const int nsm = sm_count();
-        const int64_t per_seg = p.H / tc::kHeads + p.H / tc::kHeadsB;
         int Ls = 256;
-        for (int cand : {2048, 1024, 512, 256}) {
-            if (segs_for(cand) * per_seg >= 6 * (int64_t)nsm) {
-                Ls = cand;
-                break;
+        if (!varlen) {
+            // Dense batch: the segment length, any multiple of 128 tokens up to 16384, that
+            // minimises the estimated time of the two tensor-core passes. Each pass runs its
+            // CTAs (segment x 2 heads for the chunk scan, segment x 4 heads for the segment
+            // states) in waves of one CTA per SM; a CTA costs (chunks per segment + 2) chunk
+            // steps, the 2 standing for its prologue and epilogue; a segment-state chunk step
+            // costs about 0.76 of a chunk-scan one. Ties go to the longer segment (fewer states).
+            const int64_t nsm = sm_count();
+            const int64_t nch = (p.seqlen + tc::kTile - 1) / tc::kTile;
+            const int64_t mmax = nch < 2 ? 2 : (nch < 128 ? nch : 128);
+            double best = 0.0;
+            for (int64_t m = 2; m <= mmax; ++m) {
+                const int64_t segs = (int64_t)p.nseq * ((nch + m - 1) / m);
+                const int64_t wB = (segs * (p.H / tc::kHeadsB) + nsm - 1) / nsm;
+                const int64_t wA = (segs * (p.H / tc::kHeads) + nsm - 1) / nsm;
+                const double cost = ((double)wB + 0.76 * (double)wA) * (double)(m + 2);
+                if (m == 2 || cost <= best) {
+                    best = cost;
+                    Ls = (int)(m * tc::kTile);
+                }
+            }
+        } else {
+            // Packed varlen (segment counts known only as an upper bound): the longest of
+            // 8192/.../512/256 tokens whose chunk-scan grid still fills one wave.
+            const int64_t nsm = sm_count();
+            for (int cand : {8192, 4096, 2048, 1024, 512}) {
+                if (segs_for(cand) * (p.H / tc::kHeadsB) >= nsm) {
+                    Ls = cand;
+                    break;
+                }
             }
         }
         if (const int v = g_segment_override.load()) Ls = v;
@@ -255,8 +271,8 @@ ssd_status make_plan(const ssd_dims* d, int chunk, bool varlen, Plan* pl, int64_
         p.off_first = take(sizeof(int32_t) * ((size_t)p.nseq + 1));
         p.off_count = take(sizeof(int32_t));
         p.off_states = take(sizeof(float) * ms * p.H * p.P * p.N);
-        p.off_flags = take(sizeof(int32_t) * (ms > 0 ? ms : 1) * (p.H / tc::kHeads));
-        p.off_sched = take(sizeof(tc::TcSched));
+        p.off_seg_acum = take(sizeof(float) * ms * p.H);
+        p.off_order = take(sizeof(int32_t) * (ms > 0 ? ms : 1));
     } else {
         const size_t mc = (size_t)p.max_chunks;
         p.off_table = take(sizeof(ChunkEntry) * (mc > 0 ? mc : 1));
@@ -331,31 +347,23 @@ ssd_status launch_simt(const Plan& pl, char* ws, const T* x, const float* dt_raw
 }
 
 // ---------------------------------------------------------------------------------
-// Tensor-core pipeline launch (bf16, P = 64, N = 128): the segment table, the zeroed
-// scheduling words, then one persistent kernel (one CTA per SM).
+// Tensor-core pipeline launch (bf16, P = 64, N = 128).
 ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_raw, const float* dt_bias,
                      const float* A, const void* B, const void* C, const float* D, const float* init,
                      const int32_t* cu, void* y, float* fin, cudaStream_t st) {
     auto* table = reinterpret_cast<ChunkEntry*>(ws + pl.off_table);
     auto* first = reinterpret_cast<int32_t*>(ws + pl.off_first);
     auto* count = reinterpret_cast<int32_t*>(ws + pl.off_count);
-    auto* hout = reinterpret_cast<float*>(ws + pl.off_states);
-    auto* flags = reinterpret_cast<int32_t*>(ws + pl.off_flags);
-    auto* sched = reinterpret_cast<tc::TcSched*>(ws + pl.off_sched);
-    auto* snap_first = reinterpret_cast<int32_t*>(ws + pl.off_snap_first);
+    auto* seg_state = reinterpret_cast<float*>(ws + pl.off_states);
+    auto* seg_acum = reinterpret_cast<float*>(ws + pl.off_seg_acum);
+    int32_t* order = pl.varlen ? reinterpret_cast<int32_t*>(ws + pl.off_order) : nullptr;
     const int H = pl.H, G = pl.G;
     int n = 0;
     {
         StageScope sc(ST_TABLE, st);
         k_chunk_table<<<1, kTableThreads, 0, st>>>(cu, pl.nseq, pl.T, pl.seqlen, pl.Ls, table, first, count,
-                                                   pl.snap, snap_first);
-    }
-    ++n;
-    const int64_t nflags = (pl.max_segs > 0 ? pl.max_segs : 1) * (H / tc::kHeads);
-    {
-        StageScope sc(ST_PREPARE, st);
-        tc::k_tc_prepare<<<(unsigned)std::min<int64_t>(64, (nflags + 255) / 256), 256, 0, st>>>(sched, flags,
-                                                                                               nflags);
+                                                   pl.snap, reinterpret_cast<int32_t*>(ws + pl.off_snap_first),
+                                                   order);
     }
     ++n;
     if (pl.max_segs > 0 && pl.T > 0) {
@@ -366,44 +374,36 @@ ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_ra
             !make_map3(&mc, C, tc::kN, G, T, (uint64_t)tc::kN * 2, (uint64_t)G * tc::kN * 2, 64, 1, tc::kTile) ||
             !make_map3(&my, y, tc::kP, H, T, (uint64_t)tc::kP * 2, (uint64_t)H * tc::kP * 2, 64, 1, tc::kTile))
             return fail(SSD_ERR_CUDA, "cuTensorMapEncodeTiled failed (x/B/C/y tensor maps)");
-        cudaError_t e = cudaFuncSetAttribute(tc::k_tc_prefill, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             tc::kSmem);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(k_tc_prefill)");
-        tc::TcArgs a{};
-        a.dt_raw = dt_raw;
-        a.dt_bias = dt_bias;
-        a.A = A;
-        a.D = D;
-        a.segs = table;
-        a.nsegs = count;
-        a.first = first;
-        a.init = init;
-        a.hout = hout;
-        a.final_state = fin;
-        a.y = reinterpret_cast<__nv_bfloat16*>(y);
-        a.snap = pl.snap;
-        a.snap_first = snap_first;
-        a.snap_out = pl.snap_out;
-        a.flags = flags;
-        a.sched = sched;
-        a.nseq = pl.nseq;
-        a.H = H;
-        a.G = G;
-        a.lag = g_ticket_lag.load();
-        const int64_t tickets = (pl.max_segs + a.lag) * (H / tc::kHeads + H / tc::kHeadsB);
-        const unsigned grid = (unsigned)std::min<int64_t>(sm_count(), tickets);
+        cudaError_t e = cudaFuncSetAttribute(tc::k_tc_segment_state, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             tc::kSmemA);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(tc::k_tc_chunk_scan, cudaFuncAttributeMaxDynamicSharedMemorySize, tc::kSmemB);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(tc kernels)");
         {
-            StageScope sc(ST_PREFILL, st);
-            tc::k_tc_prefill<<<grid, tc::kThreads, tc::kSmem, st>>>(mx, mb, mc, my, a);
+            StageScope sc(ST_CHUNK_STATE, st);
+            tc::k_tc_segment_state<<<(unsigned)(pl.max_segs * (H / tc::kHeads)), tc::kThreadsA, tc::kSmemA,
+                                     st>>>(mx, mb, dt_raw, dt_bias, A, table, count, H, G,
+                                                                  seg_state, seg_acum, order);
         }
         ++n;
-    }
-    // Sequences without tokens (packed calls, or seqlen 0): the final state is the
-    // initial state, or zero.
-    if (fin && (pl.varlen || pl.seqlen == 0)) {
-        StageScope sc(ST_EMPTY_FINAL, st);
-        tc::k_tc_empty_final<<<(unsigned)std::min<int64_t>(pl.nseq, 1024), 256, 0, st>>>(first, init, fin, pl.nseq,
-                                                                                       (int64_t)H * tc::kP * tc::kN);
+        {
+            StageScope sc(ST_STATE_PASSING, st);
+            tc::k_tc_segment_passing<<<dim3(pl.nseq, H, tc::kN / tc::kPassN), 256, 0, st>>>(
+                seg_state, seg_acum, first, init, fin, H, table, pl.snap,
+                reinterpret_cast<const int32_t*>(ws + pl.off_snap_first), pl.snap_out);
+        }
+        ++n;
+        {
+            StageScope sc(ST_CHUNK_SCAN, st);
+            tc::k_tc_chunk_scan<<<(unsigned)(pl.max_segs * (H / tc::kHeadsB)), tc::kThreadsB, tc::kSmemB, st>>>(mx, mb, mc, my, dt_raw, dt_bias, A, D, table, count, H,
+                                                               G, seg_state, (__nv_bfloat16*)y, order);
+        }
+        ++n;
+    } else {
+        StageScope sc(ST_STATE_PASSING, st);
+        tc::k_tc_segment_passing<<<dim3(pl.nseq, H, tc::kN / tc::kPassN), 256, 0, st>>>(
+            seg_state, seg_acum, first, init, fin, H, table, pl.snap,
+                reinterpret_cast<const int32_t*>(ws + pl.off_snap_first), pl.snap_out);
         ++n;
     }
     cudaError_t e = cudaGetLastError();
@@ -671,18 +671,6 @@ const char* ssd_scan_fwd_variant(const ssd_dims* dims, int chunk) {
 
 int ssd_last_launch_count(void) { return t_launches; }
 
-ssd_status ssd_test_flag_waits(int64_t budget_cycles, int publish) {
-    const long long b = budget_cycles > 0 ? (long long)budget_cycles : tc::kWaitBudgetCycles;
-    const int pub = publish ? 1 : 0;
-    cudaError_t e = cudaMemcpyToSymbol(tc::g_flag_wait_budget, &b, sizeof b);
-    if (e == cudaSuccess) e = cudaMemcpyToSymbol(tc::g_flag_publish, &pub, sizeof pub);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyToSymbol(flag wait settings)");
-    t_last_error.clear();
-    return SSD_OK;
-}
-
-void ssd_set_ticket_lag(int blocks) { g_ticket_lag.store(blocks >= 1 && blocks <= 64 ? blocks : 2); }
-
 void ssd_set_segment_tokens(int tokens) {
     g_segment_override.store(tokens >= tc::kTile && tokens % tc::kTile == 0 && tokens <= (1 << 20) ? tokens : 0);
 }
@@ -827,9 +815,7 @@ extern "C" ssd_status ssd_scan_fwd_noalloc(const void* x, const float* dt_raw, c
     if (s != SSD_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     // Every slot of the scratch that a kernel reads is written earlier in the same call
-    // (chunk/segment table, then states); the words that must start at zero (the
-    // tensor-core pipeline's ticket counter and per-segment flags) are cleared by a
-    // kernel of the call itself.
+    // (chunk/segment table, then states), so nothing needs clearing between calls.
     if (pl.tc)
         s = launch_tc(pl, ws, x, dt_raw, dt_bias, A, B, C, D, init_state, cu_seqlens, y, final_state, st);
     else if (pl.bf16)

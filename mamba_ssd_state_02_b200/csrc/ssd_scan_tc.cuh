@@ -1,35 +1,28 @@
 // Chunked SSD prefill on the sm_100a tensor cores (bf16 x/B/C, headdim 64, dstate 128,
-// heads per B/C group a multiple of 4), as one persistent kernel.
+// heads per B/C group a multiple of 4).
 //
 // The chunked SSD algorithm (JAX Nemotron 3 Nano page, "Key Components" 1; RL-Kernel
 // issue page, Figure 2) runs here as a two-level scan. Every sequence is cut into
 // segments of Ls tokens (a multiple of the 128-token MMA tile), anchored at the
-// sequence start, and every segment into 128-token chunks. Two kinds of work item share
-// one launch; each CTA takes items in ticket order from a counter in the workspace:
+// sequence start, and every segment into 128-token chunks:
 //
-//   state item (ssd_chunk_state + ssd_state_passing), per (segment i, 4 heads): the
-//       segment's zero-start state
-//         S_i = sum_{s in seg} exp(Acum_end - Acum_s) dt_s x_s B_s^T
+//   ssd_chunk_state (pass A): per (segment, 4 heads) the segment's zero-start state
+//       S_seg = sum_{s in seg} exp(Acum_end - Acum_s) dt_s x_s B_s^T,
 //       accumulated over the segment's chunks in TMEM by UMMA (A = B^T from the TMA
-//       tile, B = w*X written by the threads as a bf16 hi/lo pair, so the product keeps
-//       ~16 mantissa bits and the FP32 state meets 1e-3), then one link of the chain
-//         h_out(i) = exp(sum_seg dt*A) h_out(i-1) + S_i     (h_out(-1) = initial state)
-//       written for the next segment (or as the final state and snapshots), and a flag.
-//       dt = softplus(dt_raw + dt_bias) and the cumulative sums of dt*A
-//       (ssd_chunk_cumsum) are computed in the item.
-//   scan item (ssd_chunk_scan), per (segment i, 2 heads): waits for the flag of the
-//       state item of segment i-1 and, chunk by chunk, from h_out(i-1) held in the
-//       compute threads' registers (FP32):
+//       tile, B = w*X written by the threads as a bf16 hi/lo pair, so the product
+//       keeps ~16 mantissa bits: the FP32 final state is held to 1e-3). dt =
+//       softplus(dt_raw + dt_bias) and the cumulative sums of dt*A (ssd_chunk_cumsum)
+//       are computed in the same kernel.
+//   ssd_state_passing (chain): per (sequence, head, state element), sequentially over
+//       the sequence's segments, h_in(seg+1) = exp(sum_seg dt*A) h_in(seg) + S_seg,
+//       starting from the initial state; the last value is the final state.
+//   ssd_chunk_scan (pass B): per (segment, 2 heads), chunk by chunk, starting from
+//       h_in(seg) held in the compute threads' registers (FP32):
 //         CB   = C B^T                                      (UMMA, once per chunk)
 //         M    = CB o exp(Acum_t - Acum_s) dt_s, s <= t, + D on the diagonal
 //                                                           (threads, bf16 in TMEM)
 //         Y    = M X + exp(Acum_t) C h^T                    (UMMA; scaled sum by threads)
 //         h   <- exp(Acum_end) h + B^T (w X)                (UMMA + threads)
-//
-// Tickets run in blocks: block b holds the state items of segment b, then the scan items
-// of segment b - lag (lag >= 1), so a scan item starts well after the state item of the
-// previous segment that it waits for. An item only waits for items with smaller tickets,
-// which are running or done, so the waits always end.
 //
 // All exponents are <= 0 since A <= 0. TMA boxes that run past a sequence's end read
 // the next sequence's rows: their dt is forced to 0 and their y rows are not stored.
@@ -43,41 +36,19 @@ namespace tc {
 constexpr int kTile = 128;       // tokens per MMA tile (chunk)
 constexpr int kP = 64;           // headdim
 constexpr int kN = 128;          // dstate
-constexpr int kHeads = 4;        // heads per state item (a quad)
-constexpr int kHeadsB = 2;       // heads per scan item (a pair)
+constexpr int kHeads = 4;        // heads per CTA
 constexpr float kLog2e = 1.4426950408889634f;
 
+// ---------------------------------------------------------------------------------
+// Shared by both passes.
 constexpr int kRoleWarps = 2;                    // warp 0: TMA producer, warp 1: UMMA issuer
 constexpr int kComputeWarps = 16;                // four compute warpgroups (cw = 0..3)
-constexpr int kScanWarp = kRoleWarps + kComputeWarps;   // warps 18 (both items) and 19 (state items)
-constexpr int kWarps = kScanWarp + 2;
-constexpr int kThreads = 32 * kWarps;
-constexpr int kSmem = 208 * 1024 + 1024;        // dynamic shared memory (1 KB for alignment)
-constexpr int kFirstCompute = 32 * kRoleWarps;  // thread index of the first compute thread
-
-// Scheduling words of one call, zeroed by k_tc_prepare.
-struct TcSched {
-    int32_t ticket;    // next ticket
-    int32_t abort;     // set when a wait ran out: every CTA stops taking items
-    int32_t pad[2];
-};
+constexpr int kThreadsTc = 32 * (kRoleWarps + kComputeWarps);
 
 __device__ __forceinline__ void compute_bar() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
 
-__device__ __forceinline__ int ld_acquire(const int32_t* p) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void st_release(int32_t* p, int v) {
-    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// Wait on an mbarrier of this CTA's own pipeline (bounded). Its phases complete through
-// this CTA's threads, TMA copies and UMMAs only, so a wait that runs out means the
-// pipeline is broken: the error is latched and the CTA's abort flag makes every later
-// wait return at once, so all roles reach the end of the item.
+// Wait with a shared abort flag: once any wait has timed out, every later wait
+// returns at once, so all roles run to the end without blocking each other.
 __device__ __forceinline__ void wait_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
     if (mbar_try_wait(bar, parity)) return;
     const long long t0 = clock64();
@@ -91,132 +62,95 @@ __device__ __forceinline__ void wait_abort(uint64_t* bar, uint32_t parity, volat
     }
 }
 
-// Cycles a wait for another CTA's flag may take before it gives up, and whether state
-// items publish their flags: device globals so that a test of the timeout path can
-// shorten the wait and suppress publication (kWaitBudgetCycles and 1 by default).
-__device__ long long g_flag_wait_budget = kWaitBudgetCycles;
-__device__ int g_flag_publish = 1;
-
-// Wait until another CTA has published `flag` (bounded). On expiry (or once the call
-// has been aborted) the error is latched, the call's abort word is set and false is
-// returned; the caller then runs its item to the end on the data it has, so no copy
-// or UMMA of this CTA is left in flight, and takes no further tickets.
-__device__ __forceinline__ bool wait_flag(const int32_t* flag, TcSched* sched) {
-    if (ld_acquire(flag)) return true;
-    const long long t0 = clock64();
-    const long long budget = *reinterpret_cast<volatile long long*>(&g_flag_wait_budget);
-    while (!ld_acquire(flag)) {
-        if (*reinterpret_cast<volatile int32_t*>(&sched->abort) || clock64() - t0 > budget) {
-            latch_error(SSD_ERR_TIMEOUT);
-            atomicExch(&sched->abort, 1);
-            return false;
-        }
-        __nanosleep(200);
+// Inclusive scan of `a` over the 128 rows of one compute warpgroup (rows r = 32*q +
+// lane); `part` holds the four per-warp totals of that warpgroup. Two compute_bar()s.
+__device__ __forceinline__ float wg_scan(float a, int q, int lane, float* part) {
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float v = __shfl_up_sync(0xffffffffu, a, off);
+        if (lane >= off) a += v;
     }
-    return true;
-}
-
-// Wait for `flag` with every thread of the 16 compute warps: one lane polls, the
-// others wait at the compute warps' named barrier.
-__device__ __forceinline__ void compute_wait_flag(const int32_t* flag, TcSched* sched) {
-    if (threadIdx.x / 32 == kRoleWarps) {
-        if ((threadIdx.x & 31) == 0) wait_flag(flag, sched);
-        __syncwarp();
-    }
+    if (lane == 31) part[q] = a;
     compute_bar();
+    float pre = 0.f;
+    for (int w = 0; w < q; ++w) pre += part[w];
+    return a + pre;
 }
-
-// Everything one launch needs, passed once.
-struct TcArgs {
-    const float* dt_raw;
-    const float* dt_bias;
-    const float* A;
-    const float* D;
-    const ChunkEntry* segs;
-    const int32_t* nsegs;
-    const int32_t* first;      // per sequence: index of its first segment (nseq + 1 entries)
-    const float* init;         // [nseq][H][P][N] or null (zeros)
-    float* hout;               // [seg][H][P][N]: state at the end of each segment
-    float* final_state;        // [nseq][H][P][N] or null
-    __nv_bfloat16* y;
-    int64_t snap;              // snapshot interval in tokens (0: none)
-    const int32_t* snap_first;
-    float* snap_out;           // [n_snap][H][P][N]
-    int32_t* flags;            // [seg][H / 4]: hout of (segment, quad) published
-    TcSched* sched;
-    int nseq;
-    int H, G;
-    int lag;                   // scan items of segment i sit in ticket block i + lag (>= 1)
-};
-
-// Shared memory of the items. Dynamic: 208 KB of operand tiles (layout per item below);
-// static: the per-chunk scalars of the dt scans and the mbarriers.
-struct ItemShared {
-    float f[4096];             // state item: w[4][4][128]; scan item: ac2, dts, uw, ww [4][2][128]
-    float segsum[kHeads];      // state item: log2 of the segment's total decay per head
-    uint64_t bar[24];
-    int abort_flag;
-    int ticket;
-};
 
 // ---------------------------------------------------------------------------------
-// State item: segment i, heads h0 .. h0 + 3 (quad q).
+// Pass A: zero-start segment states S_seg (fp32, layout [seg][H][N][P]) and the
+// segment's total sum of dt*A (seg_acum[seg][H]). One CTA per (segment, 4 heads); the
+// chunks run from the segment end backwards so the decay to the end is a running sum.
 //
-// Warp 0 issues the TMA loads, warp 1 the UMMAs, warps 18 and 19 scan dt of heads 0-1
-// and 2-3 (up to four chunks ahead; w_s = exp(sum_{r > s in seg} dt_r A) dt_s), and
+// Warp 0 issues the TMA loads, warp 1 the UMMAs, warps 18 and 19 scan dt of heads
+// 0-1 and 2-3 (up to four chunks ahead; w_s = exp(sum_{r > s in seg} dt_r A) dt_s), and
 // the 16 compute warps write w*X as a bf16 hi/lo pair (hi in place over x, lo next to
-// it). The chunks run from the segment end backwards so the decay to the end is a
-// running sum. Heads go in pairs: per pair one batch of 8 UMMAs with N = 256 ([hi|hi|lo|
-// lo] of the two heads side by side, B^T read once) accumulates S_hi and S_lo of the
-// two heads in TMEM; while it runs the compute warps prepare the other pair. Compute
-// thread (cw, r) owns token row r and column quarter cw of every head's w*X; at the end
-// it owns state row n = r of head cw.
+// it), so the product keeps ~16 mantissa bits: the FP32 final state is held to 1e-3.
+// Heads go in pairs: per pair one batch of 8 UMMAs with N = 256 ([hi|hi|lo|lo] of the
+// two heads side by side, B^T read once) accumulates S_hi and S_lo of the two heads in
+// TMEM; while it runs the compute warps prepare the other pair. At the end S = S_hi +
+// S_lo. Compute thread (cw, r) owns token row r and column quarter cw of every head's
+// w*X.
 //
 // Shared memory: two B stages; per head pair [x/hi h0 | x/hi h1 | lo h0 | lo h1] (the
 // pair's X is reloaded as soon as its UMMAs are done). TMEM: per pair p, columns 256p
 // + [S_hi h0 | S_hi h1 | S_lo h0 | S_lo h1] (64 each).
-__device__ __forceinline__ void item_state(const CUtensorMap* map_x, const CUtensorMap* map_b, const TcArgs& a,
-                                           int i, int q, uint8_t* sm, ItemShared& sh, uint32_t tS) {
-    const int H = a.H;
+constexpr int kSmemA = 192 * 1024 + 1024;
+constexpr int kScanWarpA = kRoleWarps + kComputeWarps;         // warps 18, 19: dt scan
+constexpr int kThreadsA = 32 * (kScanWarpA + 2);
+
+__global__ void __launch_bounds__(kThreadsA, 1)
+k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
+                   const float* __restrict__ dt_raw, const float* __restrict__ dt_bias,
+                   const float* __restrict__ A, const ChunkEntry* __restrict__ segs,
+                   const int32_t* __restrict__ nsegs, int H, int G, float* __restrict__ seg_state,
+                   float* __restrict__ seg_acum, const int32_t* __restrict__ order) {
+    const int nq = H / kHeads;
+    if ((int)(blockIdx.x / nq) >= *nsegs) return;
+    const int sg = order ? order[blockIdx.x / nq] : (int)(blockIdx.x / nq);   // longest segments first
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sB = sm;                       // stage st at st*32768: [2][128 s][64 n]
     uint8_t* sP = sm + 65536;               // pair p at p*65536: x/hi of its heads, then lo; [128 s][64 p] each
     auto xs = [&](int hh) { return sP + (hh >> 1) * 65536 + (hh & 1) * 16384; };           // x, then hi
     auto los = [&](int hh) { return sP + (hh >> 1) * 65536 + 32768 + (hh & 1) * 16384; };  // lo
-    float (*wts)[kHeads][kTile] = reinterpret_cast<float (*)[kHeads][kTile]>(sh.f);
-    uint64_t* full_b = &sh.bar[0];          // [2]
-    uint64_t* empty_b = &sh.bar[2];         // [2]
-    uint64_t* full_x = &sh.bar[4];          // [2]
-    uint64_t* pair_done = &sh.bar[6];       // [2]
-    uint64_t* ops_ready = &sh.bar[8];       // [2]
-    uint64_t* w_ready = &sh.bar[10];        // [4]
-    uint64_t* w_free = &sh.bar[14];         // [4]
-    uint64_t* all_done = &sh.bar[18];
-    uint64_t* sum_ready = &sh.bar[19];
+    __shared__ __align__(16) float wts[4][kHeads][kTile];
+    __shared__ uint64_t full_b[2], empty_b[2], full_x[2], pair_done[2], ops_ready[2], w_ready[4], w_free[4], all_done;
+    __shared__ uint32_t tmem_slot;
+    __shared__ int abort_flag;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int h0 = q * kHeads, g = h0 / (H / a.G);
-    const ChunkEntry seg = a.segs[i];
+    const int h0 = (blockIdx.x % nq) * kHeads, g = h0 / (H / G);
+    const ChunkEntry seg = segs[sg];
     const int ntiles = (seg.len + kTile - 1) / kTile;
 
     if (tid == 0) {
-        for (int k = 0; k < 2; ++k) {
-            mbar_init(&full_b[k], 1);
-            mbar_init(&empty_b[k], 1);
-            mbar_init(&full_x[k], 1);
-            mbar_init(&pair_done[k], 1);
-            mbar_init(&ops_ready[k], kComputeWarps);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&full_b[i], 1);
+            mbar_init(&empty_b[i], 1);
+            mbar_init(&full_x[i], 1);
+            mbar_init(&pair_done[i], 1);
+            mbar_init(&ops_ready[i], kComputeWarps);
         }
-        for (int k = 0; k < 4; ++k) {
-            mbar_init(&w_ready[k], 2);
-            mbar_init(&w_free[k], kComputeWarps);
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(&w_ready[i], 2);
+            mbar_init(&w_free[i], kComputeWarps);
         }
-        mbar_init(all_done, 1);
-        mbar_init(sum_ready, 2);
-        sh.abort_flag = 0;
+        mbar_init(&all_done, 1);
+        abort_flag = 0;
         fence_barrier_init();
+        prefetch_tmap(&map_x);
+        prefetch_tmap(&map_b);
     }
+    if (warp == 1) {
+        tmem_alloc(&tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
     __syncthreads();
-    volatile int* abort_p = &sh.abort_flag;
+    tc_fence_after();
+    const uint32_t tS = tmem_slot;
+    volatile int* abort_p = &abort_flag;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -226,19 +160,19 @@ __device__ __forceinline__ void item_state(const CUtensorMap* map_x, const CUten
                 const int t0 = t0_of(k), st = k & 1;
                 if (k >= 2) wait_abort(&empty_b[st], ((k - 2) >> 1) & 1, abort_p);
                 mbar_arrive_expect_tx(&full_b[st], 32768);
-                tma_load_3d(sB + st * 32768, map_b, &full_b[st], 0, g, t0);
-                tma_load_3d(sB + st * 32768 + 16384, map_b, &full_b[st], 64, g, t0);
+                tma_load_3d(sB + st * 32768, &map_b, &full_b[st], 0, g, t0);
+                tma_load_3d(sB + st * 32768 + 16384, &map_b, &full_b[st], 64, g, t0);
                 if (k + 1 < ntiles) {               // next chunk's B and X into L2 meanwhile
                     const int tn = t0_of(k + 1);
-                    tma_prefetch_3d(map_b, 0, g, tn);
-                    tma_prefetch_3d(map_b, 64, g, tn);
-                    for (int hh = 0; hh < kHeads; ++hh) tma_prefetch_3d(map_x, 0, h0 + hh, tn);
+                    tma_prefetch_3d(&map_b, 0, g, tn);
+                    tma_prefetch_3d(&map_b, 64, g, tn);
+                    for (int hh = 0; hh < kHeads; ++hh) tma_prefetch_3d(&map_x, 0, h0 + hh, tn);
                 }
                 for (int pr = 0; pr < 2; ++pr) {
                     if (k >= 1) wait_abort(&pair_done[pr], (k - 1) & 1, abort_p);   // slots and lo free
                     mbar_arrive_expect_tx(&full_x[pr], 32768);
                     for (int hh = 2 * pr; hh < 2 * pr + 2; ++hh)
-                        tma_load_3d(xs(hh), map_x, &full_x[pr], 0, h0 + hh, t0);
+                        tma_load_3d(xs(hh), &map_x, &full_x[pr], 0, h0 + hh, t0);
                 }
             }
         }
@@ -263,38 +197,34 @@ __device__ __forceinline__ void item_state(const CUtensorMap* map_x, const CUten
                         umma_bf16(d, desc_add(dB, kk * kMnStep), desc_add(dp, kk * kMnStep), idesc, !(k == 0 && kk == 0));
                     umma_commit(&pair_done[pr]);
                     if (pr == 1) umma_commit(&empty_b[st]);
-                    if (pr == 1 && k == ntiles - 1) umma_commit(all_done);
+                    if (pr == 1 && k == ntiles - 1) umma_commit(&all_done);
                 }
                 __syncwarp();
             }
         }
-        // Phases no other role waits for: they complete before the item ends, so the
-        // next item can initialise the barriers again.
-        for (int k = max(0, ntiles - 2); k < ntiles; ++k) wait_abort(&empty_b[k & 1], (k >> 1) & 1, abort_p);
-        for (int pr = 0; pr < 2; ++pr) wait_abort(&pair_done[pr], (ntiles - 1) & 1, abort_p);
-    } else if (warp >= kScanWarp) {
+    } else if (warp >= kScanWarpA) {
         // ------------------------------------------------------------ dt scan
-        // Warp 18 + e scans heads 2e, 2e+1. Lane l holds tokens 4l..4l+3 of a chunk; the
+        // Warp 18 + i scans heads 2i, 2i+1. Lane l holds tokens 4l..4l+3 of a chunk; the
         // dt_raw of the next chunk is loaded while this one is scanned. suf[e] = sum of
         // dt*A after the current chunk (log2 units).
-        const int hb = 2 * (warp - kScanWarp);
+        const int hb = 2 * (warp - kScanWarpA);
         float bias[2], Ah[2], suf[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-            bias[e] = a.dt_bias[h0 + hb + e];
-            Ah[e] = a.A[h0 + hb + e] * kLog2e;
+            bias[e] = dt_bias[h0 + hb + e];
+            Ah[e] = A[h0 + hb + e] * kLog2e;
             suf[e] = 0.f;
-            if (lane == 0 && (!(a.A[h0 + hb + e] <= 0.f) || isinf(a.A[h0 + hb + e]))) latch_error(SSD_ERR_INVALID_ARG);
+            if (lane == 0 && (!(A[h0 + hb + e] <= 0.f) || isinf(A[h0 + hb + e]))) latch_error(SSD_ERR_INVALID_ARG);
         }
         float z[2][4], zn[2][4];
         auto load_dt = [&](int k, float (&zz)[2][4]) {
             const int it = ntiles - 1 - k;
             const int tlk = min(kTile, seg.len - it * kTile);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int64_t row = ((int64_t)seg.start + (int64_t)it * kTile + 4 * lane + u) * H + h0 + hb;
+            for (int i = 0; i < 4; ++i) {
+                const int64_t row = ((int64_t)seg.start + (int64_t)it * kTile + 4 * lane + i) * H + h0 + hb;
 #pragma unroll
-                for (int e = 0; e < 2; ++e) zz[e][u] = 4 * lane + u < tlk ? a.dt_raw[row + e] : 0.f;
+                for (int e = 0; e < 2; ++e) zz[e][i] = 4 * lane + i < tlk ? dt_raw[row + e] : 0.f;
             }
         };
         load_dt(0, zn);
@@ -304,16 +234,16 @@ __device__ __forceinline__ void item_state(const CUtensorMap* map_x, const CUten
 #pragma unroll
             for (int e = 0; e < 2; ++e)
 #pragma unroll
-                for (int u = 0; u < 4; ++u) z[e][u] = zn[e][u];
+                for (int i = 0; i < 4; ++i) z[e][i] = zn[e][i];
             if (k + 1 < ntiles) load_dt(k + 1, zn);
             if (k >= 4) wait_abort(&w_free[bf], ((k >> 2) - 1) & 1, abort_p);
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
                 float dtv[4], p[4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    dtv[u] = 4 * lane + u < tlk ? softplus_fast(z[e][u] + bias[e]) : 0.f;
-                    p[u] = (u ? p[u - 1] : 0.f) + dtv[u] * Ah[e];
+                for (int i = 0; i < 4; ++i) {
+                    dtv[i] = 4 * lane + i < tlk ? softplus_fast(z[e][i] + bias[e]) : 0.f;
+                    p[i] = (i ? p[i - 1] : 0.f) + dtv[i] * Ah[e];
                 }
                 float incl = p[3];
 #pragma unroll
@@ -322,22 +252,20 @@ __device__ __forceinline__ void item_state(const CUtensorMap* map_x, const CUten
                     if (lane >= off) incl += v;
                 }
                 const float tot = __shfl_sync(0xffffffffu, incl, 31);
-                const float base = suf[e] + tot - (incl - p[3]);    // decay exponent of token 4l, plus p[u] below
+                const float base = suf[e] + tot - (incl - p[3]);    // decay exponent of token 4l, plus p[i] below
                 float w[4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) w[u] = fast_exp2(base - p[u]) * dtv[u];
+                for (int i = 0; i < 4; ++i) w[i] = fast_exp2(base - p[i]) * dtv[i];
                 *reinterpret_cast<float4*>(&wts[bf][hb + e][4 * lane]) = make_float4(w[0], w[1], w[2], w[3]);
                 suf[e] += tot;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&w_ready[bf]);
         }
-        if (lane < 2) sh.segsum[hb + lane] = lane ? suf[1] : suf[0];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(sum_ready);
+        if (lane < 2) seg_acum[(int64_t)sg * H + h0 + hb + lane] = (lane ? suf[1] : suf[0]) / kLog2e;
     } else {
         // ------------------------------------------------------------ compute warps
-        const int cw = (warp - kRoleWarps) >> 2, qq = warp & 3, r = qq * 32 + lane;
+        const int cw = (warp - kRoleWarps) >> 2, q = warp & 3, r = q * 32 + lane;
         for (int k = 0; k < ntiles; ++k) {
             const int bf = k % 4;
             wait_abort(&w_ready[bf], (k >> 2) & 1, abort_p);
@@ -370,70 +298,122 @@ __device__ __forceinline__ void item_state(const CUtensorMap* map_x, const CUten
             __syncwarp();
             if (lane == 0) mbar_arrive(&w_free[bf]);
         }
-        // ---- chain link: h_out(i) = exp(sum dt*A) h_out(i-1) + S_i for head h0 + cw,
-        // state row n = r, sixteen columns p at a time.
-        const int h = h0 + cw, s = seg.seq;
-        const bool first = i == a.first[s], last = i == a.first[s + 1] - 1;
-        if (!first) compute_wait_flag(&a.flags[(i - 1) * (H / kHeads) + q], a.sched);
-        wait_abort(sum_ready, 0, abort_p);
-        wait_abort(all_done, 0, abort_p);
+        // Wait for the last UMMAs, then write S_seg of head cw: thread = state row n.
+        wait_abort(&all_done, 0, abort_p);
         tc_fence_after();
-        const float dec = fast_exp2(sh.segsum[cw]);
-        // Every state below is [P][N] (n contiguous): thread n = r touches (p, r), so a
-        // warp's accesses for one p are 128 contiguous bytes.
-        const int64_t api = ((int64_t)s * H + h) * kP * kN + r;               // (p, n = r) at api + p*kN
-        const float* hprev = a.hout + ((int64_t)(i - 1) * H + h) * kP * kN + r;
-        float* hnext = a.hout + ((int64_t)i * H + h) * kP * kN + r;
-        int64_t snap_idx = -1;
-        if (a.snap > 0) {
-            const int64_t end = (int64_t)seg.start + seg.len - a.segs[a.first[s]].start;
-            if (end % a.snap == 0) snap_idx = a.snap_first[s] + end / a.snap - 1;
-        }
-        const uint32_t thi = tS + ((uint32_t)(qq * 32) << 16) + (cw >> 1) * 256 + (cw & 1) * 64;
-        for (int c16 = 0; c16 < 4; ++c16) {
-            uint32_t vh[16], vl[16];
-            tmem_ld16(thi + 16 * c16, vh);
-            tmem_ld16(thi + 128 + 16 * c16, vl);
-            float hp[16];
-            if (!first) {
-#pragma unroll
-                for (int e = 0; e < 16; ++e) hp[e] = __ldcg(hprev + (int64_t)(16 * c16 + e) * kN);
-            } else if (a.init) {
-#pragma unroll
-                for (int e = 0; e < 16; ++e) hp[e] = a.init[api + (int64_t)(16 * c16 + e) * kN];
-            } else {
-#pragma unroll
-                for (int e = 0; e < 16; ++e) hp[e] = 0.f;
-            }
+        float* dst = seg_state + (((int64_t)sg * H + h0 + cw) * kN + r) * kP;
+        const uint32_t thi = tS + ((uint32_t)(q * 32) << 16) + (cw >> 1) * 256 + (cw & 1) * 64;
+        for (int half = 0; half < 2; ++half) {
+            uint32_t vh[32], vl[32];
+            tmem_ld32(thi + half * 32, vh);
+            tmem_ld32(thi + 128 + half * 32, vl);
             tmem_wait_ld();
-            float ho[16];
+            float4* d4 = reinterpret_cast<float4*>(dst + half * 32);
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-                ho[e] = fmaf(dec, hp[e], __uint_as_float(vh[e]) + __uint_as_float(vl[e]));
-            float* dst = !last ? hnext : a.final_state ? a.final_state + api : nullptr;
-            if (dst) {
-#pragma unroll
-                for (int e = 0; e < 16; ++e) dst[(int64_t)(16 * c16 + e) * kN] = ho[e];
-            }
-            if (snap_idx >= 0) {
-                float* so = a.snap_out + (snap_idx * H + h) * kP * kN + r;
-#pragma unroll
-                for (int e = 0; e < 16; ++e) so[(int64_t)(16 * c16 + e) * kN] = ho[e];
-            }
-        }
-        if (!last) {
-            __threadfence();
-            compute_bar();
-            if (tid == kFirstCompute && *reinterpret_cast<volatile int*>(&g_flag_publish))
-                st_release(&a.flags[i * (H / kHeads) + q], 1);
+            for (int e = 0; e < 8; ++e)
+                d4[e] = make_float4(__uint_as_float(vh[4 * e]) + __uint_as_float(vl[4 * e]),
+                                    __uint_as_float(vh[4 * e + 1]) + __uint_as_float(vl[4 * e + 1]),
+                                    __uint_as_float(vh[4 * e + 2]) + __uint_as_float(vl[4 * e + 2]),
+                                    __uint_as_float(vh[4 * e + 3]) + __uint_as_float(vl[4 * e + 3]));
         }
     }
     tc_fence_before();
     __syncthreads();
+    if (warp == 1) tmem_dealloc(tS, 512);
 }
 
 // ---------------------------------------------------------------------------------
-// Scan item: outputs y for segment i, heads h0, h0 + 1 (pair hp), chunk by chunk.
+// Chain over segments. seg_state slots are replaced by the state entering each segment
+// (h_in, layout [seg][H][N][P]); init, final_state and the snapshots use the API layout
+// [nseq][H][P][N]. A CTA owns kPassN = 8 state rows (n) x all P columns of one (sequence,
+// head); thread t walks elements t and t + 256 of that tile ([N][P] order, coalesced)
+// down the segments, four segments' loads in flight. API-layout reads and writes go
+// through a shared-memory transpose, so a warp touches 32-byte sectors it uses whole.
+constexpr int kPassN = 8;
+
+__global__ void __launch_bounds__(256)
+k_tc_segment_passing(float* __restrict__ seg_state, const float* __restrict__ seg_acum,
+                     const int32_t* __restrict__ first, const float* __restrict__ init,
+                     float* __restrict__ final_state, int H, const ChunkEntry* __restrict__ segs,
+                     int64_t snap, const int32_t* __restrict__ snap_first, float* __restrict__ snap_out) {
+    constexpr int E = kP * kPassN / 256;                   // elements per thread (2)
+    __shared__ float tile[kP][kPassN + 1];
+    const int s = blockIdx.x, h = blockIdx.y, n0 = blockIdx.z * kPassN, tid = threadIdx.x;
+    const int64_t api0 = ((int64_t)s * H + h) * kP * kN + n0;   // (p, n0 + nn) at api0 + p*kN + nn
+    // element i of thread tid: idx = tid + 256 i, n = n0 + idx / kP, p = idx % kP
+    auto api_load = [&](const float* src, float (&v)[E]) {
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+            const int idx = tid + 256 * i, p = idx / kPassN, nn = idx % kPassN;
+            tile[p][nn] = src[(int64_t)p * kN + nn];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+            const int idx = tid + 256 * i;
+            v[i] = tile[idx % kP][idx / kP];
+        }
+    };
+    auto api_store = [&](float* dst, const float (&v)[E]) {
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+            const int idx = tid + 256 * i;
+            tile[idx % kP][idx / kP] = v[i];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+            const int idx = tid + 256 * i, p = idx / kPassN, nn = idx % kPassN;
+            dst[(int64_t)p * kN + nn] = tile[p][nn];
+        }
+    };
+    float hv[E];
+    if (init) {
+        api_load(init + api0, hv);
+    } else {
+#pragma unroll
+        for (int i = 0; i < E; ++i) hv[i] = 0.f;
+    }
+    const int c0 = first[s], c1 = first[s + 1];
+    const int64_t seq0 = c1 > c0 ? segs[c0].start : 0;
+    const int64_t eoff = (int64_t)n0 * kP + tid;
+    constexpr int U = 4;
+    for (int c = c0; c < c1; c += U) {
+        float sv[U][E], dec[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (c + u < c1) {
+                const float* slot = seg_state + ((int64_t)(c + u) * H + h) * (kP * kN) + eoff;
+#pragma unroll
+                for (int i = 0; i < E; ++i) sv[u][i] = slot[256 * i];
+                dec[u] = expf(seg_acum[(int64_t)(c + u) * H + h]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (c + u < c1) {
+                float* slot = seg_state + ((int64_t)(c + u) * H + h) * (kP * kN) + eoff;
+#pragma unroll
+                for (int i = 0; i < E; ++i) {
+                    slot[256 * i] = hv[i];
+                    hv[i] = fmaf(dec[u], hv[i], sv[u][i]);
+                }
+                if (snap > 0) {                           // state after a multiple of snap tokens
+                    const int64_t end = (int64_t)segs[c + u].start + segs[c + u].len - seq0;
+                    if (end % snap == 0)
+                        api_store(snap_out + ((int64_t)(snap_first[s] + end / snap - 1) * H + h) * kP * kN + n0,
+                                  hv);
+                }
+            }
+        }
+    }
+    if (final_state) api_store(final_state + api0, hv);
+}
+
+// ---------------------------------------------------------------------------------
+// Pass B: outputs y for one (segment, 2 heads), chunk by chunk.
 //
 // Warp 0 issues the TMA loads and the y stores, warp 1 the UMMAs, and four compute
 // warpgroups (cw = 0..3) split every row's 64 columns in quarters. Compute thread
@@ -464,62 +444,77 @@ __device__ __forceinline__ void item_state(const CUtensorMap* map_x, const CUten
 // stage (reloaded as soon as the Z/S UMMAs are done), two X slots (chunk j uses slot
 // j & 1; its y tile replaces x there), bf16 h and w*X for both heads, the diagonal-block
 // decay table (16 KB).
-__device__ __forceinline__ void item_scan(const CUtensorMap* map_x, const CUtensorMap* map_b,
-                                          const CUtensorMap* map_c, const CUtensorMap* map_y, const TcArgs& a,
-                                          int i, int hp, uint8_t* sm, ItemShared& sh, uint32_t tbase) {
-    const int H = a.H;
+constexpr int kHeadsB = 2;
+constexpr int kSmemB = 208 * 1024 + 1024;
+constexpr int kScanWarp = kRoleWarps + kComputeWarps;          // warp 18: dt scan
+constexpr int kThreadsB = 32 * (kScanWarp + 1);
+
+__global__ void __launch_bounds__(kThreadsB, 1)
+k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
+                const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_y,
+                const float* __restrict__ dt_raw, const float* __restrict__ dt_bias, const float* __restrict__ A,
+                const float* __restrict__ D, const ChunkEntry* __restrict__ segs, const int32_t* __restrict__ nsegs,
+                int H, int G, const float* __restrict__ hin, __nv_bfloat16* __restrict__ y,
+                const int32_t* __restrict__ order) {
+    const int nhp = H / kHeadsB;
+    if ((int)(blockIdx.x / nhp) >= *nsegs) return;
+    const int sg = order ? order[blockIdx.x / nhp] : (int)(blockIdx.x / nhp);   // longest segments first
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sC = sm;                       // [2][128 t][64 n]   K-major
     uint8_t* sB = sm + 32768;               // [2][128 s][64 n]   K-major for C B^T, MN-major for B^T
     uint8_t* sX = sm + 65536;               // slot sl, head hh at sl*32768 + hh*16384: [128 s][64 p]
     uint8_t* sH = sm + 131072;              // head hh block at hh*16384: [128 n][64 p]  bf16 h_in
     uint8_t* sW = sm + 163840;              // head hh block at hh*16384: [128 s][64 p]  w * X
     uint8_t* sL = sm + 196608;              // head hh at hh*8192: [128 t][32] fp16 diagonal-block decays
-    float (*ac2)[kHeadsB][kTile] = reinterpret_cast<float (*)[kHeadsB][kTile]>(sh.f);
-    float (*dts)[kHeadsB][kTile] = reinterpret_cast<float (*)[kHeadsB][kTile]>(sh.f + 1024);
-    float (*uw)[kHeadsB][kTile] = reinterpret_cast<float (*)[kHeadsB][kTile]>(sh.f + 2048);
-    float (*ww)[kHeadsB][kTile] = reinterpret_cast<float (*)[kHeadsB][kTile]>(sh.f + 3072);
-    uint64_t* full_b = &sh.bar[0];
-    uint64_t* full_c = &sh.bar[1];          // [2]
-    uint64_t* s_done = &sh.bar[3];
-    uint64_t* zs_done = &sh.bar[4];
-    uint64_t* full_x = &sh.bar[5];          // [2]
-    uint64_t* cb_done = &sh.bar[7];
-    uint64_t* ops_ready = &sh.bar[8];
-    uint64_t* y0_done = &sh.bar[9];
-    uint64_t* mma_done = &sh.bar[10];
-    uint64_t* l_ready = &sh.bar[11];
-    uint64_t* dt_ready = &sh.bar[12];       // [4]
-    uint64_t* dt_free = &sh.bar[16];        // [4]
-    uint64_t* y_staged = &sh.bar[20];
+    __shared__ __align__(16) float ac2[4][kHeadsB][kTile];
+    __shared__ __align__(16) float dts[4][kHeadsB][kTile];
+    __shared__ __align__(16) float uw[4][kHeadsB][kTile];
+    __shared__ __align__(16) float ww[4][kHeadsB][kTile];
+    __shared__ uint64_t full_b, full_c[2], s_done, zs_done, full_x[2], cb_done, ops_ready, y0_done, mma_done, l_ready,
+        dt_ready[4], dt_free[4], y_staged;
+    __shared__ uint32_t tmem_slot;
+    __shared__ int abort_flag;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int h0 = hp * kHeadsB, g = h0 / (H / a.G);
-    const ChunkEntry seg = a.segs[i];
+    const int h0 = (blockIdx.x % nhp) * kHeadsB, g = h0 / (H / G);
+    const ChunkEntry seg = segs[sg];
     const int ntiles = (seg.len + kTile - 1) / kTile;
 
     if (tid == 0) {
-        mbar_init(full_b, 1);
+        mbar_init(&full_b, 1);
         mbar_init(&full_c[0], 1);
         mbar_init(&full_c[1], 1);
-        mbar_init(y0_done, 1);
-        mbar_init(s_done, 1);
-        mbar_init(zs_done, 1);
+        mbar_init(&y0_done, 1);
+        mbar_init(&s_done, 1);
+        mbar_init(&zs_done, 1);
         for (int sl = 0; sl < 2; ++sl) mbar_init(&full_x[sl], 1);
-        mbar_init(cb_done, 1);
-        mbar_init(ops_ready, kComputeWarps);
-        mbar_init(mma_done, 1);
-        for (int k = 0; k < 4; ++k) {
-            mbar_init(&dt_ready[k], 1);
-            mbar_init(&dt_free[k], kComputeWarps);
+        mbar_init(&y_staged, kComputeWarps);
+        mbar_init(&cb_done, 1);
+        mbar_init(&ops_ready, kComputeWarps);
+        mbar_init(&mma_done, 1);
+        for (int i = 0; i < 4; ++i) {
+            mbar_init(&dt_ready[i], 1);
+            mbar_init(&dt_free[i], kComputeWarps);
         }
-        mbar_init(l_ready, kComputeWarps);
-        mbar_init(y_staged, kComputeWarps);
-        sh.abort_flag = 0;
+        mbar_init(&l_ready, kComputeWarps);
+        abort_flag = 0;
         fence_barrier_init();
+        prefetch_tmap(&map_x);
+        prefetch_tmap(&map_b);
+        prefetch_tmap(&map_c);
+        prefetch_tmap(&map_y);
     }
+    if (warp == 1) {
+        tmem_alloc(&tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = tmem_slot;
     const uint32_t tZ = tbase, tS = tbase + 128, tY = tbase + 256, tM = tbase + 384;
-    volatile int* abort_p = &sh.abort_flag;
+    volatile int* abort_p = &abort_flag;
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -528,38 +523,38 @@ __device__ __forceinline__ void item_scan(const CUtensorMap* map_x, const CUtens
                 const int sl = j & 1;
                 mbar_arrive_expect_tx(&full_x[sl], 32768);
                 for (int hh = 0; hh < kHeadsB; ++hh)
-                    tma_load_3d(sX + sl * 32768 + hh * 16384, map_x, &full_x[sl], 0, h0 + hh, seg.start + j * kTile);
+                    tma_load_3d(sX + sl * 32768 + hh * 16384, &map_x, &full_x[sl], 0, h0 + hh, seg.start + j * kTile);
             };
             // B of chunk j (once the S UMMAs of chunk j-1 are done) and the two halves of
             // C (once Z is done), on separate barriers, so C B^T can start on the first
             // half. B, C and X of chunk j+1 are prefetched into L2 meanwhile.
             auto load_b = [&](int j) {
                 const int t0 = seg.start + j * kTile;
-                mbar_arrive_expect_tx(full_b, 32768);
-                tma_load_3d(sB, map_b, full_b, 0, g, t0);
-                tma_load_3d(sB + 16384, map_b, full_b, 64, g, t0);
+                mbar_arrive_expect_tx(&full_b, 32768);
+                tma_load_3d(sB, &map_b, &full_b, 0, g, t0);
+                tma_load_3d(sB + 16384, &map_b, &full_b, 64, g, t0);
             };
             auto load_c = [&](int j) {
                 const int t0 = seg.start + j * kTile;
                 for (int hf = 0; hf < 2; ++hf) {
                     mbar_arrive_expect_tx(&full_c[hf], 16384);
-                    tma_load_3d(sC + hf * 16384, map_c, &full_c[hf], 64 * hf, g, t0);
+                    tma_load_3d(sC + hf * 16384, &map_c, &full_c[hf], 64 * hf, g, t0);
                 }
                 if (j + 1 < ntiles) {
-                    tma_prefetch_3d(map_c, 0, g, t0 + kTile);
-                    tma_prefetch_3d(map_c, 64, g, t0 + kTile);
-                    tma_prefetch_3d(map_b, 0, g, t0 + kTile);
-                    tma_prefetch_3d(map_b, 64, g, t0 + kTile);
-                    for (int hh = 0; hh < kHeadsB; ++hh) tma_prefetch_3d(map_x, 0, h0 + hh, t0 + kTile);
+                    tma_prefetch_3d(&map_c, 0, g, t0 + kTile);
+                    tma_prefetch_3d(&map_c, 64, g, t0 + kTile);
+                    tma_prefetch_3d(&map_b, 0, g, t0 + kTile);
+                    tma_prefetch_3d(&map_b, 64, g, t0 + kTile);
+                    for (int hh = 0; hh < kHeadsB; ++hh) tma_prefetch_3d(&map_x, 0, h0 + hh, t0 + kTile);
                 }
             };
             // y tile of chunk j, staged by the compute warps in the chunk's X slot (full
             // chunks only; a partial last chunk is written by the threads).
             auto store_y = [&](int j) {
-                wait_abort(y_staged, j & 1, abort_p);
+                wait_abort(&y_staged, j & 1, abort_p);
                 if (seg.len - j * kTile >= kTile) {
                     for (int hh = 0; hh < kHeadsB; ++hh)
-                        tma_store_3d(map_y, sX + (j & 1) * 32768 + hh * 16384, 0, h0 + hh, seg.start + j * kTile);
+                        tma_store_3d(&map_y, sX + (j & 1) * 32768 + hh * 16384, 0, h0 + hh, seg.start + j * kTile);
                     bulk_commit_group();
                 }
             };
@@ -570,9 +565,9 @@ __device__ __forceinline__ void item_scan(const CUtensorMap* map_x, const CUtens
                 load_c(0);
             }
             for (int j = 1; j < ntiles; ++j) {
-                wait_abort(s_done, (j - 1) & 1, abort_p);          // B of chunk j-1 read
+                wait_abort(&s_done, (j - 1) & 1, abort_p);          // B of chunk j-1 read
                 load_b(j);
-                wait_abort(zs_done, (j - 1) & 1, abort_p);         // C of chunk j-1 read
+                wait_abort(&zs_done, (j - 1) & 1, abort_p);         // C of chunk j-1 read
                 load_c(j);
                 store_y(j - 1);
                 if (j + 1 < ntiles) {
@@ -595,7 +590,7 @@ __device__ __forceinline__ void item_scan(const CUtensorMap* map_x, const CUtens
         // C B^T of chunk j into the M columns (fp32): dstate columns 0..63 once B and the
         // first half of C have landed, 64..127 once the second half has.
         auto issue_cb = [&](int j) {
-            wait_abort(full_b, j & 1, abort_p);
+            wait_abort(&full_b, j & 1, abort_p);
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 wait_abort(&full_c[hf], j & 1, abort_p);
@@ -605,43 +600,40 @@ __device__ __forceinline__ void item_scan(const CUtensorMap* map_x, const CUtens
                     for (int k = 4 * hf; k < 4 * hf + 4; ++k)
                         umma_bf16(tM, desc_add(dCk, kmajor_step(128, k)), desc_add(dBk, kmajor_step(128, k)), id_cb,
                                   k > 0);
-                    if (hf == 1) umma_commit(cb_done);
+                    if (hf == 1) umma_commit(&cb_done);
                 }
                 __syncwarp();
             }
         };
         if (ntiles > 0) issue_cb(0);
         for (int it = 0; it < ntiles; ++it) {
-            wait_abort(ops_ready, it & 1, abort_p);
+            wait_abort(&ops_ready, it & 1, abort_p);
             tc_fence_after();
             const uint64_t dX0 = desc_add(dX, (it & 1) * 32768), dX1 = desc_add(dX0, 16384);
             if (elect_one()) {
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
                     umma_bf16(tS, desc_add(dBm, k * kMnStep), desc_add(dW, k * kMnStep), id_s, k > 0);
-                umma_commit(s_done);
+                umma_commit(&s_done);
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
                     umma_bf16(tZ, desc_add(dCk, kmajor_step(128, k)), desc_add(dH, k * kMnStep), id_z, k > 0);
-                umma_commit(zs_done);
+                umma_commit(&zs_done);
                 // M of head hh, sources 16k..16k+15: TMEM columns 16k + 8hh of the M block.
 #pragma unroll
                 for (int k = 0; k < 8; ++k) umma_bf16_ts(tY, tM + 16 * k, desc_add(dX0, k * kMnStep), id_y, k > 0);
-                umma_commit(y0_done);
+                umma_commit(&y0_done);
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
                     umma_bf16_ts(tY + 64, tM + 16 * k + 8, desc_add(dX1, k * kMnStep), id_y, k > 0);
-                umma_commit(mma_done);
+                umma_commit(&mma_done);
             }
             __syncwarp();
             if (it + 1 < ntiles) {
-                wait_abort(mma_done, it & 1, abort_p);     // the Y UMMAs have read M
+                wait_abort(&mma_done, it & 1, abort_p);     // the Y UMMAs have read M
                 issue_cb(it + 1);
             }
         }
-        // The last chunk's S phase is waited here (no other role waits for it), so the
-        // next item can initialise the barriers again.
-        if (ntiles > 0) wait_abort(s_done, (ntiles - 1) & 1, abort_p);
     } else if (warp == kScanWarp) {
         // ------------------------------------------------------------ dt scan
         // Chunk by chunk, up to four ahead of the compute warps: dt, the log2-scaled
@@ -650,18 +642,18 @@ __device__ __forceinline__ void item_scan(const CUtensorMap* map_x, const CUtens
         float bias[kHeadsB], Ah[kHeadsB];
 #pragma unroll
         for (int hh = 0; hh < kHeadsB; ++hh) {
-            bias[hh] = a.dt_bias[h0 + hh];
-            Ah[hh] = a.A[h0 + hh];
+            bias[hh] = dt_bias[h0 + hh];
+            Ah[hh] = A[h0 + hh];
             if (lane == 0 && (!(Ah[hh] <= 0.f) || isinf(Ah[hh]))) latch_error(SSD_ERR_INVALID_ARG);
         }
         float z[kHeadsB][4], zn[kHeadsB][4];       // dt_raw of chunk j and of chunk j+1
         auto load_dt = [&](int j, float (&zz)[kHeadsB][4]) {
             const int tlj = min(kTile, seg.len - j * kTile);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int64_t row = ((int64_t)seg.start + (int64_t)j * kTile + 4 * lane + u) * H + h0;
+            for (int i = 0; i < 4; ++i) {
+                const int64_t row = ((int64_t)seg.start + (int64_t)j * kTile + 4 * lane + i) * H + h0;
 #pragma unroll
-                for (int hh = 0; hh < kHeadsB; ++hh) zz[hh][u] = 4 * lane + u < tlj ? a.dt_raw[row + hh] : 0.f;
+                for (int hh = 0; hh < kHeadsB; ++hh) zz[hh][i] = 4 * lane + i < tlj ? dt_raw[row + hh] : 0.f;
             }
         };
         if (ntiles > 0) load_dt(0, zn);
@@ -670,7 +662,7 @@ __device__ __forceinline__ void item_scan(const CUtensorMap* map_x, const CUtens
 #pragma unroll
             for (int hh = 0; hh < kHeadsB; ++hh)
 #pragma unroll
-                for (int u = 0; u < 4; ++u) z[hh][u] = zn[hh][u];
+                for (int i = 0; i < 4; ++i) z[hh][i] = zn[hh][i];
             if (j + 1 < ntiles) load_dt(j + 1, zn);
             if (j >= 4) wait_abort(&dt_free[bf], ((j >> 2) - 1) & 1, abort_p);
             const int tlj = min(kTile, seg.len - j * kTile);
@@ -678,9 +670,9 @@ __device__ __forceinline__ void item_scan(const CUtensorMap* map_x, const CUtens
             for (int hh = 0; hh < kHeadsB; ++hh) {
                 float dtv[4], p[4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    dtv[u] = 4 * lane + u < tlj ? softplus_fast(z[hh][u] + bias[hh]) : 0.f;
-                    p[u] = (u ? p[u - 1] : 0.f) + dtv[u] * Ah[hh];
+                for (int i = 0; i < 4; ++i) {
+                    dtv[i] = 4 * lane + i < tlj ? softplus_fast(z[hh][i] + bias[hh]) : 0.f;
+                    p[i] = (i ? p[i - 1] : 0.f) + dtv[i] * Ah[hh];
                 }
                 float incl = p[3];
 #pragma unroll
@@ -691,83 +683,73 @@ __device__ __forceinline__ void item_scan(const CUtensorMap* map_x, const CUtens
                 const float excl = incl - p[3];
                 float av[4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) av[u] = (excl + p[u]) * kLog2e;
+                for (int i = 0; i < 4; ++i) av[i] = (excl + p[i]) * kLog2e;
                 const float a_blk = __shfl_sync(0xffffffffu, av[3], (lane & ~7) | 7);    // token 32b + 31
                 const float a_end = __shfl_sync(0xffffffffu, av[3], 31);                 // token 127
-                float u4[4], w[4];
+                float u[4], w[4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    u4[u] = fast_exp2(a_blk - av[u]) * dtv[u];
-                    w[u] = fast_exp2(a_end - av[u]) * dtv[u];
+                for (int i = 0; i < 4; ++i) {
+                    u[i] = fast_exp2(a_blk - av[i]) * dtv[i];
+                    w[i] = fast_exp2(a_end - av[i]) * dtv[i];
                 }
                 *reinterpret_cast<float4*>(&ac2[bf][hh][4 * lane]) = make_float4(av[0], av[1], av[2], av[3]);
                 *reinterpret_cast<float4*>(&dts[bf][hh][4 * lane]) = make_float4(dtv[0], dtv[1], dtv[2], dtv[3]);
-                *reinterpret_cast<float4*>(&uw[bf][hh][4 * lane]) = make_float4(u4[0], u4[1], u4[2], u4[3]);
+                *reinterpret_cast<float4*>(&uw[bf][hh][4 * lane]) = make_float4(u[0], u[1], u[2], u[3]);
                 *reinterpret_cast<float4*>(&ww[bf][hh][4 * lane]) = make_float4(w[0], w[1], w[2], w[3]);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&dt_ready[bf]);
         }
-    } else if (warp < kScanWarp) {
+    } else {
         // ------------------------------------------------------------ compute warpgroups
         const int q = warp & 3;                     // TMEM lane quarter of this warp
         const int r = q * 32 + lane;                // row: token t, source s or state row n
         const int cw = (warp - kRoleWarps) >> 2;    // column quarter / source block
         const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-        // Incoming state: the state item of segment i-1 (same heads), else the initial
-        // state of the sequence, else zeros.
-        const int s = seg.seq;
-        const bool first = i == a.first[s];
-        if (!first) compute_wait_flag(&a.flags[(i - 1) * (H / kHeads) + (h0 / kHeads)], a.sched);
         float h[kHeadsB][16];                       // h[head][n = r][p = 16*cw + j]
 #pragma unroll
         for (int hh = 0; hh < kHeadsB; ++hh) {
-            if (!first) {
-                const float* src = a.hout + ((int64_t)(i - 1) * H + h0 + hh) * kP * kN + (int64_t)(16 * cw) * kN + r;
+            const float4* src =
+                reinterpret_cast<const float4*>(hin + (((int64_t)sg * H + h0 + hh) * kN + r) * kP + 16 * cw);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) h[hh][j] = __ldcg(src + (int64_t)j * kN);
-            } else if (a.init) {
-                const float* src = a.init + ((int64_t)s * H + h0 + hh) * kP * kN + (int64_t)(16 * cw) * kN + r;
-#pragma unroll
-                for (int j = 0; j < 16; ++j) h[hh][j] = src[(int64_t)j * kN];
-            } else {
-#pragma unroll
-                for (int j = 0; j < 16; ++j) h[hh][j] = 0.f;
+            for (int j = 0; j < 4; ++j) {
+                const float4 v = src[j];
+                h[hh][4 * j] = v.x;
+                h[hh][4 * j + 1] = v.y;
+                h[hh][4 * j + 2] = v.z;
+                h[hh][4 * j + 3] = v.w;
             }
         }
-        const float Dh0 = a.D[h0], Dh1 = a.D[h0 + 1];
-        // Decays of the diagonal 32x32 blocks of chunk j, L[t][s] = exp(Acum_t - Acum_s) dt_s
-        // for s <= t in t's block, 0 above (fp16). Warp (cw, q) builds head cw & 1's block q,
-        // columns s = 16 (cw >> 1) + (lane & 15), rows R0 .. R0 + 15 with R0 = 16 (lane >> 4),
-        // walking down the rows: L[s][s] = dt_s, L[t][s] = L[t-1][s] d_t with d_t = exp(dt_t A)
-        // the token's own decay; a lower-half lane starts from L[R0][s] = exp(Acum_R0 -
-        // Acum_s) dt_s. So one exponential per token and row half, and a 16-step product
-        // that underflows to 0 gracefully. Row t of the table holds its block's 32 sources;
-        // 16-byte chunk c of a row sits at chunk c ^ ((t >> 1) & 3).
+        const float Dh0 = D[h0], Dh1 = D[h0 + 1];
+        // Decays of the diagonal 32x32 blocks of chunk j, L[t][s] = exp2(Acum_t - Acum_s)
+        // dt_s for s <= t in t's block (fp16). Thread (cw, r) writes row t = r of head
+        // cw & 1, sources 16 (cw >> 1) .. +15 of the block. 16-byte chunk c of a row sits
+        // at chunk c ^ ((t >> 1) & 3).
         auto diag_decays = [&](int j) {
-            const int bf = j % 4, hd = cw & 1, t0b = 32 * q;
+            const int bf = j % 4, hd = cw & 1, c0 = 2 * (cw >> 1);
             wait_abort(&dt_ready[bf], (j / 4) & 1, abort_p);
-            const int sc = 16 * (cw >> 1) + (lane & 15), R0 = 16 * (lane >> 4);
-            const int ro = R0 + (lane & 15);                                   // this lane's own row
-            const float a_ro = ac2[bf][hd][t0b + ro];
-            const float d_own = fast_exp2(a_ro - ac2[bf][hd][t0b + (ro ? ro - 1 : 0)]);   // decay of token ro
-            const float dt_s = dts[bf][hd][t0b + sc];
-            float L = sc < R0 ? fast_exp2(ac2[bf][hd][t0b + R0] - ac2[bf][hd][t0b + sc]) * dt_s : 0.f;
-            const uint32_t base = smem_u32(sL + hd * 8192) + (uint32_t)((sc & 7) * 2);
+            const float at = ac2[bf][hd][r];
+            const float4* a4 = reinterpret_cast<const float4*>(&ac2[bf][hd][32 * q + 8 * c0]);
+            const float4* d4 = reinterpret_cast<const float4*>(&dts[bf][hd][32 * q + 8 * c0]);
+            const uint32_t row = smem_u32(sL + hd * 8192 + r * 64);
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const int t = R0 + k;
-                const float d_t = __shfl_sync(0xffffffffu, d_own, (lane & 16) | k);
-                if (t == sc) L = dt_s;
-                else if (t > sc && k > 0) L *= d_t;
-                const int R = t0b + t;
-                const unsigned short hv = __half_as_ushort(__float2half_rn(t >= sc ? L : 0.f));
-                asm volatile("st.shared.b16 [%0], %1;" ::"r"(base + R * 64 + ((((sc >> 3) ^ ((R >> 1) & 3))) << 4)),
-                             "h"(hv)
-                             : "memory");
+            for (int c = 0; c < 2; ++c) {
+                uint32_t o[4];
+#pragma unroll
+                for (int k2 = 0; k2 < 2; ++k2) {
+                    const float4 as = a4[2 * c + k2], dv = d4[2 * c + k2];
+                    const int s0 = 8 * (c0 + c) + 4 * k2;   // source offset within the block
+                    const float l0 = s0 <= lane ? fast_exp2(at - as.x) * dv.x : 0.f;
+                    const float l1 = s0 + 1 <= lane ? fast_exp2(at - as.y) * dv.y : 0.f;
+                    const float l2 = s0 + 2 <= lane ? fast_exp2(at - as.z) * dv.z : 0.f;
+                    const float l3 = s0 + 3 <= lane ? fast_exp2(at - as.w) * dv.w : 0.f;
+                    o[2 * k2] = pack_f16(l0, l1);
+                    o[2 * k2 + 1] = pack_f16(l2, l3);
+                }
+                st_shared_v4(row + (((c0 + c) ^ ((r >> 1) & 3)) << 4), o[0], o[1], o[2], o[3]);
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(l_ready);
+            if (lane == 0) mbar_arrive(&l_ready);
         };
         // w*X of chunk j for both heads into shared memory.
         auto stage_wx = [&](int j) {
@@ -811,8 +793,8 @@ __device__ __forceinline__ void item_scan(const CUtensorMap* map_x, const CUtens
             const int tl = min(kTile, seg.len - it * kTile);
             const int bf = it % 4;
             wait_abort(&dt_ready[bf], (it / 4) & 1, abort_p);
-            wait_abort(l_ready, it & 1, abort_p);
-            wait_abort(cb_done, it & 1, abort_p);
+            wait_abort(&l_ready, it & 1, abort_p);
+            wait_abort(&cb_done, it & 1, abort_p);
             tc_fence_after();
             // -------- M[t][s] of both heads, t = r, in place over C B^T. Source block b
             // (32 sources) keeps its 32 columns: half j (sources 16j..16j+15 of the
@@ -888,21 +870,21 @@ __device__ __forceinline__ void item_scan(const CUtensorMap* map_x, const CUtens
             fence_proxy_async_smem();              // bf16 h and w*X of this chunk
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(ops_ready);
+            if (lane == 0) mbar_arrive(&ops_ready);
             // -------- while S and Z run: all compute warps tabulate chunk it+1's diagonal
             // decays once every warp has read chunk it's (ops_ready complete).
             if (it + 1 < ntiles) {
-                wait_abort(ops_ready, it & 1, abort_p);
+                wait_abort(&ops_ready, it & 1, abort_p);
                 diag_decays(it + 1);
             }
             // -------- S done: w*X of the next chunk (its buffer was read by this chunk's S).
             // Z done (the Y UMMAs may still run): state update, then bf16 h of the next
             // chunk (its buffer was read by this chunk's Z).
             if (it + 1 < ntiles) {
-                wait_abort(s_done, it & 1, abort_p);
+                wait_abort(&s_done, it & 1, abort_p);
                 stage_wx(it + 1);
             }
-            wait_abort(zs_done, it & 1, abort_p);
+            wait_abort(&zs_done, it & 1, abort_p);
             tc_fence_after();
 #pragma unroll
             for (int hh = 0; hh < kHeadsB; ++hh) {
@@ -923,7 +905,7 @@ __device__ __forceinline__ void item_scan(const CUtensorMap* map_x, const CUtens
             // -------- drain: y rows (into the chunk's X slot for a full chunk, else
             // straight to HBM). The TMEM loads of the next 8-column piece are issued before the
             // current one is consumed.
-            wait_abort(y0_done, it & 1, abort_p);
+            wait_abort(&y0_done, it & 1, abort_p);
             tc_fence_after();
             {
                 const bool staged = tl == kTile;
@@ -937,7 +919,7 @@ __device__ __forceinline__ void item_scan(const CUtensorMap* map_x, const CUtens
                     const int hh = piece >> 1, half = piece & 1, cur = piece & 1;
                     tmem_wait_ld();
                     if (piece == 1) {                               // head 1's Y needs all Y UMMAs
-                        wait_abort(mma_done, it & 1, abort_p);
+                        wait_abort(&mma_done, it & 1, abort_p);
                         tc_fence_after();
                     }
                     if (piece < 3) {
@@ -955,7 +937,7 @@ __device__ __forceinline__ void item_scan(const CUtensorMap* map_x, const CUtens
                         st_shared_v4(smem_u32(sX + (it & 1) * 32768 + hh * 16384) + swz(r, 2 * cw + half), o[0], o[1],
                                      o[2], o[3]);
                     } else if (r < tl) {
-                        *reinterpret_cast<uint4*>(a.y + ((t0 + r) * H + h0 + hh) * kP + 16 * cw + 8 * half) =
+                        *reinterpret_cast<uint4*>(y + ((t0 + r) * H + h0 + hh) * kP + 16 * cw + 8 * half) =
                             make_uint4(o[0], o[1], o[2], o[3]);
                     }
                 }
@@ -963,91 +945,14 @@ __device__ __forceinline__ void item_scan(const CUtensorMap* map_x, const CUtens
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(y_staged);
+                mbar_arrive(&y_staged);
                 mbar_arrive(&dt_free[bf]);          // this chunk's dt buffer is no longer read
             }
         }
     }
     tc_fence_before();
     __syncthreads();
-}
-
-// ---------------------------------------------------------------------------------
-// The persistent prefill kernel: one CTA per SM takes tickets until none are left.
-// Ticket t: block b = t / (H/4 + H/2); the first H/4 tickets of a block are the state
-// items of segment b (quads), the next H/2 the scan items of segment b - lag (pairs).
-__global__ void __launch_bounds__(kThreads, 1)
-k_tc_prefill(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
-             const __grid_constant__ CUtensorMap map_c, const __grid_constant__ CUtensorMap map_y,
-             const __grid_constant__ TcArgs a) {
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ ItemShared sh;
-    __shared__ uint32_t tmem_slot;
-    const int tid = threadIdx.x, warp = tid >> 5;
-    if (tid == 0) {
-        prefetch_tmap(&map_x);
-        prefetch_tmap(&map_b);
-        prefetch_tmap(&map_c);
-        prefetch_tmap(&map_y);
-    }
-    if (warp == 1) {
-        tmem_alloc(&tmem_slot, 512);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tbase = tmem_slot;
-    if (tid == 0) sh.abort_flag = 0;
-    const int nA = a.H / kHeads, nB = a.H / kHeadsB, per = nA + nB;
-    const int nsegs = *a.nsegs;
-    const int total = (nsegs + a.lag) * per;
-    for (;;) {
-        if (tid == 0) {
-            int t = atomicAdd(&a.sched->ticket, 1);
-            if (*reinterpret_cast<volatile int32_t*>(&a.sched->abort)) t = total;
-            sh.ticket = t;
-        }
-        __syncthreads();
-        const int t = sh.ticket;
-        if (t >= total) break;
-        const int b = t / per, r = t % per;
-        if (r < nA) {
-            if (b < nsegs) item_state(&map_x, &map_b, a, b, r, sm, sh, tbase);
-        } else if (b >= a.lag && b - a.lag < nsegs) {
-            item_scan(&map_x, &map_b, &map_c, &map_y, a, b - a.lag, r - nA, sm, sh, tbase);
-        }
-        // A broken pipeline (an mbarrier wait ran out) ends this CTA's work and the call's.
-        const bool broken = sh.abort_flag != 0;
-        if (broken && tid == 0) atomicExch(&a.sched->abort, 1);
-        __syncthreads();
-        if (broken) break;
-    }
-    tc_fence_before();
-    __syncthreads();
     if (warp == 1) tmem_dealloc(tbase, 512);
-}
-
-// Sequences without tokens: the final state is the initial state (or zero).
-__global__ void __launch_bounds__(256) k_tc_empty_final(const int32_t* __restrict__ first, const float* __restrict__ init,
-                                                       float* __restrict__ final_state, int nseq, int64_t per_seq) {
-    for (int s = blockIdx.x; s < nseq; s += gridDim.x) {
-        if (first[s] != first[s + 1]) continue;
-        float* dst = final_state + (int64_t)s * per_seq;
-        const float* src = init ? init + (int64_t)s * per_seq : nullptr;
-        for (int64_t e = threadIdx.x; e < per_seq; e += blockDim.x) dst[e] = src ? src[e] : 0.f;
-    }
-}
-
-// Zero the call's scheduling words and flags (runs before k_tc_prefill on the stream).
-__global__ void __launch_bounds__(256) k_tc_prepare(TcSched* sched, int32_t* flags, int64_t nflags) {
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i == 0) {
-        sched->ticket = 0;
-        sched->abort = 0;
-    }
-    for (int64_t k = i; k < nflags; k += (int64_t)gridDim.x * blockDim.x) flags[k] = 0;
 }
 
 }  // namespace tc

@@ -85,11 +85,8 @@ _lib.ssd_last_error.argtypes = []
 _lib.ssd_last_error.restype = ctypes.c_char_p
 _lib.ssd_scan_fwd_variant.argtypes = [ctypes.POINTER(SSDDims), ctypes.c_int]
 _lib.ssd_scan_fwd_variant.restype = ctypes.c_char_p
-_lib.ssd_test_flag_waits.argtypes = [ctypes.c_int64, ctypes.c_int]
-_lib.ssd_test_flag_waits.restype = ctypes.c_int
 _lib.ssd_set_segment_tokens.argtypes = [ctypes.c_int]
-_lib.ssd_set_ticket_lag.argtypes = [ctypes.c_int]
-_lib.ssd_set_ticket_lag.restype = None
+
 _lib.ssd_set_segment_tokens.restype = None
 _lib.ssd_scan_fwd_segment_tokens.argtypes = [ctypes.POINTER(SSDDims), ctypes.c_int]
 _lib.ssd_scan_fwd_segment_tokens.restype = ctypes.c_int
@@ -209,20 +206,9 @@ def scan_variant(dims: SSDDims, chunk: int) -> str:
     return _lib.ssd_scan_fwd_variant(ctypes.byref(dims), int(chunk)).decode()
 
 
-def test_flag_waits(budget_cycles: int = 0, publish: bool = True) -> None:
-    """Test hook: bound (in SM cycles) of the prefill's waits for other CTAs' segment
-    states, and whether those are published (see ssd_test_flag_waits in ssd.h)."""
-    _check(_lib.ssd_test_flag_waits(int(budget_cycles), 1 if publish else 0))
-
-
 def set_segment_tokens(tokens: int) -> None:
     """Force the tensor-core segment length for later calls (0 restores the planner)."""
     _lib.ssd_set_segment_tokens(int(tokens))
-
-
-def set_ticket_lag(blocks: int) -> None:
-    """Tuning knob: lag of the prefill's chunk-scan items behind its segment-state items."""
-    _lib.ssd_set_ticket_lag(int(blocks))
 
 
 def segment_tokens(dims: SSDDims, chunk: int) -> int:

@@ -144,10 +144,10 @@ def test_strict_entry_points_fail_closed_on_host(ssd):
 
 
 @pytest.mark.parametrize("batch,seqlen,H,G,expect", [
-    (1, 65536, 64, 8, 2048),      # 32 segments x 48 items: over six items per SM, L2-sized segments
-    (4, 4096, 64, 8, 512),        # 2048 would give 8 segments (384 items, under six per SM)
+    (1, 65536, 64, 8, 7296),      # 9 segments of 57 chunks: 288 chunk-scan CTAs, about two full waves
+    (4, 4096, 64, 8, 2048),       # 8 segments: 256 chunk-scan CTAs, 128 segment-state CTAs
     (256, 2048, 64, 8, 2048),     # one segment per sequence
-    (1, 2049, 8, 2, 256),         # small problem: shortest segments
+    (1, 2049, 8, 2, 256),         # small problem: shortest segments, every CTA in one wave
 ])
 def test_dense_segment_planner(ssd, batch, seqlen, H, G, expect):
     """The tensor-core segment length chosen for dense batches (host logic, no GPU; 148 SMs
@@ -158,11 +158,11 @@ def test_dense_segment_planner(ssd, batch, seqlen, H, G, expect):
 
 
 def test_varlen_segment_planner(ssd):
-    """Packed calls: the same rule on the upper bound of the segment count."""
+    """Packed calls: the longest power-of-two segment whose chunk-scan grid fills a wave."""
     d = ssd.make_dims(68177, 64, 64, 8, 128, ssd.SSD_DTYPE_BF16, nseq=16)
-    assert ssd.segment_tokens(d, 128) == 2048
+    assert ssd.segment_tokens(d, 128) == 8192
     d = ssd.make_dims(3000, 64, 64, 8, 128, ssd.SSD_DTYPE_BF16, nseq=2)
-    assert ssd.segment_tokens(d, 128) == 256
+    assert ssd.segment_tokens(d, 128) == 512
 
 
 def test_segment_override(ssd):
@@ -172,10 +172,10 @@ def test_segment_override(ssd):
         ssd.set_segment_tokens(384)
         assert ssd.segment_tokens(d, 256) == 384
         ssd.set_segment_tokens(100)        # not a multiple of 128: planner again
-        assert ssd.segment_tokens(d, 256) == 2048
+        assert ssd.segment_tokens(d, 256) == 7296
     finally:
         ssd.set_segment_tokens(0)
-    assert ssd.segment_tokens(d, 256) == 2048
+    assert ssd.segment_tokens(d, 256) == 7296
 
 
 def test_strict_binding_checks_before_the_library(ssd):

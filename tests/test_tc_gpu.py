@@ -81,30 +81,12 @@ def test_tc_zero_init_wide_dt(ssd, cuda_dev):
 
 
 @pytest.mark.parametrize("seqlens,H,G,seg", [
-    ([3000, 2000, 1], 8, 2, 128),      # 41 segments x 6 items: every CTA runs several items
-    ([1024, 1000], 64, 8, 128),        # 16 segments x 48 items, both item kinds back to back
-    ([4096] * 4, 64, 8, 512),          # the batched workload's shape and planner choice
+    ([3000, 2000, 1], 8, 2, 128),      # 41 one-chunk segments: the longest chains, more CTAs than SMs
+    ([1024, 1000], 64, 8, 128),        # 16 segments of all 64 heads: 512 chunk-scan CTAs
+    ([4096] * 4, 64, 8, 512),          # the batched workload's shape with 512-token segments
 ])
-def test_tc_many_items_per_cta(ssd, cuda_dev, seqlens, H, G, seg, segment_tokens):
-    """More work items than CTAs: each persistent CTA runs state and scan items in turn,
-    reusing its barriers, shared memory and TMEM between them."""
+def test_tc_many_segments(ssd, cuda_dev, seqlens, H, G, seg, segment_tokens):
+    """Many short segments: grids of several waves in both passes and long segment chains."""
     segment_tokens(seg)
     _check(ssd, cuda_dev, _tc_wl(seqlens, len(set(seqlens)) > 1, H=H, G=G, seed=48))
 
-
-def test_flag_wait_timeout_fails_closed(ssd, cuda_dev, segment_tokens):
-    """Segment states that are never published: every wait for one runs out after a short
-    bound, the call reports SSD_ERR_TIMEOUT through ssd_get_device_status (no hang, no
-    fault), and the next call, with the defaults restored, is correct again."""
-    w = _tc_wl([3000, 2000], True, seed=49)
-    segment_tokens(256)
-    inp = W.make_all(w)
-    try:
-        ssd.test_flag_waits(200_000, publish=False)        # about 0.1 ms per wait
-        run_gpu_scan(ssd, w, inp, cuda_dev)
-        with pytest.raises(ssd.SSDError, match="TIMEOUT"):
-            ssd.device_status()
-    finally:
-        ssd.test_flag_waits(0, publish=True)
-    ssd.device_status()                                    # the error word was cleared
-    _check(ssd, cuda_dev, w)
