@@ -219,9 +219,14 @@ ssd_status ssd_gated_rmsnorm(const void* y, const void* z, const float* weight, 
  * cudaMallocAsync. It calls no cudaMalloc, cudaFree or other allocating routine.
  *   - Size limit: if the problem needs more scratch than 32 MiB (see
  *     ssd_scan_fwd_workspace_size) it returns SSD_ERR_UNSUPPORTED and launches nothing.
+ *     Of the named workloads the tiny, batched (4 x 4096) and long-context (1 x 65536)
+ *     prefills fit; the 16-sequence packed prefill (about 48 MiB: a segment state per
+ *     sequence and segment) is refused.
  *   - Every GPU that loads the library holds those 32 MiB until the process exits.
- *   - The first call on each device looks up the array's device address (with that
- *     device current); make that first call before any stream capture.
+ *   - Each call made outside stream capture looks up the array's device address (with
+ *     the device current); a call during capture reuses the device's last lookup, so
+ *     make the first call on each device before any stream capture (a first call during
+ *     capture returns SSD_ERR_UNSUPPORTED).
  *   - All calls share the one array and it keeps the last call's contents: calls whose
  *     work can overlap on the GPU (different streams, or different host threads on one
  *     device) race on it and must be serialised by the caller. Nothing in it needs

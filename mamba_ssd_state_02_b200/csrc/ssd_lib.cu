@@ -754,7 +754,8 @@ namespace {
 
 // Scratch compiled into the library: every GPU that loads libssd holds these 32 MiB
 // until the process exits. Host code must not pass the symbol itself to a kernel (on
-// the host it is only a stand-in); the device address is looked up once per device.
+// the host it is only a stand-in); the device address is looked up with the device
+// current.
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
@@ -762,19 +763,27 @@ constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void* g_noalloc_addr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device (looked up on the first
-// call per device, with that device current).
-ssd_status noalloc_scratch(char** out) {
+// Device address of the scratch array on the current device. It is looked up on every
+// call made outside stream capture (cheap), so a context that was reset and re-created
+// since an earlier call gets the address in its own module; during capture the address
+// of the device's last lookup is used (so the first call on a device must come before
+// any capture).
+ssd_status noalloc_scratch(cudaStream_t st, char** out) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     if (dev < 0 || dev >= kMaxDevices) return fail(SSD_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    e = cudaStreamIsCapturing(st, &cap);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_addr[dev]) {
+    if (cap == cudaStreamCaptureStatusNone) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
         g_noalloc_addr[dev] = p;
+    } else if (!g_noalloc_addr[dev]) {
+        return fail(SSD_ERR_UNSUPPORTED, "first ssd_scan_fwd_noalloc call on device %d made during stream capture", dev);
     }
     *out = static_cast<char*>(g_noalloc_addr[dev]);
     return SSD_OK;
@@ -810,10 +819,10 @@ extern "C" ssd_status ssd_scan_fwd_noalloc(const void* x, const float* dt_raw, c
         t_last_error.clear();
         return SSD_OK;
     }
-    char* ws = nullptr;
-    s = noalloc_scratch(&ws);
-    if (s != SSD_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    char* ws = nullptr;
+    s = noalloc_scratch(st, &ws);
+    if (s != SSD_OK) return s;
     // Every slot of the scratch that a kernel reads is written earlier in the same call
     // (chunk/segment table, then states), so nothing needs clearing between calls.
     if (pl.tc)

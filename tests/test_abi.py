@@ -194,3 +194,20 @@ def test_strict_binding_checks_before_the_library(ssd):
     bad.len = torch.zeros(3, 8, dtype=torch.int32)
     with pytest.raises(ValueError):
         bad._check(2, 8, 64, 2, 128, torch.bfloat16, torch.device("cpu"))
+
+
+def test_noalloc_scratch_fits_the_named_prefill_workloads_except_packed(ssd):
+    """ssd_scan_fwd_noalloc has 32 MiB of scratch: the tiny, batched and long-context
+    workloads fit; the 16-sequence packed workload (one segment state per sequence and
+    per segment) does not, so that entry point refuses it (host logic, no GPU)."""
+    from mamba_ssd_state_02_b200 import workloads as W
+    limit = 32 << 20
+    for k in (0, 1, 2, 3):
+        w = W.config(k)
+        code = ssd.SSD_DTYPE_BF16 if w.dtype.itemsize == 2 else ssd.SSD_DTYPE_F32
+        if w.varlen:
+            d = ssd.make_dims(w.total_tokens, w.nheads, w.headdim, w.ngroups, w.dstate, code, nseq=w.nseq)
+        else:
+            d = ssd.make_dims(w.total_tokens, w.nheads, w.headdim, w.ngroups, w.dstate, code,
+                              batch=w.nseq, seqlen=w.seqlens[0])
+        assert (ssd.workspace_size(d, w.chunk) <= limit) == (k != 3), k

@@ -6,10 +6,11 @@ latency-critical loops where a cudaMalloc/cudaFree (or a caching allocator's slo
 in the middle of a step is not acceptable. For them the library offers
 ssd_scan_fwd_noalloc, which takes its scratch from an array compiled into the library.
 
-These tests call it through the C ABI and check that it gives the same outputs as
-ssd_scan_fwd, on two calls in a row with different problems (so the second call cannot
-lean on what the first left in the shared scratch), and that it refuses a problem whose
-scratch would not fit. This file is collected last on purpose.
+These tests call it through the C ABI and check that it gives bit for bit the same
+outputs as ssd_scan_fwd (both run the same deterministic kernels), on calls in a row with
+different problems (so a later call cannot lean on what an earlier one left in the shared
+scratch: segment tables, orders and states of a larger problem), and that it refuses a
+problem whose scratch would not fit. This file is collected last on purpose.
 """
 import ctypes
 
@@ -17,7 +18,7 @@ import pytest
 import torch
 
 from mamba_ssd_state_02_b200 import workloads as W
-from parity_util import TOL_STATE, TOL_Y, rel_err
+from parity_util import TOL_STATE, TOL_Y, oracle_scan, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -54,8 +55,31 @@ def test_noalloc_matches_scan_fwd_on_two_calls_in_a_row(ssd, cuda_dev):
         outs.append(_call(ssd.scan_fwd_noalloc, w, d))
     ssd.device_status()
     for (w, _), (y_ref, f_ref), (y, f) in zip(cases, refs, outs):
-        assert rel_err(y, y_ref) <= TOL_Y[w.dtype]
-        assert rel_err(f, f_ref) <= TOL_STATE
+        assert torch.equal(y, y_ref)
+        assert torch.equal(f, f_ref)
+
+
+def test_noalloc_smaller_tensor_core_call_after_a_larger_one(ssd, cuda_dev):
+    # A larger packed problem (more sequences, more segments, longer segment table and
+    # segment order) leaves its tables and states in the shared scratch; the smaller one
+    # after it, with other lengths, must not read any of them.
+    big_w, big = _case(cuda_dev, [2600, 5, 1300, 4100, 640], True, torch.bfloat16, 8, 64, 2, 128, 128,
+                       "normal", 93)
+    small_w, small = _case(cuda_dev, [900, 333], True, torch.bfloat16, 8, 64, 2, 128, 128, "normal", 94)
+    ssd.set_segment_tokens(256)                 # many segments in both calls
+    try:
+        y_ref, f_ref = _call(ssd.scan_fwd, small_w, small)
+        y_ref, f_ref = y_ref.clone(), f_ref.clone()
+        _call(ssd.scan_fwd_noalloc, big_w, big)
+        y, f = _call(ssd.scan_fwd_noalloc, small_w, small)
+        ssd.device_status()
+    finally:
+        ssd.set_segment_tokens(0)
+    assert torch.equal(y, y_ref)
+    assert torch.equal(f, f_ref)
+    y_o, f_o = oracle_scan(small_w, small)
+    assert rel_err(y, y_o) <= TOL_Y[small_w.dtype]
+    assert rel_err(f, f_o) <= TOL_STATE
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch(ssd, cuda_dev):
