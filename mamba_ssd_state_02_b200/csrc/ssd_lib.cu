@@ -7,6 +7,7 @@
 
 #include <cstdarg>
 #include <cstdio>
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 #include <string>
@@ -1072,6 +1073,8 @@ ssd_status launch_strict(const Plan& pl, char* ws, const T* x, const float* dt_r
     }
     ++n;
     const unsigned mc = (unsigned)pl.max_chunks;
+    if ((int64_t)mc * std::max<int64_t>(H, (int64_t)G * (Q / 32)) >= INT32_MAX)
+        return fail(SSD_ERR_UNSUPPORTED, "too many chunks for one strict call (%u chunks x %d heads)", mc, H);
     if (mc > 0) {
         {
             StageScope sc(ST_STRICT_CUMSUM, st);
@@ -1080,7 +1083,7 @@ ssd_status launch_strict(const Plan& pl, char* ws, const T* x, const float* dt_r
         }
         {
             StageScope sc(ST_STRICT_STATE, st);
-            const dim3 grid(mc, H);
+            const unsigned grid = (unsigned)((int64_t)mc * H);
             const size_t sm = chunk_state_smem(P, N, Q);
             switch (P * N / kThreads) {
 #define SSD_NOUT(V)                                                                                        \
@@ -1102,8 +1105,8 @@ ssd_status launch_strict(const Plan& pl, char* ws, const T* x, const float* dt_r
     ++n;
     if (mc > 0) {
         StageScope sc(ST_STRICT_SCAN, st);
-        scan_kernel<<<dim3(mc, G, Q / 32), kThreads, scan_smem, st>>>(x, B, C, D, dtc, acum, states, table,
-                                                                      count, H, G, N, Q, y);
+        scan_kernel<<<(unsigned)((int64_t)mc * G * (Q / 32)), kThreads, scan_smem, st>>>(
+            x, B, C, D, dtc, acum, states, table, count, H, G, N, Q, y);
         ++n;
     }
     {

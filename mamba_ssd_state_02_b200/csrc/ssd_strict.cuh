@@ -126,9 +126,10 @@ k_strict_chunk_state(const T* __restrict__ x, const T* __restrict__ B, const flo
     float* w = sm;                       // [Q]
     float* xs = w + Q;                   // [32][P]   w(last, s) x_s
     float* bs = xs + 32 * P;             // [32][N]
-    const int c = blockIdx.x;
+    // Block b: head b % H of chunk b / H, so the heads of one chunk run side by side (B in L2).
+    const int c = (int)(blockIdx.x / (unsigned)H);
     if (c >= *count) return;
-    const int h = blockIdx.y, g = h / (H / G), tid = threadIdx.x;
+    const int h = (int)(blockIdx.x % (unsigned)H), g = h / (H / G), tid = threadIdx.x;
     const ChunkEntry e = table[c];
     const float* ac = acum + ((int64_t)c * H + h) * Q;
     const float* dv = dtc + ((int64_t)c * H + h) * Q;
@@ -181,14 +182,28 @@ k_strict_passing(float* __restrict__ states, const float* __restrict__ acum, con
     }
     const int c0 = first[s], c1 = first[s + 1];
     float open = hv;
-    for (int c = c0; c < c1; ++c) {
-        const ChunkEntry e = table[c];
-        float* slot = states + ((int64_t)c * H + h) * PN + i;
-        const float sv = *slot;
-        *slot = hv;
-        open = hv;
-        hv = pass(hv, acum[((int64_t)c * H + h) * Q + e.len - 1], sv);
-        if (e.len == Q) open = hv;
+    // Four chunks' loads are issued before the four dependent updates (same arithmetic).
+    constexpr int U = 4;
+    for (int c = c0; c < c1; c += U) {
+        float sv[U], al[U];
+        int len[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (c + u < c1) {
+                len[u] = table[c + u].len;
+                sv[u] = states[((int64_t)(c + u) * H + h) * PN + i];
+                al[u] = acum[((int64_t)(c + u) * H + h) * Q + len[u] - 1];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            if (c + u < c1) {
+                states[((int64_t)(c + u) * H + h) * PN + i] = hv;
+                open = hv;
+                hv = pass(hv, al[u], sv[u]);
+                if (len[u] == Q) open = hv;
+            }
+        }
     }
     cache_state[slot0] = open;
     if (final_state) final_state[slot0] = hv;
@@ -231,12 +246,15 @@ k_strict_chunk_scan(const T* __restrict__ x, const T* __restrict__ B, const T* _
     float* dts = acs + Q;                 // [Q]
     float* hs = dts + Q;                  // [P][36]
     float* xs = hs + P * kHPad;           // [32][P]
-    const int c = blockIdx.x;
+    // Block b: tile b % (Q/32), group (b / (Q/32)) % G, chunk b / ((Q/32) G): the tiles of
+    // one (chunk, group) run side by side and share its B, incoming states and x in L2.
+    const int ntile = Q / 32;
+    const int c = (int)(blockIdx.x / (unsigned)(ntile * G));
     if (c >= *count) return;
     const ChunkEntry e = table[c];
-    const int t0 = blockIdx.z * 32;
+    const int t0 = (int)(blockIdx.x % (unsigned)ntile) * 32;
     if (t0 >= e.len) return;
-    const int g = blockIdx.y, hpg = H / G, tid = threadIdx.x;
+    const int g = (int)((blockIdx.x / (unsigned)ntile) % (unsigned)G), hpg = H / G, tid = threadIdx.x;
     const int rows = min(32, e.len - t0);
     for (int i = tid; i < 32 * N; i += kThreads) {
         const int r = i / N, nn = i % N;
@@ -340,29 +358,45 @@ k_strict_chunk_scan(const T* __restrict__ x, const T* __restrict__ B, const T* _
                 xs[i] = r < srows ? to_f32(x[((int64_t)(e.start + s0 + r) * H + h) * P + pp]) : 0.f;
             }
             __syncthreads();
+            // Coefficients of four consecutive sources are read with one 16-byte load per
+            // row; the sources are still added one at a time, left to right.
             if (s0 < t0) {                // every row of the tile sees all 32 sources
-                for (int ss = 0; ss < 32; ++ss) {
-                    float xv[TB];
+                for (int s4 = 0; s4 < 32; s4 += 4) {
+                    float4 cf4[TA];
 #pragma unroll
-                    for (int j = 0; j < TB; ++j) xv[j] = xs[ss * P + pg + j * PG];
+                    for (int i = 0; i < TA; ++i) cf4[i] = *reinterpret_cast<const float4*>(ms + (rg * TA + i) * Q + s0 + s4);
 #pragma unroll
-                    for (int i = 0; i < TA; ++i) {
-                        const float cf = ms[(rg * TA + i) * Q + s0 + ss];
+                    for (int k = 0; k < 4; ++k) {
+                        float xv[TB];
 #pragma unroll
-                        for (int j = 0; j < TB; ++j) acc[i][j] = y_step(acc[i][j], cf, xv[j]);
+                        for (int j = 0; j < TB; ++j) xv[j] = xs[(s4 + k) * P + pg + j * PG];
+#pragma unroll
+                        for (int i = 0; i < TA; ++i) {
+                            const float cf = k == 0 ? cf4[i].x : k == 1 ? cf4[i].y : k == 2 ? cf4[i].z : cf4[i].w;
+#pragma unroll
+                            for (int j = 0; j < TB; ++j) acc[i][j] = y_step(acc[i][j], cf, xv[j]);
+                        }
                     }
                 }
             } else {                      // diagonal slice: sources s <= t, s < len
-                for (int ss = 0; ss < srows; ++ss) {
-                    float xv[TB];
+                for (int s4 = 0; s4 < srows; s4 += 4) {
+                    float4 cf4[TA];
 #pragma unroll
-                    for (int j = 0; j < TB; ++j) xv[j] = xs[ss * P + pg + j * PG];
+                    for (int i = 0; i < TA; ++i) cf4[i] = *reinterpret_cast<const float4*>(ms + (rg * TA + i) * Q + s0 + s4);
 #pragma unroll
-                    for (int i = 0; i < TA; ++i) {
-                        if (ss > rg * TA + i) continue;
-                        const float cf = ms[(rg * TA + i) * Q + s0 + ss];
+                    for (int k = 0; k < 4; ++k) {
+                        const int ss = s4 + k;
+                        if (ss >= srows) break;
+                        float xv[TB];
 #pragma unroll
-                        for (int j = 0; j < TB; ++j) acc[i][j] = y_step(acc[i][j], cf, xv[j]);
+                        for (int j = 0; j < TB; ++j) xv[j] = xs[ss * P + pg + j * PG];
+#pragma unroll
+                        for (int i = 0; i < TA; ++i) {
+                            if (ss > rg * TA + i) continue;
+                            const float cf = k == 0 ? cf4[i].x : k == 1 ? cf4[i].y : k == 2 ? cf4[i].z : cf4[i].w;
+#pragma unroll
+                            for (int j = 0; j < TB; ++j) acc[i][j] = y_step(acc[i][j], cf, xv[j]);
+                        }
                     }
                 }
             }
