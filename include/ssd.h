@@ -3,8 +3,8 @@
  * step, for NVIDIA B200 (sm_100a).
  *
  * The operation. For every sequence and head h (group g = h / (H/G), heads share B
- * and C within a group "like GQA": JAX Nemotron 3 Nano page, NemotronConfig
- * `mamba_ngroups`), token by token:
+ * and C within a group, as keys/values are shared in grouped-query attention: JAX
+ * Nemotron 3 Nano page, NemotronConfig `mamba_ngroups`), token by token:
  *
  *     dt_t   = softplus(dt_raw[t,h] + dt_bias[h])          RL-Kernel issue page, Figure 2
  *     h_t    = exp(dt_t * A[h]) * h_{t-1} + dt_t * x_t B_t^T      (FP32 state, ibid. §1)
@@ -12,11 +12,11 @@
  *                                                                  "Key Components")
  *
  * starting from the caller's initial state (or zero). Prefill evaluates this with
- * the chunked SSD algorithm (JAX page, "Key Components" 1: "Chunked SSD algorithm
- * keeps memory usage bounded"; RL-Kernel issue page, Figure 2: "SSD chunked scan"),
- * decode with the per-token recurrent update (RL-Kernel issue page, §1 and §2:
- * causal_conv1d_update + selective_state_update). The state is stored [P][N] with N
- * contiguous (the transpose of B x^T).
+ * the chunked SSD algorithm, whose memory stays bounded by the chunk size (JAX page,
+ * "Key Components" 1; RL-Kernel issue page, Figure 2, the chunked SSD scan box),
+ * decode with the per-token recurrent update (RL-Kernel issue page, §1 and §2: the
+ * conv-state update followed by the selective state update). The state is stored
+ * [P][N] with N contiguous (the transpose of B x^T).
  *
  * Conventions shared by every entry point:
  *   - All tensor pointers are DEVICE pointers owned by the caller; the library never
@@ -33,7 +33,7 @@
  *     error word that ssd_get_device_status() reads and clears.
  *   - Fail closed: geometry outside the supported set returns SSD_ERR_UNSUPPORTED
  *     and nothing is launched; there is no CPU or other fallback (RL-Kernel issue
- *     page, §4.1 "fail closed on unsupported strict geometry" and §7).
+ *     page, §4.1 and §7: unsupported geometry is refused rather than approximated).
  *   - Functions are thread-safe; ssd_last_error() is per host thread.
  */
 #ifndef SSD_H
@@ -101,8 +101,8 @@ ssd_status ssd_scan_fwd_workspace_size(const ssd_dims* dims, int chunk, size_t* 
  *   init_state: [nseq,H,P,N] float32, or NULL for zero initial states.
  *   cu_seqlens: [nseq+1] int32 device array, or NULL for dense mode. Chunks are
  *     anchored at each sequence start and the state never crosses a sequence
- *     boundary (RL-Kernel issue page, §7 "sequence-anchored chunks", §8 Q4
- *     "cu_seqlens-aware chunking"); a sequence's last chunk may be partial.
+ *     boundary (RL-Kernel issue page, §7: chunks start where sequences start; §8 Q4:
+ *     chunking follows cu_seqlens); a sequence's last chunk may be partial.
  *   y: [T,H,P] output, same dtype as x (bf16 rounded to nearest even).
  *   final_state: [nseq,H,P,N] float32 output (the state after each sequence's last
  *     token; the initial state for an empty sequence), or NULL.

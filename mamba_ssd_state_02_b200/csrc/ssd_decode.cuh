@@ -1,6 +1,6 @@
-// Decode: one recurrent state update per sequence (RL-Kernel issue page, §1: "rollout
-// decode computes it as a per-token recurrent state update"; §2: the decode path is
-// causal_conv1d_update + selective_state_update).
+// Decode: one recurrent state update per sequence and token (RL-Kernel issue page, §1:
+// rollout decode advances the SSM state one token at a time; §2: the upstream decode
+// path is the conv-state update followed by the selective state update).
 //
 //   dt = softplus(dt_raw + dt_bias[h]);  h <- exp(dt*A[h]) h + dt x B^T;  y = h.C + D x
 //

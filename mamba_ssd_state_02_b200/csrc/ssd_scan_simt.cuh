@@ -1,7 +1,7 @@
 // Chunked SSD prefill, CUDA-core FP32 pipeline (all dtypes and supported dims).
 //
 // The chunked SSD algorithm (JAX Nemotron 3 Nano page, "Key Components" 1; RL-Kernel
-// issue page, Figure 2 "SSD chunked scan") splits each sequence into chunks of Q
+// issue page, Figure 2, the chunked-scan box) splits each sequence into chunks of Q
 // tokens anchored at the sequence start and evaluates the recurrence as:
 //
 //   chunk_cumsum   dt_s = softplus(dt_raw_s + dt_bias), Acum_s = sum_{r<=s in chunk} dt_r A

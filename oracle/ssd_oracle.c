@@ -6,10 +6,11 @@
  * it. It shares no code, header, table or constant with the CUDA library.
  *
  * What it computes (the recurrence the SSD pages define):
- *   per sequence s and head h, with group g = h / (H / G)      (B/C shared by head
- *   groups "like GQA", JAX Nemotron 3 Nano page, NemotronConfig `mamba_ngroups`):
+ *   per sequence s and head h, with group g = h / (H / G)      (B/C shared by groups
+ *   of heads, as keys/values are in grouped-query attention: JAX Nemotron 3 Nano page,
+ *   NemotronConfig `mamba_ngroups`):
  *     dt_t   = softplus(dt_raw[t,h] + dt_bias[h])              (RL-Kernel issue page,
- *                                                               Figure 2, "softplus(dt + dt_bias)")
+ *                                                               Figure 2: softplus of dt plus its bias)
  *     h_t    = exp(dt_t * A[h]) * h_{t-1} + dt_t * x_t B_t^T   (the SSD recurrence, FP32
  *                                                               state: RL-Kernel issue §1)
  *     y_t[p] = sum_n C_t[n] h_t[p][n] + D[h] x_t[p]            (D skip: JAX page,
