@@ -74,6 +74,11 @@ struct Plan {
     int64_t snap = 0;
     size_t off_snap_first = 0;
     float* snap_out = nullptr;
+    // tc with snapshots: segments cut at the snapshot positions into sub-segments, one
+    // state slot each (at most max_segs + T / snap); per-sequence first sub-segment and
+    // each sub-segment's end (tokens from its sequence's start)
+    int64_t max_subs = 0;
+    size_t off_sub_first = 0, off_sub_end = 0;
 };
 
 }  // namespace ssd

@@ -244,15 +244,14 @@ ssd_status make_plan(const ssd_dims* d, int chunk, bool varlen, Plan* pl, int64_
             }
         }
         if (const int v = g_segment_override.load()) Ls = v;
-        if (snap > 0) {                 // segment boundaries must fall on every snapshot
-            if (snap % tc::kTile != 0)
-                return fail(SSD_ERR_UNSUPPORTED, "snapshot_tokens (%lld) must be a multiple of %d here",
-                            (long long)snap, tc::kTile);
-            if (snap < Ls) Ls = (int)snap;
-            while (snap % Ls != 0) Ls -= tc::kTile;
-        }
+        // Snapshots cut the segments' states at multiples of snap (sub-segments), which
+        // must fall on 128-token chunk boundaries; the segment length stays as chosen.
+        if (snap > 0 && snap % tc::kTile != 0)
+            return fail(SSD_ERR_UNSUPPORTED, "snapshot_tokens (%lld) must be a multiple of %d here",
+                        (long long)snap, tc::kTile);
         p.Ls = Ls;
         p.max_segs = segs_for(Ls);
+        p.max_subs = p.max_segs + (snap > 0 ? p.T / snap : 0);
     }
     if (snap < 0) return fail(SSD_ERR_INVALID_ARG, "snapshot_tokens must be >= 0");
     if (snap > 0 && !p.tc && snap % chunk != 0)
@@ -267,13 +266,17 @@ ssd_status make_plan(const ssd_dims* d, int chunk, bool varlen, Plan* pl, int64_
         return o;
     };
     if (p.tc) {
-        const size_t ms = (size_t)p.max_segs;
+        const size_t ms = (size_t)p.max_segs, mu = (size_t)p.max_subs;
         p.off_table = take(sizeof(ChunkEntry) * (ms > 0 ? ms : 1));
         p.off_first = take(sizeof(int32_t) * ((size_t)p.nseq + 1));
         p.off_count = take(sizeof(int32_t));
-        p.off_states = take(sizeof(float) * ms * p.H * p.P * p.N);
-        p.off_seg_acum = take(sizeof(float) * ms * p.H);
+        p.off_states = take(sizeof(float) * mu * p.H * p.P * p.N);
+        p.off_seg_acum = take(sizeof(float) * mu * p.H);
         p.off_order = take(sizeof(int32_t) * (ms > 0 ? ms : 1));
+        if (snap > 0) {
+            p.off_sub_first = take(sizeof(int32_t) * ((size_t)p.nseq + 1));
+            p.off_sub_end = take(sizeof(int32_t) * (mu > 0 ? mu : 1));
+        }
     } else {
         const size_t mc = (size_t)p.max_chunks;
         p.off_table = take(sizeof(ChunkEntry) * (mc > 0 ? mc : 1));
@@ -358,13 +361,17 @@ ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_ra
     auto* seg_state = reinterpret_cast<float*>(ws + pl.off_states);
     auto* seg_acum = reinterpret_cast<float*>(ws + pl.off_seg_acum);
     int32_t* order = pl.varlen ? reinterpret_cast<int32_t*>(ws + pl.off_order) : nullptr;
+    // with snapshots the chain walks sub-segments (slot ranges sub_first), else segments
+    int32_t* sub_first = pl.snap > 0 ? reinterpret_cast<int32_t*>(ws + pl.off_sub_first) : nullptr;
+    int32_t* sub_end = pl.snap > 0 ? reinterpret_cast<int32_t*>(ws + pl.off_sub_end) : nullptr;
+    const int32_t* slot_first = sub_first ? sub_first : first;
     const int H = pl.H, G = pl.G;
     int n = 0;
     {
         StageScope sc(ST_TABLE, st);
         k_chunk_table<<<1, kTableThreads, 0, st>>>(cu, pl.nseq, pl.T, pl.seqlen, pl.Ls, table, first, count,
                                                    pl.snap, reinterpret_cast<int32_t*>(ws + pl.off_snap_first),
-                                                   order);
+                                                   order, sub_first, sub_end);
     }
     ++n;
     if (pl.max_segs > 0 && pl.T > 0) {
@@ -384,13 +391,13 @@ ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_ra
             StageScope sc(ST_CHUNK_STATE, st);
             tc::k_tc_segment_state<<<(unsigned)(pl.max_segs * (H / tc::kHeads)), tc::kThreadsA, tc::kSmemA,
                                      st>>>(mx, mb, dt_raw, dt_bias, A, table, count, H, G,
-                                                                  seg_state, seg_acum, order);
+                                                                  seg_state, seg_acum, order, first, pl.snap);
         }
         ++n;
         {
             StageScope sc(ST_STATE_PASSING, st);
-            tc::k_tc_segment_passing<<<dim3(pl.nseq, H, tc::kN / tc::kPassN), 256, 0, st>>>(
-                seg_state, seg_acum, first, init, fin, H, table, pl.snap,
+            tc::k_tc_segment_passing<<<dim3(pl.nseq, H, tc::kP * tc::kN / tc::kPassElems), 256, 0, st>>>(
+                seg_state, seg_acum, slot_first, init, fin, H, pl.Ls, pl.snap, sub_end,
                 reinterpret_cast<const int32_t*>(ws + pl.off_snap_first), pl.snap_out);
         }
         ++n;
@@ -402,9 +409,9 @@ ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_ra
         ++n;
     } else {
         StageScope sc(ST_STATE_PASSING, st);
-        tc::k_tc_segment_passing<<<dim3(pl.nseq, H, tc::kN / tc::kPassN), 256, 0, st>>>(
-            seg_state, seg_acum, first, init, fin, H, table, pl.snap,
-                reinterpret_cast<const int32_t*>(ws + pl.off_snap_first), pl.snap_out);
+        tc::k_tc_segment_passing<<<dim3(pl.nseq, H, tc::kP * tc::kN / tc::kPassElems), 256, 0, st>>>(
+            seg_state, seg_acum, slot_first, init, fin, H, pl.Ls, pl.snap, sub_end,
+            reinterpret_cast<const int32_t*>(ws + pl.off_snap_first), pl.snap_out);
         ++n;
     }
     cudaError_t e = cudaGetLastError();

@@ -28,14 +28,50 @@ namespace ssd {
 // With `order` (entries of at most 128 chunks of 128 tokens), order[k] is the entry the
 // k-th CTA of a pass takes: longest entries first (by 128-token chunks), so that CTAs of
 // unequal length finish together (longest-processing-time-first scheduling).
+// An entry's `pad` holds its index in the table. With `sub_first` (entries of the
+// tensor-core pipeline and state snapshots every `snap` tokens, snap a multiple of 128),
+// every entry is further cut at the multiples of snap that fall inside it (positions
+// counted from its sequence's start) into sub-segments, numbered in token order over the
+// whole call: `pad` becomes the number of the entry's first sub-segment, sub_first[s] that
+// of sequence s's first one (sub_first[nseq] = their count), and sub_end[k] is where
+// sub-segment k ends, counted from its sequence's start.
 constexpr int kTableThreads = 1024;
+
+// Exclusive prefix sum of v over the kTableThreads threads of the block (warp shuffles,
+// then the 32 warp totals); *total = the sum over the block. wsum: 32 shared slots, free
+// again after the next barrier.
+__device__ __forceinline__ int32_t table_scan(int32_t v, int32_t* wsum, int32_t* total) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    int32_t x = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int32_t y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x += y;
+    }
+    if (lane == 31) wsum[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+        int32_t w = wsum[lane];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int32_t y = __shfl_up_sync(0xffffffffu, w, off);
+            if (lane >= off) w += y;
+        }
+        wsum[lane] = w;
+    }
+    __syncthreads();
+    *total = wsum[31];
+    return (wid ? wsum[wid - 1] : 0) + x - v;
+}
 
 __global__ void __launch_bounds__(kTableThreads)
 k_chunk_table(const int32_t* __restrict__ cu, int32_t nseq, int64_t T, int64_t seqlen, int Q,
               ChunkEntry* __restrict__ table, int32_t* __restrict__ first,
               int32_t* __restrict__ count, int64_t snap, int32_t* __restrict__ snap_first,
-              int32_t* __restrict__ order = nullptr) {
-    __shared__ int32_t part[kTableThreads];
+              int32_t* __restrict__ order = nullptr, int32_t* __restrict__ sub_first = nullptr,
+              int32_t* __restrict__ sub_end = nullptr) {
+    static_assert(kTableThreads == 32 * 32, "table_scan assumes 32 warps");
+    __shared__ int32_t wsum[3][32];
     const int tid = threadIdx.x;
     const int per = (nseq + kTableThreads - 1) / kTableThreads;
     const int s0 = min(nseq, tid * per), s1 = min(nseq, s0 + per);
@@ -58,15 +94,8 @@ k_chunk_table(const int32_t* __restrict__ cu, int32_t nseq, int64_t T, int64_t s
         int64_t len = seq_begin(s + 1) - seq_begin(s);
         local += (int32_t)((len + Q - 1) / Q);
     }
-    part[tid] = local;
-    __syncthreads();
-    for (int off = 1; off < kTableThreads; off <<= 1) {  // inclusive Hillis-Steele scan
-        int32_t v = tid >= off ? part[tid - off] : 0;
-        __syncthreads();
-        part[tid] += v;
-        __syncthreads();
-    }
-    int32_t run = part[tid] - local;
+    int32_t nent = 0;
+    int32_t run = table_scan(local, wsum[0], &nent);
     for (int s = s0; s < s1; ++s) {
         first[s] = run;
         const int64_t b = seq_begin(s), len = seq_begin(s + 1) - b;
@@ -76,19 +105,19 @@ k_chunk_table(const int32_t* __restrict__ cu, int32_t nseq, int64_t T, int64_t s
             e.seq = s;
             e.start = (int32_t)(b + (int64_t)j * Q);
             { const int64_t rem = len - (int64_t)j * Q; e.len = (int32_t)(rem < Q ? rem : Q); }
-            e.pad = 0;
+            e.pad = run + j;
             table[run + j] = e;
         }
         run += nc;
     }
     if (tid == kTableThreads - 1) {
-        first[nseq] = part[tid];
-        *count = part[tid];
+        first[nseq] = nent;
+        *count = nent;
     }
     if (order) {                                          // counting sort by chunks, descending
         __shared__ int32_t hist[129];
         __syncthreads();                                  // every entry is written
-        const int32_t n = part[kTableThreads - 1];
+        const int32_t n = nent;
         for (int b = tid; b < 129; b += kTableThreads) hist[b] = 0;
         __syncthreads();
         for (int32_t i = tid; i < n; i += kTableThreads) atomicAdd(&hist[min(128, (table[i].len + 127) / 128)], 1);
@@ -106,23 +135,41 @@ k_chunk_table(const int32_t* __restrict__ cu, int32_t nseq, int64_t T, int64_t s
             order[atomicAdd(&hist[min(128, (table[i].len + 127) / 128)], 1)] = i;
     }
     if (snap > 0) {                                       // snapshots: floor(len / snap) per sequence
-        __syncthreads();
-        int32_t nsnap = 0;
+        int32_t nsnap = 0, tot = 0;
         for (int s = s0; s < s1; ++s) nsnap += (int32_t)((seq_begin(s + 1) - seq_begin(s)) / snap);
-        part[tid] = nsnap;
-        __syncthreads();
-        for (int off = 1; off < kTableThreads; off <<= 1) {
-            int32_t v = tid >= off ? part[tid - off] : 0;
-            __syncthreads();
-            part[tid] += v;
-            __syncthreads();
-        }
-        int32_t r2 = part[tid] - nsnap;
+        int32_t r2 = table_scan(nsnap, wsum[1], &tot);
         for (int s = s0; s < s1; ++s) {
             snap_first[s] = r2;
             r2 += (int32_t)((seq_begin(s + 1) - seq_begin(s)) / snap);
         }
-        if (tid == kTableThreads - 1) snap_first[nseq] = part[tid];
+        if (tid == kTableThreads - 1) snap_first[nseq] = tot;
+    }
+    if (snap > 0 && sub_first) {                          // sub-segments cut at multiples of snap
+        int32_t nsub = 0, tot = 0;
+        for (int s = s0; s < s1; ++s) {                   // entries plus the cuts strictly inside them
+            const int64_t len = seq_begin(s + 1) - seq_begin(s);
+            int64_t cut = snap;
+            for (int64_t r0 = 0; r0 < len; r0 += Q) {
+                const int64_t r1 = r0 + Q < len ? r0 + Q : len;
+                for (++nsub; cut < r1; cut += snap) ++nsub;
+                if (cut == r1) cut += snap;
+            }
+        }
+        int32_t k = table_scan(nsub, wsum[2], &tot);
+        for (int s = s0; s < s1; ++s) {
+            sub_first[s] = k;
+            const int64_t len = seq_begin(s + 1) - seq_begin(s);
+            int32_t c = first[s];
+            int64_t cut = snap;                                   // next multiple of snap
+            for (int64_t r0 = 0; r0 < len; r0 += Q, ++c) {
+                const int64_t r1 = r0 + Q < len ? r0 + Q : len;
+                table[c].pad = k;
+                for (; cut < r1; cut += snap) sub_end[k++] = (int32_t)cut;
+                sub_end[k++] = (int32_t)r1;
+                if (cut == r1) cut += snap;
+            }
+        }
+        if (tid == kTableThreads - 1) sub_first[nseq] = tot;
     }
 }
 

@@ -78,9 +78,10 @@ __device__ __forceinline__ float wg_scan(float a, int q, int lane, float* part) 
 }
 
 // ---------------------------------------------------------------------------------
-// Pass A: zero-start segment states S_seg (fp32, layout [seg][H][N][P]) and the
-// segment's total sum of dt*A (seg_acum[seg][H]). One CTA per (segment, 4 heads); the
+// Pass A: zero-start segment states S_seg (fp32, layout [slot][H][P][N]) and the
+// segment's total sum of dt*A (seg_acum[slot][H]). One CTA per (segment, 4 heads); the
 // chunks run from the segment end backwards so the decay to the end is a running sum.
+// With snapshots, one state and sum per piece of the segment between snapshot positions.
 //
 // Warp 0 issues the TMA loads, warp 1 the UMMAs, warps 18 and 19 scan dt of heads
 // 0-1 and 2-3 (up to four chunks ahead; w_s = exp(sum_{r > s in seg} dt_r A) dt_s), and
@@ -104,7 +105,8 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
                    const float* __restrict__ dt_raw, const float* __restrict__ dt_bias,
                    const float* __restrict__ A, const ChunkEntry* __restrict__ segs,
                    const int32_t* __restrict__ nsegs, int H, int G, float* __restrict__ seg_state,
-                   float* __restrict__ seg_acum, const int32_t* __restrict__ order) {
+                   float* __restrict__ seg_acum, const int32_t* __restrict__ order,
+                   const int32_t* __restrict__ first, int64_t snap) {
     const int nq = H / kHeads;
     if ((int)(blockIdx.x / nq) >= *nsegs) return;
     const int sg = order ? order[blockIdx.x / nq] : (int)(blockIdx.x / nq);   // longest segments first
@@ -123,6 +125,20 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
     const int h0 = (blockIdx.x % nq) * kHeads, g = h0 / (H / G);
     const ChunkEntry seg = segs[sg];
     const int ntiles = (seg.len + kTile - 1) / kTile;
+    // State slots. Without snapshots the segment has one (seg.pad). With snapshots every
+    // snap tokens the segment is cut at the multiples of snap inside it (counted from the
+    // sequence start) and each piece (sub-segment) gets its own zero-start state, in slots
+    // seg.pad, seg.pad + 1, ... in token order. Step k of the reverse walk takes chunk
+    // ntiles-1-k: it opens a piece at the piece's last chunk and closes it at its first.
+    // In 128-token chunks (segments start and snapshots fall on chunk boundaries): rc0 =
+    // the segment's first chunk within its sequence, sc = chunks per snapshot interval
+    // (0: none; capped where no sequence reaches a second interval).
+    const int sc = snap > 0 ? (int)min((int64_t)1 << 30, snap / kTile) : 0;
+    const int rc0 = sc ? (seg.start - segs[first[seg.seq]].start) / kTile : 0;
+    auto slot_of = [&](int it) -> int { return sc ? seg.pad + (rc0 + it) / sc - rc0 / sc : seg.pad; };
+    // chunk it ends a piece / starts one
+    auto opens = [&](int k) { const int it = ntiles - 1 - k; return k == 0 || (sc && (rc0 + it + 1) % sc == 0); };
+    auto closes = [&](int k) { const int it = ntiles - 1 - k; return it == 0 || (sc && (rc0 + it) % sc == 0); };
 
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
@@ -186,6 +202,7 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
             const int st = k & 1;
             wait_abort(&full_b[st], (k >> 1) & 1, abort_p);
             const uint64_t dB = smem_desc(smem_u32(sB + st * 32768), 16384, 1024);
+            const bool fresh = opens(k);            // first chunk of a piece: overwrite the accumulator
             for (int pr = 0; pr < 2; ++pr) {
                 wait_abort(&ops_ready[pr], k & 1, abort_p);
                 tc_fence_after();
@@ -194,7 +211,7 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
                 if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk)
-                        umma_bf16(d, desc_add(dB, kk * kMnStep), desc_add(dp, kk * kMnStep), idesc, !(k == 0 && kk == 0));
+                        umma_bf16(d, desc_add(dB, kk * kMnStep), desc_add(dp, kk * kMnStep), idesc, !(kk == 0 && fresh));
                     umma_commit(&pair_done[pr]);
                     if (pr == 1) umma_commit(&empty_b[st]);
                     if (pr == 1 && k == ntiles - 1) umma_commit(&all_done);
@@ -231,6 +248,7 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
         for (int k = 0; k < ntiles; ++k) {
             const int bf = k % 4, it = ntiles - 1 - k;
             const int tlk = min(kTile, seg.len - it * kTile);
+            if (opens(k)) suf[0] = suf[1] = 0.f;
 #pragma unroll
             for (int e = 0; e < 2; ++e)
 #pragma unroll
@@ -259,15 +277,40 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
                 *reinterpret_cast<float4*>(&wts[bf][hb + e][4 * lane]) = make_float4(w[0], w[1], w[2], w[3]);
                 suf[e] += tot;
             }
+            if (closes(k) && lane < 2)                          // total decay exponent of the piece
+                seg_acum[(int64_t)slot_of(it) * H + h0 + hb + lane] = (lane ? suf[1] : suf[0]) / kLog2e;
             __syncwarp();
             if (lane == 0) mbar_arrive(&w_ready[bf]);
         }
-        if (lane < 2) seg_acum[(int64_t)sg * H + h0 + hb + lane] = (lane ? suf[1] : suf[0]) / kLog2e;
     } else {
         // ------------------------------------------------------------ compute warps
         const int cw = (warp - kRoleWarps) >> 2, q = warp & 3, r = q * 32 + lane;
+        // Warpgroup cw writes the state of head cw into a slot: thread = state row n.
+        auto store_state = [&](int slot) {
+            // layout [slot][H][P][N]: for each p the warp writes 32 consecutive n
+            float* dst = seg_state + ((int64_t)slot * H + h0 + cw) * kP * kN + r;
+            const uint32_t thi = tS + ((uint32_t)(q * 32) << 16) + (cw >> 1) * 256 + (cw & 1) * 64;
+            for (int half = 0; half < 2; ++half) {
+                uint32_t vh[32], vl[32];
+                tmem_ld32(thi + half * 32, vh);
+                tmem_ld32(thi + 128 + half * 32, vl);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    dst[(half * 32 + e) * kN] = __uint_as_float(vh[e]) + __uint_as_float(vl[e]);
+            }
+        };
         for (int k = 0; k < ntiles; ++k) {
             const int bf = k % 4;
+            if (k > 0 && opens(k)) {
+                // Step k-1 closed a piece: once its UMMAs are done, store the piece's state
+                // before this step's operands are handed over (the UMMA warp waits for them
+                // and then overwrites the accumulator).
+                wait_abort(&pair_done[cw >> 1], (k - 1) & 1, abort_p);
+                tc_fence_after();
+                store_state(slot_of(ntiles - k));
+                tc_fence_before();
+            }
             wait_abort(&w_ready[bf], (k >> 2) & 1, abort_p);
             for (int pr = 0; pr < 2; ++pr) {
                 wait_abort(&full_x[pr], k & 1, abort_p);
@@ -298,24 +341,10 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
             __syncwarp();
             if (lane == 0) mbar_arrive(&w_free[bf]);
         }
-        // Wait for the last UMMAs, then write S_seg of head cw: thread = state row n.
+        // Wait for the last UMMAs, then write the state of the segment's first piece.
         wait_abort(&all_done, 0, abort_p);
         tc_fence_after();
-        float* dst = seg_state + (((int64_t)sg * H + h0 + cw) * kN + r) * kP;
-        const uint32_t thi = tS + ((uint32_t)(q * 32) << 16) + (cw >> 1) * 256 + (cw & 1) * 64;
-        for (int half = 0; half < 2; ++half) {
-            uint32_t vh[32], vl[32];
-            tmem_ld32(thi + half * 32, vh);
-            tmem_ld32(thi + 128 + half * 32, vl);
-            tmem_wait_ld();
-            float4* d4 = reinterpret_cast<float4*>(dst + half * 32);
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                d4[e] = make_float4(__uint_as_float(vh[4 * e]) + __uint_as_float(vl[4 * e]),
-                                    __uint_as_float(vh[4 * e + 1]) + __uint_as_float(vl[4 * e + 1]),
-                                    __uint_as_float(vh[4 * e + 2]) + __uint_as_float(vl[4 * e + 2]),
-                                    __uint_as_float(vh[4 * e + 3]) + __uint_as_float(vl[4 * e + 3]));
-        }
+        store_state(slot_of(0));
     }
     tc_fence_before();
     __syncthreads();
@@ -323,93 +352,88 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
 }
 
 // ---------------------------------------------------------------------------------
-// Chain over segments. seg_state slots are replaced by the state entering each segment
-// (h_in, layout [seg][H][N][P]); init, final_state and the snapshots use the API layout
-// [nseq][H][P][N]. A CTA owns kPassN = 8 state rows (n) x all P columns of one (sequence,
-// head); thread t walks elements t and t + 256 of that tile ([N][P] order, coalesced)
-// down the segments, four segments' loads in flight. API-layout reads and writes go
-// through a shared-memory transpose, so a warp touches 32-byte sectors it uses whole.
-constexpr int kPassN = 8;
+// Chain over state slots: a sequence's segments, or with snapshots the pieces its
+// segments are cut into (slots first[s] .. first[s+1]-1, in token order). The slot of
+// each segment's first piece is replaced by the state entering the segment (h_in), which
+// the chunk scan reads. Slots, init, final_state and the snapshots all use the layout
+// [.][H][P][N]. A CTA owns kPassElems consecutive elements of one (sequence, head);
+// thread t walks elements t + 256 i (i < 4) down the slots, up to eight slots' loads
+// in flight, every access coalesced.
+constexpr int kPassE = 4;                        // elements per thread
+constexpr int kPassElems = 256 * kPassE;         // elements per CTA
 
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)
 k_tc_segment_passing(float* __restrict__ seg_state, const float* __restrict__ seg_acum,
                      const int32_t* __restrict__ first, const float* __restrict__ init,
-                     float* __restrict__ final_state, int H, const ChunkEntry* __restrict__ segs,
-                     int64_t snap, const int32_t* __restrict__ snap_first, float* __restrict__ snap_out) {
-    constexpr int E = kP * kPassN / 256;                   // elements per thread (2)
-    __shared__ float tile[kP][kPassN + 1];
-    const int s = blockIdx.x, h = blockIdx.y, n0 = blockIdx.z * kPassN, tid = threadIdx.x;
-    const int64_t api0 = ((int64_t)s * H + h) * kP * kN + n0;   // (p, n0 + nn) at api0 + p*kN + nn
-    // element i of thread tid: idx = tid + 256 i, n = n0 + idx / kP, p = idx % kP
-    auto api_load = [&](const float* src, float (&v)[E]) {
-        __syncthreads();
-#pragma unroll
-        for (int i = 0; i < E; ++i) {
-            const int idx = tid + 256 * i, p = idx / kPassN, nn = idx % kPassN;
-            tile[p][nn] = src[(int64_t)p * kN + nn];
-        }
-        __syncthreads();
-#pragma unroll
-        for (int i = 0; i < E; ++i) {
-            const int idx = tid + 256 * i;
-            v[i] = tile[idx % kP][idx / kP];
-        }
-    };
-    auto api_store = [&](float* dst, const float (&v)[E]) {
-        __syncthreads();
-#pragma unroll
-        for (int i = 0; i < E; ++i) {
-            const int idx = tid + 256 * i;
-            tile[idx % kP][idx / kP] = v[i];
-        }
-        __syncthreads();
-#pragma unroll
-        for (int i = 0; i < E; ++i) {
-            const int idx = tid + 256 * i, p = idx / kPassN, nn = idx % kPassN;
-            dst[(int64_t)p * kN + nn] = tile[p][nn];
-        }
-    };
+                     float* __restrict__ final_state, int H, int Ls, int64_t snap,
+                     const int32_t* __restrict__ sub_end, const int32_t* __restrict__ snap_first,
+                     float* __restrict__ snap_out) {
+    constexpr int E = kPassE, PN = kP * kN;
+    const int s = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+    const int64_t e0 = (int64_t)blockIdx.z * kPassElems + tid;       // element of thread's i = 0
+    auto at = [&](int64_t slot) { return ((int64_t)slot * H + h) * PN + e0; };
     float hv[E];
-    if (init) {
-        api_load(init + api0, hv);
-    } else {
 #pragma unroll
-        for (int i = 0; i < E; ++i) hv[i] = 0.f;
-    }
+    for (int i = 0; i < E; ++i) hv[i] = init ? init[at(s) + 256 * i] : 0.f;
     const int c0 = first[s], c1 = first[s + 1];
-    const int64_t seq0 = c1 > c0 ? segs[c0].start : 0;
-    const int64_t eoff = (int64_t)n0 * kP + tid;
+    // Snapshot positions and segment starts, in tokens from the sequence start (int32: a
+    // sequence holds fewer than 2^31 tokens, so an interval beyond that never comes up).
+    const int sn = snap > 0 && snap <= INT32_MAX ? (int)snap : 0;
+    int prev_end = 0;                                       // where the current slot starts
+    // Groups of U slots, double-buffered: the next group's loads are in flight while
+    // this one is applied.
     constexpr int U = 4;
-    for (int c = c0; c < c1; c += U) {
-        float sv[U][E], dec[U];
+    struct Group {
+        float sv[U][E], ac[U];
+        int end[U];
+    };
+    auto load = [&](int c, Group& g) {
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             if (c + u < c1) {
-                const float* slot = seg_state + ((int64_t)(c + u) * H + h) * (kP * kN) + eoff;
 #pragma unroll
-                for (int i = 0; i < E; ++i) sv[u][i] = slot[256 * i];
-                dec[u] = expf(seg_acum[(int64_t)(c + u) * H + h]);
+                for (int i = 0; i < E; ++i) g.sv[u][i] = seg_state[at(c + u) + 256 * i];
+                g.ac[u] = seg_acum[(int64_t)(c + u) * H + h];
+                g.end[u] = sub_end ? sub_end[c + u] : 0;
             }
         }
+    };
+    auto apply = [&](int c, const Group& g) {
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             if (c + u < c1) {
-                float* slot = seg_state + ((int64_t)(c + u) * H + h) * (kP * kN) + eoff;
+                // Only a segment's first slot is read by the chunk scan.
+                if (!sub_end || prev_end % Ls == 0) {
 #pragma unroll
-                for (int i = 0; i < E; ++i) {
-                    slot[256 * i] = hv[i];
-                    hv[i] = fmaf(dec[u], hv[i], sv[u][i]);
+                    for (int i = 0; i < E; ++i) seg_state[at(c + u) + 256 * i] = hv[i];
                 }
-                if (snap > 0) {                           // state after a multiple of snap tokens
-                    const int64_t end = (int64_t)segs[c + u].start + segs[c + u].len - seq0;
-                    if (end % snap == 0)
-                        api_store(snap_out + ((int64_t)(snap_first[s] + end / snap - 1) * H + h) * kP * kN + n0,
-                                  hv);
+                const float dec = expf(g.ac[u]);
+#pragma unroll
+                for (int i = 0; i < E; ++i) hv[i] = fmaf(dec, hv[i], g.sv[u][i]);
+                if (sub_end) {                            // state after a multiple of snap tokens
+                    prev_end = g.end[u];
+                    if (sn && g.end[u] % sn == 0) {
+                        float* dst = snap_out + ((int64_t)(snap_first[s] + g.end[u] / sn - 1) * H + h) * PN + e0;
+#pragma unroll
+                        for (int i = 0; i < E; ++i) dst[256 * i] = hv[i];
+                    }
                 }
             }
         }
+    };
+    Group ga, gb;
+    if (c0 < c1) load(c0, ga);
+    for (int c = c0; c < c1; c += 2 * U) {
+        if (c + U < c1) load(c + U, gb);
+        apply(c, ga);
+        if (c + U >= c1) break;
+        if (c + 2 * U < c1) load(c + 2 * U, ga);
+        apply(c + U, gb);
     }
-    if (final_state) api_store(final_state + api0, hv);
+    if (final_state) {
+#pragma unroll
+        for (int i = 0; i < E; ++i) final_state[at(s) + 256 * i] = hv[i];
+    }
 }
 
 // ---------------------------------------------------------------------------------
@@ -709,16 +733,10 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
         float h[kHeadsB][16];                       // h[head][n = r][p = 16*cw + j]
 #pragma unroll
         for (int hh = 0; hh < kHeadsB; ++hh) {
-            const float4* src =
-                reinterpret_cast<const float4*>(hin + (((int64_t)sg * H + h0 + hh) * kN + r) * kP + 16 * cw);
+            // layout [slot][H][P][N]: for each p the warp reads 32 consecutive n
+            const float* src = hin + (((int64_t)seg.pad * H + h0 + hh) * kP + 16 * cw) * kN + r;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float4 v = src[j];
-                h[hh][4 * j] = v.x;
-                h[hh][4 * j + 1] = v.y;
-                h[hh][4 * j + 2] = v.z;
-                h[hh][4 * j + 3] = v.w;
-            }
+            for (int j = 0; j < 16; ++j) h[hh][j] = src[j * kN];
         }
         const float Dh0 = D[h0], Dh1 = D[h0 + 1];
         // Decays of the diagonal 32x32 blocks of chunk j, L[t][s] = exp2(Acum_t - Acum_s)

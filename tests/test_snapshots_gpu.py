@@ -91,3 +91,32 @@ def test_snapshot_interval_not_supported(ssd, cuda_dev):
     with pytest.raises(ssd.SSDError, match="UNSUPPORTED"):
         ssd.scan_fwd(d["x"], d["dt_raw"], d["dt_bias"], d["A"], d["B"], d["C"], d["D"],
                      cu_seqlens=d["cu_seqlens"], chunk=128, snapshot_tokens=200)
+
+
+@pytest.mark.parametrize("seqlens,varlen,seg,I", [
+    # cuts inside segments that do not line up with the segment boundaries
+    ([2600, 17, 1300, 4100, 640], True, 1024, 384),
+    ([2600, 17, 1300, 4100, 640], True, 1152, 256),
+    ([3072, 3072], False, 1536, 512),
+    # a cut after every chunk of a segment
+    ([2048, 300], True, 2048, 128),
+])
+def test_snapshots_inside_long_segments(ssd, cuda_dev, seqlens, varlen, seg, I):
+    """Tensor-core pipeline with segments longer than the interval: each segment's state is
+    cut at the snapshot positions inside it, and the chain walks the pieces."""
+    w = W.Workload("snap", nheads=8, headdim=64, ngroups=2, dstate=128, chunk=128, dtype=torch.bfloat16,
+                   seqlens=seqlens, varlen=varlen, init="normal", seed=77)
+    d = W.make_all(w)
+    ssd.set_segment_tokens(seg)
+    try:
+        y, fin, sn = _run(ssd, cuda_dev, w, d, I)
+        ssd.device_status()
+    finally:
+        ssd.set_segment_tokens(0)
+    y_ref, fin_ref, sn_ref = _oracle(w, d, I)
+    assert sn.shape == sn_ref.shape == (sum(L // I for L in seqlens), 8, 64, 128)
+    assert rel_err(y, y_ref) <= TOL_Y[torch.bfloat16]
+    assert rel_err(fin, fin_ref) <= TOL_STATE
+    for k in range(sn.shape[0]):
+        assert rel_err(sn[k], sn_ref[k]) <= TOL_STATE, k
+
