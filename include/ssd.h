@@ -339,10 +339,22 @@ int ssd_scan_fwd_segment_tokens(const ssd_dims* dims, int chunk);
  * Tuning and testing knob (process-wide): force the tensor-core pipeline's segment
  * length to `tokens` (a multiple of 128, at most 2^20) for every later call; 0 or any
  * other value restores the planner's choice. Results do not depend on it beyond
- * rounding; the workspace size does (query it after setting). Snapshot calls still
- * shorten the segment to a divisor of the snapshot interval.
+ * rounding; the workspace size does (query it after setting).
  */
 void ssd_set_segment_tokens(int tokens);
+
+/*
+ * Test hook for the fail-closed path (RL-Kernel issue page, §4.1 and §7: fail closed),
+ * process-wide, for later calls. The tensor-core prefill's warps hand work to each other
+ * through shared-memory barriers, and every wait on one is bounded (about 2 s): a wait
+ * that runs out latches SSD_ERR_TIMEOUT (read with ssd_get_device_status), the CTA's TMA
+ * and UMMA warps issue nothing more and wait (bounded) for the copies and MMAs already in
+ * flight, and the CTA exits, so the context stays usable; y and the states of that call
+ * are undefined. pass = 1 or 2 makes the UMMA warp of every CTA of the segment-state (1)
+ * or chunk-scan (2) pass first wait on a barrier that nothing arrives at, so that this
+ * wait runs out (each such call takes a few seconds); 0 (or any other value): off.
+ */
+void ssd_test_stall(int pass);
 
 
 /* Number of kernels the last successful call on this host thread enqueued. */

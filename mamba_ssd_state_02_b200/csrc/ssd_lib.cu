@@ -154,6 +154,8 @@ int sm_count() {
 
 // Segment length forced by ssd_set_segment_tokens (0: the planner chooses).
 std::atomic<int> g_segment_override{0};
+// Test hook set by ssd_test_stall: the tensor-core pass whose UMMA warp stalls (0: none).
+std::atomic<int> g_test_stall{0};
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -391,7 +393,8 @@ ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_ra
             StageScope sc(ST_CHUNK_STATE, st);
             tc::k_tc_segment_state<<<(unsigned)(pl.max_segs * (H / tc::kHeads)), tc::kThreadsA, tc::kSmemA,
                                      st>>>(mx, mb, dt_raw, dt_bias, A, table, count, H, G,
-                                                                  seg_state, seg_acum, order, first, pl.snap);
+                                                                  seg_state, seg_acum, order, first, pl.snap,
+                                                                  g_test_stall.load() == 1);
         }
         ++n;
         {
@@ -404,7 +407,8 @@ ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_ra
         {
             StageScope sc(ST_CHUNK_SCAN, st);
             tc::k_tc_chunk_scan<<<(unsigned)(pl.max_segs * (H / tc::kHeadsB)), tc::kThreadsB, tc::kSmemB, st>>>(mx, mb, mc, my, dt_raw, dt_bias, A, D, table, count, H,
-                                                               G, seg_state, (__nv_bfloat16*)y, order);
+                                                               G, seg_state, (__nv_bfloat16*)y, order,
+                                                               g_test_stall.load() == 2);
         }
         ++n;
     } else {
@@ -682,6 +686,8 @@ int ssd_last_launch_count(void) { return t_launches; }
 void ssd_set_segment_tokens(int tokens) {
     g_segment_override.store(tokens >= tc::kTile && tokens % tc::kTile == 0 && tokens <= (1 << 20) ? tokens : 0);
 }
+
+void ssd_test_stall(int pass) { g_test_stall.store(pass == 1 || pass == 2 ? pass : 0); }
 
 int ssd_scan_fwd_segment_tokens(const ssd_dims* dims, int chunk) {
     Plan pl;

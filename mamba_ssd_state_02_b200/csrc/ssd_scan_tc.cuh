@@ -45,36 +45,37 @@ constexpr int kRoleWarps = 2;                    // warp 0: TMA producer, warp 1
 constexpr int kComputeWarps = 16;                // four compute warpgroups (cw = 0..3)
 constexpr int kThreadsTc = 32 * (kRoleWarps + kComputeWarps);
 
-__device__ __forceinline__ void compute_bar() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
-
-// Wait with a shared abort flag: once any wait has timed out, every later wait
-// returns at once, so all roles run to the end without blocking each other.
-__device__ __forceinline__ void wait_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-    if (mbar_try_wait(bar, parity)) return;
+// Bounded waits with a CTA-wide abort flag. A wait that runs out latches SSD_ERR_TIMEOUT
+// and raises the flag, after which every wait in the CTA returns at once. The compute
+// and scan warps then run to the end on whatever the buffers hold: they issue no copy or
+// MMA, and the barriers they arrive on carry no transaction counts. The two issuing
+// roles stop at the first wait after the flag is up (wait_issue: an arrival made after
+// its warp saw the flag reaches them through the barrier's release/acquire, so they
+// never act on it), and at the end the TMA producer waits for the loads it has issued
+// and the UMMA warp for its MMAs (both bounded), so that no copy or MMA is in flight
+// when TMEM is freed and the CTA exits.
+__device__ __forceinline__ bool wait_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (!mbar_try_wait_sleep(bar, parity)) {
-        if (*abort_flag) return;
+        if (*abort_flag) return false;
         if (clock64() - t0 > kWaitBudgetCycles) {
             latch_error(SSD_ERR_TIMEOUT);
             *abort_flag = 1;
-            return;
+            return false;
         }
     }
+    return true;
 }
 
-// Inclusive scan of `a` over the 128 rows of one compute warpgroup (rows r = 32*q +
-// lane); `part` holds the four per-warp totals of that warpgroup. Two compute_bar()s.
-__device__ __forceinline__ float wg_scan(float a, int q, int lane, float* part) {
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const float v = __shfl_up_sync(0xffffffffu, a, off);
-        if (lane >= off) a += v;
-    }
-    if (lane == 31) part[q] = a;
-    compute_bar();
-    float pre = 0.f;
-    for (int w = 0; w < q; ++w) pre += part[w];
-    return a + pre;
+// For an issuing role: true if the phase completed and no abort has been raised.
+__device__ __forceinline__ bool wait_issue(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    return wait_abort(bar, parity, abort_flag) && !*abort_flag;
+}
+
+// The same for a whole warp (all lanes call it), warp-uniform.
+__device__ __forceinline__ bool wait_issue_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    return __all_sync(0xffffffffu, wait_issue(bar, parity, abort_flag));
 }
 
 // ---------------------------------------------------------------------------------
@@ -106,7 +107,7 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
                    const float* __restrict__ A, const ChunkEntry* __restrict__ segs,
                    const int32_t* __restrict__ nsegs, int H, int G, float* __restrict__ seg_state,
                    float* __restrict__ seg_acum, const int32_t* __restrict__ order,
-                   const int32_t* __restrict__ first, int64_t snap) {
+                   const int32_t* __restrict__ first, int64_t snap, int stall) {
     const int nq = H / kHeads;
     if ((int)(blockIdx.x / nq) >= *nsegs) return;
     const int sg = order ? order[blockIdx.x / nq] : (int)(blockIdx.x / nq);   // longest segments first
@@ -117,7 +118,8 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
     auto xs = [&](int hh) { return sP + (hh >> 1) * 65536 + (hh & 1) * 16384; };           // x, then hi
     auto los = [&](int hh) { return sP + (hh >> 1) * 65536 + 32768 + (hh & 1) * 16384; };  // lo
     __shared__ __align__(16) float wts[4][kHeads][kTile];
-    __shared__ uint64_t full_b[2], empty_b[2], full_x[2], pair_done[2], ops_ready[2], w_ready[4], w_free[4], all_done;
+    __shared__ uint64_t full_b[2], empty_b[2], full_x[2], pair_done[2], ops_ready[2], w_ready[4], w_free[4], all_done,
+        drained, stall_bar;
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
 
@@ -153,6 +155,8 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
             mbar_init(&w_free[i], kComputeWarps);
         }
         mbar_init(&all_done, 1);
+        mbar_init(&drained, 1);
+        mbar_init(&stall_bar, 1);
         abort_flag = 0;
         fence_barrier_init();
         prefetch_tmap(&map_x);
@@ -172,12 +176,15 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             auto t0_of = [&](int k) { return seg.start + (ntiles - 1 - k) * kTile; };   // k-th chunk processed
-            for (int k = 0; k < ntiles; ++k) {
+            int nb0 = 0, nb1 = 0, nx0 = 0, nx1 = 0;  // phases issued on full_b[0/1], full_x[0/1]
+            bool ok = true;
+            for (int k = 0; k < ntiles && ok; ++k) {
                 const int t0 = t0_of(k), st = k & 1;
-                if (k >= 2) wait_abort(&empty_b[st], ((k - 2) >> 1) & 1, abort_p);
+                if (k >= 2 && !wait_issue(&empty_b[st], ((k - 2) >> 1) & 1, abort_p)) break;
                 mbar_arrive_expect_tx(&full_b[st], 32768);
                 tma_load_3d(sB + st * 32768, &map_b, &full_b[st], 0, g, t0);
                 tma_load_3d(sB + st * 32768 + 16384, &map_b, &full_b[st], 64, g, t0);
+                if (st) ++nb1; else ++nb0;
                 if (k + 1 < ntiles) {               // next chunk's B and X into L2 meanwhile
                     const int tn = t0_of(k + 1);
                     tma_prefetch_3d(&map_b, 0, g, tn);
@@ -185,12 +192,22 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
                     for (int hh = 0; hh < kHeads; ++hh) tma_prefetch_3d(&map_x, 0, h0 + hh, tn);
                 }
                 for (int pr = 0; pr < 2; ++pr) {
-                    if (k >= 1) wait_abort(&pair_done[pr], (k - 1) & 1, abort_p);   // slots and lo free
+                    if (k >= 1 && !wait_issue(&pair_done[pr], (k - 1) & 1, abort_p)) {   // slots and lo free
+                        ok = false;
+                        break;
+                    }
                     mbar_arrive_expect_tx(&full_x[pr], 32768);
                     for (int hh = 2 * pr; hh < 2 * pr + 2; ++hh)
                         tma_load_3d(xs(hh), &map_x, &full_x[pr], 0, h0 + hh, t0);
+                    if (pr) ++nx1; else ++nx0;
                 }
             }
+            // The last phase issued on each barrier completes once its bytes have landed
+            // (a phase is issued only after the previous one has been consumed).
+            if (nb0) mbar_wait(&full_b[0], (nb0 - 1) & 1);
+            if (nb1) mbar_wait(&full_b[1], (nb1 - 1) & 1);
+            if (nx0) mbar_wait(&full_x[0], (nx0 - 1) & 1);
+            if (nx1) mbar_wait(&full_x[1], (nx1 - 1) & 1);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ UMMA issuer
@@ -198,13 +215,19 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
         // B MN-major with its four 64-column blocks 16 KB apart, N = 256.
         const uint32_t idesc = idesc_bf16(128, 256, 1, 1);
         const uint64_t dP = smem_desc(smem_u32(sP), 16384, 1024);
-        for (int k = 0; k < ntiles; ++k) {
+        bool ok = true;
+        for (int k = 0; k < ntiles && ok; ++k) {
             const int st = k & 1;
-            wait_abort(&full_b[st], (k >> 1) & 1, abort_p);
+            if (!wait_issue_warp(&full_b[st], (k >> 1) & 1, abort_p)) break;
             const uint64_t dB = smem_desc(smem_u32(sB + st * 32768), 16384, 1024);
             const bool fresh = opens(k);            // first chunk of a piece: overwrite the accumulator
             for (int pr = 0; pr < 2; ++pr) {
-                wait_abort(&ops_ready[pr], k & 1, abort_p);
+                // test hook (stall): before the first head pair's UMMAs, a wait that runs out
+                if ((stall && k == 0 && !wait_issue_warp(&stall_bar, 0, abort_p)) ||
+                    !wait_issue_warp(&ops_ready[pr], k & 1, abort_p)) {
+                    ok = false;
+                    break;
+                }
                 tc_fence_after();
                 const uint32_t d = tS + pr * 256;
                 const uint64_t dp = desc_add(dP, pr * 65536);
@@ -219,6 +242,10 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
                 __syncwarp();
             }
         }
+        // Every MMA issued above has completed once this commit arrives.
+        if (elect_one()) umma_commit(&drained);
+        __syncwarp();
+        mbar_wait(&drained, 0);
     } else if (warp >= kScanWarpA) {
         // ------------------------------------------------------------ dt scan
         // Warp 18 + i scans heads 2i, 2i+1. Lane l holds tokens 4l..4l+3 of a chunk; the
@@ -479,7 +506,7 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 const float* __restrict__ dt_raw, const float* __restrict__ dt_bias, const float* __restrict__ A,
                 const float* __restrict__ D, const ChunkEntry* __restrict__ segs, const int32_t* __restrict__ nsegs,
                 int H, int G, const float* __restrict__ hin, __nv_bfloat16* __restrict__ y,
-                const int32_t* __restrict__ order) {
+                const int32_t* __restrict__ order, int stall) {
     const int nhp = H / kHeadsB;
     if ((int)(blockIdx.x / nhp) >= *nsegs) return;
     const int sg = order ? order[blockIdx.x / nhp] : (int)(blockIdx.x / nhp);   // longest segments first
@@ -496,7 +523,7 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
     __shared__ __align__(16) float uw[4][kHeadsB][kTile];
     __shared__ __align__(16) float ww[4][kHeadsB][kTile];
     __shared__ uint64_t full_b, full_c[2], s_done, zs_done, full_x[2], cb_done, ops_ready, y0_done, mma_done, l_ready,
-        dt_ready[4], dt_free[4], y_staged;
+        dt_ready[4], dt_free[4], y_staged, drained, stall_bar;
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
 
@@ -522,6 +549,8 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             mbar_init(&dt_free[i], kComputeWarps);
         }
         mbar_init(&l_ready, kComputeWarps);
+        mbar_init(&drained, 1);
+        mbar_init(&stall_bar, 1);
         abort_flag = 0;
         fence_barrier_init();
         prefetch_tmap(&map_x);
@@ -543,8 +572,10 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
+            int nx0 = 0, nx1 = 0, nb = 0, nc = 0;  // phases issued on full_x[0/1], full_b, full_c[.]
             auto load_x = [&](int j) {              // X of chunk j (both heads) into slot j & 1
                 const int sl = j & 1;
+                if (sl) ++nx1; else ++nx0;
                 mbar_arrive_expect_tx(&full_x[sl], 32768);
                 for (int hh = 0; hh < kHeadsB; ++hh)
                     tma_load_3d(sX + sl * 32768 + hh * 16384, &map_x, &full_x[sl], 0, h0 + hh, seg.start + j * kTile);
@@ -554,12 +585,14 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             // half. B, C and X of chunk j+1 are prefetched into L2 meanwhile.
             auto load_b = [&](int j) {
                 const int t0 = seg.start + j * kTile;
+                ++nb;
                 mbar_arrive_expect_tx(&full_b, 32768);
                 tma_load_3d(sB, &map_b, &full_b, 0, g, t0);
                 tma_load_3d(sB + 16384, &map_b, &full_b, 64, g, t0);
             };
             auto load_c = [&](int j) {
                 const int t0 = seg.start + j * kTile;
+                ++nc;
                 for (int hf = 0; hf < 2; ++hf) {
                     mbar_arrive_expect_tx(&full_c[hf], 16384);
                     tma_load_3d(sC + hf * 16384, &map_c, &full_c[hf], 64 * hf, g, t0);
@@ -574,13 +607,14 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             };
             // y tile of chunk j, staged by the compute warps in the chunk's X slot (full
             // chunks only; a partial last chunk is written by the threads).
-            auto store_y = [&](int j) {
-                wait_abort(&y_staged, j & 1, abort_p);
+            auto store_y = [&](int j) -> bool {
+                if (!wait_issue(&y_staged, j & 1, abort_p)) return false;
                 if (seg.len - j * kTile >= kTile) {
                     for (int hh = 0; hh < kHeadsB; ++hh)
                         tma_store_3d(&map_y, sX + (j & 1) * 32768 + hh * 16384, 0, h0 + hh, seg.start + j * kTile);
                     bulk_commit_group();
                 }
+                return true;
             };
             if (ntiles > 0) {
                 load_x(0);
@@ -588,19 +622,31 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 load_b(0);
                 load_c(0);
             }
-            for (int j = 1; j < ntiles; ++j) {
-                wait_abort(&s_done, (j - 1) & 1, abort_p);          // B of chunk j-1 read
+            bool ok = true;
+            for (int j = 1; j < ntiles && ok; ++j) {
+                ok = wait_issue(&s_done, (j - 1) & 1, abort_p);     // B of chunk j-1 read
+                if (!ok) break;
                 load_b(j);
-                wait_abort(&zs_done, (j - 1) & 1, abort_p);         // C of chunk j-1 read
+                ok = wait_issue(&zs_done, (j - 1) & 1, abort_p);    // C of chunk j-1 read
+                if (!ok) break;
                 load_c(j);
-                store_y(j - 1);
-                if (j + 1 < ntiles) {
+                ok = store_y(j - 1);
+                if (ok && j + 1 < ntiles) {
                     bulk_wait_read_all();                           // slot (j+1) & 1 read by the store
                     load_x(j + 1);
                 }
             }
-            if (ntiles > 0) store_y(ntiles - 1);
+            if (ok && ntiles > 0) store_y(ntiles - 1);
             bulk_wait_all();
+            // The last phase issued on each barrier completes once its bytes have landed
+            // (a phase is issued only after the previous one has been consumed).
+            if (nx0) mbar_wait(&full_x[0], (nx0 - 1) & 1);
+            if (nx1) mbar_wait(&full_x[1], (nx1 - 1) & 1);
+            if (nb) mbar_wait(&full_b, (nb - 1) & 1);
+            if (nc) {
+                mbar_wait(&full_c[0], (nc - 1) & 1);
+                mbar_wait(&full_c[1], (nc - 1) & 1);
+            }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ UMMA issuer
@@ -613,11 +659,11 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
         const uint64_t dX = smem_desc(smem_u32(sX), 16384, 1024);
         // C B^T of chunk j into the M columns (fp32): dstate columns 0..63 once B and the
         // first half of C have landed, 64..127 once the second half has.
-        auto issue_cb = [&](int j) {
-            wait_abort(&full_b, j & 1, abort_p);
+        auto issue_cb = [&](int j) -> bool {
+            if (!wait_issue_warp(&full_b, j & 1, abort_p)) return false;
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
-                wait_abort(&full_c[hf], j & 1, abort_p);
+                if (!wait_issue_warp(&full_c[hf], j & 1, abort_p)) return false;
                 tc_fence_after();
                 if (elect_one()) {
 #pragma unroll
@@ -628,10 +674,12 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
                 }
                 __syncwarp();
             }
+            return true;
         };
-        if (ntiles > 0) issue_cb(0);
-        for (int it = 0; it < ntiles; ++it) {
-            wait_abort(&ops_ready, it & 1, abort_p);
+        // test hook (stall): before the first UMMAs, a wait that runs out
+        bool ok = !(stall && !wait_issue_warp(&stall_bar, 0, abort_p)) && (ntiles == 0 || issue_cb(0));
+        for (int it = 0; it < ntiles && ok; ++it) {
+            if (!wait_issue_warp(&ops_ready, it & 1, abort_p)) break;
             tc_fence_after();
             const uint64_t dX0 = desc_add(dX, (it & 1) * 32768), dX1 = desc_add(dX0, 16384);
             if (elect_one()) {
@@ -654,10 +702,14 @@ k_tc_chunk_scan(const __grid_constant__ CUtensorMap map_x, const __grid_constant
             }
             __syncwarp();
             if (it + 1 < ntiles) {
-                wait_abort(&mma_done, it & 1, abort_p);     // the Y UMMAs have read M
-                issue_cb(it + 1);
+                if (!wait_issue_warp(&mma_done, it & 1, abort_p)) break;   // the Y UMMAs have read M
+                ok = issue_cb(it + 1);
             }
         }
+        // Every MMA issued above has completed once this commit arrives.
+        if (elect_one()) umma_commit(&drained);
+        __syncwarp();
+        mbar_wait(&drained, 0);
     } else if (warp == kScanWarp) {
         // ------------------------------------------------------------ dt scan
         // Chunk by chunk, up to four ahead of the compute warps: dt, the log2-scaled

@@ -86,6 +86,8 @@ _lib.ssd_last_error.restype = ctypes.c_char_p
 _lib.ssd_scan_fwd_variant.argtypes = [ctypes.POINTER(SSDDims), ctypes.c_int]
 _lib.ssd_scan_fwd_variant.restype = ctypes.c_char_p
 _lib.ssd_set_segment_tokens.argtypes = [ctypes.c_int]
+_lib.ssd_test_stall.argtypes = [ctypes.c_int]
+_lib.ssd_test_stall.restype = None
 
 _lib.ssd_set_segment_tokens.restype = None
 _lib.ssd_scan_fwd_segment_tokens.argtypes = [ctypes.POINTER(SSDDims), ctypes.c_int]
@@ -209,6 +211,12 @@ def scan_variant(dims: SSDDims, chunk: int) -> str:
 def set_segment_tokens(tokens: int) -> None:
     """Force the tensor-core segment length for later calls (0 restores the planner)."""
     _lib.ssd_set_segment_tokens(int(tokens))
+
+
+def test_stall(pass_: int) -> None:
+    """Test hook: make the UMMA warp of tensor-core pass 1 (segment states) or 2 (chunk
+    scan) wait on a barrier that nothing arrives at, so that the wait runs out (0: off)."""
+    _lib.ssd_test_stall(int(pass_))
 
 
 def segment_tokens(dims: SSDDims, chunk: int) -> int:
