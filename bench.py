@@ -574,15 +574,18 @@ def bench_ours(args, rank, world, local_rank):
     ssd.device_status()
     barrier(dev)
     torch.cuda.synchronize(dev)
-    ssd.profile_enable(True)
     ev0.record(stream)
     for _ in range(strict_steps):
         strict_step()
     ev1.record(stream)
     torch.cuda.synchronize(dev)
+    strict_ms = max_over_ranks(ev0.elapsed_time(ev1) / strict_steps, dev)
+    ssd.profile_enable(True)                     # per-kernel breakdown from a second loop
+    for _ in range(strict_steps):
+        strict_step()
+    torch.cuda.synchronize(dev)
     sprof = ssd.profile_read()
     ssd.profile_enable(False)
-    strict_ms = max_over_ranks(ev0.elapsed_time(ev1) / strict_steps, dev)
     strict = {"workload": w.name, "prefill_ms_per_step": round(strict_ms, 3),
               "prefill_tokens_per_s": world * w.total_tokens / (strict_ms / 1e3),
               "slowdown_vs_default_path": round(strict_ms / ms_step, 2), "steps_timed": strict_steps,
@@ -738,16 +741,19 @@ def bench_decode(args, ssd, dev, rank, world, hbm, peak_src):
     barrier(dev)
     torch.cuda.synchronize(dev)
     s_steps = 2 * w.chunk
-    ssd.profile_enable(True)
     ev0.record(stream)
     for _ in range(s_steps):
         sstep()
     ev1.record(stream)
     torch.cuda.synchronize(dev)
+    s_ms = max_over_ranks(ev0.elapsed_time(ev1) / s_steps, dev)
+    ssd.profile_enable(True)                     # per-kernel breakdown from a second loop
+    for _ in range(s_steps):
+        sstep()
+    torch.cuda.synchronize(dev)
     sprof = ssd.profile_read()
     ssd.profile_enable(False)
     ssd.device_status()
-    s_ms = max_over_ranks(ev0.elapsed_time(ev1) / s_steps, dev)
     strict = {"ms_per_step": round(s_ms, 4), "steps_timed": s_steps, "fold_every_steps": w.chunk,
               "overhead_vs_plain_decode": round(s_ms / ms - 1.0, 4),
               "kernels_ms_per_launch": {k: round(v[1] / max(1, v[0]), 4) for k, v in sprof.items()

@@ -37,6 +37,16 @@ __device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
     return make_float4(fa.x, fa.y, fb.x, fb.y);
 }
 
+// 16-byte asynchronous global -> shared copies (cp.async): the issuing thread does not
+// wait for them; cp_async_wait<n>() waits until at most n committed groups are pending.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 // softplus(z) = log(1 + e^z), written so that neither branch overflows.
 __device__ __forceinline__ float softplus_f32(float z) {
     return z > 0.f ? z + log1pf(expf(-z)) : log1pf(expf(z));

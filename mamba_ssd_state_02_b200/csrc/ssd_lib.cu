@@ -1143,22 +1143,29 @@ ssd_status launch_strict_decode(const Plan& pl, const ssd_chunk_cache& cc, const
     using namespace strict;
     const unsigned grid = (unsigned)(pl.nseq * pl.H);
     const int H = pl.H, G = pl.G, P = pl.P, N = pl.N, Q = pl.Q;
-    const size_t dsm = decode_smem(N, Q);
+    const size_t dsm = decode_smem(H, G, N, Q);
+    if (dsm > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(k_strict_decode<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dsm);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(strict decode)");
+    }
     {
         StageScope sc(ST_STRICT_UPDATE, st);
-        k_strict_decode<T><<<grid, kDecThreads, dsm, st>>>(
+        k_strict_decode<T><<<(unsigned)(pl.nseq * pl.G), kDecThreads, dsm, st>>>(
             cc.state, static_cast<T*>(cc.x), static_cast<T*>(cc.B), cc.dt, cc.acum, cc.len, static_cast<const T*>(x),
             dt_raw, dt_bias, A, static_cast<const T*>(B), static_cast<const T*>(C), D, static_cast<T*>(y), H, G, P,
             N, Q);
     }
     {
         StageScope sc(ST_STRICT_FOLD, st);
-        const size_t sm = fold_smem(P, N, Q);
+        const size_t sm = fold_smem<T>(P, N, Q);
         switch (P * N / kThreads) {
 #define SSD_NOUT(V)                                                                                              \
-            case V: k_strict_fold<T, V><<<grid, kThreads, sm, st>>>(cc.state, static_cast<const T*>(cc.x),      \
-                                                                    static_cast<const T*>(cc.B), cc.dt, cc.acum, \
-                                                                    cc.len, H, G, P, N, Q);                     \
+            case V: if (cudaFuncSetAttribute(k_strict_fold<T, V>, cudaFuncAttributeMaxDynamicSharedMemorySize,   \
+                                             (int)sm) != cudaSuccess)                                           \
+                    return fail(SSD_ERR_CUDA, "cudaFuncSetAttribute(strict fold)");                            \
+                k_strict_fold<T, V><<<(grid + kFoldPairs - 1) / kFoldPairs, kThreads, sm, st>>>(                \
+                        cc.state, static_cast<const T*>(cc.x), static_cast<const T*>(cc.B), cc.dt, cc.acum, cc.len, \
+                        H, G, P, N, Q, (int)grid);                                                              \
                 break;
             SSD_NOUT(1) SSD_NOUT(2) SSD_NOUT(4) SSD_NOUT(8) SSD_NOUT(16) SSD_NOUT(32) SSD_NOUT(64)
 #undef SSD_NOUT

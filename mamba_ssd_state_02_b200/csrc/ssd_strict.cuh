@@ -459,12 +459,15 @@ k_strict_cache_fill(const T* __restrict__ x, const T* __restrict__ B, const floa
 }
 
 // ---------------------------------------------------------------------------------
-// Chunk-emulating decode step. One block per (sequence, head). With j = the open chunk's
-// length, the new token is position j of the open chunk: y is the prefill's y_t for t = j
-// over sources 0..j (cached 0..j-1, the new token j), and the token is appended to the
-// cache (len -> j + 1). A chunk that this fills (len == Q) is folded into the state by
-// k_strict_fold, launched right after in the same call.
-constexpr int kDecThreads = 128;
+// Chunk-emulating decode step. One block per (sequence, group): its H/G heads share
+// C_t and the cached B rows, so the dots C_t . B_s are taken once per group. With j =
+// the open chunk's length (equal across the heads), the new token is position j of the
+// open chunk: y is the prefill's y_t for t = j over sources 0..j (cached 0..j-1, the new
+// token j), and the token is appended to the cache (len -> j + 1). A chunk that this
+// fills (len == Q) is folded into the state by k_strict_fold, launched right after in
+// the same call. Threads take the dots one source each, then the coefficients
+// (C_t . B_s) w(j, s) of every head, then y[h][p] one (head, p) each.
+constexpr int kDecThreads = 512;
 
 // Left-to-right dot of the float row c[0..N) with the row b[0..N) of T, 16-byte loads.
 template <typename T>
@@ -506,130 +509,181 @@ k_strict_decode(const float* __restrict__ cstate, T* __restrict__ cx, T* __restr
                 const T* __restrict__ B, const T* __restrict__ C, const float* __restrict__ D, T* __restrict__ y,
                 int H, int G, int P, int N, int Q) {
     extern __shared__ float sm[];
-    float* cs = sm;                       // [N]  C_t
-    float* coef = cs + N;                 // [Q]
-    __shared__ float s_dt, s_acum;
-    const int bid = blockIdx.x;
-    const int s = bid / H, h = bid % H, g = h / (H / G), tid = threadIdx.x;
-    const int64_t sh = (int64_t)s * H + h;
-    const int j = clen[sh];
-    if (j < 0 || j >= Q) {                 // not a cache this step can continue
-        if (tid == 0) latch_error(SSD_ERR_INVALID_ARG);
-        return;
-    }
-    const float a = A[h];
+    const int hpg = H / G;
+    float* cs = sm;                       // [N]       C_t
+    float* dots = cs + N;                 // [Q]       C_t . B_s
+    float* coef = dots + Q;               // [hpg][Q]  (C_t . B_s) w(j, s) per head
+    float* hdt = coef + hpg * Q;          // [hpg]     the token's dt per head
+    float* hac = hdt + hpg;               // [hpg]     the token's Acum per head
+    __shared__ int s_j, s_bad;
+    const int s = blockIdx.x / G, g = blockIdx.x % G, h0 = g * hpg, tid = threadIdx.x;
     if (tid == 0) {
-        if (bad_A(a)) latch_error(SSD_ERR_INVALID_ARG);
-        const float d = dt_of(dt_raw[sh], dt_bias[h]);
-        s_dt = d;
-        s_acum = acum_next(j > 0 ? cacum[sh * Q + j - 1] : 0.f, d, a);
+        s_j = clen[(int64_t)s * H + h0];
+        s_bad = 0;
     }
-    const T* xt = x + sh * P;
+    __syncthreads();
+    const int j = s_j;
+    for (int hl = tid; hl < hpg; hl += kDecThreads) {
+        const int h = h0 + hl;
+        const int64_t sh = (int64_t)s * H + h;
+        const float a = A[h];
+        if (clen[sh] != j || j < 0 || j >= Q || bad_A(a)) {   // not a cache this step can continue
+            atomicOr(&s_bad, 1);
+            continue;
+        }
+        const float d = dt_of(dt_raw[sh], dt_bias[h]);
+        hdt[hl] = d;
+        hac[hl] = acum_next(j > 0 ? cacum[sh * Q + j - 1] : 0.f, d, a);
+    }
     const T* Bt = B + ((int64_t)s * G + g) * N;
     const T* Ct = C + ((int64_t)s * G + g) * N;
-    const T* xrow = cx + sh * Q * P;                       // cached x rows [Q][P]
     const T* brow = cB + ((int64_t)s * G + g) * Q * N;     // cached B rows [Q][N]
     for (int n = tid; n < N; n += kDecThreads) cs[n] = to_f32(Ct[n]);
     __syncthreads();
-    const float dtj = s_dt, acj = s_acum;
+    if (s_bad) {
+        if (tid == 0) latch_error(SSD_ERR_INVALID_ARG);
+        return;
+    }
 
-    // Coefficients of sources 0..j: (C_t . B_s) w(j, s).
-    for (int sidx = tid; sidx <= j; sidx += kDecThreads) {
-        const float dot = row_dot<T>(cs, sidx < j ? brow + (int64_t)sidx * N : Bt, N);
+    // C_t . B_s of sources 0..j (B_j: the token's B).
+    for (int sidx = tid; sidx <= j; sidx += kDecThreads)
+        dots[sidx] = row_dot<T>(cs, sidx < j ? brow + (int64_t)sidx * N : Bt, N);
+    __syncthreads();
+    // Coefficients of every head.
+    for (int i = tid; i < hpg * (j + 1); i += kDecThreads) {
+        const int hl = i / (j + 1), sidx = i % (j + 1);
+        const int64_t sh = (int64_t)s * H + h0 + hl;
+        const float acj = hac[hl];
         const float acs = sidx < j ? cacum[sh * Q + sidx] : acj;
-        const float dts = sidx < j ? cdt[sh * Q + sidx] : dtj;
-        coef[sidx] = mix_coef(dot, acj, acs, dts);
+        const float dts = sidx < j ? cdt[sh * Q + sidx] : hdt[hl];
+        coef[hl * Q + sidx] = mix_coef(dots[sidx], acj, acs, dts);
     }
     __syncthreads();
 
-    // y[p]: incoming-state term, sources left to right, D skip.
-    const float* hrow = cstate + sh * P * N;
-    for (int p = tid; p < P; p += kDecThreads) {
-        const float dot = row_dot<float>(cs, hrow + (int64_t)p * N, N);
-        float acc = y_begin(dot, acj);
-        const T* xp = xrow + p;
+    // y[h][p]: incoming-state term, sources left to right, D skip.
+    for (int i = tid; i < hpg * P; i += kDecThreads) {
+        const int hl = i / P, p = i % P, h = h0 + hl;
+        const int64_t sh = (int64_t)s * H + h;
+        const float* cf = coef + hl * Q;
+        const float dot = row_dot<float>(cs, cstate + (sh * P + p) * N, N);
+        float acc = y_begin(dot, hac[hl]);
+        const T* xp = cx + sh * Q * P + p;                  // cached x rows [Q][P]
         int sidx = 0;
         for (; sidx + 4 <= j; sidx += 4) {
             const float x0 = to_f32(xp[(int64_t)sidx * P]), x1 = to_f32(xp[(int64_t)(sidx + 1) * P]);
             const float x2 = to_f32(xp[(int64_t)(sidx + 2) * P]), x3 = to_f32(xp[(int64_t)(sidx + 3) * P]);
-            acc = y_step(acc, coef[sidx], x0);
-            acc = y_step(acc, coef[sidx + 1], x1);
-            acc = y_step(acc, coef[sidx + 2], x2);
-            acc = y_step(acc, coef[sidx + 3], x3);
+            acc = y_step(acc, cf[sidx], x0);
+            acc = y_step(acc, cf[sidx + 1], x1);
+            acc = y_step(acc, cf[sidx + 2], x2);
+            acc = y_step(acc, cf[sidx + 3], x3);
         }
-        for (; sidx < j; ++sidx) acc = y_step(acc, coef[sidx], to_f32(xp[(int64_t)sidx * P]));
-        const float xv = to_f32(xt[p]);
-        acc = y_step(acc, coef[j], xv);
+        for (; sidx < j; ++sidx) acc = y_step(acc, cf[sidx], to_f32(xp[(int64_t)sidx * P]));
+        const float xv = to_f32(x[sh * P + p]);
+        acc = y_step(acc, cf[j], xv);
         y[sh * P + p] = from_f32<T>(y_end(acc, D[h], xv));
     }
 
     // Append the token to the open chunk.
-    T* xdst = cx + (sh * Q + j) * P;
-    for (int p = tid; p < P; p += kDecThreads) xdst[p] = xt[p];
-    if (h % (H / G) == 0) {
-        T* bdst = cB + (((int64_t)s * G + g) * Q + j) * N;
-        for (int n = tid; n < N; n += kDecThreads) bdst[n] = Bt[n];
+    for (int i = tid; i < hpg * P; i += kDecThreads) {
+        const int64_t sh = (int64_t)s * H + h0 + i / P;
+        cx[(sh * Q + j) * P + i % P] = x[sh * P + i % P];
     }
-    if (tid == 0) {
-        cdt[sh * Q + j] = dtj;
-        cacum[sh * Q + j] = acj;
+    T* bdst = cB + (((int64_t)s * G + g) * Q + j) * N;
+    for (int n = tid; n < N; n += kDecThreads) bdst[n] = Bt[n];
+    for (int hl = tid; hl < hpg; hl += kDecThreads) {
+        const int64_t sh = (int64_t)s * H + h0 + hl;
+        cdt[sh * Q + j] = hdt[hl];
+        cacum[sh * Q + j] = hac[hl];
         clen[sh] = j + 1;
     }
 }
 
-inline size_t decode_smem(int N, int Q) { return sizeof(float) * (N + Q); }
+inline size_t decode_smem(int H, int G, int N, int Q) { return sizeof(float) * (N + Q + (H / G) * (Q + 2)); }
 
 // ---------------------------------------------------------------------------------
 // Fold of a full open chunk (len == Q) into the cache state: the prefill's chunk-state
-// and passing arithmetic, sources left to right; then len -> 0. Blocks whose chunk is
-// not full return at once. One block per (sequence, head); thread owns column
+// and passing arithmetic, sources left to right; then len -> 0. Block b looks at the
+// kFoldPairs (sequence, head) pairs kFoldPairs*b .. +kFoldPairs-1 (one load and one vote)
+// and folds the full ones one after the other, so a step that fills no chunk costs one
+// small launch. A fold walks the chunk in tiles of 32 sources: the raw x and B rows of
+// tile t+1 are copied into shared memory (16-byte asynchronous copies) while tile t is
+// used; each tile is converted once to FP32 (x scaled by w(last, s)). Thread owns column
 // n = tid % N and the NOUT consecutive rows (tid / N) * NOUT + k.
+constexpr int kFoldPairs = 8;
+
 template <typename T, int NOUT>
 __global__ void __launch_bounds__(kThreads)
 k_strict_fold(float* __restrict__ cstate, const T* __restrict__ cx, const T* __restrict__ cB,
               const float* __restrict__ cdt, const float* __restrict__ cacum, int32_t* __restrict__ clen, int H,
-              int G, int P, int N, int Q) {
-    extern __shared__ float sm[];
+              int G, int P, int N, int Q, int npairs) {
+    extern __shared__ __align__(16) float sm[];
     float* wv = sm;                       // [Q]      w(last, s)
     float* xs = wv + Q;                   // [32][P]  w(last, s) x_s
     float* bs = xs + 32 * P;              // [32][N]
-    const int bid = blockIdx.x;
-    const int s = bid / H, h = bid % H, g = h / (H / G), tid = threadIdx.x;
-    const int64_t sh = (int64_t)s * H + h;
-    if (clen[sh] != Q) return;
-    const T* xrow = cx + sh * Q * P;
-    const T* brow = cB + ((int64_t)s * G + g) * Q * N;
-    const float last = cacum[sh * Q + Q - 1];
-    for (int sidx = tid; sidx < Q; sidx += kThreads)
-        wv[sidx] = src_weight(last, cacum[sh * Q + sidx], cdt[sh * Q + sidx]);
-    const int n = tid % N, pb = (tid / N) * NOUT;
-    float acc[NOUT];
-#pragma unroll
-    for (int k = 0; k < NOUT; ++k) acc[k] = 0.f;
+    T* raw = reinterpret_cast<T*>(bs + 32 * N);   // [2][32 (P + N)] raw x rows, then B rows, of a tile
+    __shared__ int full[kFoldPairs], nfull;
+    const int tid = threadIdx.x;
+    if (tid < 32) {
+        const int pr = blockIdx.x * kFoldPairs + tid;
+        const bool f = tid < kFoldPairs && pr < npairs && clen[pr] == Q;
+        const unsigned m = __ballot_sync(0xffffffffu, f);
+        if (f) full[__popc(m & ((1u << tid) - 1u))] = pr;
+        if (tid == 0) nfull = __popc(m);
+    }
     __syncthreads();
-    for (int s0 = 0; s0 < Q; s0 += 32) {
-        for (int i = tid; i < 32 * P; i += kThreads) {
-            const int r = i / P, pp = i % P;
-            xs[r * P + pp] = state_src(wv[s0 + r], to_f32(xrow[(int64_t)(s0 + r) * P + pp]));
-        }
-        for (int i = tid; i < 32 * N; i += kThreads) {
-            const int r = i / N, nn = i % N;
-            bs[r * N + nn] = to_f32(brow[(int64_t)(s0 + r) * N + nn]);
-        }
-        __syncthreads();
-        for (int r = 0; r < 32; ++r) state_row<NOUT>(acc, xs + r * P + pb, bs[r * N + n]);
-        __syncthreads();
-    }
-    float* hout = cstate + sh * P * N;
+    constexpr int V = 16 / (int)sizeof(T);                 // elements per 16-byte copy
+    const int tile_elems = 32 * (P + N);
+    auto fold_one = [&](int64_t sh) {
+        const int s = (int)(sh / H), h = (int)(sh % H), g = h / (H / G);
+        const T* xrow = cx + sh * Q * P;
+        const T* brow = cB + ((int64_t)s * G + g) * Q * N;
+        auto fetch = [&](int t) {                           // raw rows of tile t into buffer t & 1
+            T* dst = raw + (t & 1) * tile_elems;
+            for (int i = tid; i < 32 * P / V; i += kThreads) cp_async16(dst + i * V, xrow + (int64_t)t * 32 * P + i * V);
+            for (int i = tid; i < 32 * N / V; i += kThreads)
+                cp_async16(dst + 32 * P + i * V, brow + (int64_t)t * 32 * N + i * V);
+            cp_async_commit();
+        };
+        fetch(0);
+        const float last = cacum[sh * Q + Q - 1];
+        for (int sidx = tid; sidx < Q; sidx += kThreads)
+            wv[sidx] = src_weight(last, cacum[sh * Q + sidx], cdt[sh * Q + sidx]);
+        const int n = tid % N, pb = (tid / N) * NOUT;
+        float acc[NOUT];
 #pragma unroll
-    for (int k = 0; k < NOUT; ++k) {
-        const int64_t o = (int64_t)(pb + k) * N + n;
-        hout[o] = pass(hout[o], last, acc[k]);
-    }
-    if (tid == 0) clen[sh] = 0;
+        for (int k = 0; k < NOUT; ++k) acc[k] = 0.f;
+        const int ntile = Q / 32;
+        for (int t = 0; t < ntile; ++t) {
+            if (t + 1 < ntile) {
+                fetch(t + 1);
+                cp_async_wait<1>();
+            } else {
+                cp_async_wait<0>();
+            }
+            __syncthreads();                                // tile t landed (all threads' copies); wv
+            const T* rx = raw + (t & 1) * tile_elems;
+            const T* rb = rx + 32 * P;
+            for (int i = tid; i < 32 * P; i += kThreads) xs[i] = state_src(wv[32 * t + i / P], to_f32(rx[i]));
+            for (int i = tid; i < 32 * N; i += kThreads) bs[i] = to_f32(rb[i]);
+            __syncthreads();
+            for (int r = 0; r < 32; ++r) state_row<NOUT>(acc, xs + r * P + pb, bs[r * N + n]);
+            __syncthreads();                                // xs, bs and buffer t & 1 free again
+        }
+        float* hout = cstate + sh * P * N;
+#pragma unroll
+        for (int k = 0; k < NOUT; ++k) {
+            const int64_t o = (int64_t)(pb + k) * N + n;
+            hout[o] = pass(hout[o], last, acc[k]);
+        }
+        if (tid == 0) clen[sh] = 0;
+    };
+    for (int f = 0; f < nfull; ++f) fold_one(full[f]);
 }
 
-inline size_t fold_smem(int P, int N, int Q) { return sizeof(float) * (Q + 32 * P + 32 * N); }
+template <typename T>
+inline size_t fold_smem(int P, int N, int Q) {
+    return sizeof(float) * (Q + 32 * P + 32 * N) + sizeof(T) * 2 * 32 * (P + N);
+}
 
 }  // namespace strict
 }  // namespace ssd
