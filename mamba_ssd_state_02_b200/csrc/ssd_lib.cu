@@ -1158,14 +1158,18 @@ ssd_status launch_strict_decode(const Plan& pl, const ssd_chunk_cache& cc, const
     {
         StageScope sc(ST_STRICT_FOLD, st);
         const size_t sm = fold_smem<T>(P, N, Q);
+        // a few blocks per SM, each over a stretch of at most 32 pairs
+        const int per_block = (int)std::min<int64_t>(32, std::max<int64_t>(1, ((int64_t)grid + 4 * sm_count() - 1) /
+                                                                               (4 * sm_count())));
+        const unsigned fold_grid = (unsigned)(((int64_t)grid + per_block - 1) / per_block);
         switch (P * N / kThreads) {
 #define SSD_NOUT(V)                                                                                              \
             case V: if (cudaFuncSetAttribute(k_strict_fold<T, V>, cudaFuncAttributeMaxDynamicSharedMemorySize,   \
                                              (int)sm) != cudaSuccess)                                           \
                     return fail(SSD_ERR_CUDA, "cudaFuncSetAttribute(strict fold)");                            \
-                k_strict_fold<T, V><<<(grid + kFoldPairs - 1) / kFoldPairs, kThreads, sm, st>>>(                \
+                k_strict_fold<T, V><<<fold_grid, kThreads, sm, st>>>(                                           \
                         cc.state, static_cast<const T*>(cc.x), static_cast<const T*>(cc.B), cc.dt, cc.acum, cc.len, \
-                        H, G, P, N, Q, (int)grid);                                                              \
+                        H, G, P, N, Q, (int)grid, per_block);                                                   \
                 break;
             SSD_NOUT(1) SSD_NOUT(2) SSD_NOUT(4) SSD_NOUT(8) SSD_NOUT(16) SSD_NOUT(32) SSD_NOUT(64)
 #undef SSD_NOUT

@@ -602,30 +602,29 @@ inline size_t decode_smem(int H, int G, int N, int Q) { return sizeof(float) * (
 
 // ---------------------------------------------------------------------------------
 // Fold of a full open chunk (len == Q) into the cache state: the prefill's chunk-state
-// and passing arithmetic, sources left to right; then len -> 0. Block b looks at the
-// kFoldPairs (sequence, head) pairs kFoldPairs*b .. +kFoldPairs-1 (one load and one vote)
-// and folds the full ones one after the other, so a step that fills no chunk costs one
-// small launch. A fold walks the chunk in tiles of 32 sources: the raw x and B rows of
-// tile t+1 are copied into shared memory (16-byte asynchronous copies) while tile t is
-// used; each tile is converted once to FP32 (x scaled by w(last, s)). Thread owns column
-// n = tid % N and the NOUT consecutive rows (tid / N) * NOUT + k.
-constexpr int kFoldPairs = 8;
+// and passing arithmetic, sources left to right; then len -> 0. The grid is a few blocks
+// per SM; block b looks at its stretch of at most 32 (sequence, head) pairs (one load and
+// one vote) and folds the full ones one after the other, so a step that fills no chunk
+// costs one small launch. A fold walks the chunk in tiles of 32 sources: the raw x and B
+// rows of tile t+1 are copied into shared memory (16-byte asynchronous copies) while tile
+// t is used; each tile is converted once to FP32 (x scaled by w(last, s)). Thread owns
+// column n = tid % N and the NOUT consecutive rows (tid / N) * NOUT + k.
 
 template <typename T, int NOUT>
 __global__ void __launch_bounds__(kThreads)
 k_strict_fold(float* __restrict__ cstate, const T* __restrict__ cx, const T* __restrict__ cB,
               const float* __restrict__ cdt, const float* __restrict__ cacum, int32_t* __restrict__ clen, int H,
-              int G, int P, int N, int Q, int npairs) {
+              int G, int P, int N, int Q, int npairs, int per_block) {
     extern __shared__ __align__(16) float sm[];
     float* wv = sm;                       // [Q]      w(last, s)
     float* xs = wv + Q;                   // [32][P]  w(last, s) x_s
     float* bs = xs + 32 * P;              // [32][N]
     T* raw = reinterpret_cast<T*>(bs + 32 * N);   // [2][32 (P + N)] raw x rows, then B rows, of a tile
-    __shared__ int full[kFoldPairs], nfull;
+    __shared__ int full[32], nfull;
     const int tid = threadIdx.x;
-    if (tid < 32) {
-        const int pr = blockIdx.x * kFoldPairs + tid;
-        const bool f = tid < kFoldPairs && pr < npairs && clen[pr] == Q;
+    if (tid < 32) {                       // per_block <= 32
+        const int pr = blockIdx.x * per_block + tid;
+        const bool f = tid < per_block && pr < npairs && clen[pr] == Q;
         const unsigned m = __ballot_sync(0xffffffffu, f);
         if (f) full[__popc(m & ((1u << tid) - 1u))] = pr;
         if (tid == 0) nfull = __popc(m);
