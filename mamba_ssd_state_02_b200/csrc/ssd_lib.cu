@@ -1066,10 +1066,14 @@ ssd_status launch_strict(const Plan& pl, char* ws, const T* x, const float* dt_r
     auto* acum = reinterpret_cast<float*>(ws + pl.off_acum);
     auto* states = reinterpret_cast<float*>(ws + pl.off_states);
     const int H = pl.H, G = pl.G, P = pl.P, N = pl.N, Q = pl.Q;
-    const size_t scan_smem = chunk_scan_smem(P, N, Q);
+    // Headdim 64 with heads per group a multiple of 4 (the Nemotron shape) takes the
+    // wide-tile chunk scan; both kernels give the same bits.
+    const bool wide = P == 64 && (H / G) % 4 == 0;
+    const size_t scan_smem = wide ? chunk_scan_wide_smem<T>(N, Q) : chunk_scan_smem(P, N, Q);
     void (*scan_kernel)(const T*, const T*, const T*, const float*, const float*, const float*, const float*,
                         const ChunkEntry*, const int32_t*, int, int, int, int, T*) = nullptr;
-    switch (P) {
+    switch (wide ? 0 : P) {
+        case 0: scan_kernel = k_strict_chunk_scan_wide<T>; break;
         case 16: scan_kernel = k_strict_chunk_scan<T, 16>; break;
         case 32: scan_kernel = k_strict_chunk_scan<T, 32>; break;
         case 64: scan_kernel = k_strict_chunk_scan<T, 64>; break;
@@ -1097,11 +1101,14 @@ ssd_status launch_strict(const Plan& pl, char* ws, const T* x, const float* dt_r
         {
             StageScope sc(ST_STRICT_STATE, st);
             const unsigned grid = (unsigned)((int64_t)mc * H);
-            const size_t sm = chunk_state_smem(P, N, Q);
+            const size_t sm = chunk_state_smem<T>(P, N, Q);
             switch (P * N / kThreads) {
 #define SSD_NOUT(V)                                                                                        \
-                case V: k_strict_chunk_state<T, V><<<grid, kThreads, sm, st>>>(x, B, dtc, acum, table, count, \
-                                                                              H, G, P, N, Q, states);        \
+                case V: if (cudaFuncSetAttribute(k_strict_chunk_state<T, V>,                                  \
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm) != cudaSuccess) \
+                        return fail(SSD_ERR_CUDA, "cudaFuncSetAttribute(strict chunk state)");               \
+                    k_strict_chunk_state<T, V><<<grid, kThreads, sm, st>>>(x, B, dtc, acum, table, count,     \
+                                                                          H, G, P, N, Q, states);            \
                     break;
                 SSD_NOUT(1) SSD_NOUT(2) SSD_NOUT(4) SSD_NOUT(8) SSD_NOUT(16) SSD_NOUT(32) SSD_NOUT(64)
 #undef SSD_NOUT

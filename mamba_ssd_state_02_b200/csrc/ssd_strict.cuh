@@ -115,22 +115,42 @@ k_strict_cumsum(const float* __restrict__ dt_raw, const float* __restrict__ dt_b
 // ---------------------------------------------------------------------------------
 // Prefill stage 2: chunk states S_c[p][n] (zero-start state at the chunk's last token).
 // One block per (chunk, head); thread owns column n = tid % N and the NOUT consecutive
-// rows (tid / N) * NOUT + k (NOUT = P N / 256).
+// rows (tid / N) * NOUT + k (NOUT = P N / 256). The chunk is walked in tiles of 32
+// tokens: the raw x and B rows of tile t+1 are copied into shared memory (16-byte
+// asynchronous copies) while tile t is used; each tile is converted once to FP32 (x
+// scaled by w(last, s)).
 template <typename T, int NOUT>
 __global__ void __launch_bounds__(kThreads)
 k_strict_chunk_state(const T* __restrict__ x, const T* __restrict__ B, const float* __restrict__ dtc,
                      const float* __restrict__ acum, const ChunkEntry* __restrict__ table,
                      const int32_t* __restrict__ count, int H, int G, int P, int N, int Q,
                      float* __restrict__ states) {
-    extern __shared__ float sm[];
+    extern __shared__ __align__(16) float sm[];
     float* w = sm;                       // [Q]
     float* xs = w + Q;                   // [32][P]   w(last, s) x_s
     float* bs = xs + 32 * P;             // [32][N]
+    T* raw = reinterpret_cast<T*>(bs + 32 * N);   // [2][32 (P + N)] raw x rows, then B rows, of a tile
     // Block b: head b % H of chunk b / H, so the heads of one chunk run side by side (B in L2).
     const int c = (int)(blockIdx.x / (unsigned)H);
     if (c >= *count) return;
     const int h = (int)(blockIdx.x % (unsigned)H), g = h / (H / G), tid = threadIdx.x;
     const ChunkEntry e = table[c];
+    constexpr int V = 16 / (int)sizeof(T);                 // elements per 16-byte copy
+    const int tile_elems = 32 * (P + N), ntile = (e.len + 31) / 32;
+    auto fetch = [&](int t) {                               // rows of tile t into buffer t & 1
+        T* dst = raw + (t & 1) * tile_elems;
+        const int rows = min(32, e.len - 32 * t), xp = P / V, bp = N / V;
+        for (int i = tid; i < rows * xp; i += kThreads) {
+            const int r = i / xp, k = i % xp;
+            cp_async16(dst + r * P + k * V, x + ((int64_t)(e.start + 32 * t + r) * H + h) * P + k * V);
+        }
+        for (int i = tid; i < rows * bp; i += kThreads) {
+            const int r = i / bp, k = i % bp;
+            cp_async16(dst + 32 * P + r * N + k * V, B + ((int64_t)(e.start + 32 * t + r) * G + g) * N + k * V);
+        }
+        cp_async_commit();
+    };
+    fetch(0);
     const float* ac = acum + ((int64_t)c * H + h) * Q;
     const float* dv = dtc + ((int64_t)c * H + h) * Q;
     const float last = ac[e.len - 1];
@@ -139,22 +159,22 @@ k_strict_chunk_state(const T* __restrict__ x, const T* __restrict__ B, const flo
     float acc[NOUT];
 #pragma unroll
     for (int k = 0; k < NOUT; ++k) acc[k] = 0.f;
-    __syncthreads();
-    for (int s0 = 0; s0 < e.len; s0 += 32) {
-        const int rows = min(32, e.len - s0);
-        for (int i = tid; i < rows * P; i += kThreads) {
-            const int r = i / P, pp = i % P;
-            const int64_t t = e.start + s0 + r;
-            xs[r * P + pp] = state_src(w[s0 + r], to_f32(x[(t * H + h) * P + pp]));
+    for (int t = 0; t < ntile; ++t) {
+        if (t + 1 < ntile) {
+            fetch(t + 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
         }
-        for (int i = tid; i < rows * N; i += kThreads) {
-            const int r = i / N, nn = i % N;
-            const int64_t t = e.start + s0 + r;
-            bs[r * N + nn] = to_f32(B[(t * G + g) * N + nn]);
-        }
+        __syncthreads();                                    // tile t landed (all threads' copies); w
+        const int rows = min(32, e.len - 32 * t);
+        const T* rx = raw + (t & 1) * tile_elems;
+        const T* rb = rx + 32 * P;
+        for (int i = tid; i < rows * P; i += kThreads) xs[i] = state_src(w[32 * t + i / P], to_f32(rx[i]));
+        for (int i = tid; i < rows * N; i += kThreads) bs[i] = to_f32(rb[i]);
         __syncthreads();
         for (int r = 0; r < rows; ++r) state_row<NOUT>(acc, xs + r * P + pb, bs[r * N + n]);
-        __syncthreads();
+        __syncthreads();                                    // xs, bs and buffer t & 1 free again
     }
     float* out = states + ((int64_t)c * H + h) * P * N;
 #pragma unroll
@@ -417,10 +437,202 @@ k_strict_chunk_scan(const T* __restrict__ x, const T* __restrict__ B, const T* _
     }
 }
 
+// Prefill stage 4 with wide register tiles, for P = 64 and heads per group a multiple of
+// 4: the same outputs, operations and order as k_strict_chunk_scan. One block per (chunk,
+// group, 32-row tile), 256 threads:
+//   1. C_t . B_s for the tile's rows and every source s < min(len, t0 + 32), once for the
+//      group, in 64-source slices (B rows transposed into shared memory; 4 x 2 (t, s) pairs
+//      per thread), kept s-major;
+//   2. the group's heads four at a time, 64 threads per head; thread (rg, pg) owns rows
+//      8 rg .. 8 rg + 7 and columns 4 pg .. 4 pg + 3 (32 outputs): C_t . h_in[p] in 16-wide
+//      slices of n (h_in transposed into shared memory), then the sources in 32-wide slices
+//      (the head's coefficients (C_t . B_s) w(t, s) and raw x rows in shared memory, x by
+//      asynchronous copies), then D x_t and the store.
+constexpr int kWideHS = 68;   // row stride of a transposed h_in slice (16-byte rows)
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 2)
+k_strict_chunk_scan_wide(const T* __restrict__ x, const T* __restrict__ B, const T* __restrict__ C,
+                         const float* __restrict__ D, const float* __restrict__ dtc, const float* __restrict__ acum,
+                         const float* __restrict__ hin, const ChunkEntry* __restrict__ table,
+                         const int32_t* __restrict__ count, int H, int G, int N, int Q, T* __restrict__ y) {
+    constexpr int P = 64;
+    constexpr int V = 16 / (int)sizeof(T);                 // elements per 16-byte copy
+    extern __shared__ __align__(16) float sm[];
+    float* cbs = sm;                      // [Q][32]  C_t . B_s: row s, column t (row of the tile)
+    float* ct = cbs + Q * 32;             // [N][32]  the tile's C rows, transposed
+    float* work = ct + N * 32;            // B^T slice [N][64]; or per head an h_in^T slice [16][68];
+                                          // or per head coefficients [32][32], then raw x [32][64]
+    const int ntile = Q / 32;
+    const int c = (int)(blockIdx.x / (unsigned)(ntile * G));
+    if (c >= *count) return;
+    const ChunkEntry e = table[c];
+    const int t0 = (int)(blockIdx.x % (unsigned)ntile) * 32;
+    if (t0 >= e.len) return;
+    const int g = (int)((blockIdx.x / (unsigned)ntile) % (unsigned)G), hpg = H / G, tid = threadIdx.x;
+    const int rows = min(32, e.len - t0);
+    const int nsrc = min(e.len, t0 + 32);                  // sources the tile's rows use: 0 .. nsrc-1
+    const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
+
+    // (0) The tile's C rows, transposed (zero past the chunk's end).
+    for (int i = tid; i < 32 * (N / 4); i += kThreads) {
+        const int t = i % 32, n0 = (i / 32) * 4;
+        const float4 v = t < rows ? load4(C + ((int64_t)(e.start + t0 + t) * G + g) * N + n0) : zero4;
+        ct[(n0 + 0) * 32 + t] = v.x;
+        ct[(n0 + 1) * 32 + t] = v.y;
+        ct[(n0 + 2) * 32 + t] = v.z;
+        ct[(n0 + 3) * 32 + t] = v.w;
+    }
+
+    // (1) C_t . B_s, left to right over n, 64 sources at a time.
+    {
+        const int ta = (tid % 8) * 4, sb = (tid / 8) * 2;   // rows ta..ta+3, slice sources sb, sb+1
+        for (int s0 = 0; s0 < nsrc; s0 += 64) {
+            __syncthreads();                                 // ct written; work free
+            for (int i = tid; i < 64 * (N / 4); i += kThreads) {
+                const int sl = i % 64, n0 = (i / 64) * 4;
+                const float4 v = s0 + sl < nsrc ? load4(B + ((int64_t)(e.start + s0 + sl) * G + g) * N + n0) : zero4;
+                work[(n0 + 0) * 64 + sl] = v.x;
+                work[(n0 + 1) * 64 + sl] = v.y;
+                work[(n0 + 2) * 64 + sl] = v.z;
+                work[(n0 + 3) * 64 + sl] = v.w;
+            }
+            __syncthreads();
+            float d[4][2];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) d[a][0] = d[a][1] = 0.f;
+            for (int n = 0; n < N; ++n) {
+                const float4 cv = *reinterpret_cast<const float4*>(ct + n * 32 + ta);
+                const float2 bv = *reinterpret_cast<const float2*>(work + n * 64 + sb);
+                const float cva[4] = {cv.x, cv.y, cv.z, cv.w};
+#pragma unroll
+                for (int a = 0; a < 4; ++a) {
+                    d[a][0] = dot_step(d[a][0], cva[a], bv.x);
+                    d[a][1] = dot_step(d[a][1], cva[a], bv.y);
+                }
+            }
+#pragma unroll
+            for (int b = 0; b < 2; ++b)
+                if (s0 + sb + b < nsrc)
+                    *reinterpret_cast<float4*>(cbs + (s0 + sb + b) * 32 + ta) = make_float4(d[0][b], d[1][b], d[2][b], d[3][b]);
+        }
+    }
+
+    // (2) The group's heads, four at a time.
+    const int hl = tid / 64, u = tid % 64, r0 = (u / 16) * 8, p0 = (u % 16) * 4;
+    float* hT = work + hl * (16 * kWideHS);
+    float* cf = work + hl * (32 * 32);
+    T* xs = reinterpret_cast<T*>(work + 4 * 32 * 32) + hl * (32 * P);
+    for (int hp = 0; hp < hpg; hp += 4) {
+        const int h = g * hpg + hp + hl;
+        const float* ac = acum + ((int64_t)c * H + h) * Q;
+        const float* dv = dtc + ((int64_t)c * H + h) * Q;
+        const float* hsrc = hin + ((int64_t)c * H + h) * P * N;
+        float acc[8][4];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+        // (2a) C_t . h_in[p], left to right over n, 16 at a time.
+        for (int n0 = 0; n0 < N; n0 += 16) {
+            __syncthreads();                                 // work free
+            for (int i = u; i < P * 16; i += 64) {
+                const int p = i / 16, nn = i % 16;
+                hT[nn * kWideHS + p] = hsrc[(int64_t)p * N + n0 + nn];
+            }
+            __syncthreads();
+#pragma unroll 4
+            for (int nn = 0; nn < 16; ++nn) {
+                const float4 c0 = *reinterpret_cast<const float4*>(ct + (n0 + nn) * 32 + r0);
+                const float4 c1 = *reinterpret_cast<const float4*>(ct + (n0 + nn) * 32 + r0 + 4);
+                const float4 hv = *reinterpret_cast<const float4*>(hT + nn * kWideHS + p0);
+                const float cva[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+                const float hva[4] = {hv.x, hv.y, hv.z, hv.w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) acc[i][j] = dot_step(acc[i][j], cva[i], hva[j]);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float at = ac[t0 + r0 + i];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = y_begin(acc[i][j], at);
+        }
+        // (2b) Sources s = 0..t, left to right, 32 at a time.
+        for (int s0 = 0; s0 <= t0; s0 += 32) {
+            __syncthreads();                                 // work free
+            for (int i = u; i < 32 * (P / V); i += 64) {
+                const int r = i / (P / V), k = i % (P / V);
+                if (s0 + r < e.len)
+                    cp_async16(xs + r * P + k * V, x + ((int64_t)(e.start + s0 + r) * H + h) * P + k * V);
+            }
+            cp_async_commit();
+            for (int i = u; i < 32 * 32; i += 64) {
+                const int sl = i / 32, tl = i % 32, s_ = s0 + sl, t = t0 + tl;
+                cf[i] = s_ <= t && s_ < e.len ? mix_coef(cbs[s_ * 32 + tl], ac[t], ac[s_], dv[s_]) : 0.f;
+            }
+            cp_async_wait<0>();
+            __syncthreads();
+            if (s0 < t0) {                                   // every row of the tile sees all 32 sources
+#pragma unroll 4
+                for (int k = 0; k < 32; ++k) {
+                    const float4 f0 = *reinterpret_cast<const float4*>(cf + k * 32 + r0);
+                    const float4 f1 = *reinterpret_cast<const float4*>(cf + k * 32 + r0 + 4);
+                    const float4 xv = load4(xs + k * P + p0);
+                    const float fva[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+                    const float xva[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) acc[i][j] = y_step(acc[i][j], fva[i], xva[j]);
+                }
+            } else {                                         // diagonal slice: sources s <= t
+                for (int k = 0; k < 32; ++k) {
+                    const float4 f0 = *reinterpret_cast<const float4*>(cf + k * 32 + r0);
+                    const float4 f1 = *reinterpret_cast<const float4*>(cf + k * 32 + r0 + 4);
+                    const float4 xv = load4(xs + k * P + p0);
+                    const float fva[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+                    const float xva[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        if (k > r0 + i) continue;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) acc[i][j] = y_step(acc[i][j], fva[i], xva[j]);
+                    }
+                }
+            }
+        }
+        // (2c) D skip and store.
+        const float Dh = D[h];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int tt = r0 + i;
+            if (tt >= rows) continue;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int64_t o = ((int64_t)(e.start + t0 + tt) * H + h) * P + p0 + j;
+                y[o] = from_f32<T>(y_end(acc[i][j], Dh, to_f32(x[o])));
+            }
+        }
+    }
+}
+
+template <typename T>
+inline size_t chunk_scan_wide_smem(int N, int Q) {
+    const int work_a = N * 64, work_b = 4 * 16 * kWideHS, work_c = 4 * 32 * 32 + 4 * 32 * 64 * (int)sizeof(T) / 4;
+    const int work = work_a > work_b ? (work_a > work_c ? work_a : work_c) : (work_b > work_c ? work_b : work_c);
+    return sizeof(float) * (Q * 32 + N * 32 + work);
+}
+
 inline size_t chunk_scan_smem(int P, int N, int Q) {
     return sizeof(float) * (32 * (N + 4) + scan_cb_region(N, Q) + 32 * Q + 2 * Q + P * kHPad + 32 * P);
 }
-inline size_t chunk_state_smem(int P, int N, int Q) { return sizeof(float) * (Q + 32 * P + 32 * N); }
+template <typename T>
+inline size_t chunk_state_smem(int P, int N, int Q) {
+    return sizeof(float) * (Q + 32 * P + 32 * N) + sizeof(T) * 2 * 32 * (P + N);
+}
 
 // ---------------------------------------------------------------------------------
 // Prefill stage 5: the chunk cache's open chunk (a partial last chunk's tokens) and its
