@@ -804,8 +804,10 @@ def ncu_case(args):
     W + K decode steps of 256 sequences on a random 512 MiB FP32 state; `prefill`
     runs W + K prefill calls of the long-context workload; `strict` runs W + K strict
     prefill calls of the long-context workload, then W + K chunk-emulating decode
-    steps of 256 sequences with half-full open chunks; `conv` runs W + K conv1d prologue
-    calls over the long-context workload's tokens."""
+    steps of 256 sequences with half-full open chunks; `fold` runs W + K chunk-emulating
+    decode steps of 256 sequences whose open chunks are one token short of full, so every
+    step folds every (sequence, head) chunk; `conv` runs W + K conv1d prologue calls over
+    the long-context workload's tokens."""
     from mamba_ssd_state_02_b200 import build
     build.build()
     from mamba_ssd_state_02_b200 import ssd
@@ -838,19 +840,21 @@ def ncu_case(args):
         for _ in range(args.warmup + args.steps):
             ssd.conv1d_fwd(cx, ci["weight"], ci["bias"], w.nheads, w.headdim, w.ngroups, w.dstate,
                            conv_state=ci["conv_state"], x=xo, B=bo, C=co, conv_state_out=so)
-    elif args.ncu_case == "strict":
-        # strict prefill of the long-context workload, then chunk-emulating decode steps of
-        # 256 sequences whose open chunks hold 64 tokens
-        w = W.config(PREFILL_CONFIG)
-        inp = W.make_all(w, device=dev)
-        L = w.seqlens[0]
-        r4 = lambda t: t.view(w.nseq, L, *t.shape[1:])
-        y = torch.empty_like(r4(inp["x"]))
-        cache = ssd.ChunkCache.empty(w.nseq, w.nheads, w.headdim, w.ngroups, w.dstate, w.chunk, w.dtype, dev)
-        for _ in range(args.warmup + args.steps):
-            ssd.strict_scan_fwd(r4(inp["x"]), r4(inp["dt_raw"]), inp["dt_bias"], inp["A"], r4(inp["B"]),
-                                r4(inp["C"]), inp["D"], cache, y=y)
-        del inp, y, cache
+    elif args.ncu_case in ("strict", "fold"):
+        # strict: the strict prefill of the long-context workload, then chunk-emulating
+        # decode steps of 256 sequences whose open chunks hold 64 tokens; fold: the decode
+        # steps only, every open chunk one token short of full
+        if args.ncu_case == "strict":
+            w = W.config(PREFILL_CONFIG)
+            inp = W.make_all(w, device=dev)
+            L = w.seqlens[0]
+            r4 = lambda t: t.view(w.nseq, L, *t.shape[1:])
+            y = torch.empty_like(r4(inp["x"]))
+            cache = ssd.ChunkCache.empty(w.nseq, w.nheads, w.headdim, w.ngroups, w.dstate, w.chunk, w.dtype, dev)
+            for _ in range(args.warmup + args.steps):
+                ssd.strict_scan_fwd(r4(inp["x"]), r4(inp["dt_raw"]), inp["dt_bias"], inp["A"], r4(inp["B"]),
+                                    r4(inp["C"]), inp["D"], cache, y=y)
+            del inp, y, cache
         wd = W.config(DECODE_CONFIG)
         nseq, H, P, G, N, Q = wd.nseq, wd.nheads, wd.headdim, wd.ngroups, wd.dstate, wd.chunk
         par = W.make_params(wd, device=dev)
@@ -863,11 +867,13 @@ def ncu_case(args):
         dc.B.copy_(tk["B"].view(nseq, Q, G, N).transpose(1, 2))
         dc.dt.fill_(0.01)
         dc.acum.copy_(-0.01 * torch.arange(1, Q + 1, device=dev, dtype=torch.float32).expand(nseq, H, Q))
-        dc.len.fill_(Q // 2)
+        dc.len.fill_(Q - 1 if args.ncu_case == "fold" else Q // 2)
         rows = torch.arange(nseq, device=dev, dtype=torch.int64)
         tok = W.make_tokens(wd, 0, 0, rows=rows)
         yd = torch.empty(nseq, H, P, dtype=wd.dtype, device=dev)
         for _ in range(args.warmup + args.steps):
+            if args.ncu_case == "fold":
+                dc.len.fill_(Q - 1)
             ssd.strict_state_update(dc, tok["x"], tok["dt_raw"], par["dt_bias"], par["A"], tok["B"], tok["C"],
                                     par["D"], y=yd)
     else:
@@ -891,7 +897,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--ncu-case", choices=["decode", "prefill", "strict", "conv"], default=None,
+    ap.add_argument("--ncu-case", choices=["decode", "prefill", "strict", "fold", "conv"], default=None,
                     help="run a small fixed workload for an ncu capture instead of the benchmark")
     args = ap.parse_args(argv)
     if args.ncu_case:

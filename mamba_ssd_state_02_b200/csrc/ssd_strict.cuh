@@ -68,23 +68,62 @@ __device__ __forceinline__ bool bad_A(float a) { return !(a <= 0.f) || isinf(a);
 
 constexpr int kThreads = 256;
 
-// acc[k] += xr[k] * bv for k < NOUT (one source row of a chunk state), 16-byte shared loads.
+// The register tile of a chunk-state sum S[p][n] = sum_s wx_s[p] b_s[n], sources left to
+// right, with NOUT = P N / 256 outputs per thread. When NOUT is a multiple of 4 a thread
+// owns R = NOUT / 4 consecutive rows p0.. and 4 consecutive columns n0.. (per source one
+// 16-byte load of b and R/4 of wx for 4R FMAs); otherwise one column n0 and NOUT rows.
+// acc[i][j] is output (p0 + i, n0 + j).
 template <int NOUT>
-__device__ __forceinline__ void state_row(float (&acc)[NOUT], const float* xr, float bv) {
-    if constexpr (NOUT % 4 == 0) {
-#pragma unroll
-        for (int k = 0; k < NOUT; k += 4) {
-            const float4 v = *reinterpret_cast<const float4*>(xr + k);
-            acc[k] = state_step(acc[k], v.x, bv);
-            acc[k + 1] = state_step(acc[k + 1], v.y, bv);
-            acc[k + 2] = state_step(acc[k + 2], v.z, bv);
-            acc[k + 3] = state_step(acc[k + 3], v.w, bv);
+struct StateTile {
+    static constexpr bool kWide = NOUT % 4 == 0;
+    static constexpr int R = kWide ? NOUT / 4 : NOUT, CN = kWide ? 4 : 1;
+    float acc[R][CN];
+    int p0, n0;
+    __device__ __forceinline__ StateTile(int tid, int N) {
+        if (kWide) {
+            n0 = (tid % (N / 4)) * 4;
+            p0 = (tid / (N / 4)) * R;
+        } else {
+            n0 = tid % N;
+            p0 = (tid / N) * NOUT;
         }
-    } else {
 #pragma unroll
-        for (int k = 0; k < NOUT; ++k) acc[k] = state_step(acc[k], xr[k], bv);
+        for (int i = 0; i < R; ++i)
+#pragma unroll
+            for (int j = 0; j < CN; ++j) acc[i][j] = 0.f;
     }
-}
+    // One source: xr = its wx row [P], br = its b row [N] (shared memory).
+    __device__ __forceinline__ void row(const float* xr, const float* br) {
+        float bv[CN];
+        if constexpr (kWide) {
+            const float4 b = *reinterpret_cast<const float4*>(br + n0);
+            bv[0] = b.x;
+            bv[1] = b.y;
+            bv[2] = b.z;
+            bv[3] = b.w;
+        } else {
+            bv[0] = br[n0];
+        }
+        if constexpr (R % 4 == 0) {
+#pragma unroll
+            for (int i = 0; i < R; i += 4) {
+                const float4 v = *reinterpret_cast<const float4*>(xr + p0 + i);
+                const float va[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int j = 0; j < CN; ++j) acc[i + a][j] = state_step(acc[i + a][j], va[a], bv[j]);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < R; ++i) {
+                const float v = xr[p0 + i];
+#pragma unroll
+                for (int j = 0; j < CN; ++j) acc[i][j] = state_step(acc[i][j], v, bv[j]);
+            }
+        }
+    }
+};
 
 // ---------------------------------------------------------------------------------
 // Prefill stage 1: dt and Acum per (chunk, head), left to right, [chunk][H][Q] (zero past
@@ -114,8 +153,8 @@ k_strict_cumsum(const float* __restrict__ dt_raw, const float* __restrict__ dt_b
 
 // ---------------------------------------------------------------------------------
 // Prefill stage 2: chunk states S_c[p][n] (zero-start state at the chunk's last token).
-// One block per (chunk, head); thread owns column n = tid % N and the NOUT consecutive
-// rows (tid / N) * NOUT + k (NOUT = P N / 256). The chunk is walked in tiles of 32
+// One block per (chunk, head); a thread owns a StateTile of NOUT = P N / 256 outputs.
+// The chunk is walked in tiles of 32
 // tokens: the raw x and B rows of tile t+1 are copied into shared memory (16-byte
 // asynchronous copies) while tile t is used; each tile is converted once to FP32 (x
 // scaled by w(last, s)).
@@ -155,10 +194,7 @@ k_strict_chunk_state(const T* __restrict__ x, const T* __restrict__ B, const flo
     const float* dv = dtc + ((int64_t)c * H + h) * Q;
     const float last = ac[e.len - 1];
     for (int s = tid; s < e.len; s += kThreads) w[s] = src_weight(last, ac[s], dv[s]);
-    const int n = tid % N, pb = (tid / N) * NOUT;
-    float acc[NOUT];
-#pragma unroll
-    for (int k = 0; k < NOUT; ++k) acc[k] = 0.f;
+    StateTile<NOUT> tile(tid, N);
     for (int t = 0; t < ntile; ++t) {
         if (t + 1 < ntile) {
             fetch(t + 1);
@@ -173,12 +209,14 @@ k_strict_chunk_state(const T* __restrict__ x, const T* __restrict__ B, const flo
         for (int i = tid; i < rows * P; i += kThreads) xs[i] = state_src(w[32 * t + i / P], to_f32(rx[i]));
         for (int i = tid; i < rows * N; i += kThreads) bs[i] = to_f32(rb[i]);
         __syncthreads();
-        for (int r = 0; r < rows; ++r) state_row<NOUT>(acc, xs + r * P + pb, bs[r * N + n]);
+        for (int r = 0; r < rows; ++r) tile.row(xs + r * P, bs + r * N);
         __syncthreads();                                    // xs, bs and buffer t & 1 free again
     }
     float* out = states + ((int64_t)c * H + h) * P * N;
 #pragma unroll
-    for (int k = 0; k < NOUT; ++k) out[(pb + k) * N + n] = acc[k];
+    for (int i = 0; i < StateTile<NOUT>::R; ++i)
+#pragma unroll
+        for (int j = 0; j < StateTile<NOUT>::CN; ++j) out[(tile.p0 + i) * N + tile.n0 + j] = tile.acc[i][j];
 }
 
 // ---------------------------------------------------------------------------------
@@ -819,8 +857,8 @@ inline size_t decode_smem(int H, int G, int N, int Q) { return sizeof(float) * (
 // one vote) and folds the full ones one after the other, so a step that fills no chunk
 // costs one small launch. A fold walks the chunk in tiles of 32 sources: the raw x and B
 // rows of tile t+1 are copied into shared memory (16-byte asynchronous copies) while tile
-// t is used; each tile is converted once to FP32 (x scaled by w(last, s)). Thread owns
-// column n = tid % N and the NOUT consecutive rows (tid / N) * NOUT + k.
+// t is used; each tile is converted once to FP32 (x scaled by w(last, s)). A thread owns a
+// StateTile of NOUT = P N / 256 outputs.
 
 template <typename T, int NOUT>
 __global__ void __launch_bounds__(kThreads)
@@ -859,10 +897,7 @@ k_strict_fold(float* __restrict__ cstate, const T* __restrict__ cx, const T* __r
         const float last = cacum[sh * Q + Q - 1];
         for (int sidx = tid; sidx < Q; sidx += kThreads)
             wv[sidx] = src_weight(last, cacum[sh * Q + sidx], cdt[sh * Q + sidx]);
-        const int n = tid % N, pb = (tid / N) * NOUT;
-        float acc[NOUT];
-#pragma unroll
-        for (int k = 0; k < NOUT; ++k) acc[k] = 0.f;
+        StateTile<NOUT> tile(tid, N);
         const int ntile = Q / 32;
         for (int t = 0; t < ntile; ++t) {
             if (t + 1 < ntile) {
@@ -877,15 +912,17 @@ k_strict_fold(float* __restrict__ cstate, const T* __restrict__ cx, const T* __r
             for (int i = tid; i < 32 * P; i += kThreads) xs[i] = state_src(wv[32 * t + i / P], to_f32(rx[i]));
             for (int i = tid; i < 32 * N; i += kThreads) bs[i] = to_f32(rb[i]);
             __syncthreads();
-            for (int r = 0; r < 32; ++r) state_row<NOUT>(acc, xs + r * P + pb, bs[r * N + n]);
+            for (int r = 0; r < 32; ++r) tile.row(xs + r * P, bs + r * N);
             __syncthreads();                                // xs, bs and buffer t & 1 free again
         }
         float* hout = cstate + sh * P * N;
 #pragma unroll
-        for (int k = 0; k < NOUT; ++k) {
-            const int64_t o = (int64_t)(pb + k) * N + n;
-            hout[o] = pass(hout[o], last, acc[k]);
-        }
+        for (int i = 0; i < StateTile<NOUT>::R; ++i)
+#pragma unroll
+            for (int j = 0; j < StateTile<NOUT>::CN; ++j) {
+                const int64_t o = (int64_t)(tile.p0 + i) * N + tile.n0 + j;
+                hout[o] = pass(hout[o], last, tile.acc[i][j]);
+            }
         if (tid == 0) clen[sh] = 0;
     };
     for (int f = 0; f < nfull; ++f) fold_one(full[f]);
