@@ -10,7 +10,8 @@
 // How it is met here. Both paths evaluate the chunked algorithm (chunks of Q tokens
 // anchored at the sequence start) through the functions in `namespace strict` below,
 // each a fixed sequence of correctly rounded FP32 operations (__fadd_rn, __fmul_rn,
-// __fmaf_rn: never contracted or reordered by the compiler):
+// __fmaf_rn: never contracted or reordered by the compiler) and deterministic exponentials
+// (strict_exp for the decays and weights, library expf/log1pf for softplus):
 //
 //   dt_s      = softplus(dt_raw_s + dt_bias)
 //   Acum_s    = Acum_{s-1} + dt_s A            (left to right from Acum_{-1} = 0)
@@ -41,12 +42,20 @@ __device__ __forceinline__ float dt_of(float raw, float bias) {
     const float z = __fadd_rn(raw, bias);
     return z > 0.f ? __fadd_rn(z, log1pf(expf(-z))) : log1pf(expf(z));
 }
+// exp(x) of the decays and weights: one correctly rounded multiply by log2(e), then the
+// hardware base-2 exponential (relative error ~2^-21). Deterministic, and the same function
+// on every path, which is all bitwise invariance needs.
+__device__ __forceinline__ float strict_exp(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(__fmul_rn(x, 1.4426950408889634f)));
+    return y;
+}
 __device__ __forceinline__ float acum_next(float prev, float dt, float a) {
     return __fadd_rn(prev, __fmul_rn(dt, a));
 }
 // w(t, s) = exp(Acum_t - Acum_s) dt_s
 __device__ __forceinline__ float src_weight(float acum_t, float acum_s, float dt_s) {
-    return __fmul_rn(expf(__fsub_rn(acum_t, acum_s)), dt_s);
+    return __fmul_rn(strict_exp(__fsub_rn(acum_t, acum_s)), dt_s);
 }
 // one step of a left-to-right dot product
 __device__ __forceinline__ float dot_step(float acc, float u, float v) { return __fmaf_rn(u, v, acc); }
@@ -55,14 +64,14 @@ __device__ __forceinline__ float mix_coef(float cb, float acum_t, float acum_s, 
     return __fmul_rn(cb, src_weight(acum_t, acum_s, dt_s));
 }
 // y accumulator: start from the incoming-state term, add sources left to right, add D x_t
-__device__ __forceinline__ float y_begin(float c_dot_h, float acum_t) { return __fmul_rn(c_dot_h, expf(acum_t)); }
+__device__ __forceinline__ float y_begin(float c_dot_h, float acum_t) { return __fmul_rn(c_dot_h, strict_exp(acum_t)); }
 __device__ __forceinline__ float y_step(float acc, float coef, float xs) { return __fmaf_rn(coef, xs, acc); }
 __device__ __forceinline__ float y_end(float acc, float Dh, float xt) { return __fmaf_rn(Dh, xt, acc); }
 // chunk state: source term w(last, s) x_s[p], accumulated left to right against B_s[n]
 __device__ __forceinline__ float state_src(float w, float xs) { return __fmul_rn(w, xs); }
 __device__ __forceinline__ float state_step(float acc, float wx, float b) { return __fmaf_rn(wx, b, acc); }
 // state passing across a chunk boundary
-__device__ __forceinline__ float pass(float h, float acum_last, float S) { return __fmaf_rn(expf(acum_last), h, S); }
+__device__ __forceinline__ float pass(float h, float acum_last, float S) { return __fmaf_rn(strict_exp(acum_last), h, S); }
 
 __device__ __forceinline__ bool bad_A(float a) { return !(a <= 0.f) || isinf(a); }
 
