@@ -120,3 +120,31 @@ def test_snapshots_inside_long_segments(ssd, cuda_dev, seqlens, varlen, seg, I):
     for k in range(sn.shape[0]):
         assert rel_err(sn[k], sn_ref[k]) <= TOL_STATE, k
 
+
+
+@pytest.mark.slow
+def test_snapshots_long_context_full_size(ssd, cuda_dev):
+    """The long-context workload (1 x 65536 tokens, 64 heads, chunk 256) with snapshots
+    every 2048 tokens. The planner keeps its 7296-token segments, so every segment is cut
+    into pieces at the snapshot positions. One head per B/C group is checked against the
+    oracle at all 32 snapshots, and at the final state."""
+    w = W.config(2)
+    L, I = w.seqlens[0], 2048
+    dims = ssd.make_dims(L, w.nheads, w.headdim, w.ngroups, w.dstate, ssd.SSD_DTYPE_BF16, batch=1, seqlen=L)
+    assert ssd.segment_tokens(dims, w.chunk) % I != 0          # cuts inside segments
+    inp = W.make_all(w, device=cuda_dev)
+    rs = lambda t: t.reshape(1, L, *t.shape[1:])
+    y, fin, sn = ssd.scan_fwd(rs(inp["x"]), rs(inp["dt_raw"]), inp["dt_bias"], inp["A"], rs(inp["B"]),
+                              rs(inp["C"]), inp["D"], init_state=inp["init_state"], chunk=w.chunk,
+                              snapshot_tokens=I)
+    ssd.device_status()
+    assert sn.shape == (L // I, w.nheads, w.headdim, w.dstate)
+    heads = [0, 9, 18, 27, 36, 45, 54, 63]                     # one head in each of the 8 groups
+    cpu = {k: (None if v is None else v.cpu()) for k, v in inp.items()}
+    _, fin_ref, sn_ref = O.ssd_scan(cpu["x"], cpu["dt_raw"], cpu["dt_bias"], cpu["A"], cpu["B"], cpu["C"],
+                                    cpu["D"], init_state=cpu["init_state"], batch=1,
+                                    pairs=[(0, h) for h in heads], want_y=False, snapshot_tokens=I)
+    for k, h in enumerate(heads):
+        assert rel_err(fin[0, h], fin_ref[k]) <= TOL_STATE, h
+        for m in range(L // I):
+            assert rel_err(sn[m, h], torch.as_tensor(sn_ref[k][m])) <= TOL_STATE, (h, m)
