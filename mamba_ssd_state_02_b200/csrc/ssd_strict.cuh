@@ -72,6 +72,11 @@ __device__ __forceinline__ float state_src(float w, float xs) { return __fmul_rn
 __device__ __forceinline__ float state_step(float acc, float wx, float b) { return __fmaf_rn(wx, b, acc); }
 // state passing across a chunk boundary
 __device__ __forceinline__ float pass(float h, float acum_last, float S) { return __fmaf_rn(strict_exp(acum_last), h, S); }
+// Two independent steps of the sums above at once: per component the same correctly
+// rounded FMA (u v + acc) as the scalar steps, so a tile that packs its outputs in pairs
+// produces the same bits as one that does not. Halves the issued FMA instructions.
+__device__ __forceinline__ float2 step2(float2 acc, float2 u, float2 v) { return __ffma2_rn(u, v, acc); }
+__device__ __forceinline__ float2 splat(float v) { return make_float2(v, v); }
 
 __device__ __forceinline__ bool bad_A(float a) { return !(a <= 0.f) || isinf(a); }
 
@@ -81,13 +86,15 @@ constexpr int kThreads = 256;
 // right, with NOUT = P N / 256 outputs per thread. When NOUT is a multiple of 4 a thread
 // owns R = NOUT / 4 consecutive rows p0.. and 4 consecutive columns n0.. (per source one
 // 16-byte load of b and R/4 of wx for 4R FMAs); otherwise one column n0 and NOUT rows.
-// acc[i][j] is output (p0 + i, n0 + j).
+// Rows are held in pairs (acc[i / 2][j], component i % 2), so that four rows of a source
+// update with packed FMAs; at(i, j) is output (p0 + i, n0 + j).
 template <int NOUT>
 struct StateTile {
     static constexpr bool kWide = NOUT % 4 == 0;
     static constexpr int R = kWide ? NOUT / 4 : NOUT, CN = kWide ? 4 : 1;
-    float acc[R][CN];
+    float2 acc[(R + 1) / 2][CN];
     int p0, n0;
+    __device__ __forceinline__ float& at(int i, int j) { return (i & 1) ? acc[i >> 1][j].y : acc[i >> 1][j].x; }
     __device__ __forceinline__ StateTile(int tid, int N) {
         if (kWide) {
             n0 = (tid % (N / 4)) * 4;
@@ -97,9 +104,9 @@ struct StateTile {
             p0 = (tid / N) * NOUT;
         }
 #pragma unroll
-        for (int i = 0; i < R; ++i)
+        for (int i = 0; i < (R + 1) / 2; ++i)
 #pragma unroll
-            for (int j = 0; j < CN; ++j) acc[i][j] = 0.f;
+            for (int j = 0; j < CN; ++j) acc[i][j] = make_float2(0.f, 0.f);
     }
     // One source: xr = its wx row [P], br = its b row [N] (shared memory).
     __device__ __forceinline__ void row(const float* xr, const float* br) {
@@ -114,21 +121,24 @@ struct StateTile {
             bv[0] = br[n0];
         }
         if constexpr (R % 4 == 0) {
+            float2 bb[CN];
+#pragma unroll
+            for (int j = 0; j < CN; ++j) bb[j] = splat(bv[j]);
 #pragma unroll
             for (int i = 0; i < R; i += 4) {
                 const float4 v = *reinterpret_cast<const float4*>(xr + p0 + i);
-                const float va[4] = {v.x, v.y, v.z, v.w};
+                const float2 va[2] = {make_float2(v.x, v.y), make_float2(v.z, v.w)};
 #pragma unroll
-                for (int a = 0; a < 4; ++a)
+                for (int a = 0; a < 2; ++a)
 #pragma unroll
-                    for (int j = 0; j < CN; ++j) acc[i + a][j] = state_step(acc[i + a][j], va[a], bv[j]);
+                    for (int j = 0; j < CN; ++j) acc[i / 2 + a][j] = step2(acc[i / 2 + a][j], va[a], bb[j]);
             }
         } else {
 #pragma unroll
             for (int i = 0; i < R; ++i) {
                 const float v = xr[p0 + i];
 #pragma unroll
-                for (int j = 0; j < CN; ++j) acc[i][j] = state_step(acc[i][j], v, bv[j]);
+                for (int j = 0; j < CN; ++j) at(i, j) = state_step(at(i, j), v, bv[j]);
             }
         }
     }
@@ -225,7 +235,7 @@ k_strict_chunk_state(const T* __restrict__ x, const T* __restrict__ B, const flo
 #pragma unroll
     for (int i = 0; i < StateTile<NOUT>::R; ++i)
 #pragma unroll
-        for (int j = 0; j < StateTile<NOUT>::CN; ++j) out[(tile.p0 + i) * N + tile.n0 + j] = tile.acc[i][j];
+        for (int j = 0; j < StateTile<NOUT>::CN; ++j) out[(tile.p0 + i) * N + tile.n0 + j] = tile.at(i, j);
 }
 
 // ---------------------------------------------------------------------------------
@@ -545,23 +555,24 @@ k_strict_chunk_scan_wide(const T* __restrict__ x, const T* __restrict__ B, const
                 work[(n0 + 3) * 64 + sl] = v.w;
             }
             __syncthreads();
-            float d[4][2];
+            float2 d[2][2];                                  // d[a][b]: rows ta + 2a, ta + 2a + 1; source sb + b
 #pragma unroll
-            for (int a = 0; a < 4; ++a) d[a][0] = d[a][1] = 0.f;
+            for (int a = 0; a < 2; ++a) d[a][0] = d[a][1] = make_float2(0.f, 0.f);
             for (int n = 0; n < N; ++n) {
                 const float4 cv = *reinterpret_cast<const float4*>(ct + n * 32 + ta);
                 const float2 bv = *reinterpret_cast<const float2*>(work + n * 64 + sb);
-                const float cva[4] = {cv.x, cv.y, cv.z, cv.w};
+                const float2 cva[2] = {make_float2(cv.x, cv.y), make_float2(cv.z, cv.w)};
+                const float2 bx = splat(bv.x), by = splat(bv.y);
 #pragma unroll
-                for (int a = 0; a < 4; ++a) {
-                    d[a][0] = dot_step(d[a][0], cva[a], bv.x);
-                    d[a][1] = dot_step(d[a][1], cva[a], bv.y);
+                for (int a = 0; a < 2; ++a) {
+                    d[a][0] = step2(d[a][0], cva[a], bx);
+                    d[a][1] = step2(d[a][1], cva[a], by);
                 }
             }
 #pragma unroll
             for (int b = 0; b < 2; ++b)
                 if (s0 + sb + b < nsrc)
-                    *reinterpret_cast<float4*>(cbs + (s0 + sb + b) * 32 + ta) = make_float4(d[0][b], d[1][b], d[2][b], d[3][b]);
+                    *reinterpret_cast<float4*>(cbs + (s0 + sb + b) * 32 + ta) = make_float4(d[0][b].x, d[0][b].y, d[1][b].x, d[1][b].y);
         }
     }
 
@@ -575,11 +586,11 @@ k_strict_chunk_scan_wide(const T* __restrict__ x, const T* __restrict__ B, const
         const float* ac = acum + ((int64_t)c * H + h) * Q;
         const float* dv = dtc + ((int64_t)c * H + h) * Q;
         const float* hsrc = hin + ((int64_t)c * H + h) * P * N;
-        float acc[8][4];
+        float2 acc[4][4];                                    // rows r0 + 2i, r0 + 2i + 1; column p0 + j
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+            for (int j = 0; j < 4; ++j) acc[i][j] = make_float2(0.f, 0.f);
         // (2a) C_t . h_in[p], left to right over n, 16 at a time.
         for (int n0 = 0; n0 < N; n0 += 16) {
             __syncthreads();                                 // work free
@@ -593,19 +604,20 @@ k_strict_chunk_scan_wide(const T* __restrict__ x, const T* __restrict__ B, const
                 const float4 c0 = *reinterpret_cast<const float4*>(ct + (n0 + nn) * 32 + r0);
                 const float4 c1 = *reinterpret_cast<const float4*>(ct + (n0 + nn) * 32 + r0 + 4);
                 const float4 hv = *reinterpret_cast<const float4*>(hT + nn * kWideHS + p0);
-                const float cva[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-                const float hva[4] = {hv.x, hv.y, hv.z, hv.w};
+                const float2 cva[4] = {make_float2(c0.x, c0.y), make_float2(c0.z, c0.w), make_float2(c1.x, c1.y),
+                                       make_float2(c1.z, c1.w)};
+                const float2 hva[4] = {splat(hv.x), splat(hv.y), splat(hv.z), splat(hv.w)};
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
+                for (int i = 0; i < 4; ++i)
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) acc[i][j] = dot_step(acc[i][j], cva[i], hva[j]);
+                    for (int j = 0; j < 4; ++j) acc[i][j] = step2(acc[i][j], cva[i], hva[j]);
             }
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float at = ac[t0 + r0 + i];
+        for (int i = 0; i < 4; ++i) {
+            const float a0 = ac[t0 + r0 + 2 * i], a1 = ac[t0 + r0 + 2 * i + 1];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) acc[i][j] = y_begin(acc[i][j], at);
+            for (int j = 0; j < 4; ++j) acc[i][j] = make_float2(y_begin(acc[i][j].x, a0), y_begin(acc[i][j].y, a1));
         }
         // (2b) Sources s = 0..t, left to right, 32 at a time.
         for (int s0 = 0; s0 <= t0; s0 += 32) {
@@ -628,25 +640,33 @@ k_strict_chunk_scan_wide(const T* __restrict__ x, const T* __restrict__ B, const
                     const float4 f0 = *reinterpret_cast<const float4*>(cf + k * 32 + r0);
                     const float4 f1 = *reinterpret_cast<const float4*>(cf + k * 32 + r0 + 4);
                     const float4 xv = load4(xs + k * P + p0);
-                    const float fva[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
-                    const float xva[4] = {xv.x, xv.y, xv.z, xv.w};
+                    const float2 fva[4] = {make_float2(f0.x, f0.y), make_float2(f0.z, f0.w), make_float2(f1.x, f1.y),
+                                           make_float2(f1.z, f1.w)};
+                    const float2 xva[4] = {splat(xv.x), splat(xv.y), splat(xv.z), splat(xv.w)};
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
+                    for (int i = 0; i < 4; ++i)
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) acc[i][j] = y_step(acc[i][j], fva[i], xva[j]);
+                        for (int j = 0; j < 4; ++j) acc[i][j] = step2(acc[i][j], fva[i], xva[j]);
                 }
             } else {                                         // diagonal slice: sources s <= t
                 for (int k = 0; k < 32; ++k) {
                     const float4 f0 = *reinterpret_cast<const float4*>(cf + k * 32 + r0);
                     const float4 f1 = *reinterpret_cast<const float4*>(cf + k * 32 + r0 + 4);
                     const float4 xv = load4(xs + k * P + p0);
-                    const float fva[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+                    const float2 fva[4] = {make_float2(f0.x, f0.y), make_float2(f0.z, f0.w), make_float2(f1.x, f1.y),
+                                           make_float2(f1.z, f1.w)};
                     const float xva[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        if (k > r0 + i) continue;
+                    for (int i = 0; i < 4; ++i) {
+                        // rows r0 + 2i (takes source k while k <= r0 + 2i) and r0 + 2i + 1
+                        if (k > r0 + 2 * i + 1) continue;
+                        if (k == r0 + 2 * i + 1) {
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) acc[i][j] = y_step(acc[i][j], fva[i], xva[j]);
+                            for (int j = 0; j < 4; ++j) acc[i][j].y = y_step(acc[i][j].y, fva[i].y, xva[j]);
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) acc[i][j] = step2(acc[i][j], fva[i], splat(xva[j]));
+                        }
                     }
                 }
             }
@@ -660,7 +680,8 @@ k_strict_chunk_scan_wide(const T* __restrict__ x, const T* __restrict__ B, const
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int64_t o = ((int64_t)(e.start + t0 + tt) * H + h) * P + p0 + j;
-                y[o] = from_f32<T>(y_end(acc[i][j], Dh, to_f32(x[o])));
+                const float a = (i & 1) ? acc[i >> 1][j].y : acc[i >> 1][j].x;
+                y[o] = from_f32<T>(y_end(a, Dh, to_f32(x[o])));
             }
         }
     }
@@ -726,7 +747,17 @@ k_strict_cache_fill(const T* __restrict__ x, const T* __restrict__ B, const floa
 // fills (len == Q) is folded into the state by k_strict_fold, launched right after in
 // the same call. Threads take the dots one source each, then the coefficients
 // (C_t . B_s) w(j, s) of every head, then y[h][p] one (head, p) each.
+//
+// The incoming-state term C_t . h_in[p] reads each state row left to right in one thread.
+// The group's state rows are contiguous, and they reach shared memory as slices of 16
+// columns of up to 512 rows (64 bytes per row, four 16-byte asynchronous copies; a warp
+// copies 8 whole row pieces per instruction) through a ring of three slices, the first two
+// issued before the dots and coefficients are taken. In a slice, 16-byte chunk c of row r
+// sits at chunk c ^ ((r >> 1) & 3), so that eight consecutive threads reading the same chunk
+// of their own rows hit eight different bank groups.
 constexpr int kDecThreads = 512;
+constexpr int kDecSlice = 16;         // state columns per staged slice
+constexpr int kDecStages = 3;
 
 // Left-to-right dot of the float row c[0..N) with the row b[0..N) of T, 16-byte loads.
 template <typename T>
@@ -760,22 +791,42 @@ __device__ __forceinline__ float row_dot<float>(const float* c, const float* b, 
     return d;
 }
 
+// Stage q: column slice q % nsl of the row batch q / nsl (rows 512 (q / nsl) ..), into
+// ring slot q % 3. Every thread commits one group per stage (empty past the last).
+__device__ __forceinline__ void decode_stage(float* ring, const float* st0, int q, int nst, int nsl, int rows,
+                                             int N, int tid) {
+    if (q < nst) {
+        const int rb = (q / nsl) * kDecThreads, n0 = (q % nsl) * kDecSlice, nr = min(kDecThreads, rows - rb);
+        float* dst = ring + (q % kDecStages) * (kDecThreads * kDecSlice);
+        for (int i = tid; i < nr * 4; i += kDecThreads) {
+            const int r = i >> 2, c = i & 3;
+            cp_async16(dst + r * kDecSlice + ((c ^ ((r >> 1) & 3)) << 2), st0 + (int64_t)(rb + r) * N + n0 + (c << 2));
+        }
+    }
+    cp_async_commit();
+}
+
 template <typename T>
-__global__ void __launch_bounds__(kDecThreads)
+__global__ void __launch_bounds__(kDecThreads, 2)
 k_strict_decode(const float* __restrict__ cstate, T* __restrict__ cx, T* __restrict__ cB, float* __restrict__ cdt,
                 float* __restrict__ cacum, int32_t* __restrict__ clen, const T* __restrict__ x,
                 const float* __restrict__ dt_raw, const float* __restrict__ dt_bias, const float* __restrict__ A,
                 const T* __restrict__ B, const T* __restrict__ C, const float* __restrict__ D, T* __restrict__ y,
                 int H, int G, int P, int N, int Q) {
-    extern __shared__ float sm[];
+    extern __shared__ __align__(16) float sm[];
     const int hpg = H / G;
-    float* cs = sm;                       // [N]       C_t
+    float* ring = sm;                     // [3][512][16] state slices
+    float* cs = ring + kDecStages * kDecThreads * kDecSlice;   // [N]       C_t
     float* dots = cs + N;                 // [Q]       C_t . B_s
     float* coef = dots + Q;               // [hpg][Q]  (C_t . B_s) w(j, s) per head
     float* hdt = coef + hpg * Q;          // [hpg]     the token's dt per head
     float* hac = hdt + hpg;               // [hpg]     the token's Acum per head
     __shared__ int s_j, s_bad;
     const int s = blockIdx.x / G, g = blockIdx.x % G, h0 = g * hpg, tid = threadIdx.x;
+    const int rows = hpg * P, nsl = N / kDecSlice, nst = ((rows + kDecThreads - 1) / kDecThreads) * nsl;
+    const float* st0 = cstate + ((int64_t)s * H + h0) * P * N;   // row r = hl P + p
+    decode_stage(ring, st0, 0, nst, nsl, rows, N, tid);
+    decode_stage(ring, st0, 1, nst, nsl, rows, N, tid);
     if (tid == 0) {
         s_j = clen[(int64_t)s * H + h0];
         s_bad = 0;
@@ -801,6 +852,7 @@ k_strict_decode(const float* __restrict__ cstate, T* __restrict__ cx, T* __restr
     __syncthreads();
     if (s_bad) {
         if (tid == 0) latch_error(SSD_ERR_INVALID_ARG);
+        cp_async_wait<0>();                                  // no copy left in flight at exit
         return;
     }
 
@@ -819,12 +871,34 @@ k_strict_decode(const float* __restrict__ cstate, T* __restrict__ cx, T* __restr
     }
     __syncthreads();
 
-    // y[h][p]: incoming-state term, sources left to right, D skip.
-    for (int i = tid; i < hpg * P; i += kDecThreads) {
+    // y[h][p]: incoming-state term, sources left to right, D skip. Thread tid owns row
+    // 512 b + tid of each row batch b.
+    for (int rb = 0; rb < rows; rb += kDecThreads) {
+        const int i = rb + tid;
+        float dot = 0.f;
+        for (int k = 0; k < nsl; ++k) {
+            const int q = (rb / kDecThreads) * nsl + k;
+            cp_async_wait<1>();                              // this thread's copies of stage q
+            __syncthreads();                                 // everyone's; slot (q + 2) % 3 free again
+            decode_stage(ring, st0, q + 2, nst, nsl, rows, N, tid);
+            if (i < rows) {
+                const float* src = ring + (q % kDecStages) * (kDecThreads * kDecSlice) + tid * kDecSlice;
+                const float* cn = cs + k * kDecSlice;
+                const int sw = (tid >> 1) & 3;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float4 v = *reinterpret_cast<const float4*>(src + ((c ^ sw) << 2));
+                    dot = dot_step(dot, cn[4 * c], v.x);
+                    dot = dot_step(dot, cn[4 * c + 1], v.y);
+                    dot = dot_step(dot, cn[4 * c + 2], v.z);
+                    dot = dot_step(dot, cn[4 * c + 3], v.w);
+                }
+            }
+        }
+        if (i >= rows) continue;
         const int hl = i / P, p = i % P, h = h0 + hl;
         const int64_t sh = (int64_t)s * H + h;
         const float* cf = coef + hl * Q;
-        const float dot = row_dot<float>(cs, cstate + (sh * P + p) * N, N);
         float acc = y_begin(dot, hac[hl]);
         const T* xp = cx + sh * Q * P + p;                  // cached x rows [Q][P]
         int sidx = 0;
@@ -857,7 +931,9 @@ k_strict_decode(const float* __restrict__ cstate, T* __restrict__ cx, T* __restr
     }
 }
 
-inline size_t decode_smem(int H, int G, int N, int Q) { return sizeof(float) * (N + Q + (H / G) * (Q + 2)); }
+inline size_t decode_smem(int H, int G, int N, int Q) {
+    return sizeof(float) * (kDecStages * kDecThreads * kDecSlice + N + Q + (H / G) * (Q + 2));
+}
 
 // ---------------------------------------------------------------------------------
 // Fold of a full open chunk (len == Q) into the cache state: the prefill's chunk-state
@@ -930,7 +1006,7 @@ k_strict_fold(float* __restrict__ cstate, const T* __restrict__ cx, const T* __r
 #pragma unroll
             for (int j = 0; j < StateTile<NOUT>::CN; ++j) {
                 const int64_t o = (int64_t)(tile.p0 + i) * N + tile.n0 + j;
-                hout[o] = pass(hout[o], last, tile.acc[i][j]);
+                hout[o] = pass(hout[o], last, tile.at(i, j));
             }
         if (tid == 0) clen[sh] = 0;
     };
