@@ -502,10 +502,27 @@ k_strict_chunk_scan(const T* __restrict__ x, const T* __restrict__ B, const T* _
 //      per thread), kept s-major;
 //   2. the group's heads four at a time, 64 threads per head; thread (rg, pg) owns rows
 //      8 rg .. 8 rg + 7 and columns 4 pg .. 4 pg + 3 (32 outputs): C_t . h_in[p] in 16-wide
-//      slices of n (h_in transposed into shared memory), then the sources in 32-wide slices
-//      (the head's coefficients (C_t . B_s) w(t, s) and raw x rows in shared memory, x by
-//      asynchronous copies), then D x_t and the store.
+//      slices of n (h_in transposed into shared memory by 4-byte asynchronous copies, the
+//      next slice in flight while one is used), then the sources in 32-wide slices (the
+//      head's coefficients (C_t . B_s) w(t, s) from its Acum and dt rows, staged once per
+//      head, and the raw x rows, the next slice's copies in flight), then D x_t and the store.
 constexpr int kWideHS = 68;   // row stride of a transposed h_in slice (16-byte rows)
+
+// Floats of the work region: the B^T slice of (1), two h_in^T slices per head, or the
+// coefficients and two raw x slices per head.
+template <typename T>
+__host__ __device__ inline int wide_work_floats(int N) {
+    const int a = N * 64, b = 2 * 4 * 16 * kWideHS, c = 4 * 32 * 32 + 2 * 4 * 32 * 64 * (int)sizeof(T) / 4;
+    return a > b ? (a > c ? a : c) : (b > c ? b : c);
+}
+
+// One 16-column slice of a head's h_in, transposed: hT[nn][p] = h_in[p][n0 + nn].
+__device__ __forceinline__ void wide_h_slice(float* hT, const float* hsrc, int N, int n0, int u) {
+    for (int i = u; i < 64 * 16; i += 64) {
+        const int p = i / 16, nn = i % 16;
+        cp_async4(hT + nn * kWideHS + p, hsrc + (int64_t)p * N + n0 + nn);
+    }
+}
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 2)
@@ -518,8 +535,10 @@ k_strict_chunk_scan_wide(const T* __restrict__ x, const T* __restrict__ B, const
     extern __shared__ __align__(16) float sm[];
     float* cbs = sm;                      // [Q][32]  C_t . B_s: row s, column t (row of the tile)
     float* ct = cbs + Q * 32;             // [N][32]  the tile's C rows, transposed
-    float* work = ct + N * 32;            // B^T slice [N][64]; or per head an h_in^T slice [16][68];
-                                          // or per head coefficients [32][32], then raw x [32][64]
+    float* work = ct + N * 32;            // B^T slice [N][64]; or h_in^T slices [2][4 heads][16][68];
+                                          // or coefficients [4 heads][32][32], then raw x [2][4 heads][32][64]
+    float* acs = work + wide_work_floats<T>(N);   // [4 heads][Q] Acum
+    float* dvs = acs + 4 * Q;                     // [4 heads][Q] dt
     const int ntile = Q / 32;
     const int c = (int)(blockIdx.x / (unsigned)(ntile * G));
     if (c >= *count) return;
@@ -578,32 +597,40 @@ k_strict_chunk_scan_wide(const T* __restrict__ x, const T* __restrict__ B, const
 
     // (2) The group's heads, four at a time.
     const int hl = tid / 64, u = tid % 64, r0 = (u / 16) * 8, p0 = (u % 16) * 4;
-    float* hT = work + hl * (16 * kWideHS);
     float* cf = work + hl * (32 * 32);
-    T* xs = reinterpret_cast<T*>(work + 4 * 32 * 32) + hl * (32 * P);
+    const float* ac = acs + hl * Q;
+    const float* dv = dvs + hl * Q;
+    auto hT = [&](int buf) { return work + (buf * 4 + hl) * (16 * kWideHS); };
+    auto xs = [&](int buf) { return reinterpret_cast<T*>(work + 4 * 32 * 32) + (buf * 4 + hl) * (32 * P); };
     for (int hp = 0; hp < hpg; hp += 4) {
         const int h = g * hpg + hp + hl;
-        const float* ac = acum + ((int64_t)c * H + h) * Q;
-        const float* dv = dtc + ((int64_t)c * H + h) * Q;
         const float* hsrc = hin + ((int64_t)c * H + h) * P * N;
+        __syncthreads();                                     // work, acs and dvs free
+        for (int i = u; i < Q / 4; i += 64) {
+            cp_async16(acs + hl * Q + 4 * i, acum + ((int64_t)c * H + h) * Q + 4 * i);
+            cp_async16(dvs + hl * Q + 4 * i, dtc + ((int64_t)c * H + h) * Q + 4 * i);
+        }
+        wide_h_slice(hT(0), hsrc, N, 0, u);
+        cp_async_commit();
         float2 acc[4][4];                                    // rows r0 + 2i, r0 + 2i + 1; column p0 + j
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
             for (int j = 0; j < 4; ++j) acc[i][j] = make_float2(0.f, 0.f);
         // (2a) C_t . h_in[p], left to right over n, 16 at a time.
-        for (int n0 = 0; n0 < N; n0 += 16) {
-            __syncthreads();                                 // work free
-            for (int i = u; i < P * 16; i += 64) {
-                const int p = i / 16, nn = i % 16;
-                hT[nn * kWideHS + p] = hsrc[(int64_t)p * N + n0 + nn];
-            }
+        for (int k = 0; k < N / 16; ++k) {
+            if (k > 0) __syncthreads();                      // slice k - 1 used: its buffer is free
+            if (k + 1 < N / 16) wide_h_slice(hT((k + 1) & 1), hsrc, N, 16 * (k + 1), u);
+            cp_async_commit();
+            cp_async_wait<1>();                              // slice k (and the Acum, dt rows) landed
             __syncthreads();
+            const float* hb = hT(k & 1);
+            const int n0 = 16 * k;
 #pragma unroll 4
             for (int nn = 0; nn < 16; ++nn) {
                 const float4 c0 = *reinterpret_cast<const float4*>(ct + (n0 + nn) * 32 + r0);
                 const float4 c1 = *reinterpret_cast<const float4*>(ct + (n0 + nn) * 32 + r0 + 4);
-                const float4 hv = *reinterpret_cast<const float4*>(hT + nn * kWideHS + p0);
+                const float4 hv = *reinterpret_cast<const float4*>(hb + nn * kWideHS + p0);
                 const float2 cva[4] = {make_float2(c0.x, c0.y), make_float2(c0.z, c0.w), make_float2(c1.x, c1.y),
                                        make_float2(c1.z, c1.w)};
                 const float2 hva[4] = {splat(hv.x), splat(hv.y), splat(hv.z), splat(hv.w)};
@@ -620,26 +647,37 @@ k_strict_chunk_scan_wide(const T* __restrict__ x, const T* __restrict__ B, const
             for (int j = 0; j < 4; ++j) acc[i][j] = make_float2(y_begin(acc[i][j].x, a0), y_begin(acc[i][j].y, a1));
         }
         // (2b) Sources s = 0..t, left to right, 32 at a time.
-        for (int s0 = 0; s0 <= t0; s0 += 32) {
-            __syncthreads();                                 // work free
+        const int nxs = t0 / 32 + 1;
+        auto x_slice = [&](int k) {
+            T* dst = xs(k & 1);
+            const int s0 = 32 * k;
             for (int i = u; i < 32 * (P / V); i += 64) {
-                const int r = i / (P / V), k = i % (P / V);
+                const int r = i / (P / V), q = i % (P / V);
                 if (s0 + r < e.len)
-                    cp_async16(xs + r * P + k * V, x + ((int64_t)(e.start + s0 + r) * H + h) * P + k * V);
+                    cp_async16(dst + r * P + q * V, x + ((int64_t)(e.start + s0 + r) * H + h) * P + q * V);
             }
+        };
+        __syncthreads();                                     // (2a) done: its buffers hold cf and x now
+        x_slice(0);
+        cp_async_commit();
+        for (int k = 0; k < nxs; ++k) {
+            const int s0 = 32 * k;
+            if (k > 0) __syncthreads();                      // slice k - 1 used: cf and its x buffer free
+            if (k + 1 < nxs) x_slice(k + 1);
             cp_async_commit();
             for (int i = u; i < 32 * 32; i += 64) {
                 const int sl = i / 32, tl = i % 32, s_ = s0 + sl, t = t0 + tl;
                 cf[i] = s_ <= t && s_ < e.len ? mix_coef(cbs[s_ * 32 + tl], ac[t], ac[s_], dv[s_]) : 0.f;
             }
-            cp_async_wait<0>();
+            cp_async_wait<1>();                              // x of slice k landed
             __syncthreads();
+            const T* xb = xs(k & 1);
             if (s0 < t0) {                                   // every row of the tile sees all 32 sources
 #pragma unroll 4
-                for (int k = 0; k < 32; ++k) {
-                    const float4 f0 = *reinterpret_cast<const float4*>(cf + k * 32 + r0);
-                    const float4 f1 = *reinterpret_cast<const float4*>(cf + k * 32 + r0 + 4);
-                    const float4 xv = load4(xs + k * P + p0);
+                for (int kk = 0; kk < 32; ++kk) {
+                    const float4 f0 = *reinterpret_cast<const float4*>(cf + kk * 32 + r0);
+                    const float4 f1 = *reinterpret_cast<const float4*>(cf + kk * 32 + r0 + 4);
+                    const float4 xv = load4(xb + kk * P + p0);
                     const float2 fva[4] = {make_float2(f0.x, f0.y), make_float2(f0.z, f0.w), make_float2(f1.x, f1.y),
                                            make_float2(f1.z, f1.w)};
                     const float2 xva[4] = {splat(xv.x), splat(xv.y), splat(xv.z), splat(xv.w)};
@@ -649,18 +687,18 @@ k_strict_chunk_scan_wide(const T* __restrict__ x, const T* __restrict__ B, const
                         for (int j = 0; j < 4; ++j) acc[i][j] = step2(acc[i][j], fva[i], xva[j]);
                 }
             } else {                                         // diagonal slice: sources s <= t
-                for (int k = 0; k < 32; ++k) {
-                    const float4 f0 = *reinterpret_cast<const float4*>(cf + k * 32 + r0);
-                    const float4 f1 = *reinterpret_cast<const float4*>(cf + k * 32 + r0 + 4);
-                    const float4 xv = load4(xs + k * P + p0);
+                for (int kk = 0; kk < 32; ++kk) {
+                    const float4 f0 = *reinterpret_cast<const float4*>(cf + kk * 32 + r0);
+                    const float4 f1 = *reinterpret_cast<const float4*>(cf + kk * 32 + r0 + 4);
+                    const float4 xv = load4(xb + kk * P + p0);
                     const float2 fva[4] = {make_float2(f0.x, f0.y), make_float2(f0.z, f0.w), make_float2(f1.x, f1.y),
                                            make_float2(f1.z, f1.w)};
                     const float xva[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        // rows r0 + 2i (takes source k while k <= r0 + 2i) and r0 + 2i + 1
-                        if (k > r0 + 2 * i + 1) continue;
-                        if (k == r0 + 2 * i + 1) {
+                        // rows r0 + 2i (takes source kk while kk <= r0 + 2i) and r0 + 2i + 1
+                        if (kk > r0 + 2 * i + 1) continue;
+                        if (kk == r0 + 2 * i + 1) {
 #pragma unroll
                             for (int j = 0; j < 4; ++j) acc[i][j].y = y_step(acc[i][j].y, fva[i].y, xva[j]);
                         } else {
@@ -689,9 +727,7 @@ k_strict_chunk_scan_wide(const T* __restrict__ x, const T* __restrict__ B, const
 
 template <typename T>
 inline size_t chunk_scan_wide_smem(int N, int Q) {
-    const int work_a = N * 64, work_b = 4 * 16 * kWideHS, work_c = 4 * 32 * 32 + 4 * 32 * 64 * (int)sizeof(T) / 4;
-    const int work = work_a > work_b ? (work_a > work_c ? work_a : work_c) : (work_b > work_c ? work_b : work_c);
-    return sizeof(float) * (Q * 32 + N * 32 + work);
+    return sizeof(float) * (Q * 32 + N * 32 + wide_work_floats<T>(N) + 8 * Q);
 }
 
 inline size_t chunk_scan_smem(int P, int N, int Q) {
