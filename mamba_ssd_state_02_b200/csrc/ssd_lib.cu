@@ -14,6 +14,7 @@
 #include <vector>
 
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cstdlib>
 
@@ -80,12 +81,15 @@ struct Profiler {
 };
 Profiler g_prof;
 
-// Brackets one kernel launch with events when profiling is on.
+// Brackets one kernel launch: an NVTX range named after the stage on the host timeline
+// (a no-op unless a tool such as Nsight Systems or Nsight Compute has attached), and CUDA
+// events on the stream when profiling is on.
 struct StageScope {
     int stage;
     cudaStream_t st;
     cudaEvent_t a = nullptr;
     StageScope(int s, cudaStream_t stream) : stage(s), st(stream) {
+        nvtxRangePushA(kStageName[s]);
         std::lock_guard<std::mutex> lk(g_prof.mu);
         if (!g_prof.on) return;
         if (g_prof.recs.size() >= kMaxRecords) {
@@ -96,15 +100,17 @@ struct StageScope {
         if (a) cudaEventRecord(a, st);
     }
     ~StageScope() {
-        if (!a) return;
-        std::lock_guard<std::mutex> lk(g_prof.mu);
-        cudaEvent_t b = g_prof.get();
-        if (!b) {
-            g_prof.pool.push_back(a);
-            return;
+        if (a) {
+            std::lock_guard<std::mutex> lk(g_prof.mu);
+            cudaEvent_t b = g_prof.get();
+            if (b) {
+                cudaEventRecord(b, st);
+                g_prof.recs.push_back({stage, a, b});
+            } else {
+                g_prof.pool.push_back(a);
+            }
         }
-        cudaEventRecord(b, st);
-        g_prof.recs.push_back({stage, a, b});
+        nvtxRangePop();
     }
 };
 
