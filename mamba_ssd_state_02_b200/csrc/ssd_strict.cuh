@@ -145,8 +145,10 @@ struct StateTile {
 };
 
 // ---------------------------------------------------------------------------------
-// Prefill stage 1: dt and Acum per (chunk, head), left to right, [chunk][H][Q] (zero past
-// the chunk's end). One thread per (chunk, head).
+// Prefill stage 1: dt and Acum per (chunk, head), left to right, [chunk][H][Q] (past the
+// chunk's end dt is zero and Acum holds its value at the last token). One thread per
+// (chunk, head); 16 tokens' raw dt are loaded before their 16 dependent steps, and dt, Acum
+// go out as 16-byte stores (Q is a multiple of 32).
 __global__ void __launch_bounds__(128)
 k_strict_cumsum(const float* __restrict__ dt_raw, const float* __restrict__ dt_bias, const float* __restrict__ A,
                 const ChunkEntry* __restrict__ table, const int32_t* __restrict__ count, int H, int Q,
@@ -159,14 +161,26 @@ k_strict_cumsum(const float* __restrict__ dt_raw, const float* __restrict__ dt_b
     if (bad_A(a)) latch_error(SSD_ERR_INVALID_ARG);
     const int64_t base = ((int64_t)c * H + h) * Q;
     float run = 0.f;
-    for (int r = 0; r < Q; ++r) {
-        float d = 0.f;
-        if (r < e.len) {
-            d = dt_of(dt_raw[(int64_t)(e.start + r) * H + h], bias);
-            run = acum_next(run, d, a);
+    constexpr int U = 16;
+    for (int r0 = 0; r0 < Q; r0 += U) {
+        float raw[U], dv[U], av[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) raw[u] = r0 + u < e.len ? dt_raw[(int64_t)(e.start + r0 + u) * H + h] : 0.f;
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            float d = 0.f;
+            if (r0 + u < e.len) {
+                d = dt_of(raw[u], bias);
+                run = acum_next(run, d, a);
+            }
+            dv[u] = d;
+            av[u] = run;
         }
-        dt_out[base + r] = d;
-        acum_out[base + r] = run;
+#pragma unroll
+        for (int u = 0; u < U; u += 4) {
+            *reinterpret_cast<float4*>(dt_out + base + r0 + u) = make_float4(dv[u], dv[u + 1], dv[u + 2], dv[u + 3]);
+            *reinterpret_cast<float4*>(acum_out + base + r0 + u) = make_float4(av[u], av[u + 1], av[u + 2], av[u + 3]);
+        }
     }
 }
 
