@@ -1125,7 +1125,7 @@ ssd_status launch_strict(const Plan& pl, char* ws, const T* x, const float* dt_r
     }
     {
         StageScope sc(ST_STRICT_PASSING, st);
-        k_strict_passing<<<dim3(pl.nseq, H, (P * N + kThreads - 1) / kThreads), kThreads, 0, st>>>(
+        k_strict_passing<<<dim3(pl.nseq, H, (P * N / 4 + kThreads - 1) / kThreads), kThreads, 0, st>>>(
             states, acum, table, first, resume, cc.state, cc.len, fin, H, P * N, Q);
     }
     ++n;

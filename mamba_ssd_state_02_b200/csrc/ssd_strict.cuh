@@ -254,50 +254,75 @@ k_strict_chunk_state(const T* __restrict__ x, const T* __restrict__ B, const flo
 
 // ---------------------------------------------------------------------------------
 // Prefill stage 3: state passing, sequential over a sequence's chunks, parallel over
-// (head, state element). Overwrites S_c with h_in(c), writes the final state and the
-// cache state (the state entering the sequence's open chunk: h_in of a partial last
-// chunk, else the final state). `resume`: start from cache_state, whose open chunk
-// must be empty (cache_len == 0), else SSD_ERR_UNSUPPORTED is latched (fail closed).
-__global__ void __launch_bounds__(kThreads)
+// (head, state element), four consecutive elements per thread. Overwrites S_c with
+// h_in(c), writes the final state and the cache state (the state entering the sequence's
+// open chunk: h_in of a partial last chunk, else the final state). `resume`: start from
+// cache_state, whose open chunk must be empty (cache_len == 0), else SSD_ERR_UNSUPPORTED is
+// latched (fail closed).
+__global__ void __launch_bounds__(kThreads, 4)
 k_strict_passing(float* __restrict__ states, const float* __restrict__ acum, const ChunkEntry* __restrict__ table,
                  const int32_t* __restrict__ first, int resume, float* __restrict__ cache_state,
                  const int32_t* __restrict__ cache_len, float* __restrict__ final_state, int H, int PN, int Q) {
     const int s = blockIdx.x, h = blockIdx.y;
-    const int i = blockIdx.z * kThreads + threadIdx.x;
+    const int i = (blockIdx.z * kThreads + threadIdx.x) * 4;     // elements i .. i + 3 (PN % 4 == 0)
     if (i >= PN) return;
     const int64_t slot0 = ((int64_t)s * H + h) * PN + i;
-    float hv = 0.f;
+    float hv[4] = {0.f, 0.f, 0.f, 0.f};
     if (resume) {
         if (cache_len[(int64_t)s * H + h] != 0) latch_error(SSD_ERR_UNSUPPORTED);
-        hv = cache_state[slot0];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) hv[k] = cache_state[slot0 + k];
     }
     const int c0 = first[s], c1 = first[s + 1];
-    float open = hv;
-    // Four chunks' loads are issued before the four dependent updates (same arithmetic).
+    float open[4] = {hv[0], hv[1], hv[2], hv[3]};
+    // Groups of four chunks, double-buffered: the next group's loads are in flight while
+    // this one is applied (same arithmetic per element).
     constexpr int U = 4;
-    for (int c = c0; c < c1; c += U) {
-        float sv[U], al[U];
+    struct Group {
+        float4 sv[U];
+        float al[U];
         int len[U];
+    };
+    auto load = [&](int c, Group& g) {
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             if (c + u < c1) {
-                len[u] = table[c + u].len;
-                sv[u] = states[((int64_t)(c + u) * H + h) * PN + i];
-                al[u] = acum[((int64_t)(c + u) * H + h) * Q + len[u] - 1];
+                g.len[u] = table[c + u].len;
+                g.sv[u] = *reinterpret_cast<const float4*>(states + ((int64_t)(c + u) * H + h) * PN + i);
+                g.al[u] = acum[((int64_t)(c + u) * H + h) * Q + g.len[u] - 1];
             }
         }
+    };
+    auto apply = [&](int c, const Group& g) {
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             if (c + u < c1) {
-                states[((int64_t)(c + u) * H + h) * PN + i] = hv;
-                open = hv;
-                hv = pass(hv, al[u], sv[u]);
-                if (len[u] == Q) open = hv;
+                *reinterpret_cast<float4*>(states + ((int64_t)(c + u) * H + h) * PN + i) =
+                    make_float4(hv[0], hv[1], hv[2], hv[3]);
+                const float sv[4] = {g.sv[u].x, g.sv[u].y, g.sv[u].z, g.sv[u].w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    open[k] = hv[k];
+                    hv[k] = pass(hv[k], g.al[u], sv[k]);
+                    if (g.len[u] == Q) open[k] = hv[k];
+                }
             }
         }
+    };
+    Group ga, gb;
+    if (c0 < c1) load(c0, ga);
+    for (int c = c0; c < c1; c += 2 * U) {
+        if (c + U < c1) load(c + U, gb);
+        apply(c, ga);
+        if (c + U >= c1) break;
+        if (c + 2 * U < c1) load(c + 2 * U, ga);
+        apply(c + U, gb);
     }
-    cache_state[slot0] = open;
-    if (final_state) final_state[slot0] = hv;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        cache_state[slot0 + k] = open[k];
+        if (final_state) final_state[slot0 + k] = hv[k];
+    }
 }
 
 // ---------------------------------------------------------------------------------
