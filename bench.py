@@ -417,7 +417,7 @@ def bench_ours(args, rank, world, local_rank):
                  "frac_nominal_8tbs": round(pb / 8e12 * 1e3 / ms_step, 4)}
     # The whole prefill step against its roofline (the target the workload is held to:
     # at least 60% of max(bytes / HBM bandwidth, flops / bf16 peak)).
-    north_star = {"workload": w.name, "path_frac": path_roof["frac"], "path_frac_required": 0.6,
+    path_target = {"workload": w.name, "path_frac": path_roof["frac"], "path_frac_required": 0.6,
                   "met": path_roof["frac"] >= 0.6,
                   "note": "roofline below is the dominant kernel alone; path_frac is the whole step"}
     kernels = {}
@@ -639,7 +639,7 @@ def bench_ours(args, rank, world, local_rank):
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "inputs larger than L2 (%.2f GB per step vs 126 MB L2), no flush" % (pb / 1e9),
                    "variant": variant, "segment_tokens": seg_tokens},
-        "roofline": roofline, "path_roofline": path_roof, "north_star": north_star, "kernels": kernels,
+        "roofline": roofline, "path_roofline": path_roof, "path_target": path_target, "kernels": kernels,
         "prefill_other": other_prefill,
         "clocks": clk, "e2e": e2e, "gpu_launches": launches_per_call * args.steps,
         "decode": decode,
