@@ -161,6 +161,39 @@ def test_prefill_then_decode_is_bitwise_one_shot(ssd, cuda_dev, dtype, chunk):
     _assert_cache_equal(split, full, w.ngroups, w.nheads)
 
 
+@pytest.mark.parametrize("H,G,P,N", [(8, 1, 128, 32), (16, 1, 64, 64), (4, 1, 16, 16)])
+def test_decode_geometries_bitwise_and_against_oracle(ssd, cuda_dev, H, G, P, N):
+    """The decode step streams each group's state rows (heads per group x P of them) through
+    shared memory in batches of 512 rows and slices of 16 columns: 1024 rows in two batches
+    (P = 128 or 16 heads per group), a single slice (N = 16), two slices (N = 32). Split each
+    sequence into a strict prefill and 80 decode steps (crossing chunk ends at 64 tokens);
+    the decode must give the one-shot prefill's bits and match the oracle."""
+    K, chunk = 80, 64
+    L1 = [0, 5, 64, 70]
+    w = _w([a + K for a in L1], H=H, G=G, P=P, N=N, chunk=chunk, seed=66)
+    inp = W.make_all(w, device=cuda_dev)
+    cu = inp["cu_seqlens"].tolist()
+    full = _cache(ssd, w, cuda_dev, inp["init_state"])
+    y_full, _ = ssd.strict_scan_fwd(inp["x"], inp["dt_raw"], inp["dt_bias"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                    full, resume=True, cu_seqlens=inp["cu_seqlens"])
+    split = _cache(ssd, w, cuda_dev, inp["init_state"])
+    rows = torch.cat([_seq_rows(cu, s, 0, L1[s], cuda_dev) for s in range(w.nseq)])
+    y_pre, _ = _prefill(ssd, w, inp, rows, L1, split)
+    ys = []
+    for k in range(K):
+        t = _rows(inp, torch.tensor([cu[s] + L1[s] + k for s in range(w.nseq)], device=cuda_dev))
+        ys.append(ssd.strict_state_update(split, t["x"], t["dt_raw"], inp["dt_bias"], inp["A"], t["B"], t["C"],
+                                          inp["D"]))
+    ssd.device_status()
+    dec_rows = torch.tensor([[cu[s] + L1[s] + k for s in range(w.nseq)] for k in range(K)], device=cuda_dev)
+    assert_same_bits(torch.stack(ys), y_full[dec_rows], "decode part")
+    _assert_cache_equal(split, full, w.ngroups, w.nheads)
+    cpu = {k: (None if v is None else v.cpu()) for k, v in inp.items()}
+    y_ref, _ = O.ssd_scan(cpu["x"], cpu["dt_raw"], cpu["dt_bias"], cpu["A"], cpu["B"], cpu["C"], cpu["D"],
+                          init_state=cpu["init_state"], cu_seqlens=cpu["cu_seqlens"])
+    assert rel_err(torch.stack(ys), y_ref[dec_rows.cpu()]) <= TOL_Y[w.dtype]
+
+
 def test_prefill_split_at_chunk_boundaries_is_bitwise(ssd, cuda_dev):
     chunk = 128
     L1, L2 = [256, 128, 0, 384], [300, 5, 129, 0]
