@@ -144,6 +144,41 @@ struct StateTile {
     }
 };
 
+// A tile of raw rows (n elements, rows of P) to FP32 in shared memory, 16 bytes per step:
+// dst[i] = state_src(scale[i / P], src[i]), or src[i] when scale is null. P is a power of
+// two and a multiple of the step's element count; src and dst are 16-byte aligned.
+template <typename T>
+__device__ __forceinline__ void tile_to_f32(float* dst, const T* src, int n, int P, const float* scale, int tid) {
+    constexpr int V = 16 / (int)sizeof(T);
+    const int lp = __ffs(P) - 1;
+    for (int v = tid; v < n / V; v += kThreads) {
+        const int i = v * V;
+        const uint4 u = *reinterpret_cast<const uint4*>(src + i);
+        float f[V];
+        if constexpr (V == 8) {
+            const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                f[2 * k] = __uint_as_float(w4[k] << 16);
+                f[2 * k + 1] = __uint_as_float(w4[k] & 0xffff0000u);
+            }
+        } else {
+            f[0] = __uint_as_float(u.x);
+            f[1] = __uint_as_float(u.y);
+            f[2] = __uint_as_float(u.z);
+            f[3] = __uint_as_float(u.w);
+        }
+        if (scale) {
+            const float sc = scale[i >> lp];
+#pragma unroll
+            for (int k = 0; k < V; ++k) f[k] = state_src(sc, f[k]);
+        }
+#pragma unroll
+        for (int k = 0; k < V; k += 4)
+            *reinterpret_cast<float4*>(dst + i + k) = make_float4(f[k], f[k + 1], f[k + 2], f[k + 3]);
+    }
+}
+
 // ---------------------------------------------------------------------------------
 // Prefill stage 1: dt and Acum per (chunk, head), left to right, [chunk][H][Q] (past the
 // chunk's end dt is zero and Acum holds its value at the last token). One thread per
@@ -239,8 +274,8 @@ k_strict_chunk_state(const T* __restrict__ x, const T* __restrict__ B, const flo
         const int rows = min(32, e.len - 32 * t);
         const T* rx = raw + (t & 1) * tile_elems;
         const T* rb = rx + 32 * P;
-        for (int i = tid; i < rows * P; i += kThreads) xs[i] = state_src(w[32 * t + i / P], to_f32(rx[i]));
-        for (int i = tid; i < rows * N; i += kThreads) bs[i] = to_f32(rb[i]);
+        tile_to_f32(xs, rx, rows * P, P, w + 32 * t, tid);
+        tile_to_f32(bs, rb, rows * N, N, static_cast<const float*>(nullptr), tid);
         __syncthreads();
         for (int r = 0; r < rows; ++r) tile.row(xs + r * P, bs + r * N);
         __syncthreads();                                    // xs, bs and buffer t & 1 free again
@@ -1069,8 +1104,8 @@ k_strict_fold(float* __restrict__ cstate, const T* __restrict__ cx, const T* __r
             __syncthreads();                                // tile t landed (all threads' copies); wv
             const T* rx = raw + (t & 1) * tile_elems;
             const T* rb = rx + 32 * P;
-            for (int i = tid; i < 32 * P; i += kThreads) xs[i] = state_src(wv[32 * t + i / P], to_f32(rx[i]));
-            for (int i = tid; i < 32 * N; i += kThreads) bs[i] = to_f32(rb[i]);
+            tile_to_f32(xs, rx, 32 * P, P, wv + 32 * t, tid);
+            tile_to_f32(bs, rb, 32 * N, N, static_cast<const float*>(nullptr), tid);
             __syncthreads();
             for (int r = 0; r < 32; ++r) tile.row(xs + r * P, bs + r * N);
             __syncthreads();                                // xs, bs and buffer t & 1 free again
