@@ -761,13 +761,23 @@ k_strict_chunk_scan_wide(const T* __restrict__ x, const T* __restrict__ B, const
                         for (int j = 0; j < 4; ++j) acc[i][j] = step2(acc[i][j], fva[i], xva[j]);
                 }
             } else {                                         // diagonal slice: sources s <= t
-                for (int kk = 0; kk < 32; ++kk) {
+                // Source kk reaches the thread's rows r0 .. r0 + 7 while kk <= r0 + 7, and all
+                // of them while kk <= r0.
+                for (int kk = 0; kk < r0 + 8; ++kk) {
                     const float4 f0 = *reinterpret_cast<const float4*>(cf + kk * 32 + r0);
                     const float4 f1 = *reinterpret_cast<const float4*>(cf + kk * 32 + r0 + 4);
                     const float4 xv = load4(xb + kk * P + p0);
                     const float2 fva[4] = {make_float2(f0.x, f0.y), make_float2(f0.z, f0.w), make_float2(f1.x, f1.y),
                                            make_float2(f1.z, f1.w)};
                     const float xva[4] = {xv.x, xv.y, xv.z, xv.w};
+                    if (kk <= r0) {
+                        const float2 xs2[4] = {splat(xv.x), splat(xv.y), splat(xv.z), splat(xv.w)};
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) acc[i][j] = step2(acc[i][j], fva[i], xs2[j]);
+                        continue;
+                    }
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         // rows r0 + 2i (takes source kk while kk <= r0 + 2i) and r0 + 2i + 1
