@@ -328,3 +328,44 @@ def test_strict_long_context_full_size(ssd, cuda_dev):
     assert rel_err(torch.stack([fin[0, h] for _, h in pairs]), fin_ref) <= TOL_STATE
     assert int(cache.len.max()) == 0                      # 65536 is a multiple of the chunk
     assert_same_bits(cache.state, fin, "cache state = final state on a chunk boundary")
+
+
+def test_strict_decode_full_batch_bitwise(ssd, cuda_dev):
+    """The chunk-emulating decode at the shape the benchmark times it: 256 sequences, 64
+    heads (8 groups), headdim 64, dstate 128, chunk 128 (2048 blocks). Each sequence is
+    split after 100 to 227 tokens (all different open-chunk lengths) into a strict prefill
+    and 60 decode steps, so that most sequences cross a chunk end and are folded mid-batch.
+    The decode must give the one-shot prefill's bits; three sequences also go through the
+    oracle."""
+    w0 = W.config(4)
+    K, nseq = 60, 256
+    L1 = [100 + (s * 37) % 128 for s in range(nseq)]
+    w = W.Workload("strict_decode_full", nheads=w0.nheads, headdim=w0.headdim, ngroups=w0.ngroups,
+                   dstate=w0.dstate, chunk=w0.chunk, dtype=w0.dtype, seqlens=[a + K for a in L1], varlen=True,
+                   init="normal", seed=67)
+    inp = W.make_all(w, device=cuda_dev)
+    cu = inp["cu_seqlens"].tolist()
+    full = _cache(ssd, w, cuda_dev, inp["init_state"])
+    y_full, _ = ssd.strict_scan_fwd(inp["x"], inp["dt_raw"], inp["dt_bias"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                    full, resume=True, cu_seqlens=inp["cu_seqlens"])
+    split = _cache(ssd, w, cuda_dev, inp["init_state"])
+    rows = torch.cat([_seq_rows(cu, s, 0, L1[s], cuda_dev) for s in range(nseq)])
+    _prefill(ssd, w, inp, rows, L1, split)
+    ys = []
+    for k in range(K):
+        t = _rows(inp, torch.tensor([cu[s] + L1[s] + k for s in range(nseq)], device=cuda_dev))
+        ys.append(ssd.strict_state_update(split, t["x"], t["dt_raw"], inp["dt_bias"], inp["A"], t["B"], t["C"],
+                                          inp["D"]))
+    ssd.device_status()
+    dec_rows = torch.tensor([[cu[s] + L1[s] + k for s in range(nseq)] for k in range(K)], device=cuda_dev)
+    got = torch.stack(ys)
+    assert_same_bits(got, y_full[dec_rows], "decode part")
+    _assert_cache_equal(split, full, w.ngroups, w.nheads)
+    for s in (0, 97, 255):
+        sub = {k: (None if v is None else v.cpu()) for k, v in inp.items()}
+        a, b = cu[s], cu[s + 1]
+        y_ref, _ = O.ssd_scan(sub["x"][a:b], sub["dt_raw"][a:b], sub["dt_bias"], sub["A"], sub["B"][a:b],
+                              sub["C"][a:b], sub["D"], init_state=sub["init_state"][s:s + 1],
+                              cu_seqlens=torch.tensor([0, b - a], dtype=torch.int32))
+        assert rel_err(got[:, s].cpu(), y_ref[L1[s]:L1[s] + K]) <= TOL_Y[w.dtype]
+
