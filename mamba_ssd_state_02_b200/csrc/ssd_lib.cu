@@ -375,13 +375,15 @@ ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_ra
     const int32_t* slot_first = sub_first ? sub_first : first;
     const int H = pl.H, G = pl.G;
     int n = 0;
-    {
+    // A dense batch without snapshots: the segment-state pass writes the table itself.
+    const bool dense_table = !pl.varlen && pl.snap <= 0 && pl.max_segs > 0 && pl.T > 0;
+    if (!dense_table) {
         StageScope sc(ST_TABLE, st);
         k_chunk_table<<<1, kTableThreads, 0, st>>>(cu, pl.nseq, pl.T, pl.seqlen, pl.Ls, table, first, count,
                                                    pl.snap, reinterpret_cast<int32_t*>(ws + pl.off_snap_first),
                                                    order, sub_first, sub_end);
+        ++n;
     }
-    ++n;
     if (pl.max_segs > 0 && pl.T > 0) {
         CUtensorMap mx, mb, mc, my;
         const uint64_t T = (uint64_t)pl.T;
@@ -400,7 +402,8 @@ ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_ra
             tc::k_tc_segment_state<<<(unsigned)(pl.max_segs * (H / tc::kHeads)), tc::kThreadsA, tc::kSmemA,
                                      st>>>(mx, mb, dt_raw, dt_bias, A, table, count, H, G,
                                                                   seg_state, seg_acum, order, first, pl.snap,
-                                                                  g_test_stall.load() == 1);
+                                                                  g_test_stall.load() == 1, pl.nseq,
+                                                                  dense_table ? pl.seqlen : 0, pl.Ls);
         }
         ++n;
         {

@@ -104,12 +104,34 @@ constexpr int kThreadsA = 32 * (kScanWarpA + 2);
 __global__ void __launch_bounds__(kThreadsA, 1)
 k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_b,
                    const float* __restrict__ dt_raw, const float* __restrict__ dt_bias,
-                   const float* __restrict__ A, const ChunkEntry* __restrict__ segs,
-                   const int32_t* __restrict__ nsegs, int H, int G, float* __restrict__ seg_state,
+                   const float* __restrict__ A, ChunkEntry* __restrict__ segs,
+                   int32_t* __restrict__ nsegs, int H, int G, float* __restrict__ seg_state,
                    float* __restrict__ seg_acum, const int32_t* __restrict__ order,
-                   const int32_t* __restrict__ first, int64_t snap, int stall) {
+                   int32_t* __restrict__ first, int64_t snap, int stall, int nseq, int64_t dense_len, int Ls) {
     const int nq = H / kHeads;
-    if ((int)(blockIdx.x / nq) >= *nsegs) return;
+    // A dense batch without snapshots needs no table kernel: segment sg is piece sg % nps of
+    // sequence sg / nps (nps = segments per sequence), computed here from the grid (one CTA
+    // per (segment, 4 heads), exactly), and the first head quad's CTA writes the segment's
+    // table entry, the sequence's first segment and the count for the kernels that follow.
+    ChunkEntry dseg{0, 0, 0, 0};
+    if (dense_len > 0) {
+        const int nps = (int)((dense_len + Ls - 1) / Ls), sgd = (int)(blockIdx.x / nq);
+        const int sq = sgd / nps, k = sgd % nps;
+        dseg.seq = sq;
+        dseg.start = (int32_t)((int64_t)sq * dense_len + (int64_t)k * Ls);
+        dseg.len = (int32_t)min((int64_t)Ls, dense_len - (int64_t)k * Ls);
+        dseg.pad = sgd;
+        if (blockIdx.x % nq == 0 && threadIdx.x == 0) {
+            segs[sgd] = dseg;
+            if (k == 0) first[sq] = sgd;
+            if (sgd == nseq * nps - 1) {
+                first[nseq] = nseq * nps;
+                *nsegs = nseq * nps;
+            }
+        }
+    } else if ((int)(blockIdx.x / nq) >= *nsegs) {
+        return;
+    }
     const int sg = order ? order[blockIdx.x / nq] : (int)(blockIdx.x / nq);   // longest segments first
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -125,7 +147,7 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h0 = (blockIdx.x % nq) * kHeads, g = h0 / (H / G);
-    const ChunkEntry seg = segs[sg];
+    const ChunkEntry seg = dense_len > 0 ? dseg : segs[sg];
     const int ntiles = (seg.len + kTile - 1) / kTile;
     // State slots. Without snapshots the segment has one (seg.pad). With snapshots every
     // snap tokens the segment is cut at the multiples of snap inside it (counted from the
