@@ -385,9 +385,10 @@ ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_ra
         ++n;
     }
     if (pl.max_segs > 0 && pl.T > 0) {
-        CUtensorMap mx, mb, mc, my;
+        CUtensorMap mx, mxa, mb, mc, my;
         const uint64_t T = (uint64_t)pl.T;
         if (!make_map3(&mx, x, tc::kP, H, T, (uint64_t)tc::kP * 2, (uint64_t)H * tc::kP * 2, 64, 1, tc::kTile) ||
+            !make_map3(&mxa, x, tc::kP, H, T, (uint64_t)tc::kP * 2, (uint64_t)H * tc::kP * 2, 64, 1, tc::kTile / 2) ||
             !make_map3(&mb, B, tc::kN, G, T, (uint64_t)tc::kN * 2, (uint64_t)G * tc::kN * 2, 64, 1, tc::kTile) ||
             !make_map3(&mc, C, tc::kN, G, T, (uint64_t)tc::kN * 2, (uint64_t)G * tc::kN * 2, 64, 1, tc::kTile) ||
             !make_map3(&my, y, tc::kP, H, T, (uint64_t)tc::kP * 2, (uint64_t)H * tc::kP * 2, 64, 1, tc::kTile))
@@ -400,7 +401,7 @@ ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_ra
         {
             StageScope sc(ST_CHUNK_STATE, st);
             tc::k_tc_segment_state<<<(unsigned)(pl.max_segs * (H / tc::kHeads)), tc::kThreadsA, tc::kSmemA,
-                                     st>>>(mx, mb, dt_raw, dt_bias, A, table, count, H, G,
+                                     st>>>(mxa, mb, dt_raw, dt_bias, A, table, count, H, G,
                                                                   seg_state, seg_acum, order, first, pl.snap,
                                                                   g_test_stall.load() == 1, pl.nseq,
                                                                   dense_table ? pl.seqlen : 0, pl.Ls);

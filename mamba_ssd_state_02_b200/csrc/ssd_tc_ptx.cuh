@@ -131,6 +131,10 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
 }
 
 // Make generic-proxy shared-memory writes visible to the async proxy (UMMA, TMA).
+// Hardware barrier `id` (1..15) among `count` threads (whole warps) of the CTA.
+__device__ __forceinline__ void named_barrier(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
