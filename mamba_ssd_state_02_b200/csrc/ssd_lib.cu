@@ -388,7 +388,7 @@ ssd_status launch_tc(const Plan& pl, char* ws, const void* x, const float* dt_ra
         CUtensorMap mx, mxa, mb, mc, my;
         const uint64_t T = (uint64_t)pl.T;
         if (!make_map3(&mx, x, tc::kP, H, T, (uint64_t)tc::kP * 2, (uint64_t)H * tc::kP * 2, 64, 1, tc::kTile) ||
-            !make_map3(&mxa, x, tc::kP, H, T, (uint64_t)tc::kP * 2, (uint64_t)H * tc::kP * 2, 64, 1, tc::kTile / 2) ||
+            !make_map3(&mxa, x, tc::kP, H, T, (uint64_t)tc::kP * 2, (uint64_t)H * tc::kP * 2, 64, 1, tc::kXRows) ||
             !make_map3(&mb, B, tc::kN, G, T, (uint64_t)tc::kN * 2, (uint64_t)G * tc::kN * 2, 64, 1, tc::kTile) ||
             !make_map3(&mc, C, tc::kN, G, T, (uint64_t)tc::kN * 2, (uint64_t)G * tc::kN * 2, 64, 1, tc::kTile) ||
             !make_map3(&my, y, tc::kP, H, T, (uint64_t)tc::kP * 2, (uint64_t)H * tc::kP * 2, 64, 1, tc::kTile))

@@ -98,6 +98,8 @@ __device__ __forceinline__ bool wait_issue_warp(uint64_t* bar, uint32_t parity, 
 // pair's X is reloaded as soon as its UMMAs are done). TMEM: per pair p, columns 256p
 // + [S_hi h0 | S_hi h1 | S_lo h0 | S_lo h1] (64 each).
 constexpr int kSmemA = 192 * 1024 + 1024;
+constexpr int kXParts = 2;                    // x slot parts per chunk (2 or 4; 4 measured slower)
+constexpr int kXRows = kTile / kXParts;       // token rows per part
 constexpr int kScanWarpA = kRoleWarps + kComputeWarps;         // warps 18, 19: dt scan
 constexpr int kThreadsA = 32 * (kScanWarpA + 2);
 
@@ -140,11 +142,11 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
     auto xs = [&](int hh) { return sP + (hh >> 1) * 65536 + (hh & 1) * 16384; };           // x, then hi
     auto los = [&](int hh) { return sP + (hh >> 1) * 65536 + 32768 + (hh & 1) * 16384; };  // lo
     __shared__ __align__(16) float wts[4][kHeads][kTile];
-    // x slots by (head pair, 64-token half): the half's rows are loaded, formed into hi/lo
-    // and read by its four K-steps on barriers of their own, so a half is reloaded for the
-    // next chunk while the other half's UMMAs still run.
-    __shared__ uint64_t full_b[2], empty_b[2], full_x[2][2], pair_done[2][2], ops_ready[2][2], w_ready[4], w_free[4],
-        all_done,
+    // x slots by (head pair, part of kXParts token rows): a part's rows are loaded, formed
+    // into hi/lo and read by its K-steps on barriers of their own, so a part is reloaded for
+    // the next chunk while the later parts' UMMAs still run.
+    __shared__ uint64_t full_b[2], empty_b[2], full_x[2][kXParts], pair_done[2][kXParts], ops_ready[2][kXParts],
+        w_ready[4], w_free[4], all_done,
         drained, stall_bar;
     __shared__ uint32_t tmem_slot;
     __shared__ int abort_flag;
@@ -172,10 +174,10 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
         for (int i = 0; i < 2; ++i) {
             mbar_init(&full_b[i], 1);
             mbar_init(&empty_b[i], 1);
-            for (int hf = 0; hf < 2; ++hf) {
+            for (int hf = 0; hf < kXParts; ++hf) {
                 mbar_init(&full_x[i][hf], 1);
                 mbar_init(&pair_done[i][hf], 1);
-                mbar_init(&ops_ready[i][hf], kComputeWarps / 2);
+                mbar_init(&ops_ready[i][hf], kComputeWarps / kXParts);
             }
         }
         for (int i = 0; i < 4; ++i) {
@@ -204,7 +206,7 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             auto t0_of = [&](int k) { return seg.start + (ntiles - 1 - k) * kTile; };   // k-th chunk processed
-            int nb0 = 0, nb1 = 0, nx[2][2] = {{0, 0}, {0, 0}};   // phases issued on full_b[.], full_x[.][.]
+            int nb0 = 0, nb1 = 0, nx[2][kXParts] = {};      // phases issued on full_b[.], full_x[.][.]
             bool ok = true;
             for (int k = 0; k < ntiles && ok; ++k) {
                 const int t0 = t0_of(k), st = k & 1;
@@ -217,21 +219,20 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
                     const int tn = t0_of(k + 1);
                     tma_prefetch_3d(&map_b, 0, g, tn);
                     tma_prefetch_3d(&map_b, 64, g, tn);
-                    for (int hh = 0; hh < kHeads; ++hh) {
-                        tma_prefetch_3d(&map_x, 0, h0 + hh, tn);
-                        tma_prefetch_3d(&map_x, 0, h0 + hh, tn + kTile / 2);
-                    }
+                    for (int hh = 0; hh < kHeads; ++hh)
+                        for (int hf = 0; hf < kXParts; ++hf) tma_prefetch_3d(&map_x, 0, h0 + hh, tn + hf * kXRows);
                 }
                 for (int pr = 0; pr < 2 && ok; ++pr) {
-                    for (int hf = 0; hf < 2; ++hf) {
-                        // the half's slot rows (x, then hi) and lo rows are free
+                    for (int hf = 0; hf < kXParts; ++hf) {
+                        // the part's slot rows (x, then hi) and lo rows are free
                         if (k >= 1 && !wait_issue(&pair_done[pr][hf], (k - 1) & 1, abort_p)) {
                             ok = false;
                             break;
                         }
-                        mbar_arrive_expect_tx(&full_x[pr][hf], 16384);
+                        mbar_arrive_expect_tx(&full_x[pr][hf], 2 * kXRows * 128);
                         for (int hh = 2 * pr; hh < 2 * pr + 2; ++hh)
-                            tma_load_3d(xs(hh) + hf * 8192, &map_x, &full_x[pr][hf], 0, h0 + hh, t0 + hf * (kTile / 2));
+                            tma_load_3d(xs(hh) + hf * kXRows * 128, &map_x, &full_x[pr][hf], 0, h0 + hh,
+                                        t0 + hf * kXRows);
                         ++nx[pr][hf];
                     }
                 }
@@ -241,7 +242,7 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
             if (nb0) mbar_wait(&full_b[0], (nb0 - 1) & 1);
             if (nb1) mbar_wait(&full_b[1], (nb1 - 1) & 1);
             for (int pr = 0; pr < 2; ++pr)
-                for (int hf = 0; hf < 2; ++hf)
+                for (int hf = 0; hf < kXParts; ++hf)
                     if (nx[pr][hf]) mbar_wait(&full_x[pr][hf], (nx[pr][hf] - 1) & 1);
         }
     } else if (warp == 1) {
@@ -257,7 +258,7 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
             const uint64_t dB = smem_desc(smem_u32(sB + st * 32768), 16384, 1024);
             const bool fresh = opens(k);            // first chunk of a piece: overwrite the accumulator
             for (int pr = 0; pr < 2 && ok; ++pr) {
-                for (int hf = 0; hf < 2; ++hf) {
+                for (int hf = 0; hf < kXParts; ++hf) {
                     // test hook (stall): before the first head pair's UMMAs, a wait that runs out
                     if ((stall && k == 0 && hf == 0 && !wait_issue_warp(&stall_bar, 0, abort_p)) ||
                         !wait_issue_warp(&ops_ready[pr][hf], k & 1, abort_p)) {
@@ -269,12 +270,12 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
                     const uint64_t dp = desc_add(dP, pr * 65536);
                     if (elect_one()) {
 #pragma unroll
-                        for (int kk = 4 * hf; kk < 4 * hf + 4; ++kk)
+                        for (int kk = hf * (8 / kXParts); kk < (hf + 1) * (8 / kXParts); ++kk)
                             umma_bf16(d, desc_add(dB, kk * kMnStep), desc_add(dp, kk * kMnStep), idesc,
                                       !(kk == 0 && fresh));
                         umma_commit(&pair_done[pr][hf]);
-                        if (pr == 1 && hf == 1) umma_commit(&empty_b[st]);
-                        if (pr == 1 && hf == 1 && k == ntiles - 1) umma_commit(&all_done);
+                        if (pr == 1 && hf == kXParts - 1) umma_commit(&empty_b[st]);
+                        if (pr == 1 && hf == kXParts - 1 && k == ntiles - 1) umma_commit(&all_done);
                     }
                     __syncwarp();
                 }
@@ -371,7 +372,7 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
                 // Step k-1 closed a piece: once its UMMAs are done, store the piece's state
                 // before this step's operands are handed over (the UMMA warp waits for them
                 // and then overwrites the accumulator).
-                wait_abort(&pair_done[cw >> 1][1], (k - 1) & 1, abort_p);   // covers the pair's earlier MMAs
+                wait_abort(&pair_done[cw >> 1][kXParts - 1], (k - 1) & 1, abort_p);   // covers earlier MMAs
                 tc_fence_after();
                 store_state(slot_of(ntiles - k));
                 tc_fence_before();
@@ -381,7 +382,7 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
             }
             wait_abort(&w_ready[bf], (k >> 2) & 1, abort_p);
             for (int pr = 0; pr < 2; ++pr) {
-                wait_abort(&full_x[pr][q >> 1], k & 1, abort_p);     // rows r = 32 q + lane: half q >> 1
+                wait_abort(&full_x[pr][q / (4 / kXParts)], k & 1, abort_p);   // rows r = 32 q + lane
 #pragma unroll
                 for (int hh = 2 * pr; hh < 2 * pr + 2; ++hh) {
                     const float w = wts[bf][hh][r];
@@ -404,7 +405,7 @@ k_tc_segment_state(const __grid_constant__ CUtensorMap map_x, const __grid_const
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&ops_ready[pr][q >> 1]);
+                if (lane == 0) mbar_arrive(&ops_ready[pr][q / (4 / kXParts)]);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&w_free[bf]);
