@@ -90,3 +90,12 @@ def test_tc_many_segments(ssd, cuda_dev, seqlens, H, G, seg, segment_tokens):
     segment_tokens(seg)
     _check(ssd, cuda_dev, _tc_wl(seqlens, len(set(seqlens)) > 1, H=H, G=G, seed=48))
 
+
+@pytest.mark.parametrize("seg", [384, 1024])
+def test_tc_dense_table_from_the_grid(ssd, cuda_dev, seg, segment_tokens):
+    """A dense batch builds its segment table inside the segment-state pass (no table
+    kernel): three sequences of 1000 tokens cut into segments of 384 (three per sequence,
+    the last ragged) or 1024 (one, shorter than the segment)."""
+    segment_tokens(seg)
+    _check(ssd, cuda_dev, _tc_wl([1000] * 3, False, seed=49, dt_range=(1e-4, 0.5)))
+
