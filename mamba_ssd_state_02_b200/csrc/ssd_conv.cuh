@@ -154,7 +154,7 @@ __device__ __forceinline__ T* conv_dst(int64_t row, int c0, int HP, int GN, T* x
 // Prefill: block (token tile of kConvTokens, channel tile). seq_begin(s) gives packed
 // token offsets (cu_seqlens, or s * seqlen for a dense batch).
 template <typename T, int K>
-__global__ void __launch_bounds__(kConvThreads, 3)
+__global__ void __launch_bounds__(kConvThreads, 2)
 k_conv1d_fwd(const T* __restrict__ in, const float* __restrict__ w, const float* __restrict__ bias,
              const T* __restrict__ st_in, const int32_t* __restrict__ cu, int32_t nseq, int64_t T_,
              int64_t seqlen, int Dc, int HP, int GN, T* __restrict__ x, T* __restrict__ B,
@@ -184,61 +184,24 @@ k_conv1d_fwd(const T* __restrict__ in, const float* __restrict__ w, const float*
     else
 #pragma unroll
         for (int j = 0; j < 8; ++j) bv[j] = 0.f;
-    // Window: win[k] = input k positions before the current token (k = 1..K-1).
-    float win[K][8];
-    auto load_state = [&](int seq) {            // previous K-1 inputs of sequence seq's start
+    // History of the last K inputs as a circular buffer: the input of token t0 + i sits in
+    // hist[i % K], so the input k positions before it is hist[(i - k) % K]. The token loop
+    // runs in groups of K with the position in the group a compile-time constant, so every
+    // index is fixed and the window slides without register moves.
+    float hist[K][8];
+    auto state_in = [&](int seq, int k, float (&dst)[8]) {   // input k positions before seq's start
 #pragma unroll
-        for (int k = 1; k < K; ++k)
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-                win[k][j] = st_in ? to_f32(st_in[((int64_t)seq * Dc + c0 + j) * (K - 1) + (K - 1 - k)]) : 0.f;
+        for (int j = 0; j < 8; ++j)
+            dst[j] = st_in ? to_f32(st_in[((int64_t)seq * Dc + c0 + j) * (K - 1) + (K - 1 - k)]) : 0.f;
     };
     // Initial window for t0: inputs t0-1 .. t0-K+1, from the sequence, or from its
     // incoming state for positions before the sequence start.
 #pragma unroll
     for (int k = 1; k < K; ++k) {
         const int64_t tp = t0 - k;
-        if (tp >= sb) {
-            load8(in + tp * Dc + c0, win[k]);
-        } else {
-            const int64_t back = sb - tp;               // 1 .. K-1 positions before sb
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-                win[k][j] = st_in ? to_f32(st_in[((int64_t)s * Dc + c0 + j) * (K - 1) + (K - 1 - back)]) : 0.f;
-        }
+        if (tp >= sb) load8(in + tp * Dc + c0, hist[(K - k) % K]);
+        else state_in(s, (int)(sb - tp), hist[(K - k) % K]);
     }
-    // One token: output from the window, then slide the window; at a sequence's last
-    // token, the final conv state.
-    auto step = [&](int64_t t, const float (&cur)[8]) {
-        float o[8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int j = 2 * i;
-            float2 acc = tc::ffma2(make_float2(wk[K - 1][j], wk[K - 1][j + 1]), make_float2(cur[j], cur[j + 1]),
-                                   make_float2(bv[j], bv[j + 1]));
-#pragma unroll
-            for (int k = 1; k < K; ++k)
-                acc = tc::ffma2(make_float2(wk[K - 1 - k][j], wk[K - 1 - k][j + 1]),
-                                make_float2(win[k][j], win[k][j + 1]), acc);
-            const float2 v = silu2<T>(acc);
-            o[j] = v.x;
-            o[j + 1] = v.y;
-        }
-        store8(dst + t * dstride, o);
-#pragma unroll
-        for (int k = K - 1; k >= 2; --k)
-#pragma unroll
-            for (int j = 0; j < 8; ++j) win[k][j] = win[k - 1][j];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) win[1][j] = cur[j];
-        if (t == se - 1 && st_out) {
-#pragma unroll
-            for (int k = 1; k < K; ++k)
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    st_out[((int64_t)s * Dc + c0 + j) * (K - 1) + (K - 1 - k)] = from_f32<T>(win[k][j]);
-        }
-    };
     constexpr int R = conv_ring<T, K>();
     T* const ring = reinterpret_cast<T*>(sw);
     auto slot = [&](int k) { return ring + ((int64_t)k * kConvThreads + threadIdx.x) * 8; };
@@ -253,20 +216,49 @@ k_conv1d_fwd(const T* __restrict__ in, const float* __restrict__ w, const float*
         if (t0 + k < t1) issue(t0 + k, k);
         cp_async_commit();
     }
-    for (int64_t t = t0; t < t1; ++t) {
-        const int k = (int)(t - t0) & (R - 1);
-        cp_async_wait<R - 1>();                  // token t's group (the oldest pending) is done
-        float cur[8];
-        load8(slot(k), cur);
-        while (t >= se) {                        // next sequence (skipping empty ones)
-            ++s;
-            sb = seq_begin(s);
-            se = seq_begin(s + 1);
-            load_state(s);
+    for (int64_t tg = t0; tg < t1; tg += K) {
+#pragma unroll
+        for (int u = 0; u < K; ++u) {
+            const int64_t t = tg + u;
+            if (t >= t1) break;
+            const int kr = (int)(t - t0) & (R - 1);
+            cp_async_wait<R - 1>();              // token t's group (the oldest pending) is done
+            load8(slot(kr), hist[u]);
+            while (t >= se) {                    // next sequence (skipping empty ones)
+                ++s;
+                sb = seq_begin(s);
+                se = seq_begin(s + 1);
+#pragma unroll
+                for (int k = 1; k < K; ++k) state_in(s, k, hist[(u - k + K) % K]);
+            }
+            // Output: bias + taps over the inputs t-K+1 .. t, then SiLU; the final conv state
+            // (the last K-1 inputs) at a sequence's last token.
+            float o[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int j = 2 * i;
+                float2 acc = tc::ffma2(make_float2(wk[K - 1][j], wk[K - 1][j + 1]),
+                                       make_float2(hist[u][j], hist[u][j + 1]), make_float2(bv[j], bv[j + 1]));
+#pragma unroll
+                for (int k = 1; k < K; ++k)
+                    acc = tc::ffma2(make_float2(wk[K - 1 - k][j], wk[K - 1 - k][j + 1]),
+                                    make_float2(hist[(u - k + K) % K][j], hist[(u - k + K) % K][j + 1]), acc);
+                const float2 v = silu2<T>(acc);
+                o[j] = v.x;
+                o[j + 1] = v.y;
+            }
+            store8(dst + t * dstride, o);
+            if (t == se - 1 && st_out) {
+#pragma unroll
+                for (int k = 1; k < K; ++k)
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        st_out[((int64_t)s * Dc + c0 + j) * (K - 1) + (K - 1 - k)] =
+                            from_f32<T>(hist[(u - (k - 1) + K) % K][j]);
+            }
+            if (t + R < t1) issue(t + R, kr);   // slot kr was consumed above
+            cp_async_commit();
         }
-        step(t, cur);                            // consumes slot k before it is refilled
-        if (t + R < t1) issue(t + R, k);
-        cp_async_commit();
     }
 }
 
