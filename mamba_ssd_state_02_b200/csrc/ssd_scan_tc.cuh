@@ -88,15 +88,15 @@ __device__ __forceinline__ bool wait_issue_warp(uint64_t* bar, uint32_t parity, 
 // 0-1 and 2-3 (up to four chunks ahead; w_s = exp(sum_{r > s in seg} dt_r A) dt_s), and
 // the 16 compute warps write w*X as a bf16 hi/lo pair (hi in place over x, lo next to
 // it), so the product keeps ~16 mantissa bits: the FP32 final state is held to 1e-3.
-// Heads go in pairs: per pair one batch of 8 UMMAs with N = 256 ([hi|hi|lo|lo] of the
-// two heads side by side, B^T read once) accumulates S_hi and S_lo of the two heads in
-// TMEM; while it runs the compute warps prepare the other pair. At the end S = S_hi +
-// S_lo. Compute thread (cw, r) owns token row r and column quarter cw of every head's
-// w*X.
+// Heads go in pairs: per pair 8 UMMAs with N = 256 ([hi|hi|lo|lo] of the two heads side
+// by side, B^T read once) accumulate S_hi and S_lo of the two heads in TMEM, issued in
+// two batches of 4, one per 64-token half of the chunk; while they run the compute warps
+// prepare the other half or pair. At the end S = S_hi + S_lo. Compute thread (cw, r)
+// owns token row r (half r / 64) and column quarter cw of every head's w*X.
 //
-// Shared memory: two B stages; per head pair [x/hi h0 | x/hi h1 | lo h0 | lo h1] (the
-// pair's X is reloaded as soon as its UMMAs are done). TMEM: per pair p, columns 256p
-// + [S_hi h0 | S_hi h1 | S_lo h0 | S_lo h1] (64 each).
+// Shared memory: two B stages; per head pair [x/hi h0 | x/hi h1 | lo h0 | lo h1], each
+// half of a pair's rows reloaded as soon as that half's UMMAs are done. TMEM: per pair p,
+// columns 256p + [S_hi h0 | S_hi h1 | S_lo h0 | S_lo h1] (64 each).
 constexpr int kSmemA = 192 * 1024 + 1024;
 constexpr int kXParts = 2;                    // x slot parts per chunk (2 or 4; 4 measured slower)
 constexpr int kXRows = kTile / kXParts;       // token rows per part
