@@ -793,8 +793,10 @@ k_strict_chunk_scan_wide(const T* __restrict__ x, const T* __restrict__ B, const
                 }
             }
         }
-        // (2c) D skip and store.
+        // (2c) D skip and store. x_t of the tile's rows is the last (diagonal) source slice,
+        // still in shared memory (it starts at t0).
         const float Dh = D[h];
+        const T* xl = xs((nxs - 1) & 1);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int tt = r0 + i;
@@ -803,7 +805,7 @@ k_strict_chunk_scan_wide(const T* __restrict__ x, const T* __restrict__ B, const
             for (int j = 0; j < 4; ++j) {
                 const int64_t o = ((int64_t)(e.start + t0 + tt) * H + h) * P + p0 + j;
                 const float a = (i & 1) ? acc[i >> 1][j].y : acc[i >> 1][j].x;
-                y[o] = from_f32<T>(y_end(a, Dh, to_f32(x[o])));
+                y[o] = from_f32<T>(y_end(a, Dh, to_f32(xl[tt * P + p0 + j])));
             }
         }
     }
